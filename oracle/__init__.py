@@ -1,0 +1,182 @@
+"""CPU oracle for the AWQ per-layer scale search (numpy front end).
+
+TEST INFRASTRUCTURE ONLY.  The tests, ``__graft_entry__.smoke()`` and the
+bench's CPU-baseline leg are the only code allowed to import this package; the
+library's product path never does.  The arithmetic lives in plain C
+(``awq_oracle.c``), built here with gcc on first use.
+
+Each wrapper names the passage of the AWQ pages it follows; see the C file's
+header for the page list and the readings taken where the pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "awq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle_awq.so")
+
+STAT_MEAN = 0
+STAT_MAX = 1
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (IEEE fp32 quantiser: no fast-math, no FMA
+    contraction).  Returns the path of the shared library."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-std=c11", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
+               "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        I = ctypes.c_int
+        F = ctypes.c_float
+        lib.oracle_act_stats.argtypes = [P, I64, I64, I, P]
+        lib.oracle_act_stats.restype = None
+        lib.oracle_scales.argtypes = [P, I64, F, P]
+        lib.oracle_scales.restype = None
+        lib.oracle_quantize.argtypes = [P, P, I64, I64, I, I, P, P]
+        lib.oracle_quantize.restype = None
+        lib.oracle_pack.argtypes = [P, I64, I64, I, P]
+        lib.oracle_pack.restype = None
+        lib.oracle_loss_cols.argtypes = [P, P, P, I64, I64, I64, I, I, I, P, I64, P]
+        lib.oracle_loss_cols.restype = None
+        lib.oracle_search.argtypes = [P, P, P, I64, I64, I64, P, I, I, I, P, I64, P, P]
+        lib.oracle_search.restype = I
+        lib.oracle_literal_loss.argtypes = [P, P, P, I64, I64, I64, I, I]
+        lib.oracle_literal_loss.restype = ctypes.c_longdouble
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = I
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _as_bf16_bits(X) -> np.ndarray:
+    """Accept a torch bf16 tensor or a uint16 array of bf16 bit patterns."""
+    if isinstance(X, np.ndarray):
+        assert X.dtype == np.uint16
+        return np.ascontiguousarray(X)
+    import torch
+    assert X.dtype == torch.bfloat16
+    return np.ascontiguousarray(X.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def _f32(a) -> np.ndarray:
+    if not isinstance(a, np.ndarray):
+        a = a.detach().cpu().numpy()
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def act_stats(X, stat: int = STAT_MEAN) -> np.ndarray:
+    """a_j = mean_i |X_ij| (or max), fp64.  compassingai.com concept page,
+    "statistical basis of salient channels"."""
+    Xb = _as_bf16_bits(X)
+    N, D = Xb.shape
+    a = np.empty(D, dtype=np.float64)
+    _load().oracle_act_stats(_ptr(Xb), N, D, stat, _ptr(a))
+    return a
+
+
+def scales(a, alpha: float) -> np.ndarray:
+    """s_j = a_j^alpha (floored), fp32.  compassingai.com concept page, flow
+    step 3."""
+    a = _f32(a)
+    s = np.empty_like(a)
+    _load().oracle_scales(_ptr(a), a.shape[0], float(alpha), _ptr(s))
+    return s
+
+
+def quantize(W, s, bits: int, group: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Codes q [D_in, D_out] (int8) and deltas [D_in/group, D_out] (fp32) of
+    diag(s).W.  compassingai.com concept page, "quantisation math"."""
+    W = _f32(W)
+    D_in, D_out = W.shape
+    s = None if s is None else _f32(s)
+    q = np.empty((D_in, D_out), dtype=np.int8)
+    d = np.empty((D_in // group, D_out), dtype=np.float32)
+    _load().oracle_quantize(_ptr(W), _ptr(s), D_in, D_out, bits, group, _ptr(q), _ptr(d))
+    return q, d
+
+
+def pack(q: np.ndarray, bits: int) -> np.ndarray:
+    """uint32 [D_in/8, D_out]: 8 offset-binary codes per word, row 8k8+i in
+    nibble i."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    D_in, D_out = q.shape
+    out = np.empty((D_in // 8, D_out), dtype=np.uint32)
+    _load().oracle_pack(_ptr(q), D_in, D_out, bits, _ptr(out))
+    return out
+
+
+def loss_cols(X, W, s, bits: int, group: int, cols: Optional[Sequence[int]] = None,
+              quantize_w: bool = True) -> np.ndarray:
+    """Per-column share of ||X S^-1 Q(S W) - X W||^2 (fp64) for one scale
+    vector.  compassingai.com concept page, flow step 4c."""
+    Xb = _as_bf16_bits(X)
+    W = _f32(W)
+    N, D_in = Xb.shape
+    D_out = W.shape[1]
+    s = None if s is None else _f32(s)
+    c = None if cols is None else np.ascontiguousarray(cols, dtype=np.int64)
+    nc = D_out if c is None else c.shape[0]
+    out = np.empty(nc, dtype=np.float64)
+    _load().oracle_loss_cols(_ptr(Xb), _ptr(W), _ptr(s), N, D_in, D_out, bits, group,
+                             1 if quantize_w else 0, _ptr(c), 0 if c is None else nc, _ptr(out))
+    return out
+
+
+def search(X, W, a, alphas, bits: int, group: int, cols: Optional[Sequence[int]] = None,
+           want_cols: bool = False):
+    """Grid search over alpha: returns (L [n_alpha] fp64, best index[, L_col]).
+
+    compassingai.com concept page, flow steps 3-5; mudrobot.github.io notes,
+    "searching the optimal scale" (alpha* = argmin L(s_X^alpha) on [0, 1])."""
+    Xb = _as_bf16_bits(X)
+    W = _f32(W)
+    a = _f32(a)
+    al = _f32(alphas)
+    N, D_in = Xb.shape
+    D_out = W.shape[1]
+    c = None if cols is None else np.ascontiguousarray(cols, dtype=np.int64)
+    nc = D_out if c is None else c.shape[0]
+    L = np.empty(al.shape[0], dtype=np.float64)
+    Lc = np.empty((al.shape[0], nc), dtype=np.float64) if want_cols else None
+    best = _load().oracle_search(_ptr(Xb), _ptr(W), _ptr(a), N, D_in, D_out, _ptr(al), al.shape[0],
+                                 bits, group, _ptr(c), 0 if c is None else nc, _ptr(L), _ptr(Lc))
+    if want_cols:
+        return L, int(best), Lc
+    return L, int(best)
+
+
+def literal_loss(X, W, s, bits: int, group: int) -> float:
+    """||(X S^-1) Q(S W) - X W||_F^2 with every matrix materialised, in long
+    double (tiny layers only)."""
+    Xb = _as_bf16_bits(X)
+    W = _f32(W)
+    s = _f32(s)
+    N, D_in = Xb.shape
+    return float(_load().oracle_literal_loss(_ptr(Xb), _ptr(W), _ptr(s), N, D_in, W.shape[1], bits, group))

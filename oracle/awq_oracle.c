@@ -1,0 +1,323 @@
+/*
+ * awq_oracle.c -- plain, slow, obviously-correct CPU oracle for the AWQ
+ * per-layer activation-aware scale search.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the library's product path may load,
+ * call or link this file.  Only the tests, the smoke check and the bench's
+ * CPU-baseline leg use it.  It shares no code, header, table or constant with
+ * the CUDA path.
+ *
+ * Sources (each function names the passage it follows):
+ *   [P1] compassingai.com, "AWQ (Activation-aware Weight Quantization)" concept
+ *        page: "quantisation math" section (absmax symmetric b-bit group
+ *        quantiser), "statistical basis of salient channels" (activation_scale
+ *        = mean|X| or max), "full scale-optimisation flow" steps 1-6.
+ *   [P2] mudrobot.github.io, AWQ paper notes: "analysing the quantisation
+ *        error" (Q(w) = delta * Round(w / delta)) and "searching the optimal
+ *        scale" (L(s) = ||Q(W diag(s)) (diag(s)^-1 X) - W X||, s = s_X^alpha).
+ *
+ * Precision: the statistic and the loss are computed in fp64 (the loss via
+ * explicit loops, no BLAS).  The quantiser is defined on fp32 values with
+ * every operation correctly rounded (IEEE single, no contraction): that is the
+ * only reading under which "identical INT4 codes" is well defined.  Build with
+ * -O2 -fno-fast-math -ffp-contract=off.
+ *
+ * Readings taken where the pages are silent (see the design notes):
+ *   - delta = max|w| / (2^(b-1) - 1) with the clamp to +-(2^(b-1) - 1) of P1;
+ *     P2's max|w| / 2^(N-1) is a variant, not used here.
+ *   - round = round-half-to-even (IEEE default).
+ *   - an all-zero group has delta = 0 and all codes 0.
+ *   - a_j is floored at 1e-6 * max_j a_j (fp32 product) so that a dead channel
+ *     does not make S^-1 infinite; if every a_j is 0 the scales are all 1.
+ *   - s_j = (float) pow((double) a_j, (double) alpha).
+ *   - codes are stored offset-binary u = q + 2^(b-1), eight per 32-bit word,
+ *     nibble i (bits 4i..4i+3) = row 8*k8 + i of the column.
+ */
+#include <float.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_STAT_MEAN 0
+#define ORACLE_STAT_MAX 1
+
+static double bf16_bits_to_double(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* [P1] "statistical basis of salient channels": for every input channel j,
+ * activation_scale[j] = mean_i |X[i, j]| (or max_i |X[i, j]|).  [P2] "searching
+ * the optimal scale": s_X is the per-channel average activation magnitude. */
+void oracle_act_stats(const uint16_t *X, int64_t N, int64_t D, int stat, double *a)
+{
+    for (int64_t j = 0; j < D; ++j)
+        a[j] = 0.0;
+    for (int64_t i = 0; i < N; ++i) {
+        const uint16_t *row = X + i * D;
+        for (int64_t j = 0; j < D; ++j) {
+            double v = fabs(bf16_bits_to_double(row[j]));
+            if (stat == ORACLE_STAT_MAX) {
+                if (v > a[j])
+                    a[j] = v;
+            } else {
+                a[j] += v;
+            }
+        }
+    }
+    if (stat != ORACLE_STAT_MAX && N > 0)
+        for (int64_t j = 0; j < D; ++j)
+            a[j] /= (double)N;
+}
+
+/* [P1] flow step 3: s_j(alpha) = activation_scale[j]^alpha.  [P2]: s = s_X^alpha.
+ * Floor reading: see the header. */
+void oracle_scales(const float *a, int64_t D, float alpha, float *s)
+{
+    float amax = 0.0f;
+    for (int64_t j = 0; j < D; ++j)
+        if (a[j] > amax)
+            amax = a[j];
+    const float floor_ = 1e-6f * amax;
+    for (int64_t j = 0; j < D; ++j) {
+        float aj;
+        if (amax == 0.0f)
+            aj = 1.0f;
+        else
+            aj = a[j] > floor_ ? a[j] : floor_;
+        s[j] = (float)pow((double)aj, (double)alpha);
+    }
+}
+
+/* [P1] "quantisation math", steps 1-3, applied to one group of one column of
+ * W' = diag(s) W ([P1] flow step 4a):
+ *   w'_k  = fl32(s_k * w_k)
+ *   delta = fl32(max_k |w'_k| / (2^(b-1) - 1))
+ *   q_k   = clamp(round(fl32(w'_k / delta)), -(2^(b-1)-1), 2^(b-1)-1)
+ * s == NULL means s_k = 1 (no scaling). */
+static void quantize_group(const float *W, const float *s, int64_t D_out, int64_t n,
+                           int64_t k0, int group, int bits, int8_t *q, float *delta)
+{
+    const int qmax = (1 << (bits - 1)) - 1;
+    float m = 0.0f;
+    for (int k = 0; k < group; ++k) {
+        float w = W[(k0 + k) * D_out + n];
+        float wp = s ? s[k0 + k] * w : w;
+        float am = fabsf(wp);
+        if (am > m)
+            m = am;
+    }
+    const float d = m / (float)qmax;
+    *delta = d;
+    for (int k = 0; k < group; ++k) {
+        int code = 0;
+        if (d != 0.0f) {
+            float w = W[(k0 + k) * D_out + n];
+            float wp = s ? s[k0 + k] * w : w;
+            float t = wp / d;
+            float r = nearbyintf(t); /* round half to even in the default mode */
+            if (r > (float)qmax)
+                r = (float)qmax;
+            if (r < (float)-qmax)
+                r = (float)-qmax;
+            code = (int)r;
+        }
+        q[k] = (int8_t)code;
+    }
+}
+
+/* Quantise every (group, column) of diag(s) W.  q: [D_in][D_out] codes in
+ * [-qmax, qmax]; delta: [D_in/group][D_out]. */
+void oracle_quantize(const float *W, const float *s, int64_t D_in, int64_t D_out,
+                     int bits, int group, int8_t *q, float *delta)
+{
+    int8_t *col = (int8_t *)malloc((size_t)group);
+    for (int64_t n = 0; n < D_out; ++n) {
+        for (int64_t g = 0; g < D_in / group; ++g) {
+            quantize_group(W, s, D_out, n, g * group, group, bits, col, &delta[g * D_out + n]);
+            for (int k = 0; k < group; ++k)
+                q[(g * group + k) * D_out + n] = col[k];
+        }
+    }
+    free(col);
+}
+
+/* Pack codes: word (k8, n) holds rows 8*k8 .. 8*k8+7 of column n, row 8*k8+i in
+ * bits 4i..4i+3 as u = q + 2^(b-1).  [P1] "inference-time equivalent":
+ * W_quantized = Quantize(diag(s*) W) stored as INT4. */
+void oracle_pack(const int8_t *q, int64_t D_in, int64_t D_out, int bits, uint32_t *packed)
+{
+    const int off = 1 << (bits - 1);
+    for (int64_t k8 = 0; k8 < D_in / 8; ++k8) {
+        for (int64_t n = 0; n < D_out; ++n) {
+            uint32_t word = 0;
+            for (int i = 0; i < 8; ++i) {
+                int u = (int)q[(8 * k8 + i) * D_out + n] + off;
+                word |= ((uint32_t)u & 0xFu) << (4 * i);
+            }
+            packed[k8 * D_out + n] = word;
+        }
+    }
+}
+
+/* [P1] flow step 4c for a set of output columns:
+ *   L_n = sum_i ( sum_k x_ik * e_kn )^2,   e_kn = q_kn * delta_gn / s_k - w_kn
+ * which is column n's share of ||X S^-1 Q(S W) - X W||^2 (exact algebra: the
+ * k-th row of S^-1 Q(SW) is q_kn delta_gn / s_k).  All in fp64.
+ * quantize == 0 replaces Q by the identity (w'_k itself), for the
+ * cancellation check. */
+static double column_loss(const double *Xd, const float *W, const float *s,
+                          int64_t N, int64_t D_in, int64_t D_out, int64_t n,
+                          int bits, int group, int quantize, double *e, int8_t *qcol)
+{
+    for (int64_t g = 0; g < D_in / group; ++g) {
+        const int64_t k0 = g * group;
+        if (quantize) {
+            float d;
+            quantize_group(W, s, D_out, n, k0, group, bits, qcol, &d);
+            for (int k = 0; k < group; ++k) {
+                double sk = s ? (double)s[k0 + k] : 1.0;
+                e[k0 + k] = (double)qcol[k] * (double)d / sk - (double)W[(k0 + k) * D_out + n];
+            }
+        } else {
+            for (int k = 0; k < group; ++k) {
+                float w = W[(k0 + k) * D_out + n];
+                float wp = s ? s[k0 + k] * w : w;
+                double sk = s ? (double)s[k0 + k] : 1.0;
+                e[k0 + k] = (double)wp / sk - (double)w;
+            }
+        }
+    }
+    double acc = 0.0;
+    for (int64_t i = 0; i < N; ++i) {
+        const double *xr = Xd + i * D_in;
+        double y = 0.0;
+        for (int64_t k = 0; k < D_in; ++k)
+            y += xr[k] * e[k];
+        acc += y * y;
+    }
+    return acc;
+}
+
+static double *x_to_double(const uint16_t *X, int64_t N, int64_t D_in)
+{
+    double *Xd = (double *)malloc((size_t)(N * D_in) * sizeof(double));
+    for (int64_t i = 0; i < N * D_in; ++i)
+        Xd[i] = bf16_bits_to_double(X[i]);
+    return Xd;
+}
+
+/* Per-column losses for one scale vector s (NULL = all ones).  cols == NULL
+ * means every column; otherwise L_col[c] is the loss of column cols[c]. */
+void oracle_loss_cols(const uint16_t *X, const float *W, const float *s,
+                      int64_t N, int64_t D_in, int64_t D_out, int bits, int group,
+                      int quantize, const int64_t *cols, int64_t ncols, double *L_col)
+{
+    double *Xd = x_to_double(X, N, D_in);
+    const int64_t nc = cols ? ncols : D_out;
+#pragma omp parallel
+    {
+        double *e = (double *)malloc((size_t)D_in * sizeof(double));
+        int8_t *qcol = (int8_t *)malloc((size_t)group);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t c = 0; c < nc; ++c) {
+            int64_t n = cols ? cols[c] : c;
+            L_col[c] = column_loss(Xd, W, s, N, D_in, D_out, n, bits, group, quantize, e, qcol);
+        }
+        free(e);
+        free(qcol);
+    }
+    free(Xd);
+}
+
+/* [P1] flow steps 3-5 for one layer: for every alpha on the grid, s = a^alpha,
+ * quantise diag(s) W per group, L(alpha) = ||X S^-1 Q(SW) - X W||^2, and
+ * alpha* = argmin L (the smallest index among exact minima).
+ * L: [n_alpha]; L_col: [n_alpha][ncols] (may be NULL); restricted to the
+ * columns in cols when cols != NULL (L then sums those columns only).
+ * Returns the argmin index. */
+int oracle_search(const uint16_t *X, const float *W, const float *a,
+                  int64_t N, int64_t D_in, int64_t D_out,
+                  const float *alphas, int n_alpha, int bits, int group,
+                  const int64_t *cols, int64_t ncols, double *L, double *L_col)
+{
+    const int64_t nc = cols ? ncols : D_out;
+    float *s = (float *)malloc((size_t)D_in * sizeof(float));
+    double *lc = (double *)malloc((size_t)nc * sizeof(double));
+    int best = 0;
+    for (int ai = 0; ai < n_alpha; ++ai) {
+        oracle_scales(a, D_in, alphas[ai], s);
+        oracle_loss_cols(X, W, s, N, D_in, D_out, bits, group, 1, cols, ncols, lc);
+        double sum = 0.0;
+        for (int64_t c = 0; c < nc; ++c) {
+            sum += lc[c];
+            if (L_col)
+                L_col[(int64_t)ai * nc + c] = lc[c];
+        }
+        L[ai] = sum;
+        if (L[ai] < L[best])
+            best = ai;
+    }
+    free(lc);
+    free(s);
+    return best;
+}
+
+/* The literal two-product form of [P1] flow step 4c for tiny layers:
+ * materialise S^-1 (D_in x D_in), W_hat' = Q(S W) (D_in x D_out, codes times
+ * delta), then L = ||(X S^-1) W_hat' - X W||_F^2, all in long double. */
+long double oracle_literal_loss(const uint16_t *X, const float *W, const float *s,
+                                int64_t N, int64_t D_in, int64_t D_out, int bits, int group)
+{
+    long double *Sinv = (long double *)calloc((size_t)(D_in * D_in), sizeof(long double));
+    long double *What = (long double *)malloc((size_t)(D_in * D_out) * sizeof(long double));
+    long double *XS = (long double *)malloc((size_t)(N * D_in) * sizeof(long double));
+    int8_t *q = (int8_t *)malloc((size_t)(D_in * D_out));
+    float *delta = (float *)malloc((size_t)(D_in / group * D_out) * sizeof(float));
+    for (int64_t k = 0; k < D_in; ++k)
+        Sinv[k * D_in + k] = 1.0L / (long double)s[k];
+    oracle_quantize(W, s, D_in, D_out, bits, group, q, delta);
+    for (int64_t k = 0; k < D_in; ++k)
+        for (int64_t n = 0; n < D_out; ++n)
+            What[k * D_out + n] = (long double)q[k * D_out + n] * (long double)delta[(k / group) * D_out + n];
+    for (int64_t i = 0; i < N; ++i)
+        for (int64_t c = 0; c < D_in; ++c) {
+            long double acc = 0.0L;
+            for (int64_t k = 0; k < D_in; ++k)
+                acc += (long double)bf16_bits_to_double(X[i * D_in + k]) * Sinv[k * D_in + c];
+            XS[i * D_in + c] = acc;
+        }
+    long double L = 0.0L;
+    for (int64_t i = 0; i < N; ++i)
+        for (int64_t n = 0; n < D_out; ++n) {
+            long double yq = 0.0L, y = 0.0L;
+            for (int64_t k = 0; k < D_in; ++k) {
+                yq += XS[i * D_in + k] * What[k * D_out + n];
+                y += (long double)bf16_bits_to_double(X[i * D_in + k]) * (long double)W[k * D_out + n];
+            }
+            L += (yq - y) * (yq - y);
+        }
+    free(Sinv);
+    free(What);
+    free(XS);
+    free(q);
+    free(delta);
+    return L;
+}
+
+/* Number of OpenMP threads the loss loops use (reported with CPU timings). */
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,271 @@
+"""Pins that tie the CPU oracle to what the AWQ pages and plain mathematics
+fix, independently of the oracle's own code.
+
+Each test names the passage or the mathematical fact it checks:
+hand-worked examples from the pages' quantiser definition (golden files),
+special cases that reduce to a textbook routine (alpha = 0 is plain RTN),
+exact identities (S^-1 and S cancel without quantisation; power-of-two scale
+invariance; sign symmetry), bounds (|q| <= qmax, |error| <= delta / 2), a
+library check of the loss (numpy fp64 matmul) and brute force on tiny layers.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from post_weight_only_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16(x: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+
+
+def _small(N, D_in, D_out, seed=0, **kw):
+    return synth.layer_inputs(synth.small_layer(N, D_in, D_out, seed=seed, **kw))
+
+
+def _rtn_numpy(W: np.ndarray, bits: int, group: int):
+    """Plain round-to-nearest absmax group quantiser written with numpy float32
+    primitives (the RTN baseline of the mudrobot.github.io notes, "baselines")."""
+    qmax = np.float32(2 ** (bits - 1) - 1)
+    D_in, D_out = W.shape
+    Wg = W.reshape(D_in // group, group, D_out).astype(np.float32)
+    m = np.abs(Wg).max(axis=1)                                   # [G, D_out]
+    d = (m / qmax).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = (Wg / d[:, None, :]).astype(np.float32)
+    q = np.clip(np.round(t), -qmax, qmax)                         # np.round: half to even
+    q = np.where(d[:, None, :] == 0, 0, q).astype(np.int8)
+    return q.reshape(D_in, D_out), d
+
+
+# --------------------------------------------------------------------------
+# Hand-worked examples (golden files)
+# --------------------------------------------------------------------------
+
+def test_hand_group_codes_pack_and_delta():
+    g = json.load(open(os.path.join(GOLDEN, "hand_group_b4_g128.json")))
+    W = np.zeros((128, 1), dtype=np.float32)
+    W[:7, 0] = np.array(g["w_rows_0_to_6"], dtype=np.float32)
+    q, d = oracle.quantize(W, None, g["bits"], g["group"])
+    assert d[0, 0] == np.float32(g["delta"])
+    assert q[:8, 0].tolist() == g["q_rows_0_to_7"]
+    assert (q[8:, 0] == 0).all()
+    packed = oracle.pack(q, g["bits"])
+    assert packed.shape == (16, 1)
+    assert int(packed[0, 0]) == int(g["packed_word_0"], 16)
+    assert all(int(v) == int(g["packed_words_1_to_15"], 16) for v in packed[1:, 0])
+    err = q[:6, 0].astype(np.float64) * float(d[0, 0]) - W[:6, 0].astype(np.float64)
+    assert err.tolist() == g["errors_rows_0_to_5"]
+
+
+def test_hand_group_loss_and_tie_break():
+    g = json.load(open(os.path.join(GOLDEN, "hand_group_b4_g128.json")))
+    W = np.zeros((128, 1), dtype=np.float32)
+    W[:7, 0] = np.array(g["w_rows_0_to_6"], dtype=np.float32)
+    X = _bf16(np.ones((1, 128), dtype=np.float32))
+    a = oracle.act_stats(X)
+    assert (a == 1.0).all()
+    alphas = synth.alpha_grid(20).numpy()
+    L, best = oracle.search(X, W, a.astype(np.float32), alphas, 4, 128)
+    expect = (-0.0625 + 0.125 - float(np.float32(0.1))) ** 2
+    assert np.allclose(L, expect, rtol=1e-14, atol=0)
+    assert len(set(L.tolist())) == 1          # bit-identical for every alpha
+    assert best == g["alpha_star_index"]
+
+
+def test_scalar_example_page3():
+    g = json.load(open(os.path.join(GOLDEN, "scalar_example_page3.json")))
+    W = np.zeros((g["group"], 1), dtype=np.float32)
+    W[:2, 0] = np.array(g["group_values"], dtype=np.float32)
+    q, d = oracle.quantize(W, None, g["bits"], g["group"])
+    assert d[0, 0] == np.float32(g["delta"])
+    assert q[:2, 0].tolist() == g["q"]
+    w_hat = float(q[1, 0]) * float(d[0, 0])
+    assert w_hat == g["w_hat_of_1.23"]
+    assert abs((w_hat - float(np.float32(1.23))) - g["error_of_1.23"]) < 1e-7
+
+
+# --------------------------------------------------------------------------
+# Special cases and identities
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (3, 128), (4, 64), (2, 32)])
+def test_alpha_zero_is_plain_rtn(bits, group):
+    """alpha = 0 gives s = 1 exactly, i.e. no scaling: the codes degenerate to
+    plain RTN (compassingai.com concept page, "scale search": alpha = 0 means
+    no scaling, plain uniform quantisation)."""
+    X, W = _small(64, 256, 40, seed=3)
+    a = oracle.act_stats(X).astype(np.float32)
+    s0 = oracle.scales(a, 0.0)
+    assert (s0 == 1.0).all()
+    q, d = oracle.quantize(W, s0, bits, group)
+    q_rtn, d_rtn = _rtn_numpy(W.numpy(), bits, group)
+    assert np.array_equal(q, q_rtn)
+    assert np.array_equal(d, d_rtn)
+    L, _, Lc = oracle.search(X, W, a, np.array([0.0], dtype=np.float32), bits, group, want_cols=True)
+    L_plain = oracle.loss_cols(X, W, None, bits, group)
+    assert np.array_equal(Lc[0], L_plain)          # column by column, bit for bit
+    assert np.isclose(L[0], L_plain.sum(), rtol=1e-13)
+
+
+def test_cancellation_without_quantisation():
+    """With Q replaced by the identity, X S^-1 (S W) = X W: the transform is
+    exactly equivalent (compassingai.com concept page, "core mechanism";
+    laojiahuo2003.github.io notes, AWQ section: W'x' = Wx).  Only the fp32
+    rounding of s*w is left, ~2^-24 relative."""
+    X, W = _small(32, 256, 24, seed=5)
+    a = oracle.act_stats(X).astype(np.float32)
+    Y = X.double() @ W.double()
+    ref = float((Y * Y).sum())
+    for alpha in (0.0, 0.35, 1.0):
+        s = oracle.scales(a, alpha)
+        L = oracle.loss_cols(X, W, s, 4, 128, quantize_w=False).sum()
+        assert L <= 1e-12 * ref
+
+
+def test_power_of_two_scale_invariance_and_sign_symmetry():
+    """The absmax definition makes the codes invariant to s -> 2^t s (delta
+    scales by 2^t, exactly in fp32) and antisymmetric in W -> -W; the loss is
+    unchanged in both cases."""
+    X, W = _small(32, 256, 24, seed=7)
+    a = oracle.act_stats(X).astype(np.float32)
+    s = oracle.scales(a, 0.5)
+    q, d = oracle.quantize(W, s, 4, 128)
+    for t in (-3, 5):
+        q2, d2 = oracle.quantize(W, (s * np.float32(2.0 ** t)).astype(np.float32), 4, 128)
+        assert np.array_equal(q, q2)
+        assert np.array_equal(d2, (d * np.float32(2.0 ** t)).astype(np.float32))
+    qn, dn = oracle.quantize(-W, s, 4, 128)
+    assert np.array_equal(qn, -q) and np.array_equal(dn, d)
+    L1 = oracle.loss_cols(X, W, s, 4, 128).sum()
+    L2 = oracle.loss_cols(X, W, (s * np.float32(8.0)).astype(np.float32), 4, 128).sum()
+    L3 = oracle.loss_cols(X, -W, s, 4, 128).sum()
+    assert np.isclose(L1, L2, rtol=1e-12) and np.isclose(L1, L3, rtol=1e-12)
+
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (3, 128), (4, 64), (2, 32), (3, 32)])
+def test_quantiser_bounds(bits, group):
+    """|q| <= 2^(b-1)-1 (the clamp of the concept page), |w' - q delta| <=
+    delta/2 (the rounding error lies in [0, 0.5] steps: mudrobot.github.io notes,
+    "analysing the quantisation error"), and every non-zero group reaches
+    |q| = qmax at its largest element."""
+    X, W = _small(16, 512, 64, seed=11)
+    a = oracle.act_stats(X).astype(np.float32)
+    s = oracle.scales(a, 0.6)
+    q, d = oracle.quantize(W, s, bits, group)
+    qmax = 2 ** (bits - 1) - 1
+    assert np.abs(q.astype(np.int32)).max() <= qmax
+    Wp = (s[:, None].astype(np.float32) * W.numpy()).astype(np.float32)
+    dd = np.repeat(d, group, axis=0).astype(np.float64)
+    err = np.abs(Wp.astype(np.float64) - q.astype(np.float64) * dd)
+    assert (err <= dd / 2 * (1 + 1e-6)).all()
+    qg = np.abs(q.astype(np.int32)).reshape(-1, group, q.shape[1]).max(axis=1)
+    assert (qg[d > 0] == qmax).all()
+
+
+def test_rounding_error_statistics():
+    """The rounding error, in units of delta, is roughly uniform on [0, 0.5]
+    with mean ~0.25 (mudrobot.github.io notes, "analysing the quantisation
+    error", item 1).  Statistical, loose tolerance."""
+    W = synth.make_w(4096, 64, 0.02, 123)
+    q, d = oracle.quantize(W, None, 4, 128)
+    dd = np.repeat(d, 128, axis=0).astype(np.float64)
+    r = np.abs(W.numpy().astype(np.float64) - q * dd) / dd
+    assert abs(r.mean() - 0.25) < 0.01
+    hist, _ = np.histogram(r, bins=5, range=(0, 0.5))
+    frac = hist / hist.sum()
+    assert np.all(np.abs(frac - 0.2) < 0.02)
+
+
+# --------------------------------------------------------------------------
+# Statistic, scales, packing
+# --------------------------------------------------------------------------
+
+def test_act_stats_matches_numpy():
+    X, _ = _small(100, 264, 8, seed=2)
+    xf = X.float().numpy().astype(np.float64)
+    assert np.allclose(oracle.act_stats(X, oracle.STAT_MEAN), np.abs(xf).mean(axis=0), rtol=1e-14)
+    assert np.array_equal(oracle.act_stats(X, oracle.STAT_MAX), np.abs(xf).max(axis=0))
+
+
+def test_scales_special_values():
+    a = np.array([0.5, 2.0, 0.0, 3.0], dtype=np.float32)
+    assert (oracle.scales(a, 0.0) == 1.0).all()
+    s1 = oracle.scales(a, 1.0)
+    assert s1[0] == 0.5 and s1[1] == 2.0 and s1[3] == 3.0
+    assert s1[2] == np.float32(1e-6) * np.float32(3.0)          # floored dead channel
+    sh = oracle.scales(a, 0.5)
+    assert sh[1] == np.float32(np.sqrt(2.0))
+    assert (oracle.scales(np.zeros(4, np.float32), 0.7) == 1.0).all()
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_pack_roundtrip(bits):
+    rng = np.random.default_rng(0)
+    qmax = 2 ** (bits - 1) - 1
+    q = rng.integers(-qmax, qmax + 1, size=(64, 12)).astype(np.int8)
+    p = oracle.pack(q, bits)
+    u = np.stack([(p >> (4 * i)) & 0xF for i in range(8)], axis=1)   # [D_in/8, 8, D_out]
+    back = u.reshape(64, 12).astype(np.int32) - 2 ** (bits - 1)
+    assert np.array_equal(back, q.astype(np.int32))
+
+
+# --------------------------------------------------------------------------
+# The loss: library check, literal form, brute-force argmin
+# --------------------------------------------------------------------------
+
+def test_loss_matches_numpy_matmul():
+    X, W = _small(48, 256, 20, seed=9)
+    a = oracle.act_stats(X).astype(np.float32)
+    s = oracle.scales(a, 0.45)
+    q, d = oracle.quantize(W, s, 4, 128)
+    E = q.astype(np.float64) * np.repeat(d, 128, axis=0).astype(np.float64) / s[:, None].astype(np.float64) \
+        - W.numpy().astype(np.float64)
+    Y = X.float().numpy().astype(np.float64) @ E
+    ref = (Y * Y).sum(axis=0)
+    got = oracle.loss_cols(X, W, s, 4, 128)
+    assert np.allclose(got, ref, rtol=1e-11)
+    cols = [3, 17, 0]
+    assert np.allclose(oracle.loss_cols(X, W, s, 4, 128, cols=cols), ref[cols], rtol=1e-11)
+
+
+@pytest.mark.parametrize("D_in,D_out,N,seed", [(128, 4, 8, 0), (256, 8, 16, 1), (256, 3, 5, 2)])
+def test_literal_form_and_brute_force_argmin(D_in, D_out, N, seed):
+    """Materialise S^-1 and Q(S W) and evaluate ||X S^-1 Q(SW) - X W||^2
+    literally (long double) for every alpha: it must equal the oracle's
+    column-sum form, and the argmin over the grid must agree."""
+    X, W = _small(N, D_in, D_out, seed=seed, n_outlier=2)
+    a = oracle.act_stats(X).astype(np.float32)
+    alphas = synth.alpha_grid(20).numpy()
+    L, best = oracle.search(X, W, a, alphas, 4, 128)
+    lit = np.array([oracle.literal_loss(X, W, oracle.scales(a, al), 4, 128) for al in alphas])
+    assert np.allclose(L, lit, rtol=1e-9)
+    assert best == int(np.argmin(lit))
+
+
+def test_search_column_subset_sums():
+    X, W = _small(40, 256, 16, seed=4)
+    a = oracle.act_stats(X).astype(np.float32)
+    alphas = synth.alpha_grid(4).numpy()
+    L, best, Lc = oracle.search(X, W, a, alphas, 3, 64, want_cols=True)
+    assert np.allclose(Lc.sum(axis=1), L, rtol=1e-13)
+    cols = [1, 7, 15]
+    Ls, _, Lcs = oracle.search(X, W, a, alphas, 3, 64, cols=cols, want_cols=True)
+    assert np.allclose(Lcs, Lc[:, cols], rtol=1e-13)
+    assert np.allclose(Ls, Lc[:, cols].sum(axis=1), rtol=1e-13)
+
+
+def test_outlier_channels_pull_alpha_up():
+    """Sanity (not a pin): on a layer with strong outlier channels the search
+    picks alpha > 0, i.e. scaling beats plain RTN (the pages' central claim)."""
+    X, W = _small(128, 512, 32, seed=1, n_outlier=5)
+    a = oracle.act_stats(X).astype(np.float32)
+    alphas = synth.alpha_grid(20).numpy()
+    L, best = oracle.search(X, W, a, alphas, 4, 128)
+    assert best > 0 and L[best] < L[0]
