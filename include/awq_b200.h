@@ -1,0 +1,234 @@
+/*
+ * awq_b200.h -- C ABI of the B200 (sm_100a) AWQ per-layer scale search.
+ *
+ * The library evaluates, for ONE linear layer Y = X W, the activation-aware
+ * scale search of AWQ and quantises the weights with the chosen scales:
+ *   1. a_j = mean_i |X_ij| (or max)                       -> awq_act_stats
+ *   2. s_j(alpha) = a_j^alpha for every alpha on a grid    -> awq_scales
+ *   3. W' = diag(s) W, symmetric absmax per-group b-bit quantisation along D_in
+ *   4. L(alpha) = || X S^-1 Q(S W) - X W ||^2
+ *   5. alpha* = argmin L                                   -> awq_search (2-5)
+ *   6. the final INT codes + per-group scales for s*       -> awq_quantize_pack
+ * Passages: compassingai.com AWQ concept page, "statistical basis of salient
+ * channels" (step 1), "full scale-optimisation flow" steps 1-6 (steps 2-5),
+ * "quantisation math" (step 3), "inference-time equivalent" (step 6);
+ * mudrobot.github.io AWQ notes, "searching the optimal scale" (s = s_X^alpha,
+ * alpha* = argmin over [0, 1]).
+ *
+ * Conventions for every call:
+ *   - Matrices are dense row-major.  X: N x D_in bf16 (raw 16-bit patterns),
+ *     W: D_in x D_out fp32 (the Y = X W orientation: scales act on the rows of
+ *     W, groups run along D_in).
+ *   - Every pointer argument is a DEVICE pointer owned by the caller unless
+ *     its comment says "host".  Device pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     only enqueue work; they are asynchronous with respect to the host and
+ *     do not synchronise.  The library allocates no device memory: scratch
+ *     space comes from a caller-provided workspace whose size is queried.
+ *   - The return value is an awq_status.  A non-OK status from argument
+ *     checking is returned before any work is enqueued; awq_get_last_error()
+ *     then describes it.  Errors found on the device (a wait that timed out)
+ *     are written to the caller's device status word (see awq_search).
+ *   - Inputs are assumed finite; NaN or Inf inputs give unspecified (but
+ *     memory-safe) results.
+ *   - Supported bit widths are 2, 3 and 4 (codes are stored as 4-bit
+ *     offset-binary values); group sizes are 32, 64 and 128.
+ */
+#ifndef AWQ_B200_H
+#define AWQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define AWQ_API __attribute__((visibility("default")))
+#else
+#define AWQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  AWQ_OK = 0,
+  AWQ_EINVAL = 1,        /* bad size, null pointer, bad enum value */
+  AWQ_EALIGN = 2,        /* a device pointer is not 16-byte aligned */
+  AWQ_EUNSUPPORTED = 3,  /* bits/group/n_alpha outside the supported set, or no sm_100 device */
+  AWQ_EWORKSPACE = 4,    /* workspace too small or null */
+  AWQ_ECUDA = 5,         /* a CUDA call failed; awq_get_last_error() has its message */
+  AWQ_ETIMEOUT = 6       /* device only: a pipeline wait gave up (written to the status word) */
+} awq_status;
+
+enum { AWQ_STAT_MEAN = 0, AWQ_STAT_MAX = 1 };
+
+/*
+ * How awq_search evaluates L(alpha) = || X S^-1 Q(S W) - X W ||^2 on the tensor
+ * cores (identical in exact arithmetic):
+ *   AWQ_LOSS_ERROR      L = || X E ||^2 with E = S^-1 Q(S W) - W formed per
+ *                       weight in fp32 (from the quantiser's rounding residual,
+ *                       kept to 1/128 of a quantisation step) and rounded to
+ *                       bf16 once; the default, and the more accurate form.
+ *   AWQ_LOSS_REFERENCE  the reference output X W is computed once per tile by
+ *                       the same GEMM (bf16 W) and subtracted from
+ *                       X S^-1 Q(S W) (bf16 operands) in the epilogue.
+ */
+enum { AWQ_LOSS_ERROR = 0, AWQ_LOSS_REFERENCE = 1 };
+
+/* Largest alpha grid accepted by awq_search. */
+#define AWQ_MAX_ALPHA 64
+
+/*
+ * Activation statistic (compassingai.com AWQ concept page, "statistical basis
+ * of salient channels": activation_scale[j] = mean(|X_calib[:, j]|), or max;
+ * mudrobot.github.io notes: s_X is the average per-channel magnitude).
+ *   X     [N][D_in] bf16, 1 <= N <= 2^24, 8 <= D_in <= 2^20, D_in % 8 == 0
+ *   stat  AWQ_STAT_MEAN: a_j = (sum_i |X_ij|) / N, summed in fp32 in a fixed
+ *         order (bit-reproducible); AWQ_STAT_MAX: a_j = max_i |X_ij| (exact)
+ *   a     [D_in] fp32 output
+ */
+AWQ_API int awq_act_stats(const void* X, int64_t N, int64_t D_in, int stat, float* a, void* stream);
+
+/*
+ * Scale vector for one alpha (compassingai.com concept page, flow step 3:
+ * s_j = activation_scale[j]^alpha; step 6: s* = activation_scale^alpha*).
+ *   s_j = (float) pow((double) max(a_j, 1e-6f * max_i a_i), (double) alpha)
+ *   (all ones when every a_j is 0).  alpha = 0 gives exactly 1.
+ *   a  [D_in] fp32;  s  [D_in] fp32 output;  alpha is a host value.
+ */
+AWQ_API int awq_scales(const float* a, int64_t D_in, float alpha, float* s, void* stream);
+
+/* Same, with alpha read from device memory (e.g. the alpha_star output of
+ * awq_search), so that search -> scales -> pack needs no host round trip. */
+AWQ_API int awq_scales_dev(const float* a, int64_t D_in, const float* alpha_dev, float* s, void* stream);
+
+/*
+ * Bytes of workspace awq_search needs for this shape on the current device
+ * (0 if the arguments are invalid).
+ */
+AWQ_API size_t awq_search_workspace_size(int64_t N, int64_t D_in, int64_t D_out, int n_alpha, int bits, int group,
+                                         int loss_form);
+
+/*
+ * The grid search (compassingai.com concept page, flow steps 3-5;
+ * mudrobot.github.io notes, "searching the optimal scale").  For every alpha
+ * in the grid it forms s = a^alpha, quantises diag(s) W per group of `group`
+ * rows to `bits` bits (delta = max|w'| / (2^(b-1)-1), round half to even,
+ * clamp to +-(2^(b-1)-1)) and evaluates
+ *     L(alpha) = || X S^-1 Q(S W) - X W ||^2
+ * with bf16 operands and fp32 accumulation on the tensor cores, in the form
+ * chosen by loss_form (AWQ_LOSS_ERROR or AWQ_LOSS_REFERENCE); the squared
+ * error is summed in fp32 per 128 tokens and in fp64 above that, in a fixed
+ * order.
+ *   X           [N][D_in] bf16;  W [D_in][D_out] fp32;  a [D_in] fp32
+ *   alpha_grid  HOST array of n_alpha fp32 values, 1 <= n_alpha <= 64
+ *   bits        2, 3 or 4;  group 32, 64 or 128;  D_in % group == 0,
+ *               D_in <= 2^20, D_out % 4 == 0, D_out <= 2^24, 1 <= N <= 2^24
+ *   loss_form   AWQ_LOSS_ERROR or AWQ_LOSS_REFERENCE
+ *   L           [n_alpha] fp64 output (device)
+ *   L_col       [n_alpha][D_out] fp64 output: each column's share of L
+ *               (may be NULL)
+ *   alpha_star  [1] fp32 output: alpha_grid[argmin L] (smallest index on ties)
+ *   alpha_idx   [1] int32 output: argmin L
+ *   workspace   at least awq_search_workspace_size(...) bytes, 256-byte aligned
+ *   status      [1] int32 device status word (may be NULL): set to 0 by the
+ *               call, then AWQ_ETIMEOUT | (site << 8) if a pipeline wait gave
+ *               up; the outputs are then invalid.  Read it after the stream
+ *               has been synchronised.
+ */
+AWQ_API int awq_search(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
+                       const float* alpha_grid, int n_alpha, int bits, int group, int loss_form, double* L,
+                       double* L_col, float* alpha_star, int32_t* alpha_idx, void* workspace, size_t workspace_bytes,
+                       int32_t* status, void* stream);
+
+/* One layer of a batched search (see awq_search for the meaning of each field). */
+typedef struct {
+  const void* X;
+  const float* W;
+  const float* a;
+  int64_t N, D_in, D_out;
+  double* L;          /* [n_alpha] */
+  double* L_col;      /* [n_alpha][D_out] or NULL */
+  float* alpha_star;  /* [1] */
+  int32_t* alpha_idx; /* [1] */
+} awq_layer;
+
+/* Bytes of workspace awq_search_batched needs (the largest single layer). */
+AWQ_API size_t awq_search_batched_workspace_size(const awq_layer* layers, int n_layers, int n_alpha, int bits,
+                                                 int group, int loss_form);
+
+/*
+ * Independent searches for several layers with one call (compassingai.com
+ * concept page, flow note: each layer is searched independently).  `layers`
+ * is a HOST array of n_layers descriptors; every layer gets its own L and
+ * alpha*.  The layers run one after another on `stream`, sharing the
+ * workspace.
+ */
+AWQ_API int awq_search_batched(const awq_layer* layers, int n_layers, const float* alpha_grid, int n_alpha,
+                               int bits, int group, int loss_form, void* workspace, size_t workspace_bytes,
+                               int32_t* status, void* stream);
+
+/*
+ * Final quantise + pack for a given scale vector (compassingai.com concept
+ * page, "inference-time equivalent": W_quantized = Quantize(diag(s*) W), s*
+ * kept as metadata).  Bit-exact IEEE fp32 arithmetic:
+ *   w' = fl(s_k w_kn), delta = fl(max|w'| / (2^(b-1)-1)),
+ *   q = clamp(rne(fl(w' / delta))), an all-zero group has delta = 0, q = 0.
+ *   W       [D_in][D_out] fp32;  s [D_in] fp32
+ *   packed  [D_in/8][D_out] uint32 output: word (k8, n) holds rows
+ *           8*k8 .. 8*k8+7 of column n, row 8*k8+i in bits 4i..4i+3 as the
+ *           offset-binary value u = q + 2^(bits-1)
+ *   scales  [D_in/group][D_out] fp32 output: delta of each (group, column)
+ */
+AWQ_API int awq_quantize_pack(const float* W, const float* s, int64_t D_in, int64_t D_out, int bits, int group,
+                      uint32_t* packed, float* scales, void* stream);
+
+/*
+ * The layer's reference output Y = X bf16(W) computed by the search's own
+ * tensor-core GEMM (the X W term of the loss, concept page flow step 4c), fp32.
+ *   Y          [N][D_out] fp32 output
+ *   workspace  at least awq_layer_output_workspace_size(...) bytes
+ */
+AWQ_API size_t awq_layer_output_workspace_size(int64_t N, int64_t D_in, int64_t D_out);
+AWQ_API int awq_layer_output(const void* X, const float* W, int64_t N, int64_t D_in, int64_t D_out, float* Y,
+                     void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
+
+/*
+ * Failure-detection self test: launches one CTA that waits on a barrier no one
+ * ever arrives at, with the same bounded wait the search kernel uses.  After
+ * about timeout_ns nanoseconds the wait gives up and AWQ_ETIMEOUT | (site << 8)
+ * is written to *status (device int32).  Nothing hangs or traps.
+ */
+AWQ_API int awq_selftest_wait_timeout(int32_t* status, int64_t timeout_ns, void* stream);
+
+/*
+ * Stage timing.  While enabled, every entry point records a pair of CUDA
+ * events on its stream around each kernel it launches; awq_profile_read waits
+ * for the recorded events and returns, per stage, the summed device time in
+ * milliseconds and the number of launches since the last reset.  Stages:
+ */
+enum {
+  AWQ_STAGE_ACT_STATS = 0,     /* awq_act_stats */
+  AWQ_STAGE_SCALE_TABLE = 1,   /* s = a^alpha (and 1/s) for the alpha grid, or one alpha */
+  AWQ_STAGE_SEARCH_CODES = 2,  /* per-alpha INT codes + deltas of diag(s) W */
+  AWQ_STAGE_SEARCH_GEMM = 3,   /* the fused tensor-core loss GEMM */
+  AWQ_STAGE_LOSS_REDUCE = 4,   /* L(alpha), argmin */
+  AWQ_STAGE_QUANTIZE_PACK = 5, /* awq_quantize_pack */
+  AWQ_STAGE_WEIGHT_PAIRS = 6,  /* bf16 copy of W for awq_layer_output */
+  AWQ_NUM_STAGES = 7
+};
+AWQ_API int awq_profile_enable(int on);
+AWQ_API int awq_profile_reset(void);
+AWQ_API int awq_profile_read(int stage, double* total_ms, int32_t* launches);
+
+/* Message describing the last non-OK status returned on this thread. */
+AWQ_API const char* awq_get_last_error(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+AWQ_API int awq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AWQ_B200_H */

@@ -1,0 +1,348 @@
+"""Thin Python binding of the C ABI in ``include/awq_b200.h``.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library ``libawq_b200.so`` built in this package directory.  PyTorch supplies
+device memory and the current stream.  There is no CPU fallback: importing this
+module raises if the library is missing, and every call raises on a non-OK
+status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libawq_b200.so")
+
+AWQ_OK, AWQ_EINVAL, AWQ_EALIGN, AWQ_EUNSUPPORTED, AWQ_EWORKSPACE, AWQ_ECUDA, AWQ_ETIMEOUT = range(7)
+STAT_MEAN, STAT_MAX = 0, 1
+LOSS_ERROR, LOSS_REFERENCE = 0, 1
+MAX_ALPHA = 64
+
+EXPORTS = (
+    "awq_act_stats", "awq_scales", "awq_scales_dev", "awq_search_workspace_size", "awq_search",
+    "awq_search_batched_workspace_size", "awq_search_batched", "awq_quantize_pack",
+    "awq_layer_output_workspace_size", "awq_layer_output", "awq_selftest_wait_timeout",
+    "awq_get_last_error", "awq_version", "awq_profile_enable", "awq_profile_reset", "awq_profile_read",
+)
+STAGES = ("act_stats", "scale_table", "search_codes", "search_gemm", "loss_reduce", "quantize_pack",
+          "weight_pairs")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m post_weight_only_b200.build` "
+        "(nvcc, sm_100a); there is no fallback implementation")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+P = ctypes.c_void_p
+I64 = ctypes.c_int64
+I = ctypes.c_int
+F = ctypes.c_float
+SZ = ctypes.c_size_t
+
+
+class AwqLayer(ctypes.Structure):
+    _fields_ = [("X", P), ("W", P), ("a", P), ("N", I64), ("D_in", I64), ("D_out", I64),
+                ("L", P), ("L_col", P), ("alpha_star", P), ("alpha_idx", P)]
+
+
+def _sig(name, res, args):
+    fn = getattr(_lib, name)
+    fn.restype = res
+    fn.argtypes = args
+    return fn
+
+
+_act_stats = _sig("awq_act_stats", I, [P, I64, I64, I, P, P])
+_scales = _sig("awq_scales", I, [P, I64, F, P, P])
+_scales_dev = _sig("awq_scales_dev", I, [P, I64, P, P, P])
+_search_ws = _sig("awq_search_workspace_size", SZ, [I64, I64, I64, I, I, I, I])
+_search = _sig("awq_search", I, [P, P, P, I64, I64, I64, P, I, I, I, I, P, P, P, P, P, SZ, P, P])
+_batched_ws = _sig("awq_search_batched_workspace_size", SZ, [ctypes.POINTER(AwqLayer), I, I, I, I, I])
+_batched = _sig("awq_search_batched", I, [ctypes.POINTER(AwqLayer), I, P, I, I, I, I, P, SZ, P, P])
+_pack = _sig("awq_quantize_pack", I, [P, P, I64, I64, I, I, P, P, P])
+_out_ws = _sig("awq_layer_output_workspace_size", SZ, [I64, I64, I64])
+_out = _sig("awq_layer_output", I, [P, P, I64, I64, I64, P, P, SZ, P, P])
+_selftest = _sig("awq_selftest_wait_timeout", I, [P, I64, P])
+_last_error = _sig("awq_get_last_error", ctypes.c_char_p, [])
+_prof_enable = _sig("awq_profile_enable", I, [I])
+_prof_reset = _sig("awq_profile_reset", I, [])
+_prof_read = _sig("awq_profile_read", I, [I, P, P])
+_version = _sig("awq_version", I, [])
+
+
+class AwqError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"awq status {code}: {msg}")
+        self.code = code
+
+
+def _check(rc: int) -> None:
+    if rc != AWQ_OK:
+        raise AwqError(rc, _last_error().decode(errors="replace"))
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _dev(t: torch.Tensor, dtype: torch.dtype, name: str) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.contiguous()
+
+
+def version() -> int:
+    return int(_version())
+
+
+def act_stats(X: torch.Tensor, stat: int = STAT_MEAN) -> torch.Tensor:
+    """a_j = mean_i |X_ij| (or max): ``awq_act_stats``."""
+    X = _dev(X, torch.bfloat16, "X")
+    N, D = X.shape
+    a = torch.empty(D, dtype=torch.float32, device=X.device)
+    _check(_act_stats(_ptr(X), N, D, stat, _ptr(a), _stream()))
+    return a
+
+
+def scales(a: torch.Tensor, alpha) -> torch.Tensor:
+    """s = a^alpha (floored): ``awq_scales`` for a host alpha, ``awq_scales_dev``
+    when alpha is a one-element CUDA tensor."""
+    a = _dev(a, torch.float32, "a")
+    s = torch.empty_like(a)
+    if isinstance(alpha, torch.Tensor):
+        al = _dev(alpha.reshape(1), torch.float32, "alpha")
+        _check(_scales_dev(_ptr(a), a.numel(), _ptr(al), _ptr(s), _stream()))
+    else:
+        _check(_scales(_ptr(a), a.numel(), float(alpha), _ptr(s), _stream()))
+    return s
+
+
+def search_workspace_size(N: int, D_in: int, D_out: int, n_alpha: int, bits: int, group: int,
+                          loss_form: int = LOSS_ERROR) -> int:
+    n = int(_search_ws(N, D_in, D_out, n_alpha, bits, group, loss_form))
+    if n == 0:
+        raise AwqError(AWQ_EINVAL, _last_error().decode(errors="replace"))
+    return n
+
+
+@dataclass
+class SearchResult:
+    L: torch.Tensor                 # [n_alpha] fp64
+    alpha_star: torch.Tensor        # [1] fp32
+    alpha_idx: torch.Tensor         # [1] int32
+    L_col: Optional[torch.Tensor]   # [n_alpha, D_out] fp64 or None
+    status: torch.Tensor            # [1] int32 device status word
+
+
+class Workspace:
+    """A reusable device workspace (grown on demand, 256-byte aligned)."""
+
+    def __init__(self, device=None):
+        self.buf = None
+        self.device = device
+
+    def get(self, nbytes: int, device) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes or self.buf.device != device:
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        return self.buf
+
+
+_default_ws = Workspace()
+
+
+def search(X: torch.Tensor, W: torch.Tensor, a: torch.Tensor, alpha_grid: Sequence[float], bits: int = 4,
+           group: int = 128, want_cols: bool = False, workspace: Optional[Workspace] = None,
+           check_status: bool = True, loss_form: int = LOSS_ERROR) -> SearchResult:
+    """Grid search over alpha for one layer: ``awq_search``."""
+    X = _dev(X, torch.bfloat16, "X")
+    W = _dev(W, torch.float32, "W")
+    a = _dev(a, torch.float32, "a")
+    N, D_in = X.shape
+    D_out = W.shape[1]
+    grid = (ctypes.c_float * len(alpha_grid))(*[float(v) for v in alpha_grid])
+    A = len(alpha_grid)
+    dev = X.device
+    L = torch.empty(A, dtype=torch.float64, device=dev)
+    Lc = torch.empty(A, D_out, dtype=torch.float64, device=dev) if want_cols else None
+    astar = torch.empty(1, dtype=torch.float32, device=dev)
+    aidx = torch.empty(1, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    nbytes = search_workspace_size(N, D_in, D_out, A, bits, group, loss_form)
+    ws = (workspace or _default_ws).get(nbytes, dev)
+    _check(_search(_ptr(X), _ptr(W), _ptr(a), N, D_in, D_out, grid, A, bits, group, loss_form, _ptr(L), _ptr(Lc),
+                   _ptr(astar), _ptr(aidx), _ptr(ws), ws.numel(), _ptr(status), _stream()))
+    res = SearchResult(L, astar, aidx, Lc, status)
+    if check_status:
+        check_device_status(status)
+    return res
+
+
+def check_device_status(status: torch.Tensor) -> None:
+    v = int(status.item())
+    if v != 0:
+        raise AwqError(v & 0xFF, f"device status {v:#x} (code {v & 0xFF}, site {v >> 8})")
+
+
+def search_batched(layers, alpha_grid: Sequence[float], bits: int = 4, group: int = 128,
+                   want_cols: bool = False, workspace: Optional[Workspace] = None, loss_form: int = LOSS_ERROR):
+    """Independent searches of several layers in one call: ``awq_search_batched``.
+    ``layers`` is a sequence of (X, W, a).  Returns one SearchResult per layer."""
+    A = len(alpha_grid)
+    grid = (ctypes.c_float * A)(*[float(v) for v in alpha_grid])
+    descs = (AwqLayer * len(layers))()
+    results, keep = [], []
+    dev = None
+    for i, (X, W, a) in enumerate(layers):
+        X = _dev(X, torch.bfloat16, "X")
+        W = _dev(W, torch.float32, "W")
+        a = _dev(a, torch.float32, "a")
+        dev = X.device
+        N, D_in = X.shape
+        D_out = W.shape[1]
+        L = torch.empty(A, dtype=torch.float64, device=dev)
+        Lc = torch.empty(A, D_out, dtype=torch.float64, device=dev) if want_cols else None
+        astar = torch.empty(1, dtype=torch.float32, device=dev)
+        aidx = torch.empty(1, dtype=torch.int32, device=dev)
+        keep += [X, W, a]
+        descs[i] = AwqLayer(_ptr(X), _ptr(W), _ptr(a), N, D_in, D_out, _ptr(L), _ptr(Lc), _ptr(astar), _ptr(aidx))
+        results.append(SearchResult(L, astar, aidx, Lc, None))
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    nbytes = int(_batched_ws(descs, len(layers), A, bits, group, loss_form))
+    if nbytes == 0:
+        raise AwqError(AWQ_EINVAL, _last_error().decode(errors="replace"))
+    ws = (workspace or _default_ws).get(nbytes, dev)
+    _check(_batched(descs, len(layers), grid, A, bits, group, loss_form, _ptr(ws), ws.numel(), _ptr(status),
+                    _stream()))
+    check_device_status(status)
+    for r in results:
+        r.status = status
+    return results
+
+
+def quantize_pack(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int = 128):
+    """INT codes (offset binary, 8 per uint32 word) + per-group scales:
+    ``awq_quantize_pack``.  Returns (packed int32 view [D_in/8, D_out],
+    scales fp32 [D_in/group, D_out])."""
+    W = _dev(W, torch.float32, "W")
+    s = _dev(s, torch.float32, "s")
+    D_in, D_out = W.shape
+    packed = torch.empty(D_in // 8, D_out, dtype=torch.int32, device=W.device)
+    sc = torch.empty(D_in // group, D_out, dtype=torch.float32, device=W.device)
+    _check(_pack(_ptr(W), _ptr(s), D_in, D_out, bits, group, _ptr(packed), _ptr(sc), _stream()))
+    return packed, sc
+
+
+def layer_output(X: torch.Tensor, W: torch.Tensor, workspace: Optional[Workspace] = None) -> torch.Tensor:
+    """Y = X bf16(W) on the search's tensor-core GEMM: ``awq_layer_output``."""
+    X = _dev(X, torch.bfloat16, "X")
+    W = _dev(W, torch.float32, "W")
+    N, D_in = X.shape
+    D_out = W.shape[1]
+    Y = torch.empty(N, D_out, dtype=torch.float32, device=X.device)
+    status = torch.zeros(1, dtype=torch.int32, device=X.device)
+    nbytes = int(_out_ws(N, D_in, D_out))
+    if nbytes == 0:
+        raise AwqError(AWQ_EINVAL, _last_error().decode(errors="replace"))
+    ws = (workspace or _default_ws).get(nbytes, X.device)
+    _check(_out(_ptr(X), _ptr(W), N, D_in, D_out, _ptr(Y), _ptr(ws), ws.numel(), _ptr(status), _stream()))
+    check_device_status(status)
+    return Y
+
+
+def selftest_wait_timeout(timeout_ns: int = 1_000_000) -> int:
+    """Run the bounded-wait self test; returns the device status word."""
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _check(_selftest(_ptr(status), int(timeout_ns), _stream()))
+    torch.cuda.synchronize()
+    return int(status.item())
+
+
+def last_error() -> str:
+    return _last_error().decode(errors="replace")
+
+
+def profile_enable(on: bool = True) -> None:
+    """Record CUDA events around every kernel the library launches."""
+    _check(_prof_enable(1 if on else 0))
+
+
+def profile_reset() -> None:
+    _check(_prof_reset())
+
+
+def profile_read() -> dict:
+    """{stage: (total device ms, launches)} since the last reset."""
+    out = {}
+    for i, name in enumerate(STAGES):
+        ms = ctypes.c_double(0.0)
+        n = ctypes.c_int32(0)
+        _check(_prof_read(i, ctypes.byref(ms), ctypes.byref(n)))
+        out[name] = (ms.value, n.value)
+    return out
+
+
+@dataclass
+class LayerResult:
+    a: torch.Tensor             # [D_in] activation statistic
+    search: SearchResult        # L(alpha), alpha*, status
+    s_star: torch.Tensor        # [D_in] scales for alpha*
+    packed: torch.Tensor        # [D_in/8, D_out] int32 words of offset-binary codes
+    scales: torch.Tensor        # [D_in/group, D_out] fp32 deltas
+
+
+def quantize_layer(X: torch.Tensor, W: torch.Tensor, alpha_grid: Sequence[float], bits: int = 4,
+                   group: int = 128, stat: int = STAT_MEAN, workspace: Optional[Workspace] = None,
+                   want_cols: bool = False, loss_form: int = LOSS_ERROR) -> LayerResult:
+    """The whole per-layer path on the device, with no host synchronisation:
+    statistic -> grid search -> s* = a^alpha* (alpha* read on the device) ->
+    quantise + pack.  Check ``result.search.status`` after synchronising."""
+    a = act_stats(X, stat)
+    res = search(X, W, a, alpha_grid, bits, group, want_cols=want_cols, workspace=workspace, check_status=False,
+                 loss_form=loss_form)
+    s_star = scales(a, res.alpha_star)
+    packed, sc = quantize_pack(W, s_star, bits, group)
+    return LayerResult(a, res, s_star, packed, sc)
+
+
+def quantize_layer_host(X_host: torch.Tensor, W_host: torch.Tensor, alpha_grid: Sequence[float], bits: int = 4,
+                        group: int = 128, stat: int = STAT_MEAN, device="cuda",
+                        workspace: Optional[Workspace] = None, out: Optional[dict] = None,
+                        loss_form: int = LOSS_ERROR) -> dict:
+    """The per-layer path from host buffers to host buffers: copies X and W to
+    the device (pinned host memory gives asynchronous copies), runs
+    :func:`quantize_layer`, copies L, alpha*, the packed codes and the scales
+    back, synchronises the stream and checks the device status word."""
+    X = X_host.to(device, non_blocking=True)
+    W = W_host.to(device, non_blocking=True)
+    r = quantize_layer(X, W, alpha_grid, bits, group, stat, workspace, loss_form=loss_form)
+    if out is None:
+        pin = X_host.is_pinned()
+        out = {
+            "L": torch.empty(r.search.L.shape, dtype=r.search.L.dtype, pin_memory=pin),
+            "alpha_star": torch.empty(1, dtype=torch.float32, pin_memory=pin),
+            "status": torch.empty(1, dtype=torch.int32, pin_memory=pin),
+            "packed": torch.empty(r.packed.shape, dtype=r.packed.dtype, pin_memory=pin),
+            "scales": torch.empty(r.scales.shape, dtype=r.scales.dtype, pin_memory=pin),
+        }
+    out["L"].copy_(r.search.L, non_blocking=True)
+    out["alpha_star"].copy_(r.search.alpha_star, non_blocking=True)
+    out["status"].copy_(r.search.status, non_blocking=True)
+    out["packed"].copy_(r.packed, non_blocking=True)
+    out["scales"].copy_(r.scales, non_blocking=True)
+    torch.cuda.current_stream().synchronize()
+    v = int(out["status"][0])
+    if v != 0:
+        raise AwqError(v & 0xFF, f"device status {v:#x}")
+    return out

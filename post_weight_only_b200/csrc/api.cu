@@ -1,0 +1,483 @@
+// api.cu -- the C ABI (include/awq_b200.h): argument checking, workspace
+// layout, and the launch sequence of each entry point.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/awq_b200.h"
+#include "internal.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int fail_cuda(cudaError_t e, const char* what) {
+  return fail(AWQ_ECUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+constexpr int64_t kMaxDim = int64_t(1) << 24;
+// Kernels index groups and 64-channel slabs of D_in with gridDim.y (< 65536).
+constexpr int64_t kMaxDin = int64_t(1) << 20;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Current device: its SM count, and whether it is an sm_100 part.
+int device_info(int* num_sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  int major = 0;
+  e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaDeviceGetAttribute");
+  if (major != 10) return fail(AWQ_EUNSUPPORTED, "device %d has compute capability %d.x; this library is built for sm_100a", dev, major);
+  e = cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaDeviceGetAttribute");
+  return AWQ_OK;
+}
+
+uint64_t timeout_ns() {
+  static uint64_t t = 0;
+  if (t == 0) {
+    uint64_t ms = 2000;
+    if (const char* env = getenv("AWQ_TIMEOUT_MS")) {
+      long long v = atoll(env);
+      if (v > 0) ms = static_cast<uint64_t>(v);
+    }
+    t = ms * 1000000ull;
+  }
+  return t;
+}
+
+struct SearchLayout {
+  size_t s_tab, r_tab, codes, delta, w_pairs, yref, partial, blk, status, total;
+  int grid, Tt, nblk;
+};
+
+SearchLayout search_layout(int64_t N, int64_t D_in, int64_t D_out, int A, int group, int form, int num_sms) {
+  SearchLayout L{};
+  awq::SearchShape sh{static_cast<int>(N), static_cast<int>(D_in), static_cast<int>(D_out), A, 4, group, form};
+  const bool ref = form == AWQ_LOSS_REFERENCE;
+  L.grid = awq::search_grid_size(sh, num_sms);
+  L.Tt = awq::search_token_tiles(static_cast<int>(N));
+  L.nblk = awq::loss_reduce_blocks(D_out);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += round_up(bytes, 256);
+    return o;
+  };
+  const size_t a = static_cast<size_t>(A);
+  L.s_tab = take(a * D_in * 4);
+  L.r_tab = take(a * D_in * 4);
+  L.codes = take(a * (D_in / (ref ? 8 : 4)) * D_out * 4);
+  L.delta = take(A > 0 ? a * (D_in / group) * D_out * 4 : 0);
+  L.w_pairs = take(ref ? static_cast<size_t>(D_in / 2) * D_out * 4 : 0);
+  L.yref = take(A > 0 && ref ? static_cast<size_t>(L.grid) * 128 * 256 * 4 : 0);
+  L.partial = take(a * L.Tt * D_out * 4);
+  L.blk = take(a * L.nblk * 8);
+  L.status = take(4);
+  L.total = off;
+  return L;
+}
+
+int check_form(int form) {
+  if (form != AWQ_LOSS_ERROR && form != AWQ_LOSS_REFERENCE)
+    return fail(AWQ_EINVAL, "loss_form = %d: use AWQ_LOSS_ERROR or AWQ_LOSS_REFERENCE", form);
+  return AWQ_OK;
+}
+
+int check_quant_args(int bits, int group) {
+  if (bits < 2 || bits > 4) return fail(AWQ_EUNSUPPORTED, "bits = %d: supported bit widths are 2, 3 and 4", bits);
+  if (group != 32 && group != 64 && group != 128)
+    return fail(AWQ_EUNSUPPORTED, "group = %d: supported group sizes are 32, 64 and 128", group);
+  return AWQ_OK;
+}
+
+int check_layer_shape(int64_t N, int64_t D_in, int64_t D_out) {
+  if (N < 1 || N > kMaxDim) return fail(AWQ_EINVAL, "N = %lld: need 1 <= N <= 2^24", (long long)N);
+  if (D_in < 8 || D_in > kMaxDin || D_in % 8) return fail(AWQ_EINVAL, "D_in = %lld: need a multiple of 8 in [8, 2^20]", (long long)D_in);
+  if (D_out < 4 || D_out > kMaxDim || D_out % 4) return fail(AWQ_EINVAL, "D_out = %lld: need a multiple of 4 in [4, 2^24]", (long long)D_out);
+  // Tiles of 128 output columns x 256 tokens are numbered with 32-bit ints.
+  if (((D_out + 127) / 128) * ((N + 255) / 256) > (int64_t(1) << 30))
+    return fail(AWQ_EINVAL, "N x D_out = %lld x %lld is too large", (long long)N, (long long)D_out);
+  return AWQ_OK;
+}
+
+int check_ptr(const void* p, const char* name, size_t align) {
+  if (!p) return fail(AWQ_EINVAL, "%s is NULL", name);
+  if (!aligned(p, align)) return fail(AWQ_EALIGN, "%s is not %zu-byte aligned", name, align);
+  return AWQ_OK;
+}
+
+// ---------------------------------------------------------------- stage timing
+struct ProfRec {
+  int stage;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof_pending;
+double g_prof_ms[AWQ_NUM_STAGES] = {};
+int g_prof_n[AWQ_NUM_STAGES] = {};
+
+// Brackets one kernel launch with events when profiling is on.
+struct StageTimer {
+  int stage;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr, b = nullptr;
+  StageTimer(int stage_, cudaStream_t st_) : stage(stage_), st(st_) {
+    if (!g_prof_on) return;
+    if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) {
+      a = b = nullptr;
+      return;
+    }
+    cudaEventRecord(a, st);
+  }
+  ~StageTimer() {
+    if (!a) return;
+    cudaEventRecord(b, st);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_pending.push_back({stage, a, b});
+  }
+};
+
+void prof_collect() {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : g_prof_pending) {
+    float ms = 0.0f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+      g_prof_ms[r.stage] += ms;
+      g_prof_n[r.stage] += 1;
+    }
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  g_prof_pending.clear();
+}
+
+#define AWQ_TRY(expr)            \
+  do {                           \
+    int _rc = (expr);            \
+    if (_rc != AWQ_OK) return _rc; \
+  } while (0)
+
+// The search for one layer with a workspace already checked; does not reset
+// the status word.
+int search_one(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
+               const awq::AlphaList& alphas, int A, int bits, int group, int form, double* L, double* L_col,
+               float* alpha_star, int32_t* alpha_idx, uint8_t* ws, int32_t* status, cudaStream_t st,
+               int num_sms) {
+  const SearchLayout lay = search_layout(N, D_in, D_out, A, group, form, num_sms);
+  float* s_tab = reinterpret_cast<float*>(ws + lay.s_tab);
+  float* r_tab = reinterpret_cast<float*>(ws + lay.r_tab);
+  uint32_t* codes = reinterpret_cast<uint32_t*>(ws + lay.codes);
+  float* delta = reinterpret_cast<float*>(ws + lay.delta);
+  uint32_t* w_pairs = form == AWQ_LOSS_REFERENCE ? reinterpret_cast<uint32_t*>(ws + lay.w_pairs) : nullptr;
+  float* yref = reinterpret_cast<float*>(ws + lay.yref);
+  float* partial = reinterpret_cast<float*>(ws + lay.partial);
+  double* blk = reinterpret_cast<double*>(ws + lay.blk);
+
+  cudaError_t e;
+  {
+    StageTimer t(AWQ_STAGE_SCALE_TABLE, st);
+    e = awq::launch_scale_table(a, D_in, alphas, nullptr, A, s_tab, r_tab, st);
+  }
+  if (e != cudaSuccess) return fail_cuda(e, "scale table kernel");
+  {
+    StageTimer t(AWQ_STAGE_SEARCH_CODES, st);
+    e = awq::launch_search_codes(W, s_tab, D_in, D_out, A, bits, group, form, codes, delta, w_pairs, st);
+  }
+  if (e != cudaSuccess) return fail_cuda(e, "search codes kernel");
+  awq::SearchShape sh{static_cast<int>(N), static_cast<int>(D_in), static_cast<int>(D_out), A, bits, group, form};
+  awq::SearchBuffers b{X, w_pairs, codes, delta, r_tab, yref, partial, nullptr, status};
+  const char* what = "search kernel";
+  int rc;
+  {
+    StageTimer t(AWQ_STAGE_SEARCH_GEMM, st);
+    rc = awq::launch_search(sh, b, lay.grid, timeout_ns(), st, &e, &what);
+  }
+  if (rc != AWQ_OK) return e != cudaSuccess ? fail_cuda(e, what) : fail(rc, "%s failed", what);
+  {
+    StageTimer t(AWQ_STAGE_LOSS_REDUCE, st);
+    e = awq::launch_loss_reduce(partial, A, lay.Tt, D_out, L_col, blk, lay.nblk, alphas, L, alpha_star,
+                                alpha_idx, st);
+  }
+  if (e != cudaSuccess) return fail_cuda(e, "loss reduction kernels");
+  return AWQ_OK;
+}
+
+int check_search_args(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
+                      const float* alpha_grid, int n_alpha, int bits, int group, int form, double* L, double* L_col,
+                      float* alpha_star, int32_t* alpha_idx) {
+  AWQ_TRY(check_layer_shape(N, D_in, D_out));
+  AWQ_TRY(check_quant_args(bits, group));
+  AWQ_TRY(check_form(form));
+  if (D_in % group) return fail(AWQ_EINVAL, "D_in = %lld is not a multiple of group = %d", (long long)D_in, group);
+  if (n_alpha < 1 || n_alpha > AWQ_MAX_ALPHA) return fail(AWQ_EUNSUPPORTED, "n_alpha = %d: need 1..%d", n_alpha, AWQ_MAX_ALPHA);
+  if (!alpha_grid) return fail(AWQ_EINVAL, "alpha_grid is NULL");
+  AWQ_TRY(check_ptr(X, "X", 16));
+  AWQ_TRY(check_ptr(W, "W", 16));
+  AWQ_TRY(check_ptr(a, "a", 16));
+  AWQ_TRY(check_ptr(L, "L", 8));
+  if (L_col) AWQ_TRY(check_ptr(L_col, "L_col", 8));
+  AWQ_TRY(check_ptr(alpha_star, "alpha_star", 4));
+  AWQ_TRY(check_ptr(alpha_idx, "alpha_idx", 4));
+  return AWQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* awq_get_last_error(void) { return g_last_error.c_str(); }
+
+int awq_version(void) { return 100; }
+
+int awq_act_stats(const void* X, int64_t N, int64_t D_in, int stat, float* a, void* stream) {
+  if (N < 1 || N > kMaxDim) return fail(AWQ_EINVAL, "N = %lld: need 1 <= N <= 2^24", (long long)N);
+  if (D_in < 8 || D_in > kMaxDin || D_in % 8) return fail(AWQ_EINVAL, "D_in = %lld: need a multiple of 8 in [8, 2^20]", (long long)D_in);
+  if (stat != AWQ_STAT_MEAN && stat != AWQ_STAT_MAX) return fail(AWQ_EINVAL, "stat = %d: use AWQ_STAT_MEAN or AWQ_STAT_MAX", stat);
+  AWQ_TRY(check_ptr(X, "X", 16));
+  AWQ_TRY(check_ptr(a, "a", 16));
+  int sms = 0;
+  AWQ_TRY(device_info(&sms));
+  cudaError_t e;
+  {
+    StageTimer t(AWQ_STAGE_ACT_STATS, static_cast<cudaStream_t>(stream));
+    e = awq::launch_act_stats(static_cast<const uint16_t*>(X), N, D_in, stat, a, static_cast<cudaStream_t>(stream));
+  }
+  return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "act_stats kernel");
+}
+
+static int scales_common(const float* a, int64_t D_in, float alpha, const float* alpha_dev, float* s, void* stream) {
+  if (D_in < 1 || D_in > kMaxDim) return fail(AWQ_EINVAL, "D_in = %lld out of range", (long long)D_in);
+  AWQ_TRY(check_ptr(a, "a", 4));
+  AWQ_TRY(check_ptr(s, "s", 4));
+  int sms = 0;
+  AWQ_TRY(device_info(&sms));
+  awq::AlphaList al{};
+  al.v[0] = alpha;
+  cudaError_t e;
+  {
+    StageTimer t(AWQ_STAGE_SCALE_TABLE, static_cast<cudaStream_t>(stream));
+    e = awq::launch_scale_table(a, D_in, al, alpha_dev, 1, s, nullptr, static_cast<cudaStream_t>(stream));
+  }
+  return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "scale table kernel");
+}
+
+int awq_scales(const float* a, int64_t D_in, float alpha, float* s, void* stream) {
+  return scales_common(a, D_in, alpha, nullptr, s, stream);
+}
+
+int awq_scales_dev(const float* a, int64_t D_in, const float* alpha_dev, float* s, void* stream) {
+  AWQ_TRY(check_ptr(alpha_dev, "alpha_dev", 4));
+  return scales_common(a, D_in, 0.0f, alpha_dev, s, stream);
+}
+
+size_t awq_search_workspace_size(int64_t N, int64_t D_in, int64_t D_out, int n_alpha, int bits, int group,
+                                 int loss_form) {
+  if (check_layer_shape(N, D_in, D_out) != AWQ_OK || check_quant_args(bits, group) != AWQ_OK) return 0;
+  if (check_form(loss_form) != AWQ_OK) return 0;
+  if (D_in % group || n_alpha < 1 || n_alpha > AWQ_MAX_ALPHA) return 0;
+  int sms = 0;
+  if (device_info(&sms) != AWQ_OK) return 0;
+  return search_layout(N, D_in, D_out, n_alpha, group, loss_form, sms).total;
+}
+
+int awq_search(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
+               const float* alpha_grid, int n_alpha, int bits, int group, int loss_form, double* L, double* L_col,
+               float* alpha_star, int32_t* alpha_idx, void* workspace, size_t workspace_bytes, int32_t* status,
+               void* stream) {
+  AWQ_TRY(check_search_args(X, W, a, N, D_in, D_out, alpha_grid, n_alpha, bits, group, loss_form, L, L_col,
+                            alpha_star, alpha_idx));
+  int sms = 0;
+  AWQ_TRY(device_info(&sms));
+  const SearchLayout lay = search_layout(N, D_in, D_out, n_alpha, group, loss_form, sms);
+  if (!workspace) return fail(AWQ_EWORKSPACE, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(AWQ_EALIGN, "workspace is not 256-byte aligned");
+  if (workspace_bytes < lay.total)
+    return fail(AWQ_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, lay.total);
+  if (status && !aligned(status, 4)) return fail(AWQ_EALIGN, "status is not 4-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* st_word = status ? status : reinterpret_cast<int32_t*>(ws + lay.status);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(st_word, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(status)");
+  awq::AlphaList al{};
+  for (int i = 0; i < n_alpha; ++i) al.v[i] = alpha_grid[i];
+  return search_one(X, W, a, N, D_in, D_out, al, n_alpha, bits, group, loss_form, L, L_col, alpha_star, alpha_idx,
+                    ws, st_word, st, sms);
+}
+
+size_t awq_search_batched_workspace_size(const awq_layer* layers, int n_layers, int n_alpha, int bits, int group,
+                                         int loss_form) {
+  if (!layers || n_layers < 1) return 0;
+  size_t m = 0;
+  for (int i = 0; i < n_layers; ++i) {
+    size_t s = awq_search_workspace_size(layers[i].N, layers[i].D_in, layers[i].D_out, n_alpha, bits, group,
+                                         loss_form);
+    if (s == 0) return 0;
+    if (s > m) m = s;
+  }
+  return m + 256;   // + the batch's own status word after the largest layout
+}
+
+int awq_search_batched(const awq_layer* layers, int n_layers, const float* alpha_grid, int n_alpha, int bits,
+                       int group, int loss_form, void* workspace, size_t workspace_bytes, int32_t* status,
+                       void* stream) {
+  if (!layers || n_layers < 1) return fail(AWQ_EINVAL, "layers is NULL or n_layers < 1");
+  for (int i = 0; i < n_layers; ++i) {
+    const awq_layer& l = layers[i];
+    int rc = check_search_args(l.X, l.W, l.a, l.N, l.D_in, l.D_out, alpha_grid, n_alpha, bits, group, loss_form,
+                               l.L, l.L_col, l.alpha_star, l.alpha_idx);
+    if (rc != AWQ_OK) return fail(rc, "layer %d: %s", i, g_last_error.c_str());
+  }
+  int sms = 0;
+  AWQ_TRY(device_info(&sms));
+  size_t need = 0;
+  for (int i = 0; i < n_layers; ++i) {
+    size_t s = search_layout(layers[i].N, layers[i].D_in, layers[i].D_out, n_alpha, group, loss_form, sms).total;
+    if (s > need) need = s;
+  }
+  if (!workspace) return fail(AWQ_EWORKSPACE, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(AWQ_EALIGN, "workspace is not 256-byte aligned");
+  if (workspace_bytes < need + 256)
+    return fail(AWQ_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need + 256);
+  if (status && !aligned(status, 4)) return fail(AWQ_EALIGN, "status is not 4-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Every layer's layout ends at or before `need`; the batch status word sits after it.
+  int32_t* st_word = status ? status : reinterpret_cast<int32_t*>(ws + need);
+  cudaError_t e = cudaMemsetAsync(st_word, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(status)");
+  awq::AlphaList al{};
+  for (int i = 0; i < n_alpha; ++i) al.v[i] = alpha_grid[i];
+  for (int i = 0; i < n_layers; ++i) {
+    const awq_layer& l = layers[i];
+    int rc = search_one(l.X, l.W, l.a, l.N, l.D_in, l.D_out, al, n_alpha, bits, group, loss_form, l.L, l.L_col,
+                        l.alpha_star, l.alpha_idx, ws, st_word, st, sms);
+    if (rc != AWQ_OK) return rc;
+  }
+  return AWQ_OK;
+}
+
+int awq_quantize_pack(const float* W, const float* s, int64_t D_in, int64_t D_out, int bits, int group,
+                      uint32_t* packed, float* scales, void* stream) {
+  AWQ_TRY(check_quant_args(bits, group));
+  if (D_in < group || D_in > kMaxDin || D_in % group)
+    return fail(AWQ_EINVAL, "D_in = %lld: need a positive multiple of group = %d", (long long)D_in, group);
+  if (D_out < 1 || D_out > kMaxDim) return fail(AWQ_EINVAL, "D_out = %lld out of range", (long long)D_out);
+  AWQ_TRY(check_ptr(W, "W", 16));
+  AWQ_TRY(check_ptr(s, "s", 16));
+  AWQ_TRY(check_ptr(packed, "packed", 16));
+  AWQ_TRY(check_ptr(scales, "scales", 16));
+  int sms = 0;
+  AWQ_TRY(device_info(&sms));
+  cudaError_t e;
+  {
+    StageTimer t(AWQ_STAGE_QUANTIZE_PACK, static_cast<cudaStream_t>(stream));
+    e = awq::launch_quantize_pack(W, s, D_in, D_out, bits, group, packed, scales, static_cast<cudaStream_t>(stream));
+  }
+  return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "quantize_pack kernel");
+}
+
+size_t awq_layer_output_workspace_size(int64_t N, int64_t D_in, int64_t D_out) {
+  if (check_layer_shape(N, D_in, D_out) != AWQ_OK) return 0;
+  int sms = 0;
+  if (device_info(&sms) != AWQ_OK) return 0;
+  return search_layout(N, D_in, D_out, 0, 128, AWQ_LOSS_REFERENCE, sms).total;
+}
+
+int awq_layer_output(const void* X, const float* W, int64_t N, int64_t D_in, int64_t D_out, float* Y,
+                     void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  AWQ_TRY(check_layer_shape(N, D_in, D_out));
+  AWQ_TRY(check_ptr(X, "X", 16));
+  AWQ_TRY(check_ptr(W, "W", 16));
+  AWQ_TRY(check_ptr(Y, "Y", 16));
+  int sms = 0;
+  AWQ_TRY(device_info(&sms));
+  const SearchLayout lay = search_layout(N, D_in, D_out, 0, 128, AWQ_LOSS_REFERENCE, sms);
+  if (!workspace) return fail(AWQ_EWORKSPACE, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(AWQ_EALIGN, "workspace is not 256-byte aligned");
+  if (workspace_bytes < lay.total)
+    return fail(AWQ_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, lay.total);
+  if (status && !aligned(status, 4)) return fail(AWQ_EALIGN, "status is not 4-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* st_word = status ? status : reinterpret_cast<int32_t*>(ws + lay.status);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(st_word, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(status)");
+  uint32_t* w_pairs = reinterpret_cast<uint32_t*>(ws + lay.w_pairs);
+  {
+    StageTimer t(AWQ_STAGE_WEIGHT_PAIRS, st);
+    e = awq::launch_weight_pairs(W, D_in, D_out, w_pairs, st);
+  }
+  if (e != cudaSuccess) return fail_cuda(e, "weight pairs kernel");
+  awq::SearchShape sh{static_cast<int>(N), static_cast<int>(D_in), static_cast<int>(D_out), 0, 4, 128,
+                      AWQ_LOSS_REFERENCE};
+  awq::SearchBuffers b{X, w_pairs, nullptr, nullptr, nullptr, nullptr, nullptr, Y, st_word};
+  const char* what = "search kernel (reference output)";
+  int rc;
+  {
+    StageTimer t(AWQ_STAGE_SEARCH_GEMM, st);
+    rc = awq::launch_search(sh, b, lay.grid, timeout_ns(), st, &e, &what);
+  }
+  if (rc != AWQ_OK) return e != cudaSuccess ? fail_cuda(e, what) : fail(rc, "%s failed", what);
+  return AWQ_OK;
+}
+
+int awq_profile_enable(int on) {
+  g_prof_on = on != 0;
+  return AWQ_OK;
+}
+
+int awq_profile_reset(void) {
+  prof_collect();
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (int i = 0; i < AWQ_NUM_STAGES; ++i) {
+    g_prof_ms[i] = 0.0;
+    g_prof_n[i] = 0;
+  }
+  return AWQ_OK;
+}
+
+int awq_profile_read(int stage, double* total_ms, int32_t* launches) {
+  if (stage < 0 || stage >= AWQ_NUM_STAGES) return fail(AWQ_EINVAL, "stage = %d out of range", stage);
+  prof_collect();
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (total_ms) *total_ms = g_prof_ms[stage];
+  if (launches) *launches = g_prof_n[stage];
+  return AWQ_OK;
+}
+
+int awq_selftest_wait_timeout(int32_t* status, int64_t timeout_ns_arg, void* stream) {
+  AWQ_TRY(check_ptr(status, "status", 4));
+  if (timeout_ns_arg < 1000 || timeout_ns_arg > 10000000000LL)
+    return fail(AWQ_EINVAL, "timeout_ns = %lld: need 1 us .. 10 s", (long long)timeout_ns_arg);
+  int sms = 0;
+  AWQ_TRY(device_info(&sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(status)");
+  e = awq::launch_wait_timeout_selftest(status, static_cast<uint64_t>(timeout_ns_arg), st);
+  return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "self-test kernel");
+}
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+// internal.cuh -- launch helpers shared by the C-ABI layer (api.cu) and the
+// kernel files.  Not part of the public interface.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace awq {
+
+constexpr int kMaxAlpha = 64;
+
+// Loss forms of the search (see search.cu).
+constexpr int kFormError = 0;        // L = ||X E||^2 with E = S^-1 Q(S W) - W as the MMA operand
+constexpr int kFormReference = 1;    // L = ||X S^-1 Q(S W) - X W||^2, reference output subtracted
+
+struct AlphaList {
+  float v[kMaxAlpha];
+};
+
+// ---- act_stats.cu
+cudaError_t launch_act_stats(const uint16_t* X, int64_t N, int64_t D, int stat, float* a, cudaStream_t st);
+
+// ---- scales.cu
+// s_tab [A][D] (may be null), r_tab [A][D] = fl32(1 / s) (may be null).
+// alpha_dev != null: a single alpha read from device memory (A must be 1).
+cudaError_t launch_scale_table(const float* a, int64_t D, const AlphaList& alphas, const float* alpha_dev, int A,
+                               float* s_tab, float* r_tab, cudaStream_t st);
+
+// ---- quant.cu
+// Search-side quantiser, per alpha: the codes (error form: 7-bit rounding
+// residuals, 4 per word; reference form: 4-bit codes in interleaved nibble
+// order), the per-group deltas (error form: times 2^-7), and the bf16 pairs
+// of W (may be null).  See quant.cu.
+cudaError_t launch_search_codes(const float* W, const float* s_tab, int64_t D_in, int64_t D_out, int A, int bits,
+                                int group, int form, uint32_t* codes, float* delta, uint32_t* w_pairs,
+                                cudaStream_t st);
+// bf16 pairs of W for the reference pass: w_pairs[k/2][n] = (bf16 w[k][n],
+// bf16 w[k+1][n]) as the low and high halves.
+cudaError_t launch_weight_pairs(const float* W, int64_t D_in, int64_t D_out, uint32_t* w_pairs, cudaStream_t st);
+// Final quantise + pack for one given scale vector s (natural nibble order).
+cudaError_t launch_quantize_pack(const float* W, const float* s, int64_t D_in, int64_t D_out, int bits, int group,
+                                 uint32_t* packed, float* scales, cudaStream_t st);
+
+// ---- reduce.cu
+cudaError_t launch_loss_reduce(const float* partial, int A, int H, int64_t D_out, double* L_col, double* blk,
+                               int nblk, const AlphaList& alphas, double* L, float* alpha_star, int* alpha_idx,
+                               cudaStream_t st);
+int loss_reduce_blocks(int64_t D_out);
+
+// ---- search.cu
+struct SearchShape {
+  int N, D_in, D_out, A, bits, group, form;
+};
+struct SearchBuffers {
+  const void* X;              // bf16 [N][D_in]
+  const uint32_t* w_pairs;    // [D_in/2][D_out]
+  const uint32_t* codes;      // [A][D_in/4][D_out] (error form) or [A][D_in/8][D_out]
+  const float* delta;         // [A][D_in/group][D_out]
+  const float* r_tab;         // [A][D_in] fp32 1/s
+  float* yref;                // [grid][128*256]
+  float* partial;             // [A][Tt][D_out]
+  float* y_out;               // gemm-only mode: [N][D_out]
+  int* status;
+};
+int search_grid_size(const SearchShape& sh, int num_sms);
+int search_token_tiles(int N);
+// Returns 0 on success, otherwise an awq error code; *cerr gets the CUDA error.
+int launch_search(const SearchShape& sh, const SearchBuffers& b, int grid, uint64_t timeout_ns, cudaStream_t st,
+                  cudaError_t* cerr, const char** what);
+
+// Self-test of the bounded wait: one CTA waits on an mbarrier that nothing
+// arrives at, gives up after timeout_ns and records the timeout in *status.
+cudaError_t launch_wait_timeout_selftest(int* status, uint64_t timeout_ns, cudaStream_t st);
+
+}  // namespace awq

@@ -1,0 +1,113 @@
+"""The C-ABI library builds, loads and exports every symbol its header
+declares; host-side argument checks reject bad calls before any device work
+(no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "awq_b200.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from post_weight_only_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^AWQ_API\s+[\w\s\*]+?\b(awq_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("awq_act_stats", "awq_search", "awq_quantize_pack", "awq_scales", "awq_get_last_error"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_lists_every_export():
+    from post_weight_only_b200 import awq
+    assert sorted(awq.EXPORTS) == declared_functions()
+
+
+def _err(lib):
+    lib.awq_get_last_error.restype = ctypes.c_char_p
+    return lib.awq_get_last_error().decode()
+
+
+def test_argument_checks_without_gpu(lib):
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    f = lib.awq_act_stats
+    f.argtypes = [P, I64, I64, I, P, P]
+    f.restype = I
+    fake = 0x10000  # never dereferenced: checks run first
+    assert f(fake, 0, 64, 0, fake, None) == 1            # N = 0
+    assert "N = 0" in _err(lib)
+    assert f(fake, 16, 12, 0, fake, None) == 1           # D_in not a multiple of 8
+    assert f(fake, 16, 64, 7, fake, None) == 1           # bad stat
+    assert f(fake + 4, 16, 64, 0, fake, None) == 2       # misaligned X
+    assert f(None, 16, 64, 0, fake, None) == 1           # NULL X
+
+    s = lib.awq_search
+    s.argtypes = [P, P, P, I64, I64, I64, P, I, I, I, I, P, P, P, P, P, ctypes.c_size_t, P, P]
+    s.restype = I
+    grid = (ctypes.c_float * 3)(0.0, 0.5, 1.0)
+    args = dict(X=fake, W=fake, a=fake, N=64, D_in=256, D_out=64, grid=grid, A=3, bits=4, group=128, form=0,
+                L=fake, Lc=None, astar=fake, aidx=fake, ws=fake, wsb=1 << 20, st=None, stream=None)
+
+    def call(**kw):
+        d = dict(args, **kw)
+        return s(d["X"], d["W"], d["a"], d["N"], d["D_in"], d["D_out"], d["grid"], d["A"], d["bits"], d["group"],
+                 d["form"], d["L"], d["Lc"], d["astar"], d["aidx"], d["ws"], d["wsb"], d["st"], d["stream"])
+
+    assert call(bits=5) == 3
+    assert call(bits=1) == 3
+    assert call(group=96) == 3
+    assert call(D_in=192) == 1                            # not a multiple of group 128
+    assert call(A=0) == 3
+    assert call(A=65) == 3
+    assert call(D_out=6) == 1
+    assert call(N=0) == 1
+    assert call(W=fake + 8) == 2
+    assert call(grid=None) == 1
+    assert call(form=2) == 1
+
+    q = lib.awq_quantize_pack
+    q.argtypes = [P, P, I64, I64, I, I, P, P, P]
+    q.restype = I
+    assert q(fake, fake, 256, 64, 4, 100, fake, fake, None) == 3
+    assert q(fake, fake, 200, 64, 4, 128, fake, fake, None) == 1
+    assert q(fake, fake, 256, 64, 6, 128, fake, fake, None) == 3
+
+    t = lib.awq_selftest_wait_timeout
+    t.argtypes = [P, I64, P]
+    t.restype = I
+    assert t(fake, 10, None) == 1                          # timeout below 1 us
+
+
+def test_no_device_is_reported_not_crashed(lib):
+    """On a machine without a usable sm_100 GPU a well-formed call fails with
+    AWQ_ECUDA or AWQ_EUNSUPPORTED; it never falls back to a CPU path."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    f = lib.awq_act_stats
+    f.argtypes = [P, I64, I64, I, P, P]
+    f.restype = I
+    rc = f(0x10000, 16, 64, 0, 0x10000, None)
+    assert rc in (3, 5)
+
+
+def test_version(lib):
+    lib.awq_version.restype = ctypes.c_int
+    assert lib.awq_version() >= 100
