@@ -67,7 +67,7 @@ enum { AWQ_STAT_MEAN = 0, AWQ_STAT_MAX = 1 };
  * cores (identical in exact arithmetic):
  *   AWQ_LOSS_ERROR      L = || X E ||^2 with E = S^-1 Q(S W) - W formed per
  *                       weight in fp32 (from the quantiser's rounding residual,
- *                       kept to 1/128 of a quantisation step) and rounded to
+ *                       kept to 1/256 of a quantisation step) and rounded to
  *                       bf16 once; the default, and the more accurate form.
  *   AWQ_LOSS_REFERENCE  the reference output X W is computed once per tile by
  *                       the same GEMM (bf16 W) and subtracted from

@@ -9,7 +9,7 @@
 #include <string>
 #include <vector>
 
-#include "../../include/awq_b200.h"
+#include "awq_b200.h"
 #include "internal.cuh"
 
 namespace {

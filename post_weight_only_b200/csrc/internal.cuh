@@ -28,9 +28,9 @@ cudaError_t launch_scale_table(const float* a, int64_t D, const AlphaList& alpha
                                float* s_tab, float* r_tab, cudaStream_t st);
 
 // ---- quant.cu
-// Search-side quantiser, per alpha: the codes (error form: 7-bit rounding
+// Search-side quantiser, per alpha: the codes (error form: 8-bit rounding
 // residuals, 4 per word; reference form: 4-bit codes in interleaved nibble
-// order), the per-group deltas (error form: times 2^-7), and the bf16 pairs
+// order), the per-group deltas (error form: times 2^-8), and the bf16 pairs
 // of W (may be null).  See quant.cu.
 cudaError_t launch_search_codes(const float* W, const float* s_tab, int64_t D_in, int64_t D_out, int A, int bits,
                                 int group, int form, uint32_t* codes, float* delta, uint32_t* w_pairs,

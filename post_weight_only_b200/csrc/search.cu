@@ -12,17 +12,17 @@
 //   error form (default)  the MMA operand is the weight error itself,
 //       E = S^-1 Q(S W) - W,  E_kn = (q_kn - w'_kn / delta) * delta / s_k,
 //       and L = ||X E||^2.  The quantiser's rounding residual
-//       e' = q - w'/delta (in [-1/2, 1/2]) arrives as a 7-bit fixed-point code
-//       per weight (made once per alpha by quant.cu); the subtraction happens
-//       in fp32 before the one rounding to bf16, so the bf16 rounding error is
-//       relative to E, not to W.
+//       e' = q - w'/delta (in [-1/2, 1/2]) arrives as an 8-bit fixed-point code
+//       per weight (made once per alpha by quant.cu) and E is formed in fp32
+//       and rounded to bf16 once, so the bf16 rounding error is relative to E,
+//       not to W.
 //   reference form        the literal two-product form: the reference output
 //       X W is computed once per tile by the same GEMM (bf16 W), parked in a
 //       per-CTA scratch that stays in L2, and every alpha pass computes
 //       X S^-1 Q(S W) from 4-bit codes and subtracts it in the epilogue.
 //
 // Orientation.  The MMA computes the transposed product D = A B with
-//   A = weight tile (M = 128 output columns of the layer, K = D_in),
+//   A = weight tile (M = 256 output columns of the layer, K = D_in),
 //   B = X^T tile    (N = 256 calibration tokens,          K = D_in),
 // so that the operand that changes with alpha is the A operand, which
 // tcgen05.mma reads straight from tensor memory.  Weight producer warps decode
@@ -30,16 +30,28 @@
 // tcgen05.st: the produced tile never touches shared memory, which stays free
 // for the TMA stream of X.  Each produced weight is reused by 256 tokens.
 //
-// Roles (448 threads, one CTA per SM, persistent):
-//   warp 0      TMA: X tile (256 tokens x 64 k, 128B-swizzled) and, on its own
-//               barrier, the side data of the stage (codes, deltas, 1/s; the
-//               bf16 weights for a reference pass)
-//   warp 1      allocates TMEM; lane 0 issues tcgen05.mma (M128 N256 K16)
+// CTA pairs.  Two CTAs of a cluster run one tcgen05.mma.cta_group::2 (M 256,
+// N 256, K 16), issued by the leader: each CTA holds 128 of the 256 weight
+// columns in its TMEM (A operand and accumulator) and stages 128 of the 256
+// tokens of the X tile in its shared memory (B operand), which the pair's
+// tensor cores share.  So each SM streams half an X tile per stage, which
+// keeps the shared-memory pipe (TMA writes, MMA reads, producer reads) well
+// below saturation.  Both CTAs' X copies complete on the leader's barrier; the
+// producers and epilogues of both CTAs arrive on the leader's barriers; the
+// leader's commits arrive on the barriers of both CTAs (multicast).  No TMA
+// load uses cluster multicast.
+//
+// Roles (480 threads per CTA, one CTA per SM, persistent):
+//   warp 0      TMA: this CTA's X half-tile (128 tokens x 64 k, 128B-swizzled)
+//   warp 14     TMA of the side data (codes, deltas, 1/s; the bf16 weights for
+//               a reference pass), on its own, deeper ring
+//   warp 1      allocates TMEM (pair); lane 0 of the leader issues the MMAs
 //   warps 2-9   weight producers: two per TMEM lane quarter, taking even and
 //               odd stages in turn, so that one's tcgen05.st overlaps the
 //               other's decoding
 //   warps 10-13 epilogue, one per TMEM lane quarter (256 tokens each)
-// TMEM: columns [0, 256) accumulator, [256, 384) four 32-column A stages.
+// TMEM: columns [0, 256) accumulator, [256, 512) eight (error form) or four
+// 32-column A stages.
 //
 // Work: a unit is (128 output columns) x (256 tokens); per unit the passes
 // are the alphas (after the reference pass in the reference form).  Units are
@@ -61,22 +73,37 @@
 namespace awq {
 namespace {
 
-constexpr int kBM = 128;                 // output columns per tile (MMA M, TMEM lanes)
-constexpr int kBN = 256;                 // tokens per tile (MMA N)
+constexpr int kBM = 128;                 // output columns per CTA (TMEM lanes); a pair covers 256
+constexpr int kPairM = 256;              // MMA M: output columns per CTA pair
+constexpr int kBN = 256;                 // tokens per tile (MMA N); each CTA stages 128
+constexpr int kHalfN = kBN / 2;
 constexpr int kBK = 64;                  // k per stage: one 128-byte swizzle row of bf16
-constexpr int kStages = 4;
+constexpr int kXStages = 6;              // ring of X half-tiles in shared memory
 constexpr int kACol0 = 256;              // first TMEM column of the A stages
 constexpr int kTmemCols = 512;
-constexpr int kXStageBytes = kBN * kBK * 2;      // 32 KiB
-constexpr int kAuxStageBytes = 16384;            // bf16 W pairs (16 KiB) or codes+deltas+1/s
+constexpr int kXStageBytes = kHalfN * kBK * 2;   // 16 KiB: this CTA's 128 tokens x 64 k
 constexpr int kAuxCodesOff = 0;                  // error form [16][128] u32, reference form [8][128] u32
 constexpr int kAuxDeltaOff = 8192;               // [<=2][128] f32
 constexpr int kAuxROff = 9216;                   // [64] f32 (1/s of the stage's rows)
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;
 constexpr int kEpiWarps = 4;
 constexpr int kProdWarps = 8;
-constexpr int kProdPerStage = 4;         // producer warps that fill one stage (one per lane quarter)
-constexpr int kSmemBytes = kStages * (kXStageBytes + kAuxStageBytes) + 1024 /*barriers*/ + 1024 /*align*/;
+constexpr int kProdPerStage = 4;         // producer warps of one CTA that fill one stage
+constexpr int kAuxTmaWarp = 14;
+constexpr uint16_t kPairMask = 0x3;
+
+// The weight (A operand) ring is decoupled from the X ring and deeper: the
+// side data of a stage can only be requested once the MMA has released the
+// stage, and it then goes through a TMA round trip and the producers' decode
+// before the MMA needs it again, so that ring holds eight stages (TMEM columns
+// 256..511) in the error form.  The reference form's reference pass needs
+// 16 KiB of side data per stage, so it keeps four.
+template <int kForm>
+struct Ring {
+  static constexpr int kAStages = kForm == kFormError ? 8 : 4;
+  static constexpr int kAuxBytes = kForm == kFormError ? 10240 : 16384;
+  static constexpr int kSmemBytes = kXStages * kXStageBytes + kAStages * kAuxBytes + 1024 /*barriers*/ + 1024 /*align*/;
+};
 
 enum Site { kSiteTmaEmpty = 1, kSiteMmaAccEmpty, kSiteMmaFull, kSiteMmaAReady, kSiteProdFull, kSiteEpiAccFull,
             kSiteDrainTma, kSiteDrainMma, kSiteSelfTest };
@@ -95,8 +122,8 @@ struct Segment {
   int u, a0, a1;     // unit, alpha range [a0, a1)
 };
 
-// The sequence of segments a CTA processes.  Every role walks the same
-// sequence, so ring positions and barrier phases agree.
+// The sequence of segments a CTA pair processes.  Every role of both CTAs
+// walks the same sequence, so ring positions and barrier phases agree.
 struct Schedule {
   int U, A, G, c;
   int full_waves, head;
@@ -159,49 +186,59 @@ __device__ __forceinline__ bool is_ref_pass(const Segment& sg, int pass) {
 __device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
 __device__ __forceinline__ __nv_bfloat162 as_bf16x2(uint32_t v) { return *reinterpret_cast<__nv_bfloat162*>(&v); }
 
-// One bf16 pair of A-operand values, rows (k, k+1) of one column:
-//   v     the two codes as bf16 values 128 + u (exact small integers)
-//   off2  the code offset (128 + bias) in both halves, so v - off2 is the
-//         signed integer code exactly
-//   c     fl32(delta / s_k) per row (times 2^-7 for the 7-bit error codes),
-//         rounded to bf16 once per element, then the product once more.
-// Both roundings are per element: no rounding error is shared by a whole row
-// or a whole group of the operand.
+// One bf16 pair of reference-form A-operand values, rows (k, k+1) of one
+// column: v holds the two 4-bit codes as bf16 values 128 + u (exact small
+// integers), off2 the code offset 128 + 2^(b-1) in both halves, so v - off2 is
+// the signed code q exactly; c = fl32(delta / s_k) is rounded to bf16 once per
+// element and q * c once more.  No rounding error is shared by a whole row or
+// a whole group of the operand.
 __device__ __forceinline__ uint32_t decode_pair(uint32_t v, uint32_t off2, float c_lo, float c_hi) {
   const __nv_bfloat162 q = __hsub2(as_bf16x2(v), as_bf16x2(off2));
   return bf16x2_bits(__hmul2(q, __floats2bfloat162_rn(c_lo, c_hi)));
 }
 
 template <int kForm>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     search_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmWp,
                   const __grid_constant__ CUtensorMap tmCodes, const __grid_constant__ CUtensorMap tmDelta,
                   const __grid_constant__ CUtensorMap tmR, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int kAS = Ring<kForm>::kAStages;
+  constexpr int kAuxStageBytes = Ring<kForm>::kAuxBytes;
   uint8_t* xs = smem;
-  uint8_t* aux = smem + kStages * kXStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(aux + kStages * kAuxStageBytes);
-  uint64_t* xfull = bars;                   // X tile landed
-  uint64_t* afull = bars + kStages;         // side data landed
-  uint64_t* aready = bars + 2 * kStages;    // A operand written to TMEM
-  uint64_t* empty = bars + 3 * kStages;     // the MMAs of the stage completed
-  uint64_t* acc_full = bars + 4 * kStages;
-  uint64_t* acc_empty = acc_full + 1;
+  uint8_t* aux = smem + kXStages * kXStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(aux + kAS * kAuxStageBytes);
+  // Every CTA holds the full set; xfull, aready and acc_empty are used in the
+  // leader (rank 0) only, where both CTAs' copies and warps arrive.
+  uint64_t* xfull = bars;                   // both X halves landed (leader)       [kXStages]
+  uint64_t* xempty = xfull + kXStages;      // MMAs done with the X stage          [kXStages]
+  uint64_t* afull = xempty + kXStages;      // this CTA's side data landed         [kAS]
+  uint64_t* aready = afull + kAS;           // both CTAs' A stages written (leader) [kAS]
+  uint64_t* aempty = aready + kAS;          // MMAs done with the A stage          [kAS]
+  uint64_t* acc_full = aempty + kAS;
+  uint64_t* acc_empty = acc_full + 1;       // both CTAs' epilogues drained (leader)
   uint64_t* mma_done = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kXStages; ++s) {
       mbar_init(&xfull[s], 1);
+      mbar_init(&xempty[s], 1);
+    }
+    for (int s = 0; s < kAS; ++s) {
       mbar_init(&afull[s], 1);
-      mbar_init(&aready[s], kProdPerStage);
-      mbar_init(&empty[s], 1);
+      mbar_init(&aready[s], 2 * kProdPerStage);
+      mbar_init(&aempty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kEpiWarps);
+    mbar_init(acc_empty, 2 * kEpiWarps);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -216,24 +253,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();       // barriers of both CTAs initialised, TMEM of both allocated
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const uint64_t tmo = p.timeout_ns;
+  bool aborted = false;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == kAuxTmaWarp) {
+    // ------------------------------------------------------------ TMA: X half-tiles (warp 0), side data (warp 14)
     if (lane == 0) {
-      Schedule sch(p.U, p.A, gridDim.x, blockIdx.x);
+      const bool is_x = warp == 0;
+      const int nst = is_x ? kXStages : kAS;
+      uint64_t* emptyb = is_x ? xempty : aempty;
+      Schedule sch(p.U, p.A, npairs, pair);
       Segment sg;
       uint32_t it = 0;
-      int last_round[kStages];
+      int last_round[kAS > kXStages ? kAS : kXStages];
 #pragma unroll
-      for (int s = 0; s < kStages; ++s) last_round[s] = -1;
+      for (int s = 0; s < (kAS > kXStages ? kAS : kXStages); ++s) last_round[s] = -1;
       bool ok = true;
       const uint32_t ref_bytes = 32 * kBM * 4;
       const uint32_t code_rows = kForm == kFormError ? kBK / 4 : kBK / 8;
@@ -241,48 +283,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (ok && sch.next(sg)) {
         int wt, tt;
         unit_tiles(p, sg.u, wt, tt);
+        const int col0 = wt * kPairM + static_cast<int>(rank) * kBM;     // this CTA's weight columns
+        const int tok0 = tt * kBN + static_cast<int>(rank) * kHalfN;     // this CTA's tokens
         for (int pass = first_pass<kForm>(sg); ok && pass < sg.a1; ++pass) {
           const bool ref = is_ref_pass<kForm>(sg, pass);
           for (int kb = 0; kb < p.KB; ++kb, ++it) {
-            const int s = it % kStages;
-            const uint32_t r = it / kStages;
-            if (!wait_bounded(&empty[s], (r & 1) ^ 1, abort_flag, p.status, kSiteTmaEmpty, tmo)) {
+            const int s = it % nst;
+            const uint32_t r = it / nst;
+            if (!wait_bounded(&emptyb[s], (r & 1) ^ 1, abort_flag, p.status, kSiteTmaEmpty, tmo)) {
               ok = false;
               break;
             }
-            uint8_t* ad = aux + s * kAuxStageBytes;
-            // Side data first: the weight producers wait only for it.
-            if (ref) {
-              mbar_arrive_expect_tx(&afull[s], ref_bytes);
-              tma_load_2d(ad, &tmWp, &afull[s], wt * kBM, kb * (kBK / 2));
+            if (is_x) {
+              // Both halves complete on the leader's barrier, which expects the
+              // bytes of both.
+              if (leader) mbar_arrive_expect_tx(&xfull[s], 2 * kXStageBytes);
+              tma_load_2d_pair(xs + s * kXStageBytes, &tmX, mapa_shared(smem_u32(&xfull[s]), 0), kb * kBK, tok0);
             } else {
-              mbar_arrive_expect_tx(&afull[s], alpha_bytes);
-              tma_load_3d(ad + kAuxCodesOff, &tmCodes, &afull[s], wt * kBM, kb * code_rows, pass);
-              tma_load_3d(ad + kAuxDeltaOff, &tmDelta, &afull[s], wt * kBM, (kb * kBK) / p.group, pass);
-              tma_load_2d(ad + kAuxROff, &tmR, &afull[s], kb * kBK, pass);
+              uint8_t* ad = aux + s * kAuxStageBytes;
+              if (ref) {
+                mbar_arrive_expect_tx(&afull[s], ref_bytes);
+                tma_load_2d(ad, &tmWp, &afull[s], col0, kb * (kBK / 2));
+              } else {
+                mbar_arrive_expect_tx(&afull[s], alpha_bytes);
+                tma_load_3d(ad + kAuxCodesOff, &tmCodes, &afull[s], col0, kb * code_rows, pass);
+                tma_load_3d(ad + kAuxDeltaOff, &tmDelta, &afull[s], col0, (kb * kBK) / p.group, pass);
+                tma_load_2d(ad + kAuxROff, &tmR, &afull[s], kb * kBK, pass);
+              }
             }
-            mbar_arrive_expect_tx(&xfull[s], kXStageBytes);
-            tma_load_2d(xs + s * kXStageBytes, &tmX, &xfull[s], kb * kBK, tt * kBN);
             last_round[s] = static_cast<int>(r);
           }
         }
       }
-      // Never leave the CTA with a copy still writing into shared memory: wait
-      // for the last fill of every stage (already complete on a normal exit).
+      aborted = !ok;
+      // Never leave the CTA with a copy still writing into shared memory.
       volatile int no_abort = 0;
-      for (int s = 0; s < kStages; ++s)
-        if (last_round[s] >= 0) {
-          wait_bounded(&afull[s], last_round[s] & 1, &no_abort, p.status, kSiteDrainTma, tmo);
-          wait_bounded(&xfull[s], last_round[s] & 1, &no_abort, p.status, kSiteDrainTma, tmo);
-        }
+      if (!is_x) {
+        for (int s = 0; s < nst; ++s)
+          if (last_round[s] >= 0) wait_bounded(&afull[s], last_round[s] & 1, &no_abort, p.status, kSiteDrainTma, tmo);
+      } else if (leader) {
+        // The leader's xfull counts both halves of every round it armed.
+        for (int s = 0; s < nst; ++s)
+          if (last_round[s] >= 0)
+            wait_bounded(&xfull[s], last_round[s] & 1, &no_abort, p.status, kSiteDrainTma, tmo);
+      }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      Schedule sch(p.U, p.A, gridDim.x, blockIdx.x);
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && leader) {
+      Schedule sch(p.U, p.A, npairs, pair);
       Segment sg;
       uint32_t it = 0, acc_it = 0;
-      const uint32_t idesc = idesc_bf16_f32(kBM, kBN);
+      const uint32_t idesc = idesc_bf16_f32(kPairM, kBN);
       bool ok = true;
       while (ok && sch.next(sg)) {
         for (int pass = first_pass<kForm>(sg); ok && pass < sg.a1; ++pass, ++acc_it) {
@@ -292,27 +344,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           for (int kb = 0; kb < p.KB; ++kb, ++it) {
-            const int s = it % kStages;
-            const uint32_t r = it / kStages;
-            if (!wait_bounded(&xfull[s], r & 1, abort_flag, p.status, kSiteMmaFull, tmo) ||
-                !wait_bounded(&aready[s], r & 1, abort_flag, p.status, kSiteMmaAReady, tmo)) {
+            const int sx = it % kXStages, sa = it % kAS;
+            if (!wait_bounded(&xfull[sx], (it / kXStages) & 1, abort_flag, p.status, kSiteMmaFull, tmo) ||
+                !wait_bounded(&aready[sa], (it / kAS) & 1, abort_flag, p.status, kSiteMmaAReady, tmo)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint64_t bdesc = sw128_kmajor_desc(smem_u32(xs + s * kXStageBytes));
-            const uint32_t a_tmem = tbase + kACol0 + s * (kBK / 2);
+            const uint64_t bdesc = sw128_kmajor_desc(smem_u32(xs + sx * kXStageBytes));
+            const uint32_t a_tmem = tbase + kACol0 + sa * (kBK / 2);
 #pragma unroll
             for (int j = 0; j < kBK / 16; ++j)
-              mma_ts_f16(tbase, a_tmem + j * 8, bdesc + 2 * j, idesc, (kb | j) != 0 ? 1u : 0u);
-            mma_commit(&empty[s]);
+              mma_ts_f16_pair(tbase, a_tmem + j * 8, bdesc + 2 * j, idesc, (kb | j) != 0 ? 1u : 0u);
+            mma_commit_pair_multicast(&xempty[sx], kPairMask);
+            mma_commit_pair_multicast(&aempty[sa], kPairMask);
           }
           if (!ok) break;
-          mma_commit(acc_full);
+          mma_commit_pair_multicast(acc_full, kPairMask);
         }
       }
-      // All MMAs must have finished before TMEM is released.
-      mma_commit(mma_done);
+      aborted = !ok;
+      // All MMAs (which write both CTAs' TMEM) must have finished before
+      // either CTA releases its TMEM.
+      mma_commit_pair_multicast(mma_done, kPairMask);
+    }
+    if (lane == 0) {
       volatile int no_abort = 0;
       wait_bounded(mma_done, 0, &no_abort, p.status, kSiteDrainMma, tmo);
     }
@@ -322,20 +378,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const uint32_t parity = static_cast<uint32_t>((warp - 2) >> 2);   // this warp fills stages it % 2 == parity
     const int nl = q * 32 + lane;
-    Schedule sch(p.U, p.A, gridDim.x, blockIdx.x);
+    Schedule sch(p.U, p.A, npairs, pair);
     Segment sg;
     uint32_t it = 0;
     bool ok = true;
     const uint32_t off2 = static_cast<uint32_t>(p.off_bf16x2);
     const bool two_groups = p.gpb == 2;   // group 32: a 64-k stage spans two groups
     const uint32_t lane_addr = tbase + (static_cast<uint32_t>(q * 32) << 16) + kACol0;
+    const uint32_t aready_leader = mapa_shared(smem_u32(aready), 0);
     while (ok && sch.next(sg)) {
       for (int pass = first_pass<kForm>(sg); ok && pass < sg.a1; ++pass) {
         const bool ref = is_ref_pass<kForm>(sg, pass);
         for (int kb = 0; kb < p.KB; ++kb, ++it) {
           if ((it & 1u) != parity) continue;
-          const int s = it % kStages;
-          const uint32_t r = it / kStages;
+          const int s = it % kAS;
+          const uint32_t r = it / kAS;
           // The tcgen05.st below is warp-collective: take the outcome of the
           // wait as a warp, never split the warp on a timeout.
           const bool got = wait_bounded(&afull[s], r & 1, abort_flag, p.status, kSiteProdFull, tmo);
@@ -355,10 +412,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i) out[i] = cw[i * kBM + nl];
             tmem_st32(st_addr, out);
           } else if (kForm == kFormError) {
-            // Word j holds the 7-bit codes u = k + 64 of rows 4j .. 4j+3 as
-            // bytes; one byte permute turns two of them into the bf16 pair
-            // (128 + u0, 128 + u1).  Two 16-column halves keep the live set
+            // Word j holds the 8-bit codes u = 256 e' + 128 of rows 4j .. 4j+3.
+            // A byte permute places u in the mantissa of the float 2^23 + u;
+            // subtracting 2^23 + 128 leaves k = 256 e' exactly, and
+            // E = k * (delta 2^-8 / s_k) is formed in fp32 (packed pairs) and
+            // rounded to bf16 once.  Two 16-column halves keep the live set
             // small.
+            const float2 bias = make_float2(-8388736.0f, -8388736.0f);    // -(2^23 + 128)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
               uint32_t out[16];
@@ -368,10 +428,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t word = cw[j * kBM + nl];
                 const float d = dl[(two_groups ? hh : 0) * kBM + nl];
                 const float4 rv = rf[j];
-                const uint32_t v0 = __byte_perm(word, 0x43u, 0x4140u);
-                const uint32_t v1 = __byte_perm(word, 0x43u, 0x4342u);
-                out[2 * jj] = decode_pair(v0, off2, __fmul_rn(d, rv.x), __fmul_rn(d, rv.y));
-                out[2 * jj + 1] = decode_pair(v1, off2, __fmul_rn(d, rv.z), __fmul_rn(d, rv.w));
+                const float2 c01 = __fmul2_rn(make_float2(d, d), make_float2(rv.x, rv.y));
+                const float2 c23 = __fmul2_rn(make_float2(d, d), make_float2(rv.z, rv.w));
+                const float2 k01 = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(word, 0x4B000000u, 0x7440u)),
+                                                          __uint_as_float(__byte_perm(word, 0x4B000000u, 0x7441u))),
+                                              bias);
+                const float2 k23 = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(word, 0x4B000000u, 0x7442u)),
+                                                          __uint_as_float(__byte_perm(word, 0x4B000000u, 0x7443u))),
+                                              bias);
+                const float2 e01 = __fmul2_rn(k01, c01);
+                const float2 e23 = __fmul2_rn(k23, c23);
+                out[2 * jj] = bf16x2_bits(__floats2bfloat162_rn(e01.x, e01.y));
+                out[2 * jj + 1] = bf16x2_bits(__floats2bfloat162_rn(e23.x, e23.y));
               }
               tmem_st16(st_addr + hh * 16, out);
             }
@@ -402,25 +470,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&aready[s]);
+          if (lane == 0) mbar_arrive_cluster(aready_leader + s * 8);
         }
       }
     }
+    aborted = !ok;
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int nl = q * 32 + lane;
-    Schedule sch(p.U, p.A, gridDim.x, blockIdx.x);
+    Schedule sch(p.U, p.A, npairs, pair);
     Segment sg;
     uint32_t acc_it = 0;
     bool ok = true;
     float4* yref = reinterpret_cast<float4*>(p.yref + static_cast<size_t>(blockIdx.x) * (kBM * kBN));
     const uint32_t lane_addr = tbase + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
     const int H = p.Tt;
     while (ok && sch.next(sg)) {
       int wt, tt;
       unit_tiles(p, sg.u, wt, tt);
-      const int n = wt * kBM + nl;
+      const int n = wt * kPairM + static_cast<int>(rank) * kBM + nl;
       for (int pass = first_pass<kForm>(sg); ok && pass < sg.a1; ++pass, ++acc_it) {
         const bool ref = is_ref_pass<kForm>(sg, pass);
         const bool got = wait_bounded(acc_full, acc_it & 1, abort_flag, p.status, kSiteEpiAccFull, tmo);
@@ -431,9 +501,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (kForm == kFormError) {
           // Four 64-column quarters: load both chunks of a quarter, then square
-          // and sum them; release the accumulator after the last load.  (With
-          // 448 threads a thread has at most 128 registers, too few to hold
-          // more than 64 columns besides the rest of its state.)
+          // and sum them; release the accumulator after the last load.  (A
+          // thread has at most 128 registers, too few to hold more than 64
+          // columns besides the rest of its state.)
           float s0 = 0.0f, s1 = 0.0f;
 #pragma unroll 1
           for (int h4 = 0; h4 < 4; ++h4) {
@@ -444,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (h4 == 3) {
               tc_fence_before();
               __syncwarp();
-              if (lane == 0) mbar_arrive(acc_empty);
+              if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
             }
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
@@ -478,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty);
+          if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
         } else {
           float sum = 0.0f;
 #pragma unroll 1
@@ -504,17 +574,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty);
+          if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
           if (n < p.D_out) p.partial[(static_cast<size_t>(pass) * H + tt) * p.D_out + n] = sum;
         }
       }
     }
+    aborted = !ok;
   }
 
+  // After a timeout a copy issued by this CTA may still be landing in this
+  // CTA's shared memory with no barrier here to show it: give it time (a
+  // TMA round trip is a few microseconds) before the pair goes away.
+  if (aborted || *abort_flag) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) __nanosleep(1000);
+  }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();       // no CTA of the pair leaves while the other may still use its memory
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tbase, kTmemCols);
+  if (warp == 1) tmem_dealloc_pair(tbase, kTmemCols);
 }
 
 __global__ void wait_timeout_selftest_kernel(int* status, unsigned long long timeout_ns) {
@@ -565,11 +644,11 @@ cudaError_t launch_form(int grid, const CUtensorMap& mX, const CUtensorMap& mWp,
   cudaGetDevice(&dev);
   if (attr_set_device != dev) {
     cudaError_t e = cudaFuncSetAttribute(search_kernel<kForm>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
+                                         Ring<kForm>::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set_device = dev;
   }
-  search_kernel<kForm><<<grid, kThreads, kSmemBytes, st>>>(mX, mWp, mC, mD, mR, p);
+  search_kernel<kForm><<<grid, kThreads, Ring<kForm>::kSmemBytes, st>>>(mX, mWp, mC, mD, mR, p);
   return cudaGetLastError();
 }
 
@@ -577,10 +656,13 @@ cudaError_t launch_form(int grid, const CUtensorMap& mX, const CUtensorMap& mWp,
 
 int search_token_tiles(int N) { return (N + kBN - 1) / kBN; }
 
+// Number of CTAs (two per pair): one pair per unit of work, at most one CTA
+// per SM.
 int search_grid_size(const SearchShape& sh, int num_sms) {
-  const long long U = static_cast<long long>((sh.D_out + kBM - 1) / kBM) * search_token_tiles(sh.N);
+  const long long U = static_cast<long long>((sh.D_out + kPairM - 1) / kPairM) * search_token_tiles(sh.N);
   const long long work = sh.A > 0 ? U * sh.A : U;
-  return static_cast<int>(work < num_sms ? work : num_sms);
+  const long long pairs = num_sms / 2;
+  return 2 * static_cast<int>(work < pairs ? work : pairs);
 }
 
 int launch_search(const SearchShape& sh, const SearchBuffers& b, int grid, uint64_t timeout_ns, cudaStream_t st,
@@ -592,7 +674,7 @@ int launch_search(const SearchShape& sh, const SearchBuffers& b, int grid, uint6
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(sh.D_in), static_cast<uint64_t>(sh.N)};
     const uint64_t str[1] = {static_cast<uint64_t>(sh.D_in) * 2};
-    const uint32_t box[2] = {kBK, kBN};
+    const uint32_t box[2] = {kBK, kHalfN};
     if (!make_map(&mX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, b.X, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) {
       *what = "tensor map for X";
       return kECuda;
@@ -660,13 +742,13 @@ int launch_search(const SearchShape& sh, const SearchBuffers& b, int grid, uint6
     p.off_bf16x2 = static_cast<int>(h | (h << 16));
   }
   p.Tt = search_token_tiles(sh.N);
-  p.Wt = (sh.D_out + kBM - 1) / kBM;
+  p.Wt = (sh.D_out + kPairM - 1) / kPairM;
   p.U = p.Wt * p.Tt;
   p.KB = (sh.D_in + kBK - 1) / kBK;
   p.gpb = gpb;
   p.gemm_only = gemm_only ? 1 : 0;
   {
-    // Concurrent CTAs (one wave) either share token tiles (weight-minor
+    // Concurrent pairs (one wave) either share token tiles (weight-minor
     // numbering: all of X stays hot, plus the codes of a few weight tiles)
     // or weight tiles (token-minor: the codes of one alpha stay hot, plus a
     // few token tiles of X).  Keep the smaller working set.

@@ -70,7 +70,7 @@ def _rounding_bound(X, W, a, alpha, bits, group, form="error", cols=None, k_sigm
     if form == "reference":
         var = (2.0 * w_hat ** 2 + w ** 2) * U_BF16 ** 2 / 3.0
     else:
-        var = (2.0 ** -8 * step) ** 2 / 3.0 + 2.0 * (E * U_BF16) ** 2 / 3.0
+        var = (2.0 ** -9 * step) ** 2 / 3.0 + 2.0 * (E * U_BF16) ** 2 / 3.0
     G = x.T @ (x @ E)
     cross_sd = np.sqrt(4.0 * (var * G ** 2).sum(axis=0))          # per column
     quad = ((x ** 2).sum(axis=0)[:, None] * var).sum(axis=0)       # per column
