@@ -194,6 +194,34 @@ AWQ_API int awq_layer_output(const void* X, const float* W, int64_t N, int64_t D
                      void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
 
 /*
+ * awq_search without a caller-provided workspace, for callers that cannot
+ * allocate device memory: code that runs where the allocator must not be
+ * called (an engine or plugin host that owns all device memory and hands out
+ * only the buffers of a call, a real-time path with a fixed memory budget).
+ * The AWQ pages have no counterpart; this is an interface convenience.
+ *
+ * The scratch space is a file-scope device array of AWQ_NOALLOC_SCRATCH_BYTES
+ * (32 MiB) inside the library: every GPU that loads the library holds it until
+ * the process exits.  Shapes whose awq_search_workspace_size exceeds it are
+ * rejected with AWQ_EWORKSPACE and a message giving both sizes; they need
+ * awq_search.  Arguments, outputs and results are those of awq_search.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; each call writes every scratch byte it reads before reading it
+ *     and clears the status word it uses.  Calls that may overlap on the GPU
+ *     (different streams, or different host threads) race on the array: order
+ *     them on one stream.
+ *   - Nothing is allocated: no cudaMalloc, no cudaFree, no allocating library
+ *     routine (leave stage timing, which creates CUDA events, switched off).
+ */
+#define AWQ_NOALLOC_SCRATCH_BYTES (32u << 20)
+AWQ_API int awq_search_noalloc(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
+                               const float* alpha_grid, int n_alpha, int bits, int group, int loss_form, double* L,
+                               double* L_col, float* alpha_star, int32_t* alpha_idx, int32_t* status, void* stream);
+
+/*
  * Failure-detection self test: launches one CTA that waits on a barrier no one
  * ever arrives at, with the same bounded wait the search kernel uses.  After
  * about timeout_ns nanoseconds the wait gives up and AWQ_ETIMEOUT | (site << 8)

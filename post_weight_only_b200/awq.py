@@ -28,6 +28,7 @@ EXPORTS = (
     "awq_search_batched_workspace_size", "awq_search_batched", "awq_quantize_pack",
     "awq_layer_output_workspace_size", "awq_layer_output", "awq_selftest_wait_timeout",
     "awq_get_last_error", "awq_version", "awq_profile_enable", "awq_profile_reset", "awq_profile_read",
+    "awq_search_noalloc",
 )
 STAGES = ("act_stats", "scale_table", "search_codes", "search_gemm", "loss_reduce", "quantize_pack",
           "weight_pairs")

@@ -242,6 +242,32 @@ int check_search_args(const void* X, const float* W, const float* a, int64_t N, 
   return AWQ_OK;
 }
 
+// ---------------------------------------------------------------- scratch without allocation
+// Scratch for awq_search_noalloc: a file-scope device array.  Host code must
+// not use its name as a device address; the address comes from
+// cudaGetSymbolAddress, once per device, with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[AWQ_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(AWQ_EUNSUPPORTED, "device %d: at most %d devices", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(no-allocation scratch)");
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return AWQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -465,6 +491,35 @@ int awq_profile_read(int stage, double* total_ms, int32_t* launches) {
   if (total_ms) *total_ms = g_prof_ms[stage];
   if (launches) *launches = g_prof_n[stage];
   return AWQ_OK;
+}
+
+int awq_search_noalloc(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
+                       const float* alpha_grid, int n_alpha, int bits, int group, int loss_form, double* L,
+                       double* L_col, float* alpha_star, int32_t* alpha_idx, int32_t* status, void* stream) {
+  AWQ_TRY(check_search_args(X, W, a, N, D_in, D_out, alpha_grid, n_alpha, bits, group, loss_form, L, L_col,
+                            alpha_star, alpha_idx));
+  int sms = 0;
+  AWQ_TRY(device_info(&sms));
+  const SearchLayout lay = search_layout(N, D_in, D_out, n_alpha, group, loss_form, sms);
+  if (lay.total > AWQ_NOALLOC_SCRATCH_BYTES)
+    return fail(AWQ_EWORKSPACE,
+                "awq_search_noalloc: this shape needs %zu bytes of scratch, the built-in scratch holds %u; "
+                "use awq_search with a workspace",
+                lay.total, static_cast<unsigned>(AWQ_NOALLOC_SCRATCH_BYTES));
+  if (status && !aligned(status, 4)) return fail(AWQ_EALIGN, "status is not 4-byte aligned");
+  void* scratch = nullptr;
+  AWQ_TRY(noalloc_scratch(&scratch));
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  int32_t* st_word = status ? status : reinterpret_cast<int32_t*>(ws + lay.status);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Every scratch byte the search reads it writes first in the same call;
+  // only the status word has to start at zero.
+  cudaError_t e = cudaMemsetAsync(st_word, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(status)");
+  awq::AlphaList al{};
+  for (int i = 0; i < n_alpha; ++i) al.v[i] = alpha_grid[i];
+  return search_one(X, W, a, N, D_in, D_out, al, n_alpha, bits, group, loss_form, L, L_col, alpha_star, alpha_idx,
+                    ws, st_word, st, sms);
 }
 
 int awq_selftest_wait_timeout(int32_t* status, int64_t timeout_ns_arg, void* stream) {
