@@ -5,7 +5,7 @@
                     [--workload NAME]
 
 One step is one pass of the whole per-layer path over one synthetic layer:
-activation statistic -> alpha grid search (scale table, per-alpha codes, the
+activation statistic -> alpha grid search (scale table, per-alpha bf16 operand, the
 fused tensor-core loss GEMM, loss reduction + argmin) -> s* = a^alpha* ->
 final quantise + pack.  The default workload is the LLaMA-7B-shaped attention
 projection (X 4096 x 4096 bf16, W 4096 x 4096 fp32, 4-bit g128, 21 alphas).
@@ -39,13 +39,12 @@ if ROOT not in sys.path:
 METRIC = "AWQ search α-candidates/s per layer; eff. TFLOP/s and % of B200 bf16 peak"
 UNIT = "alpha-candidates/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 8   # act_stats, scale table, codes, loss GEMM, 2 x reduce, s*, pack
 
 
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="llama7b_attn_proj")
@@ -88,9 +87,10 @@ def committed_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 200 ms while the
-    timed region runs."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clocks and throttle reasons, sampled every 20 ms around the
+    timed region; only the samples taken inside the region (by their
+    timestamps against the host clock at its start and end) are reported."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -98,6 +98,7 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
 
     def start(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -105,15 +106,31 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "20"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
         time.sleep(0.3)
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    @staticmethod
+    def _stamp(text):
+        import datetime
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(text, fmt).timestamp()
+            except ValueError:
+                pass
+        return None
+
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
+        time.sleep(0.1)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -126,17 +143,25 @@ class ClockSampler:
                 if len(parts) >= 9:
                     rows.append(parts)
         os.unlink(self.path)
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        inside = [r for r in rows if (t := self._stamp(r[0])) is not None and self.t0 is not None
+                  and self.t0 - 0.02 <= t <= self.t1 + 0.02]
+        use = inside or rows
+        sm = [v for r in use if (v := num(r[1])) is not None]
+        smax = [v for r in rows if (v := num(r[2])) is not None]
+        power = [v for r in use if (v := num(r[3])) is not None]
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
-        # "under load": samples drawing at least half of the peak power seen
-        loaded = [s for s, p in zip(sm, power) if power and p >= 0.5 * max(power)] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+        reasons = sorted({names[i] for r in use for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
                 "power_w_max": max(power) if power else None,
-                "samples": len(rows), "reasons": reasons}
+                "samples": len(use), "samples_in_timed_region": len(inside),
+                "interval_ms": 20, "reasons": reasons}
 
 
 def layer_for_rank(wl, rank):
@@ -280,12 +305,14 @@ def run_ours(args):
     awq.profile_reset()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier()
+    clocks.mark_start()
     for k in range(args.steps):
         flush.zero_()                      # evict X and W from L2 before every step
         ev[k][0].record()
         r = step()
         ev[k][1].record()
     barrier()
+    clocks.mark_end()
     clk = clocks.stop()
     prof = awq.profile_read()
     awq.profile_enable(False)
@@ -340,8 +367,10 @@ def run_ours(args):
     stats_bytes = layer.N * layer.D_in * 2 + layer.D_in * 4
     pack_bytes = layer.D_in * layer.D_out * 4 + layer.D_in * 4 + (layer.D_in // 8) * layer.D_out * 4 + \
         (layer.D_in // group) * layer.D_out * 4
+    # W once, s and 1/s per alpha, the bf16 operand per alpha
+    operand_bytes = layer.D_in * layer.D_out * 4 + A * layer.D_in * 8 + A * layer.D_in * layer.D_out * 2
     kernels = {name: {"total_ms": ms, "launches": n} for name, (ms, n) in prof.items() if n}
-    launches = KERNELS_PER_STEP * args.steps
+    launches = sum(n for _, n in prof.values())     # the library's launches in the timed region
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -351,7 +380,8 @@ def run_ours(args):
         "eff_tflops": flops * world / (ms_per_step / 1e3) / 1e12,
         "pct_bf16_peak_step": flops / (ms_per_step / 1e3) / 1e12 / peak,
         "roofline": roof,
-        "hbm_kernels": {"act_stats": hbm("act_stats", stats_bytes), "quantize_pack": hbm("quantize_pack", pack_bytes)},
+        "hbm_kernels": {"act_stats": hbm("act_stats", stats_bytes), "quantize_pack": hbm("quantize_pack", pack_bytes),
+                        "search_operand": hbm("search_operand", operand_bytes)},
         "kernels": kernels,
         "e2e": {"value": A * world / (e2e_per_step / 1e3), "unit": UNIT, "ms_per_step": e2e_per_step,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

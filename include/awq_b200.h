@@ -238,11 +238,11 @@ AWQ_API int awq_selftest_wait_timeout(int32_t* status, int64_t timeout_ns, void*
 enum {
   AWQ_STAGE_ACT_STATS = 0,     /* awq_act_stats */
   AWQ_STAGE_SCALE_TABLE = 1,   /* s = a^alpha (and 1/s) for the alpha grid, or one alpha */
-  AWQ_STAGE_SEARCH_CODES = 2,  /* per-alpha INT codes + deltas of diag(s) W */
+  AWQ_STAGE_SEARCH_OPERAND = 2, /* per-alpha bf16 GEMM operand: S^-1 Q(S W) - W, or S^-1 Q(S W) */
   AWQ_STAGE_SEARCH_GEMM = 3,   /* the fused tensor-core loss GEMM */
   AWQ_STAGE_LOSS_REDUCE = 4,   /* L(alpha), argmin */
   AWQ_STAGE_QUANTIZE_PACK = 5, /* awq_quantize_pack */
-  AWQ_STAGE_WEIGHT_PAIRS = 6,  /* bf16 copy of W for awq_layer_output */
+  AWQ_STAGE_WEIGHT_T = 6,      /* bf16 W^T: reference pass of the search, awq_layer_output */
   AWQ_NUM_STAGES = 7
 };
 AWQ_API int awq_profile_enable(int on);

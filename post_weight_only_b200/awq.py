@@ -30,8 +30,8 @@ EXPORTS = (
     "awq_get_last_error", "awq_version", "awq_profile_enable", "awq_profile_reset", "awq_profile_read",
     "awq_search_noalloc",
 )
-STAGES = ("act_stats", "scale_table", "search_codes", "search_gemm", "loss_reduce", "quantize_pack",
-          "weight_pairs")
+STAGES = ("act_stats", "scale_table", "search_operand", "search_gemm", "loss_reduce", "quantize_pack",
+          "weight_t")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(

@@ -66,8 +66,8 @@ uint64_t timeout_ns() {
 }
 
 struct SearchLayout {
-  size_t s_tab, r_tab, codes, delta, w_pairs, yref, partial, blk, status, total;
-  int grid, Tt, nblk;
+  size_t s_tab, r_tab, op, wt, yref, partial, blk, status, total;
+  int grid, H, nblk;
 };
 
 SearchLayout search_layout(int64_t N, int64_t D_in, int64_t D_out, int A, int group, int form, int num_sms) {
@@ -75,7 +75,7 @@ SearchLayout search_layout(int64_t N, int64_t D_in, int64_t D_out, int A, int gr
   awq::SearchShape sh{static_cast<int>(N), static_cast<int>(D_in), static_cast<int>(D_out), A, 4, group, form};
   const bool ref = form == AWQ_LOSS_REFERENCE;
   L.grid = awq::search_grid_size(sh, num_sms);
-  L.Tt = awq::search_token_tiles(static_cast<int>(N));
+  L.H = awq::search_partial_rows(static_cast<int>(N));
   L.nblk = awq::loss_reduce_blocks(D_out);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -86,11 +86,10 @@ SearchLayout search_layout(int64_t N, int64_t D_in, int64_t D_out, int A, int gr
   const size_t a = static_cast<size_t>(A);
   L.s_tab = take(a * D_in * 4);
   L.r_tab = take(a * D_in * 4);
-  L.codes = take(a * (D_in / (ref ? 8 : 4)) * D_out * 4);
-  L.delta = take(A > 0 ? a * (D_in / group) * D_out * 4 : 0);
-  L.w_pairs = take(ref ? static_cast<size_t>(D_in / 2) * D_out * 4 : 0);
+  L.op = take(a * D_out * D_in * 2);
+  L.wt = take(ref ? static_cast<size_t>(D_out) * D_in * 2 : 0);
   L.yref = take(A > 0 && ref ? static_cast<size_t>(L.grid) * 128 * 256 * 4 : 0);
-  L.partial = take(a * L.Tt * D_out * 4);
+  L.partial = take(a * L.H * D_out * 4);
   L.blk = take(a * L.nblk * 8);
   L.status = take(4);
   L.total = off;
@@ -187,9 +186,8 @@ int search_one(const void* X, const float* W, const float* a, int64_t N, int64_t
   const SearchLayout lay = search_layout(N, D_in, D_out, A, group, form, num_sms);
   float* s_tab = reinterpret_cast<float*>(ws + lay.s_tab);
   float* r_tab = reinterpret_cast<float*>(ws + lay.r_tab);
-  uint32_t* codes = reinterpret_cast<uint32_t*>(ws + lay.codes);
-  float* delta = reinterpret_cast<float*>(ws + lay.delta);
-  uint32_t* w_pairs = form == AWQ_LOSS_REFERENCE ? reinterpret_cast<uint32_t*>(ws + lay.w_pairs) : nullptr;
+  uint16_t* op = reinterpret_cast<uint16_t*>(ws + lay.op);
+  uint16_t* wt = form == AWQ_LOSS_REFERENCE ? reinterpret_cast<uint16_t*>(ws + lay.wt) : nullptr;
   float* yref = reinterpret_cast<float*>(ws + lay.yref);
   float* partial = reinterpret_cast<float*>(ws + lay.partial);
   double* blk = reinterpret_cast<double*>(ws + lay.blk);
@@ -201,12 +199,17 @@ int search_one(const void* X, const float* W, const float* a, int64_t N, int64_t
   }
   if (e != cudaSuccess) return fail_cuda(e, "scale table kernel");
   {
-    StageTimer t(AWQ_STAGE_SEARCH_CODES, st);
-    e = awq::launch_search_codes(W, s_tab, D_in, D_out, A, bits, group, form, codes, delta, w_pairs, st);
+    StageTimer t(AWQ_STAGE_SEARCH_OPERAND, st);
+    e = awq::launch_search_operand(W, s_tab, r_tab, D_in, D_out, A, bits, group, form, op, st);
   }
-  if (e != cudaSuccess) return fail_cuda(e, "search codes kernel");
+  if (e != cudaSuccess) return fail_cuda(e, "search operand kernel");
+  if (wt) {
+    StageTimer t(AWQ_STAGE_WEIGHT_T, st);
+    e = awq::launch_weight_t(W, D_in, D_out, wt, st);
+  }
+  if (e != cudaSuccess) return fail_cuda(e, "weight transpose kernel");
   awq::SearchShape sh{static_cast<int>(N), static_cast<int>(D_in), static_cast<int>(D_out), A, bits, group, form};
-  awq::SearchBuffers b{X, w_pairs, codes, delta, r_tab, yref, partial, nullptr, status};
+  awq::SearchBuffers b{X, wt, op, yref, partial, nullptr, status};
   const char* what = "search kernel";
   int rc;
   {
@@ -216,7 +219,7 @@ int search_one(const void* X, const float* W, const float* a, int64_t N, int64_t
   if (rc != AWQ_OK) return e != cudaSuccess ? fail_cuda(e, what) : fail(rc, "%s failed", what);
   {
     StageTimer t(AWQ_STAGE_LOSS_REDUCE, st);
-    e = awq::launch_loss_reduce(partial, A, lay.Tt, D_out, L_col, blk, lay.nblk, alphas, L, alpha_star,
+    e = awq::launch_loss_reduce(partial, A, lay.H, D_out, L_col, blk, lay.nblk, alphas, L, alpha_star,
                                 alpha_idx, st);
   }
   if (e != cudaSuccess) return fail_cuda(e, "loss reduction kernels");
@@ -450,15 +453,15 @@ int awq_layer_output(const void* X, const float* W, int64_t N, int64_t D_in, int
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(st_word, 0, sizeof(int32_t), st);
   if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(status)");
-  uint32_t* w_pairs = reinterpret_cast<uint32_t*>(ws + lay.w_pairs);
+  uint16_t* wt = reinterpret_cast<uint16_t*>(ws + lay.wt);
   {
-    StageTimer t(AWQ_STAGE_WEIGHT_PAIRS, st);
-    e = awq::launch_weight_pairs(W, D_in, D_out, w_pairs, st);
+    StageTimer t(AWQ_STAGE_WEIGHT_T, st);
+    e = awq::launch_weight_t(W, D_in, D_out, wt, st);
   }
-  if (e != cudaSuccess) return fail_cuda(e, "weight pairs kernel");
+  if (e != cudaSuccess) return fail_cuda(e, "weight transpose kernel");
   awq::SearchShape sh{static_cast<int>(N), static_cast<int>(D_in), static_cast<int>(D_out), 0, 4, 128,
                       AWQ_LOSS_REFERENCE};
-  awq::SearchBuffers b{X, w_pairs, nullptr, nullptr, nullptr, nullptr, nullptr, Y, st_word};
+  awq::SearchBuffers b{X, wt, nullptr, nullptr, nullptr, Y, st_word};
   const char* what = "search kernel (reference output)";
   int rc;
   {

@@ -28,16 +28,13 @@ cudaError_t launch_scale_table(const float* a, int64_t D, const AlphaList& alpha
                                float* s_tab, float* r_tab, cudaStream_t st);
 
 // ---- quant.cu
-// Search-side quantiser, per alpha: the codes (error form: 8-bit rounding
-// residuals, 4 per word; reference form: 4-bit codes in interleaved nibble
-// order), the per-group deltas (error form: times 2^-8), and the bf16 pairs
-// of W (may be null).  See quant.cu.
-cudaError_t launch_search_codes(const float* W, const float* s_tab, int64_t D_in, int64_t D_out, int A, int bits,
-                                int group, int form, uint32_t* codes, float* delta, uint32_t* w_pairs,
-                                cudaStream_t st);
-// bf16 pairs of W for the reference pass: w_pairs[k/2][n] = (bf16 w[k][n],
-// bf16 w[k+1][n]) as the low and high halves.
-cudaError_t launch_weight_pairs(const float* W, int64_t D_in, int64_t D_out, uint32_t* w_pairs, cudaStream_t st);
+// The search's A operand for every alpha, bf16 [A][D_out][D_in]: error form
+// (S^-1 Q(S W) - W)^T, reference form (S^-1 Q(S W))^T.  See quant.cu.
+cudaError_t launch_search_operand(const float* W, const float* s_tab, const float* r_tab, int64_t D_in,
+                                  int64_t D_out, int A, int bits, int group, int form, uint16_t* op,
+                                  cudaStream_t st);
+// bf16 W^T [D_out][D_in] for the reference output X W.
+cudaError_t launch_weight_t(const float* W, int64_t D_in, int64_t D_out, uint16_t* wt, cudaStream_t st);
 // Final quantise + pack for one given scale vector s (natural nibble order).
 cudaError_t launch_quantize_pack(const float* W, const float* s, int64_t D_in, int64_t D_out, int bits, int group,
                                  uint32_t* packed, float* scales, cudaStream_t st);
@@ -54,17 +51,17 @@ struct SearchShape {
 };
 struct SearchBuffers {
   const void* X;              // bf16 [N][D_in]
-  const uint32_t* w_pairs;    // [D_in/2][D_out]
-  const uint32_t* codes;      // [A][D_in/4][D_out] (error form) or [A][D_in/8][D_out]
-  const float* delta;         // [A][D_in/group][D_out]
-  const float* r_tab;         // [A][D_in] fp32 1/s
+  const uint16_t* wt;         // bf16 W^T [D_out][D_in] (reference pass, gemm-only mode)
+  const uint16_t* op;         // bf16 [A][D_out][D_in], the per-alpha operand
   float* yref;                // [grid][128*256]
-  float* partial;             // [A][Tt][D_out]
+  float* partial;             // [A][search_partial_rows(N)][D_out]
   float* y_out;               // gemm-only mode: [N][D_out]
   int* status;
 };
 int search_grid_size(const SearchShape& sh, int num_sms);
 int search_token_tiles(int N);
+// Rows of loss partials per alpha: one per 128-token half of a token tile.
+int search_partial_rows(int N);
 // Returns 0 on success, otherwise an awq error code; *cerr gets the CUDA error.
 int launch_search(const SearchShape& sh, const SearchBuffers& b, int grid, uint64_t timeout_ns, cudaStream_t st,
                   cudaError_t* cerr, const char** what);
