@@ -16,6 +16,7 @@ import pytest
 import torch
 
 import oracle
+from gpu_bounds import check_alpha, rounding_bound
 from post_weight_only_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -39,52 +40,15 @@ def _oracle_a(X):
     return oracle.act_stats(X).astype(np.float32)
 
 
-U_BF16 = 2.0 ** -8     # largest relative rounding error of one bf16 rounding
 FORMS = ("error", "reference")
-
-
-def _rounding_bound(X, W, a, alpha, bits, group, form="error", cols=None, k_sigma=6.0):
-    """Tolerance on |L_gpu - L| derived from the arithmetic of the CUDA path.
-
-    The tensor cores see bf16 operands.  Reference form: the dequantised
-    weight q * delta / s_k is rounded twice (once as c = delta / s_k, once as
-    q * c) and the reference weight once, so the noise eta on a weight has
-    variance var <= (2 w_hat^2 + w^2) U^2 / 3.  Error form: the operand is
-    E = e' * delta / s_k with the rounding residual e' kept to 1/128 of a step
-    (error <= 2^-8 delta / s_k) and then rounded twice relative to E, so
-    var <= (2^-8 delta / s_k)^2 / 3 + 2 E^2 U^2 / 3.  With independent
-    errors,  L_gpu - L = 2 <XE, X eta> + ||X eta||^2:  the first term has
-    variance 4 sum_kn var_kn (X^T X E)_kn^2, the second the mean
-    sum_kn (sum_i x_ik^2) var_kn.  The bound is k_sigma standard deviations of
-    the first plus three times the mean of the second.  E, s, q and delta come
-    from the oracle."""
-    s = oracle.scales(a, alpha).astype(np.float64)
-    q, d = oracle.quantize(W, s.astype(np.float32), bits, group)
-    w = W.numpy().astype(np.float64)
-    step = np.repeat(d, group, axis=0).astype(np.float64) / s[:, None]      # delta / s_k
-    w_hat = q.astype(np.float64) * step
-    E = w_hat - w
-    x = X.float().numpy().astype(np.float64)
-    if cols is not None:
-        E, w, w_hat, step = E[:, cols], w[:, cols], w_hat[:, cols], step[:, cols]
-    if form == "reference":
-        var = (2.0 * w_hat ** 2 + w ** 2) * U_BF16 ** 2 / 3.0
-    else:
-        var = (2.0 ** -9 * step) ** 2 / 3.0 + 2.0 * (E * U_BF16) ** 2 / 3.0
-    G = x.T @ (x @ E)
-    cross_sd = np.sqrt(4.0 * (var * G ** 2).sum(axis=0))          # per column
-    quad = ((x ** 2).sum(axis=0)[:, None] * var).sum(axis=0)       # per column
-    return k_sigma * cross_sd + 3.0 * quad
+_rounding_bound = rounding_bound
 
 
 def _form_id(form, awq):
     return awq.LOSS_ERROR if form == "error" else awq.LOSS_REFERENCE
 
 
-def _check_alpha(L_or, best_or, idx_gpu):
-    if idx_gpu == best_or:
-        return
-    assert L_or[idx_gpu] <= 1.01 * L_or[best_or], (idx_gpu, best_or, L_or[idx_gpu], L_or[best_or])
+_check_alpha = check_alpha
 
 
 # ------------------------------------------------------------------ statistic
