@@ -23,8 +23,10 @@
  *     its comment says "host".  Device pointers must be 16-byte aligned.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
  *     only enqueue work; they are asynchronous with respect to the host and
- *     do not synchronise.  The library allocates no device memory: scratch
- *     space comes from a caller-provided workspace whose size is queried.
+ *     do not synchronise.  Scratch space comes from a caller-provided
+ *     workspace whose size is queried; the one exception is awq_act_stats,
+ *     which takes a small stream-ordered scratch from the device's default
+ *     memory pool (see there).  The library calls no other allocator.
  *   - The return value is an awq_status.  A non-OK status from argument
  *     checking is returned before any work is enqueued; awq_get_last_error()
  *     then describes it.  Errors found on the device (a wait that timed out)
@@ -66,9 +68,9 @@ enum { AWQ_STAT_MEAN = 0, AWQ_STAT_MAX = 1 };
  * How awq_search evaluates L(alpha) = || X S^-1 Q(S W) - X W ||^2 on the tensor
  * cores (identical in exact arithmetic):
  *   AWQ_LOSS_ERROR      L = || X E ||^2 with E = S^-1 Q(S W) - W formed per
- *                       weight in fp32 (from the quantiser's rounding residual,
- *                       kept to 1/256 of a quantisation step) and rounded to
- *                       bf16 once; the default, and the more accurate form.
+ *                       weight in fp32 from the quantiser's exact rounding
+ *                       residual and rounded to bf16 once; the default, and
+ *                       the more accurate form.
  *   AWQ_LOSS_REFERENCE  the reference output X W is computed once per tile by
  *                       the same GEMM (bf16 W) and subtracted from
  *                       X S^-1 Q(S W) (bf16 operands) in the epilogue.
@@ -86,6 +88,11 @@ enum { AWQ_LOSS_ERROR = 0, AWQ_LOSS_REFERENCE = 1 };
  *   stat  AWQ_STAT_MEAN: a_j = (sum_i |X_ij|) / N, summed in fp32 in a fixed
  *         order (bit-reproducible); AWQ_STAT_MAX: a_j = max_i |X_ij| (exact)
  *   a     [D_in] fp32 output
+ * When the rows are split over several CTAs (the usual case: the work is cut
+ * into about one CTA per SM), the per-CTA partial rows go to a scratch of at
+ * most (number of SMs) x 1024 floats (about 0.6 MB on B200) taken with
+ * cudaMallocAsync and released with cudaFreeAsync on `stream` (capturable in
+ * a CUDA graph); a failure of that allocation returns AWQ_ECUDA.
  */
 AWQ_API int awq_act_stats(const void* X, int64_t N, int64_t D_in, int stat, float* a, void* stream);
 

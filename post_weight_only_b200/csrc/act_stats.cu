@@ -5,31 +5,39 @@
 // AWQ notes, "searching the optimal scale" (s_X = average magnitude per
 // channel).
 //
-// HBM-bound column reduction over a row-major bf16 matrix.  One cluster of 8
-// CTAs owns a slab of 64 channels (128 bytes of every row); each warp reads
-// four rows per instruction (8 lanes x 16 bytes per row) and keeps eight such
-// loads in flight.  Every thread accumulates 8 channels in fp32 over its rows;
-// the CTA folds its 32 row-lanes in a fixed order in shared memory, and CTA
-// rank 0 folds the 8 CTA totals of the cluster through distributed shared
-// memory, again in a fixed order.  No atomics and no scratch memory: the result
-// is bit-for-bit reproducible for a given shape.
+// HBM-bound column reduction over a row-major bf16 matrix, in one wave of CTA
+// pairs (clusters of two, one CTA per SM).  The channels are cut into slabs
+// whose width is a multiple of 64 channels, so that every row segment a CTA
+// reads is whole 128-byte lines (segments that straddle lines cost a third
+// more time on B200), as many slabs as there are pairs or fewer; the two CTAs
+// of a pair split the slab's rows.  Inside a CTA a thread owns one 8-channel
+// chunk and one row lane and streams its rows through private slots in shared
+// memory with 16-byte asynchronous copies, sixteen rows in flight, so the data
+// in flight costs no registers and needs no barrier (a thread reads back only
+// its own copies).  The row lanes fold in two fixed-order steps in shared
+// memory and the pair folds its two halves through distributed shared memory,
+// again in a fixed order: no atomics, no scratch in global memory, and the
+// result is bit-for-bit reproducible for a given shape.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include "internal.cuh"
+#include "ptx.cuh"
 
 namespace cg = cooperative_groups;
 
 namespace awq {
 namespace {
 
-constexpr int kCluster = 8;
-constexpr int kThreads = 256;
-constexpr int kSlab = 64;                // channels per cluster
-constexpr int kLanesPerRow = kSlab / 8;  // 16-byte chunks per row slab
-constexpr int kRowLanesCta = kThreads / kLanesPerRow;
-constexpr int kRowLanes = kCluster * kRowLanesCta;
-constexpr int kUnroll = 8;
+constexpr int kThreads = 512;
+constexpr int kCluster = 2;                              // CTAs per slab: the row split
+constexpr int kSlabAlign = 64;                           // channels: one 128-byte line of bf16
+constexpr int kMaxSlabChunks = 2048;                     // 8-channel chunks per slab at most
+constexpr int kRowsPerStage = 4;
+constexpr int kStages = 4;
+constexpr int kDepth = kRowsPerStage * kStages;          // rows in flight per thread
+constexpr int kRingBytes = kDepth * kThreads * 16;       // 128 KiB
+constexpr int kSmemBytes = kRingBytes + kMaxSlabChunks * 8 * 4 /*channel totals*/;
 
 __device__ __forceinline__ void unpack8_abs(const uint4& v, float (&x)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -48,65 +56,136 @@ __device__ __forceinline__ void fold8(float (&acc)[8], const uint4& v) {
   for (int e = 0; e < 8; ++e) acc[e] = kMax ? fmaxf(acc[e], x[e]) : acc[e] + x[e];
 }
 
+// Cluster blockIdx.x / kCluster owns channels [slab * W, min(D, (slab + 1) * W)).
 template <bool kMax>
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads)
-    act_stats_kernel(const uint16_t* __restrict__ X, int64_t N, int64_t D, float* __restrict__ a) {
-  __shared__ float part[kRowLanesCta][kSlab + 1];
-  __shared__ float cta_total[kSlab];
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
+    act_stats_kernel(const uint16_t* __restrict__ X, int64_t N, int64_t D, int64_t slab_ch, float* __restrict__ a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint4* ring = reinterpret_cast<uint4*>(smem);
+  float* fold = reinterpret_cast<float*>(smem);                 // reuses the ring after the stream
+  float* tot = reinterpret_cast<float*>(smem + kRingBytes);     // this CTA's channel totals
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
-  const int chunk = threadIdx.x % kLanesPerRow;
-  const int rl = threadIdx.x / kLanesPerRow;               // row-lane within the CTA
-  const int64_t ch0 = static_cast<int64_t>(blockIdx.y) * kSlab + chunk * 8;
-  const int row_lane = rank * kRowLanesCta + rl;
+  const int t = threadIdx.x;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x / kCluster) * slab_ch;     // first channel of the slab
+  const int64_t c1 = c0 + slab_ch < D ? c0 + slab_ch : D;
+  const int nck = static_cast<int>((c1 - c0) / 8);              // chunks, >= 1
+  const int RL = nck < kThreads ? kThreads / nck : 1;           // row lanes
+  const int lanes = nck * RL;
+  const int64_t r0 = N * rank / kCluster, r1 = N * (rank + 1) / kCluster;
+  const int64_t stride = D / 8;                                 // uint4 per row
 
-  float acc[8];
+  const int rounds = (lanes + kThreads - 1) / kThreads;       // > 1 only with one row lane
+  for (int j = 0; j < rounds; ++j) {
+    const int L = t + j * kThreads;
+    const bool active = L < lanes;
+    const int ck = active ? L % nck : 0, rl = active ? L / nck : 0;
+    float acc[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-
-  if (ch0 < D) {
-    const uint4* base = reinterpret_cast<const uint4*>(X + ch0);
-    const int64_t stride = D / 8;   // uint4 per row
-    int64_t r = row_lane;
-    for (; r + (kUnroll - 1) * kRowLanes < N; r += kUnroll * kRowLanes) {
-      uint4 v[kUnroll];
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+    if (active) {
+      const int64_t first = r0 + rl;
+      const int nr = first < r1 ? static_cast<int>((r1 - first + RL - 1) / RL) : 0;   // rows of this lane
+      const int nst = (nr + kRowsPerStage - 1) / kRowsPerStage;
+      const uint4* src = reinterpret_cast<const uint4*>(X) + c0 / 8 + ck + first * stride;
+      const int64_t step = static_cast<int64_t>(RL) * stride;
+      auto issue = [&](int g) {
+        if (g < nst) {
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) v[u] = __ldcs(base + (r + u * kRowLanes) * stride);
+          for (int q = 0; q < kRowsPerStage; ++q) {
+            const int i = g * kRowsPerStage + q;
+            if (i < nr) cp_async16(ring + (i & (kDepth - 1)) * kThreads + t, src + i * step, 16u);
+          }
+        }
+        cp_async_commit();
+      };
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) fold8<kMax>(acc, v[u]);
+      for (int g = 0; g < kStages - 1; ++g) issue(g);
+      for (int g = 0; g < nst; ++g) {
+        issue(g + kStages - 1);
+        cp_async_wait<kStages - 1>();      // this thread's rows of stage g have landed
+#pragma unroll
+        for (int q = 0; q < kRowsPerStage; ++q) {
+          const int i = g * kRowsPerStage + q;
+          if (i < nr) fold8<kMax>(acc, ring[(i & (kDepth - 1)) * kThreads + t]);
+        }
+      }
+      cp_async_wait<0>();
     }
-    for (; r < N; r += kRowLanes) fold8<kMax>(acc, __ldcs(base + r * stride));
+    if (RL == 1) {
+      // one row lane: a lane's sums are the CTA's totals for its chunk
+      if (active) {
+        float4* d4 = reinterpret_cast<float4*>(tot + ck * 8);
+        d4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        d4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      }
+    } else {
+      // several row lanes (then a single round): fold them in order through
+      // the ring, which every thread has finished streaming through
+      __syncthreads();
+      if (active) {
+        float4* f4 = reinterpret_cast<float4*>(fold + (static_cast<int64_t>(rl) * nck + ck) * 8);
+        f4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        f4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      }
+      __syncthreads();
+      // Step 1: P parts per channel, part p folding row lanes p, p + P, ...
+      // in order; step 2: the P parts in order.
+      const int nch = nck * 8;
+      const int P = nch < kThreads ? kThreads / nch : 1;
+      float* parts = fold + kThreads * 8;                     // after the row-lane sums
+      if (t < P * nch) {
+        const int c = t % nch, pp = t / nch;
+        float sum = fold[pp * nch + c];
+        for (int l = pp + P; l < RL; l += P) sum = kMax ? fmaxf(sum, fold[l * nch + c]) : sum + fold[l * nch + c];
+        parts[pp * nch + c] = sum;
+      }
+      __syncthreads();
+      for (int c = t; c < nch; c += kThreads) {
+        float sum = parts[c];
+        for (int pp = 1; pp < P; ++pp) sum = kMax ? fmaxf(sum, parts[pp * nch + c]) : sum + parts[pp * nch + c];
+        tot[c] = sum;
+      }
+    }
   }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) part[rl][chunk * 8 + e] = acc[e];
-  __syncthreads();
-  if (threadIdx.x < kSlab) {
-    float t = part[0][threadIdx.x];
-#pragma unroll
-    for (int l = 1; l < kRowLanesCta; ++l) t = kMax ? fmaxf(t, part[l][threadIdx.x]) : t + part[l][threadIdx.x];
-    cta_total[threadIdx.x] = t;
-  }
+  // The pair folds in rank order; CTA q writes the channels c with c % 2 == q.
+  const int nch = nck * 8;
   cluster.sync();
-  if (rank == 0 && threadIdx.x < kSlab) {
-    float t = 0.0f;
-    for (int q = 0; q < kCluster; ++q) {
-      const float* remote = cluster.map_shared_rank(cta_total, q);
-      t = kMax ? fmaxf(t, remote[threadIdx.x]) : t + remote[threadIdx.x];
-    }
-    const int64_t j = static_cast<int64_t>(blockIdx.y) * kSlab + threadIdx.x;
-    if (j < D) a[j] = kMax ? t : __fdiv_rn(t, static_cast<float>(N));
+  const float* part0 = cluster.map_shared_rank(tot, 0);
+  const float* part1 = cluster.map_shared_rank(tot, 1);
+  for (int c = rank + kCluster * t; c < nch; c += kCluster * kThreads) {
+    const float sum = kMax ? fmaxf(part0[c], part1[c]) : part0[c] + part1[c];
+    a[c0 + c] = kMax ? sum : __fdiv_rn(sum, static_cast<float>(N));
   }
-  cluster.sync();   // keep every CTA's shared memory alive until rank 0 has read it
+  cluster.sync();   // each CTA's shared memory stays alive until the other has read it
 }
 
 }  // namespace
 
-cudaError_t launch_act_stats(const uint16_t* X, int64_t N, int64_t D, int stat, float* a, cudaStream_t st) {
-  dim3 grid(kCluster, static_cast<unsigned>((D + kSlab - 1) / kSlab));
+cudaError_t launch_act_stats(const uint16_t* X, int64_t N, int64_t D, int stat, float* a, int num_sms,
+                             cudaStream_t st) {
+  static int attr_set_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_set_device != dev) {
+    for (auto fn : {act_stats_kernel<false>, act_stats_kernel<true>}) {
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      if (e != cudaSuccess) return e;
+    }
+    attr_set_device = dev;
+  }
+  // Slab width: D / (pairs that fit) rounded up to whole lines, at most
+  // kMaxSlabChunks chunks.
+  const int64_t pairs = num_sms >= 2 ? num_sms / 2 : 1;
+  int64_t slab = (D + pairs - 1) / pairs;
+  slab = (slab + kSlabAlign - 1) / kSlabAlign * kSlabAlign;
+  if (slab > static_cast<int64_t>(kMaxSlabChunks) * 8) slab = static_cast<int64_t>(kMaxSlabChunks) * 8;
+  const int64_t slabs = (D + slab - 1) / slab;
+  const dim3 grid(static_cast<unsigned>(slabs * kCluster));
   if (stat == 1)
-    act_stats_kernel<true><<<grid, kThreads, 0, st>>>(X, N, D, a);
+    act_stats_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(X, N, D, slab, a);
   else
-    act_stats_kernel<false><<<grid, kThreads, 0, st>>>(X, N, D, a);
+    act_stats_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(X, N, D, slab, a);
   return cudaGetLastError();
 }
 

@@ -290,7 +290,7 @@ int awq_act_stats(const void* X, int64_t N, int64_t D_in, int stat, float* a, vo
   cudaError_t e;
   {
     StageTimer t(AWQ_STAGE_ACT_STATS, static_cast<cudaStream_t>(stream));
-    e = awq::launch_act_stats(static_cast<const uint16_t*>(X), N, D_in, stat, a, static_cast<cudaStream_t>(stream));
+    e = awq::launch_act_stats(static_cast<const uint16_t*>(X), N, D_in, stat, a, sms, static_cast<cudaStream_t>(stream));
   }
   return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "act_stats kernel");
 }
@@ -422,7 +422,7 @@ int awq_quantize_pack(const float* W, const float* s, int64_t D_in, int64_t D_ou
   cudaError_t e;
   {
     StageTimer t(AWQ_STAGE_QUANTIZE_PACK, static_cast<cudaStream_t>(stream));
-    e = awq::launch_quantize_pack(W, s, D_in, D_out, bits, group, packed, scales, static_cast<cudaStream_t>(stream));
+    e = awq::launch_quantize_pack(W, s, D_in, D_out, bits, group, packed, scales, sms, static_cast<cudaStream_t>(stream));
   }
   return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "quantize_pack kernel");
 }

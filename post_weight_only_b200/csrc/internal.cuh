@@ -19,7 +19,10 @@ struct AlphaList {
 };
 
 // ---- act_stats.cu
-cudaError_t launch_act_stats(const uint16_t* X, int64_t N, int64_t D, int stat, float* a, cudaStream_t st);
+// Uses a stream-ordered scratch of at most about num_sms x 1024 floats (from
+// the device's default memory pool) when the rows are split over CTAs.
+cudaError_t launch_act_stats(const uint16_t* X, int64_t N, int64_t D, int stat, float* a, int num_sms,
+                             cudaStream_t st);
 
 // ---- scales.cu
 // s_tab [A][D] (may be null), r_tab [A][D] = fl32(1 / s) (may be null).
@@ -37,7 +40,7 @@ cudaError_t launch_search_operand(const float* W, const float* s_tab, const floa
 cudaError_t launch_weight_t(const float* W, int64_t D_in, int64_t D_out, uint16_t* wt, cudaStream_t st);
 // Final quantise + pack for one given scale vector s (natural nibble order).
 cudaError_t launch_quantize_pack(const float* W, const float* s, int64_t D_in, int64_t D_out, int bits, int group,
-                                 uint32_t* packed, float* scales, cudaStream_t st);
+                                 uint32_t* packed, float* scales, int num_sms, cudaStream_t st);
 
 // ---- reduce.cu
 cudaError_t launch_loss_reduce(const float* partial, int A, int H, int64_t D_out, double* L_col, double* blk,

@@ -200,6 +200,29 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 
 }  // namespace awq
 
+// ---------------------------------------------------------------- cp.async and dependent launches
+namespace awq {
+
+// 16-byte asynchronous copy global -> shared; src_bytes < 16 zero-fills the
+// rest (0: a pure zero fill, the source is not read).
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
+
+// Programmatic dependent launch: the primary lets its dependent grid start
+// early; the dependent waits for the primary's completion (and its memory)
+// before touching the primary's output.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+}  // namespace awq
+
 // ---------------------------------------------------------------- CTA pairs (cluster of 2)
 namespace awq {
 

@@ -52,7 +52,11 @@ _check_alpha = check_alpha
 
 
 # ------------------------------------------------------------------ statistic
-@pytest.mark.parametrize("N,D", [(1, 8), (7, 264), (300, 520), (4096, 4096), (1000, 11008)])
+@pytest.mark.parametrize("N,D", [
+    (1, 8), (7, 264), (300, 520), (4096, 4096), (1000, 11008),
+    (1, 4096),                                    # one row: the second CTA of each pair has none
+    (3, 262144), (2, 524288), (1, 1048576),       # one row lane per chunk; one, two, four rounds
+])
 def test_act_stats(awq, N, D):
     X, _ = _layer(N, D, 8, seed=N)
     Xd = X.cuda()
@@ -101,6 +105,22 @@ def test_quantize_pack_bit_exact(awq, bits, group, D_in, D_out):
     q_or, d_or = oracle.quantize(W, s, bits, group)
     p_or = oracle.pack(q_or, bits)
     assert np.array_equal(packed.cpu().numpy().view(np.uint32), p_or)
+    assert np.array_equal(sc.cpu().numpy(), d_or)
+
+
+@pytest.mark.parametrize("bits,group,D_in,D_out", [
+    (4, 128, 256, 203),    # D_out % 4 != 0: the untiled kernel
+    (4, 128, 128, 1),      # one column (untiled)
+    (4, 32, 96, 200),      # the last 128-row tile reaches past D_in
+    (3, 64, 192, 132),     # same, two groups per tile
+    (4, 64, 320, 4100),    # ragged last column tile
+])
+def test_quantize_pack_ragged(awq, bits, group, D_in, D_out):
+    X, W = _layer(16, D_in, D_out, seed=D_in + D_out)
+    s = oracle.scales(_oracle_a(X), 0.4)
+    packed, sc = awq.quantize_pack(W.cuda(), torch.from_numpy(s).cuda(), bits, group)
+    q_or, d_or = oracle.quantize(W, s, bits, group)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), oracle.pack(q_or, bits))
     assert np.array_equal(sc.cpu().numpy(), d_or)
 
 
