@@ -53,6 +53,10 @@ def _load():
         lib.oracle_scales.restype = None
         lib.oracle_quantize.argtypes = [P, P, I64, I64, I, I, P, P]
         lib.oracle_quantize.restype = None
+        lib.oracle_quantize_clip.argtypes = [P, P, P, I64, I64, I, I, P, P]
+        lib.oracle_quantize_clip.restype = None
+        lib.oracle_clip_loss.argtypes = [P, P, P, I64, I64, I64, P, I, I, I, P, I64, P, P]
+        lib.oracle_clip_loss.restype = None
         lib.oracle_pack.argtypes = [P, I64, I64, I, P]
         lib.oracle_pack.restype = None
         lib.oracle_loss_cols.argtypes = [P, P, P, I64, I64, I64, I, I, I, P, I64, P]
@@ -110,16 +114,46 @@ def scales(a, alpha: float) -> np.ndarray:
     return s
 
 
-def quantize(W, s, bits: int, group: int) -> Tuple[np.ndarray, np.ndarray]:
+def quantize(W, s, bits: int, group: int, clip=None) -> Tuple[np.ndarray, np.ndarray]:
     """Codes q [D_in, D_out] (int8) and deltas [D_in/group, D_out] (fp32) of
-    diag(s).W.  compassingai.com concept page, "quantisation math"."""
+    diag(s).W.  compassingai.com concept page, "quantisation math".  clip:
+    optional [D_in/group, D_out] fp32 clip ratios (the group maximum is
+    replaced by fl32(clip * max) before delta is formed)."""
     W = _f32(W)
     D_in, D_out = W.shape
     s = None if s is None else _f32(s)
     q = np.empty((D_in, D_out), dtype=np.int8)
     d = np.empty((D_in // group, D_out), dtype=np.float32)
-    _load().oracle_quantize(_ptr(W), _ptr(s), D_in, D_out, bits, group, _ptr(q), _ptr(d))
+    if clip is None:
+        _load().oracle_quantize(_ptr(W), _ptr(s), D_in, D_out, bits, group, _ptr(q), _ptr(d))
+    else:
+        c = _f32(clip)
+        assert c.shape == (D_in // group, D_out)
+        _load().oracle_quantize_clip(_ptr(W), _ptr(s), _ptr(c), D_in, D_out, bits, group, _ptr(q), _ptr(d))
     return q, d
+
+
+def clip_search(X, W, s, clip_grid, bits: int, group: int, cols: Optional[Sequence[int]] = None,
+                want_loss: bool = False):
+    """Weight-clipping search (mudrobot.github.io notes, "searching the optimal
+    scale": weight clipping to minimise the quantisation MSE): for every clip
+    ratio of the grid, group and column, the fp64 squared error of that group's
+    share of the layer output.  Returns (best [D_in/group, nc] int32 grid
+    indices, loss [n_clip, D_in/group, nc] fp64 or None)."""
+    Xb = _as_bf16_bits(X)
+    W = _f32(W)
+    s = None if s is None else _f32(s)
+    grid = _f32(clip_grid)
+    N, D_in = Xb.shape
+    D_out = W.shape[1]
+    c = None if cols is None else np.ascontiguousarray(cols, dtype=np.int64)
+    nc = D_out if c is None else c.shape[0]
+    G = D_in // group
+    best = np.empty((G, nc), dtype=np.int32)
+    loss = np.empty((grid.shape[0], G, nc), dtype=np.float64) if want_loss else None
+    _load().oracle_clip_loss(_ptr(Xb), _ptr(W), _ptr(s), N, D_in, D_out, _ptr(grid), grid.shape[0], bits, group,
+                             _ptr(c), 0 if c is None else nc, _ptr(loss), _ptr(best))
+    return best, loss
 
 
 def pack(q: np.ndarray, bits: int) -> np.ndarray:

@@ -101,9 +101,13 @@ void oracle_scales(const float *a, int64_t D, float alpha, float *s)
  *   w'_k  = fl32(s_k * w_k)
  *   delta = fl32(max_k |w'_k| / (2^(b-1) - 1))
  *   q_k   = clamp(round(fl32(w'_k / delta)), -(2^(b-1)-1), 2^(b-1)-1)
- * s == NULL means s_k = 1 (no scaling). */
+ * s == NULL means s_k = 1 (no scaling).  clip is the weight-clipping ratio
+ * ([P2] "searching the optimal scale": weight clipping to minimise the
+ * quantisation MSE): the group maximum m is replaced by fl32(clip * m) before
+ * delta is formed, and the clamp then bounds the codes of the clipped weights.
+ * clip = 1 leaves m unchanged (fl32(1 * m) = m). */
 static void quantize_group(const float *W, const float *s, int64_t D_out, int64_t n,
-                           int64_t k0, int group, int bits, int8_t *q, float *delta)
+                           int64_t k0, int group, int bits, float clip, int8_t *q, float *delta)
 {
     const int qmax = (1 << (bits - 1)) - 1;
     float m = 0.0f;
@@ -114,6 +118,7 @@ static void quantize_group(const float *W, const float *s, int64_t D_out, int64_
         if (am > m)
             m = am;
     }
+    m = clip * m;
     const float d = m / (float)qmax;
     *delta = d;
     for (int k = 0; k < group; ++k) {
@@ -134,19 +139,27 @@ static void quantize_group(const float *W, const float *s, int64_t D_out, int64_
 }
 
 /* Quantise every (group, column) of diag(s) W.  q: [D_in][D_out] codes in
- * [-qmax, qmax]; delta: [D_in/group][D_out]. */
-void oracle_quantize(const float *W, const float *s, int64_t D_in, int64_t D_out,
-                     int bits, int group, int8_t *q, float *delta)
+ * [-qmax, qmax]; delta: [D_in/group][D_out].  clip: [D_in/group][D_out] clip
+ * ratios, or NULL for none. */
+void oracle_quantize_clip(const float *W, const float *s, const float *clip, int64_t D_in, int64_t D_out,
+                          int bits, int group, int8_t *q, float *delta)
 {
     int8_t *col = (int8_t *)malloc((size_t)group);
     for (int64_t n = 0; n < D_out; ++n) {
         for (int64_t g = 0; g < D_in / group; ++g) {
-            quantize_group(W, s, D_out, n, g * group, group, bits, col, &delta[g * D_out + n]);
+            quantize_group(W, s, D_out, n, g * group, group, bits, clip ? clip[g * D_out + n] : 1.0f, col,
+                           &delta[g * D_out + n]);
             for (int k = 0; k < group; ++k)
                 q[(g * group + k) * D_out + n] = col[k];
         }
     }
     free(col);
+}
+
+void oracle_quantize(const float *W, const float *s, int64_t D_in, int64_t D_out,
+                     int bits, int group, int8_t *q, float *delta)
+{
+    oracle_quantize_clip(W, s, NULL, D_in, D_out, bits, group, q, delta);
 }
 
 /* Pack codes: word (k8, n) holds rows 8*k8 .. 8*k8+7 of column n, row 8*k8+i in
@@ -181,7 +194,7 @@ static double column_loss(const double *Xd, const float *W, const float *s,
         const int64_t k0 = g * group;
         if (quantize) {
             float d;
-            quantize_group(W, s, D_out, n, k0, group, bits, qcol, &d);
+            quantize_group(W, s, D_out, n, k0, group, bits, 1.0f, qcol, &d);
             for (int k = 0; k < group; ++k) {
                 double sk = s ? (double)s[k0 + k] : 1.0;
                 e[k0 + k] = (double)qcol[k] * (double)d / sk - (double)W[(k0 + k) * D_out + n];
@@ -320,4 +333,62 @@ int oracle_num_threads(void)
 #else
     return 1;
 #endif
+}
+
+/* Weight clipping search ([P2] "searching the optimal scale": after the scale
+ * search, weight clipping is applied to minimise the quantisation MSE).
+ * Reading: per (group, column) and per clip ratio c_i of a given grid, the
+ * mean squared error of that group's share of the layer output,
+ *   loss[i][g][n] = sum_t ( sum_{k in g} x_tk e_k )^2,
+ *   e_k = q_k * delta / s_k - w_kn,   q, delta from quantize_group(clip = c_i),
+ * in fp64; best[g][n] = argmin_i loss[i][g][n], the lowest index on exact
+ * ties.  cols == NULL means every column (else column cols[c] in slot c);
+ * loss may be NULL. */
+void oracle_clip_loss(const uint16_t *X, const float *W, const float *s, int64_t N, int64_t D_in, int64_t D_out,
+                      const float *clip, int n_clip, int bits, int group, const int64_t *cols, int64_t ncols,
+                      double *loss, int32_t *best)
+{
+    double *Xd = x_to_double(X, N, D_in);
+    const int64_t nc = cols ? ncols : D_out;
+    const int64_t G = D_in / group;
+#pragma omp parallel
+    {
+        double *e = (double *)malloc((size_t)group * sizeof(double));
+        int8_t *qg = (int8_t *)malloc((size_t)group);
+#pragma omp for schedule(dynamic, 1) collapse(2)
+        for (int64_t c = 0; c < nc; ++c) {
+            for (int64_t g = 0; g < G; ++g) {
+                const int64_t n = cols ? cols[c] : c;
+                const int64_t k0 = g * group;
+                double lbest = 0.0;
+                int ibest = 0;
+                for (int i = 0; i < n_clip; ++i) {
+                    float d;
+                    quantize_group(W, s, D_out, n, k0, group, bits, clip[i], qg, &d);
+                    for (int k = 0; k < group; ++k) {
+                        double sk = s ? (double)s[k0 + k] : 1.0;
+                        e[k] = (double)qg[k] * (double)d / sk - (double)W[(k0 + k) * D_out + n];
+                    }
+                    double acc = 0.0;
+                    for (int64_t t = 0; t < N; ++t) {
+                        const double *xr = Xd + t * D_in + k0;
+                        double y = 0.0;
+                        for (int k = 0; k < group; ++k)
+                            y += xr[k] * e[k];
+                        acc += y * y;
+                    }
+                    if (loss)
+                        loss[((int64_t)i * G + g) * nc + c] = acc;
+                    if (i == 0 || acc < lbest) {
+                        lbest = acc;
+                        ibest = i;
+                    }
+                }
+                best[g * nc + c] = ibest;
+            }
+        }
+        free(e);
+        free(qg);
+    }
+    free(Xd);
 }

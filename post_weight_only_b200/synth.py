@@ -22,7 +22,7 @@ from typing import List, Optional, Tuple
 import torch
 
 __all__ = [
-    "LayerSpec", "Workload", "WORKLOADS", "alpha_grid", "make_x", "make_w",
+    "LayerSpec", "Workload", "WORKLOADS", "alpha_grid", "clip_grid", "make_x", "make_w",
     "layer_inputs", "workload",
 ]
 
@@ -37,6 +37,14 @@ def alpha_grid(n_intervals: int) -> torch.Tensor:
     """
     k = torch.arange(n_intervals + 1, dtype=torch.float64)
     return (k / n_intervals).to(torch.float32)
+
+
+def clip_grid(n_intervals: int = 20, lo: float = 0.5) -> torch.Tensor:
+    """Weight-clipping ratios from 1 (no clipping, index 0) down to `lo` in
+    n_intervals equal steps: c_i = 1 - (1 - lo) i / n_intervals, formed in fp64
+    and rounded once to fp32."""
+    i = torch.arange(n_intervals + 1, dtype=torch.float64)
+    return (1.0 - (1.0 - lo) * i / n_intervals).to(torch.float32)
 
 
 @dataclass(frozen=True)
