@@ -191,6 +191,42 @@ AWQ_API int awq_quantize_pack(const float* W, const float* s, int64_t D_in, int6
                       uint32_t* packed, float* scales, void* stream);
 
 /*
+ * Weight-clipping search, the step after the scale search (mudrobot.github.io
+ * AWQ notes, "searching the optimal scale": weight clipping is applied to
+ * minimise the quantisation MSE).  For every group g of `group` rows, output
+ * column n and clip ratio c = clip_grid[i], the group maximum of
+ * W' = diag(s) W is replaced by fl32(c * max) before delta = max / qmax is
+ * formed, codes are clamped to +-qmax, and the objective is the squared error
+ * of the group's share of the layer output,
+ *     L_i(g, n) = || X_g (S^-1 Q_c(S W) - W)_{g,n} ||^2 = e^T (X_g^T X_g) e,
+ * evaluated on the tensor cores in the Gram form (bf16 X_g^T X_g blocks, bf16
+ * operand, fp32 accumulation).  The chosen ratio is the argmin over i, the
+ * lowest index on ties (put c = 1, no clipping, first).
+ *   X          [N][D_in] bf16;  W [D_in][D_out] fp32;  s [D_in] fp32 (e.g. s*)
+ *   clip_grid  HOST array of n_clip fp32 ratios in (0, 1], 1 <= n_clip <= 64
+ *   bits       2, 3 or 4;  group 64 or 128;  D_in % group == 0, D_out % 4 == 0
+ *   clip       [D_in/group][D_out] fp32 output: the chosen ratio
+ *   clip_idx   [D_in/group][D_out] int32 output: its grid index (may be NULL)
+ *   loss       [n_clip][D_in/group][D_out] fp32 output: every L_i (may be NULL)
+ *   workspace  at least awq_clip_search_workspace_size(...) bytes, 256-byte aligned
+ *   status     as for awq_search (may be NULL)
+ */
+AWQ_API size_t awq_clip_search_workspace_size(int64_t N, int64_t D_in, int64_t D_out, int n_clip, int bits,
+                                              int group);
+AWQ_API int awq_clip_search(const void* X, const float* W, const float* s, int64_t N, int64_t D_in, int64_t D_out,
+                            const float* clip_grid, int n_clip, int bits, int group, float* clip, int32_t* clip_idx,
+                            float* loss, void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
+
+/*
+ * awq_quantize_pack with a clip ratio per (group, column) (the output of
+ * awq_clip_search): the group maximum of diag(s) W is replaced by
+ * fl32(clip * max) before delta is formed and codes are clamped to +-qmax;
+ * otherwise as awq_quantize_pack.  clip: [D_in/group][D_out] fp32 (device).
+ */
+AWQ_API int awq_quantize_pack_clip(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out,
+                                   int bits, int group, uint32_t* packed, float* scales, void* stream);
+
+/*
  * The layer's reference output Y = X bf16(W) computed by the search's own
  * tensor-core GEMM (the X W term of the loss, concept page flow step 4c), fp32.
  *   Y          [N][D_out] fp32 output
@@ -250,7 +286,10 @@ enum {
   AWQ_STAGE_LOSS_REDUCE = 4,   /* L(alpha), argmin */
   AWQ_STAGE_QUANTIZE_PACK = 5, /* awq_quantize_pack */
   AWQ_STAGE_WEIGHT_T = 6,      /* bf16 W^T: reference pass of the search, awq_layer_output */
-  AWQ_NUM_STAGES = 7
+  AWQ_STAGE_CLIP_GRAM = 7,     /* awq_clip_search: X^T and the group Gram blocks X_g^T X_g */
+  AWQ_STAGE_CLIP_OPERAND = 8,  /* awq_clip_search: bf16 operand per clip ratio */
+  AWQ_STAGE_CLIP_LOSS = 9,     /* awq_clip_search: e^T H_g e per (ratio, group, column), argmin */
+  AWQ_NUM_STAGES = 10
 };
 AWQ_API int awq_profile_enable(int on);
 AWQ_API int awq_profile_reset(void);

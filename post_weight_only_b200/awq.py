@@ -28,10 +28,10 @@ EXPORTS = (
     "awq_search_batched_workspace_size", "awq_search_batched", "awq_quantize_pack",
     "awq_layer_output_workspace_size", "awq_layer_output", "awq_selftest_wait_timeout",
     "awq_get_last_error", "awq_version", "awq_profile_enable", "awq_profile_reset", "awq_profile_read",
-    "awq_search_noalloc",
+    "awq_search_noalloc", "awq_clip_search_workspace_size", "awq_clip_search", "awq_quantize_pack_clip",
 )
 STAGES = ("act_stats", "scale_table", "search_operand", "search_gemm", "loss_reduce", "quantize_pack",
-          "weight_t")
+          "weight_t", "clip_gram", "clip_operand", "clip_loss")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -75,6 +75,9 @@ _prof_enable = _sig("awq_profile_enable", I, [I])
 _prof_reset = _sig("awq_profile_reset", I, [])
 _prof_read = _sig("awq_profile_read", I, [I, P, P])
 _version = _sig("awq_version", I, [])
+_clip_ws = _sig("awq_clip_search_workspace_size", SZ, [I64, I64, I64, I, I, I])
+_clip = _sig("awq_clip_search", I, [P, P, P, I64, I64, I64, P, I, I, I, P, P, P, P, SZ, P, P])
+_pack_clip = _sig("awq_quantize_pack_clip", I, [P, P, P, I64, I64, I, I, P, P, P])
 
 
 class AwqError(RuntimeError):
@@ -188,6 +191,57 @@ def search(X: torch.Tensor, W: torch.Tensor, a: torch.Tensor, alpha_grid: Sequen
     if check_status:
         check_device_status(status)
     return res
+
+
+@dataclass
+class ClipResult:
+    clip: torch.Tensor                  # [D_in/group, D_out] fp32 chosen ratio
+    idx: torch.Tensor                   # [D_in/group, D_out] int32 grid index
+    loss: Optional[torch.Tensor]        # [n_clip, D_in/group, D_out] fp32, if asked for
+    status: torch.Tensor
+
+
+def clip_search(X: torch.Tensor, W: torch.Tensor, s: torch.Tensor, clip_grid: Sequence[float], bits: int = 4,
+                group: int = 128, want_loss: bool = False, workspace: Optional[Workspace] = None,
+                check_status: bool = True) -> ClipResult:
+    """Weight-clipping search after the scale search: ``awq_clip_search``."""
+    X = _dev(X, torch.bfloat16, "X")
+    W = _dev(W, torch.float32, "W")
+    s = _dev(s, torch.float32, "s")
+    N, D_in = X.shape
+    D_out = W.shape[1]
+    C = len(clip_grid)
+    grid = (ctypes.c_float * C)(*[float(v) for v in clip_grid])
+    dev = X.device
+    G = D_in // group
+    clip = torch.empty(G, D_out, dtype=torch.float32, device=dev)
+    idx = torch.empty(G, D_out, dtype=torch.int32, device=dev)
+    loss = torch.empty(C, G, D_out, dtype=torch.float32, device=dev) if want_loss else None
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    nbytes = int(_clip_ws(N, D_in, D_out, C, bits, group))
+    if nbytes == 0:
+        raise AwqError(AWQ_EINVAL, _last_error().decode(errors="replace"))
+    ws = (workspace or _default_ws).get(nbytes, dev)
+    _check(_clip(_ptr(X), _ptr(W), _ptr(s), N, D_in, D_out, grid, C, bits, group, _ptr(clip), _ptr(idx), _ptr(loss),
+                 _ptr(ws), ws.numel(), _ptr(status), _stream()))
+    res = ClipResult(clip, idx, loss, status)
+    if check_status:
+        check_device_status(status)
+    return res
+
+
+def quantize_pack_clip(W: torch.Tensor, s: torch.Tensor, clip: torch.Tensor, bits: int = 4, group: int = 128):
+    """``awq_quantize_pack_clip``: the final pack with a clip ratio per
+    (group, column).  Returns (packed int32 view [D_in/8, D_out], scales fp32
+    [D_in/group, D_out])."""
+    W = _dev(W, torch.float32, "W")
+    s = _dev(s, torch.float32, "s")
+    clip = _dev(clip, torch.float32, "clip")
+    D_in, D_out = W.shape
+    packed = torch.empty(D_in // 8, D_out, dtype=torch.int32, device=W.device)
+    sc = torch.empty(D_in // group, D_out, dtype=torch.float32, device=W.device)
+    _check(_pack_clip(_ptr(W), _ptr(s), _ptr(clip), D_in, D_out, bits, group, _ptr(packed), _ptr(sc), _stream()))
+    return packed, sc
 
 
 def check_device_status(status: torch.Tensor) -> None:

@@ -422,9 +422,44 @@ int awq_quantize_pack(const float* W, const float* s, int64_t D_in, int64_t D_ou
   cudaError_t e;
   {
     StageTimer t(AWQ_STAGE_QUANTIZE_PACK, static_cast<cudaStream_t>(stream));
-    e = awq::launch_quantize_pack(W, s, D_in, D_out, bits, group, packed, scales, sms, static_cast<cudaStream_t>(stream));
+    e = awq::launch_quantize_pack(W, s, nullptr, D_in, D_out, bits, group, packed, scales, sms,
+                                   static_cast<cudaStream_t>(stream));
   }
   return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "quantize_pack kernel");
+}
+
+// ---------------------------------------------------------------- weight-clipping search
+struct ClipLayout {
+  size_t xt, hb, r, op, status, total;
+  int64_t Np;
+};
+
+static ClipLayout clip_layout(int64_t N, int64_t D_in, int64_t D_out, int n_clip, int group) {
+  ClipLayout L{};
+  L.Np = (N + 7) / 8 * 8;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += round_up(bytes, 256);
+    return o;
+  };
+  L.xt = take(static_cast<size_t>(D_in) * L.Np * 2);
+  L.hb = take(static_cast<size_t>(D_in) * group * 2);
+  L.r = take(static_cast<size_t>(D_in) * 4);
+  L.op = take(static_cast<size_t>(n_clip) * D_out * D_in * 2);
+  L.status = take(4);
+  L.total = off;
+  return L;
+}
+
+static int check_clip_args(int64_t N, int64_t D_in, int64_t D_out, int n_clip, int bits, int group) {
+  AWQ_TRY(check_layer_shape(N, D_in, D_out));
+  if (bits < 2 || bits > 4) return fail(AWQ_EUNSUPPORTED, "bits = %d: supported bit widths are 2, 3 and 4", bits);
+  if (group != 64 && group != 128)
+    return fail(AWQ_EUNSUPPORTED, "group = %d: the clipping search supports groups of 64 and 128", group);
+  if (D_in % group) return fail(AWQ_EINVAL, "D_in = %lld is not a multiple of group = %d", (long long)D_in, group);
+  if (n_clip < 1 || n_clip > AWQ_MAX_ALPHA) return fail(AWQ_EUNSUPPORTED, "n_clip = %d: need 1..%d", n_clip, AWQ_MAX_ALPHA);
+  return AWQ_OK;
 }
 
 size_t awq_layer_output_workspace_size(int64_t N, int64_t D_in, int64_t D_out) {
@@ -536,6 +571,91 @@ int awq_selftest_wait_timeout(int32_t* status, int64_t timeout_ns_arg, void* str
   if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(status)");
   e = awq::launch_wait_timeout_selftest(status, static_cast<uint64_t>(timeout_ns_arg), st);
   return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "self-test kernel");
+}
+
+
+size_t awq_clip_search_workspace_size(int64_t N, int64_t D_in, int64_t D_out, int n_clip, int bits, int group) {
+  if (check_clip_args(N, D_in, D_out, n_clip, bits, group) != AWQ_OK) return 0;
+  return clip_layout(N, D_in, D_out, n_clip, group).total;
+}
+
+int awq_clip_search(const void* X, const float* W, const float* s, int64_t N, int64_t D_in, int64_t D_out,
+                    const float* clip_grid, int n_clip, int bits, int group, float* clip, int32_t* clip_idx,
+                    float* loss, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  AWQ_TRY(check_clip_args(N, D_in, D_out, n_clip, bits, group));
+  if (!clip_grid) return fail(AWQ_EINVAL, "clip_grid is NULL");
+  for (int i = 0; i < n_clip; ++i)
+    if (!(clip_grid[i] > 0.0f && clip_grid[i] <= 1.0f))
+      return fail(AWQ_EINVAL, "clip_grid[%d] = %g: ratios must lie in (0, 1]", i, (double)clip_grid[i]);
+  AWQ_TRY(check_ptr(X, "X", 16));
+  AWQ_TRY(check_ptr(W, "W", 16));
+  AWQ_TRY(check_ptr(s, "s", 16));
+  AWQ_TRY(check_ptr(clip, "clip", 4));
+  if (clip_idx) AWQ_TRY(check_ptr(clip_idx, "clip_idx", 4));
+  if (loss) AWQ_TRY(check_ptr(loss, "loss", 4));
+  int sms = 0;
+  AWQ_TRY(device_info(&sms));
+  const ClipLayout lay = clip_layout(N, D_in, D_out, n_clip, group);
+  if (!workspace) return fail(AWQ_EWORKSPACE, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(AWQ_EALIGN, "workspace is not 256-byte aligned");
+  if (workspace_bytes < lay.total)
+    return fail(AWQ_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, lay.total);
+  if (status && !aligned(status, 4)) return fail(AWQ_EALIGN, "status is not 4-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* st_word = status ? status : reinterpret_cast<int32_t*>(ws + lay.status);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(st_word, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(status)");
+  uint16_t* xt = reinterpret_cast<uint16_t*>(ws + lay.xt);
+  uint16_t* hb = reinterpret_cast<uint16_t*>(ws + lay.hb);
+  float* r = reinterpret_cast<float*>(ws + lay.r);
+  uint16_t* op = reinterpret_cast<uint16_t*>(ws + lay.op);
+  awq::AlphaList clips{};
+  for (int i = 0; i < n_clip; ++i) clips.v[i] = clip_grid[i];
+  const char* what = "clipping search";
+  int rc = AWQ_OK;
+  {
+    StageTimer t(AWQ_STAGE_CLIP_GRAM, st);
+    e = awq::launch_xt(static_cast<const uint16_t*>(X), N, D_in, lay.Np, xt, st);
+    if (e == cudaSuccess) e = awq::launch_recip(s, D_in, r, st);
+    if (e == cudaSuccess) rc = awq::launch_gram(xt, D_in, lay.Np, group, hb, st_word, timeout_ns(), st, &e, &what);
+  }
+  if (e != cudaSuccess) return fail_cuda(e, what);
+  if (rc != AWQ_OK) return fail(rc, "%s failed", what);
+  {
+    StageTimer t(AWQ_STAGE_CLIP_OPERAND, st);
+    e = awq::launch_clip_operand(W, s, r, D_in, D_out, clips, n_clip, bits, group, op, st);
+  }
+  if (e != cudaSuccess) return fail_cuda(e, "clipping operand kernel");
+  {
+    StageTimer t(AWQ_STAGE_CLIP_LOSS, st);
+    rc = awq::launch_clip_loss(op, hb, D_in, D_out, group, clips, n_clip, clip, clip_idx, loss, sms, st_word,
+                               timeout_ns(), st, &e, &what);
+  }
+  if (rc != AWQ_OK) return e != cudaSuccess ? fail_cuda(e, what) : fail(rc, "%s failed", what);
+  return AWQ_OK;
+}
+
+int awq_quantize_pack_clip(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out, int bits,
+                           int group, uint32_t* packed, float* scales, void* stream) {
+  AWQ_TRY(check_quant_args(bits, group));
+  if (D_in < group || D_in > kMaxDin || D_in % group)
+    return fail(AWQ_EINVAL, "D_in = %lld: need a positive multiple of group = %d", (long long)D_in, group);
+  if (D_out < 1 || D_out > kMaxDim) return fail(AWQ_EINVAL, "D_out = %lld out of range", (long long)D_out);
+  AWQ_TRY(check_ptr(W, "W", 16));
+  AWQ_TRY(check_ptr(s, "s", 16));
+  AWQ_TRY(check_ptr(clip, "clip", 4));
+  AWQ_TRY(check_ptr(packed, "packed", 16));
+  AWQ_TRY(check_ptr(scales, "scales", 16));
+  int sms = 0;
+  AWQ_TRY(device_info(&sms));
+  cudaError_t e;
+  {
+    StageTimer t(AWQ_STAGE_QUANTIZE_PACK, static_cast<cudaStream_t>(stream));
+    e = awq::launch_quantize_pack(W, s, clip, D_in, D_out, bits, group, packed, scales, sms,
+                                  static_cast<cudaStream_t>(stream));
+  }
+  return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "quantize_pack kernel (clipped)");
 }
 
 }  // extern "C"

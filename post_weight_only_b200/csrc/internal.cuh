@@ -36,11 +36,18 @@ cudaError_t launch_scale_table(const float* a, int64_t D, const AlphaList& alpha
 cudaError_t launch_search_operand(const float* W, const float* s_tab, const float* r_tab, int64_t D_in,
                                   int64_t D_out, int A, int bits, int group, int form, uint16_t* op,
                                   cudaStream_t st);
+// The clipping search's operand for every clip ratio c of `clips`, bf16
+// [n_clip][D_out][D_in]: (S^-1 Q_c(S W) - W)^T with the group maximum scaled
+// by c and codes clamped; s and r = 1/s are single rows [D_in].
+cudaError_t launch_clip_operand(const float* W, const float* s, const float* r, int64_t D_in, int64_t D_out,
+                                const AlphaList& clips, int n_clip, int bits, int group, uint16_t* op,
+                                cudaStream_t st);
 // bf16 W^T [D_out][D_in] for the reference output X W.
 cudaError_t launch_weight_t(const float* W, int64_t D_in, int64_t D_out, uint16_t* wt, cudaStream_t st);
-// Final quantise + pack for one given scale vector s (natural nibble order).
-cudaError_t launch_quantize_pack(const float* W, const float* s, int64_t D_in, int64_t D_out, int bits, int group,
-                                 uint32_t* packed, float* scales, int num_sms, cudaStream_t st);
+// Final quantise + pack for one given scale vector s (natural nibble order);
+// clip [D_in/group][D_out] (may be null) scales each group maximum.
+cudaError_t launch_quantize_pack(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out,
+                                 int bits, int group, uint32_t* packed, float* scales, int num_sms, cudaStream_t st);
 
 // ---- reduce.cu
 cudaError_t launch_loss_reduce(const float* partial, int A, int H, int64_t D_out, double* L_col, double* blk,
@@ -68,6 +75,26 @@ int search_partial_rows(int N);
 // Returns 0 on success, otherwise an awq error code; *cerr gets the CUDA error.
 int launch_search(const SearchShape& sh, const SearchBuffers& b, int grid, uint64_t timeout_ns, cudaStream_t st,
                   cudaError_t* cerr, const char** what);
+
+// bf16 TMA map (128-byte swizzle) over rows of `inner` contiguous elements,
+// `rows` rows, `planes` planes (0: a 2-D map); box box_inner x box_rows.
+bool make_bf16_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t planes,
+                   uint32_t box_inner, uint32_t box_rows);
+
+// ---- clip.cu (the weight-clipping search)
+// XT [D][Np] = X^T, tokens padded with zeros to Np (a multiple of 8).
+cudaError_t launch_xt(const uint16_t* X, int64_t N, int64_t D, int64_t Np, uint16_t* XT, cudaStream_t st);
+// r = 1 / s (IEEE).
+cudaError_t launch_recip(const float* s, int64_t D, float* r, cudaStream_t st);
+// Hb [D_in/group][group][group] bf16: the diagonal Gram blocks X_g^T X_g.
+int launch_gram(const uint16_t* XT, int64_t D_in, int64_t Np, int group, uint16_t* Hb, int* status,
+                uint64_t timeout_ns, cudaStream_t st, cudaError_t* cerr, const char** what);
+// Per (group, column): the clip ratio of `clips` with the smallest e^T H_g e
+// (lowest index on ties) -> clip_out [groups][D_out]; idx_out, loss_out
+// [n_clip][groups][D_out] may be null.
+int launch_clip_loss(const uint16_t* op, const uint16_t* Hb, int64_t D_in, int64_t D_out, int group,
+                     const AlphaList& clips, int n_clip, float* clip_out, int* idx_out, float* loss_out, int num_sms,
+                     int* status, uint64_t timeout_ns, cudaStream_t st, cudaError_t* cerr, const char** what);
 
 // Self-test of the bounded wait: one CTA waits on an mbarrier that nothing
 // arrives at, gives up after timeout_ns and records the timeout in *status.

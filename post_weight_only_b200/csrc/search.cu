@@ -460,23 +460,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// A bf16 K-major map: rows of `inner` elements (contiguous), `rows` rows,
-// optionally `planes` planes of rows x inner; box = 64 x 128 (x 1), 128-byte
-// swizzle.
-bool make_kmajor_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t planes) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const uint64_t dims[3] = {inner, rows, planes};
-  const uint64_t str[2] = {inner * 2, inner * 2 * rows};
-  const uint32_t box[3] = {kBK, kBM, 1};
-  const uint32_t estr[3] = {1, 1, 1};
-  const cuuint32_t rank = planes > 0 ? 3 : 2;
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, str, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int kForm>
 cudaError_t launch_form(int grid, const CUtensorMap& mX, const CUtensorMap& mWt, const CUtensorMap& mOp,
                         const Params& p, cudaStream_t st) {
@@ -494,6 +477,24 @@ cudaError_t launch_form(int grid, const CUtensorMap& mX, const CUtensorMap& mWt,
 }
 
 }  // namespace
+
+// A bf16 map: rows of `inner` elements (contiguous), `rows` rows, optionally
+// `planes` planes of rows x inner; box box_inner x box_rows (x 1), 128-byte
+// swizzle (box_inner = 64: one swizzle row).
+bool make_bf16_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t planes,
+                   uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t dims[3] = {inner, rows, planes};
+  const uint64_t str[2] = {inner * 2, inner * 2 * rows};
+  const uint32_t box[3] = {box_inner, box_rows, 1};
+  const uint32_t estr[3] = {1, 1, 1};
+  const cuuint32_t rank = planes > 0 ? 3 : 2;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, str, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 int search_token_tiles(int N) { return (N + kBN - 1) / kBN; }
 
@@ -514,12 +515,12 @@ int launch_search(const SearchShape& sh, const SearchBuffers& b, int grid, uint6
   const bool gemm_only = sh.A == 0;
   const int form = gemm_only ? kFormReference : sh.form;
   CUtensorMap mX, mWt, mOp;
-  if (!make_kmajor_map(&mX, b.X, static_cast<uint64_t>(sh.D_in), static_cast<uint64_t>(sh.N), 0)) {
+  if (!make_bf16_map(&mX, b.X, static_cast<uint64_t>(sh.D_in), static_cast<uint64_t>(sh.N), 0, kBK, kBM)) {
     *what = "tensor map for X";
     return kECuda;
   }
   if (form == kFormReference) {
-    if (!make_kmajor_map(&mWt, b.wt, static_cast<uint64_t>(sh.D_in), static_cast<uint64_t>(sh.D_out), 0)) {
+    if (!make_bf16_map(&mWt, b.wt, static_cast<uint64_t>(sh.D_in), static_cast<uint64_t>(sh.D_out), 0, kBK, kBM)) {
       *what = "tensor map for the bf16 weights";
       return kECuda;
     }
@@ -527,8 +528,8 @@ int launch_search(const SearchShape& sh, const SearchBuffers& b, int grid, uint6
     mWt = mX;   // never read by the error form
   }
   if (!gemm_only) {
-    if (!make_kmajor_map(&mOp, b.op, static_cast<uint64_t>(sh.D_in), static_cast<uint64_t>(sh.D_out),
-                         static_cast<uint64_t>(sh.A))) {
+    if (!make_bf16_map(&mOp, b.op, static_cast<uint64_t>(sh.D_in), static_cast<uint64_t>(sh.D_out),
+                       static_cast<uint64_t>(sh.A), kBK, kBM)) {
       *what = "tensor map for the per-alpha operand";
       return kECuda;
     }

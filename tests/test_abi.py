@@ -81,6 +81,33 @@ def test_argument_checks_without_gpu(lib):
     assert call(grid=None) == 1
     assert call(form=2) == 1
 
+    c = lib.awq_clip_search
+    c.argtypes = [P, P, P, I64, I64, I64, P, I, I, I, P, P, P, P, ctypes.c_size_t, P, P]
+    c.restype = I
+    cgrid = (ctypes.c_float * 3)(1.0, 0.75, 0.5)
+    cargs = dict(X=fake, W=fake, s=fake, N=64, D_in=256, D_out=64, grid=cgrid, C=3, bits=4, group=128, clip=fake,
+                 idx=None, loss=None, ws=fake, wsb=1 << 20, st=None, stream=None)
+
+    def ccall(**kw):
+        d = dict(cargs, **kw)
+        return c(d["X"], d["W"], d["s"], d["N"], d["D_in"], d["D_out"], d["grid"], d["C"], d["bits"], d["group"],
+                 d["clip"], d["idx"], d["loss"], d["ws"], d["wsb"], d["st"], d["stream"])
+
+    assert ccall(group=32) == 3                           # the clipping search takes groups of 64 and 128
+    assert ccall(bits=5) == 3
+    assert ccall(C=0) == 3
+    assert ccall(D_in=192) == 1
+    assert ccall(grid=None) == 1
+    assert ccall(grid=(ctypes.c_float * 3)(1.0, 0.0, 0.5)) == 1         # ratios must lie in (0, 1]
+    assert ccall(grid=(ctypes.c_float * 3)(1.0, 1.5, 0.5)) == 1
+    assert ccall(clip=None) == 1
+    assert ccall(s=fake + 4) == 2
+    cws = lib.awq_clip_search_workspace_size
+    cws.argtypes = [I64, I64, I64, I, I, I]
+    cws.restype = ctypes.c_size_t
+    assert cws(64, 256, 64, 3, 4, 32) == 0
+    assert cws(64, 256, 64, 3, 4, 128) > 0                 # the layout needs no device
+
     q = lib.awq_quantize_pack
     q.argtypes = [P, P, I64, I64, I, I, P, P, P]
     q.restype = I
