@@ -52,6 +52,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clip", action="store_true", help="skip timing the weight-clipping search")
     ap.add_argument("--no-at-scale", action="store_true",
                     help="skip timing the statistic and pack kernels on the 70B block's largest operands")
     ap.add_argument("--loss-form", choices=("error", "reference"), default="error")
@@ -411,6 +412,47 @@ def run_ours(args):
         del xs_b, ws_b
         torch.cuda.empty_cache()
 
+    # ---------------- the weight-clipping search that follows the scale search
+    # (not part of the step): the same layer at s*, 21 ratios from 1 down to 0.5
+    clip_info = None
+    if not args.no_clip:
+        cgrid = synth.clip_grid(20).tolist()
+        cws = awq.Workspace()
+        for _ in range(2):
+            awq.clip_search(X, W, r.s_star, cgrid, bits, group, workspace=cws)
+        torch.cuda.synchronize()
+        reps = 10
+        times = []
+        for _ in range(reps):
+            flush.zero_()
+            flush_sink.add_(flush.amax())
+            ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ea.record()
+            cr = awq.clip_search(X, W, r.s_star, cgrid, bits, group, workspace=cws, check_status=False)
+            eb.record()
+            times.append((ea, eb))
+        torch.cuda.synchronize()
+        awq.check_device_status(cr.status)
+        call_ms = sum(a_.elapsed_time(b_) for a_, b_ in times) / reps
+        awq.profile_enable(True)
+        awq.profile_reset()
+        for _ in range(3):
+            awq.clip_search(X, W, r.s_star, cgrid, bits, group, workspace=cws, check_status=False)
+        cprof = awq.profile_read()
+        awq.profile_enable(False)
+        C = len(cgrid)
+        op_bytes = C * layer.D_in * layer.D_out * 2
+        loss_ms = cprof["clip_loss"][0] / max(cprof["clip_loss"][1], 1)
+        clip_info = {
+            "ms_per_call": call_ms, "n_clip": C,
+            "stages_ms": {k: cprof[k][0] / max(cprof[k][1], 1) for k in ("clip_gram", "clip_operand", "clip_loss")},
+            "loss_kernel": {"algorithmic_bytes": op_bytes, "achieved_gbs": op_bytes / (loss_ms / 1e3) / 1e9,
+                            "frac_hbm": op_bytes / (loss_ms / 1e3) / 1e9 / float(load_peaks()[0]["hbm_gbs"]),
+                            "mma_tflops": 2.0 * group * layer.D_in * layer.D_out * C / (loss_ms / 1e3) / 1e12},
+            "mean_ratio": float(cr.clip.mean().item()),
+            "frac_clipped": float((cr.idx > 0).float().mean().item()),
+        }
+
     def hbm(stage, nbytes):
         ms, n = prof[stage]
         if n == 0:
@@ -443,6 +485,7 @@ def run_ours(args):
         "hbm_kernels": {"act_stats": hbm("act_stats", stats_bytes), "quantize_pack": hbm("quantize_pack", pack_bytes),
                         "search_operand": hbm("search_operand", operand_bytes)},
         "hbm_kernels_at_scale": at_scale or None,
+        "clip_search": clip_info,
         "kernels": kernels,
         "e2e": {"value": A * world / (e2e_per_step / 1e3), "unit": UNIT, "ms_per_step": e2e_per_step,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
