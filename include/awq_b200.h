@@ -191,6 +191,30 @@ AWQ_API int awq_quantize_pack(const float* W, const float* s, int64_t D_in, int6
                       uint32_t* packed, float* scales, void* stream);
 
 /*
+ * Joint search of linears that share one input and therefore one scale vector
+ * (mudrobot.github.io AWQ notes: 1/s is fused into the previous operator, so
+ * q/k/v after one LayerNorm, or gate/up, take the same s).  The objective is
+ * the sum of the layers' losses,
+ *     L(alpha) = sum_l || X S^-1 Q(S W_l) - X W_l ||^2,
+ * and alpha* its argmin.  Since a layer's loss is a sum over its output
+ * columns, this is exactly the search of the layers' weights side by side
+ * ([D_in][sum_l D_out_l], copied into the workspace).
+ *   Ws        HOST array of n_layers device pointers, W_l [D_in][D_outs[l]] fp32
+ *   D_outs    HOST array: each a multiple of 4; 1 <= n_layers <= 16
+ *   L         [n_alpha] fp64 output: the joint loss
+ *   L_layers  [n_layers][n_alpha] fp64 output: each layer's loss (may be NULL)
+ *   other arguments and limits as for awq_search; workspace at least
+ *   awq_search_joint_workspace_size(...) bytes.
+ */
+AWQ_API size_t awq_search_joint_workspace_size(int64_t N, int64_t D_in, const int64_t* D_outs, int n_layers,
+                                               int n_alpha, int bits, int group, int loss_form);
+AWQ_API int awq_search_joint(const void* X, const float* const* Ws, const int64_t* D_outs, int n_layers,
+                             const float* a, int64_t N, int64_t D_in, const float* alpha_grid, int n_alpha, int bits,
+                             int group, int loss_form, double* L, double* L_layers, float* alpha_star,
+                             int32_t* alpha_idx, void* workspace, size_t workspace_bytes, int32_t* status,
+                             void* stream);
+
+/*
  * Weight-clipping search, the step after the scale search (mudrobot.github.io
  * AWQ notes, "searching the optimal scale": weight clipping is applied to
  * minimise the quantisation MSE).  For every group g of `group` rows, output

@@ -214,3 +214,16 @@ def literal_loss(X, W, s, bits: int, group: int) -> float:
     s = _f32(s)
     N, D_in = Xb.shape
     return float(_load().oracle_literal_loss(_ptr(Xb), _ptr(W), _ptr(s), N, D_in, W.shape[1], bits, group))
+
+
+def search_joint(X, Ws, a, alphas, bits: int, group: int):
+    """Joint search of linears sharing one input and one scale vector
+    (mudrobot.github.io AWQ notes: 1/s is fused into the previous operator, so
+    q/k/v, or gate/up, take the same s): L(alpha) = sum_l L_l(alpha), each
+    L_l the single-layer loss above; alpha* = argmin, lowest index on ties.
+    Returns (L [n_alpha], best, L_layers [n_layers, n_alpha])."""
+    per = np.stack([search(X, W, a, alphas, bits, group)[0] for W in Ws])
+    L = per.sum(axis=0)
+    best = int(np.flatnonzero(L == L.min())[0])
+    return L, best, per
+

@@ -29,6 +29,7 @@ EXPORTS = (
     "awq_layer_output_workspace_size", "awq_layer_output", "awq_selftest_wait_timeout",
     "awq_get_last_error", "awq_version", "awq_profile_enable", "awq_profile_reset", "awq_profile_read",
     "awq_search_noalloc", "awq_clip_search_workspace_size", "awq_clip_search", "awq_quantize_pack_clip",
+    "awq_search_joint_workspace_size", "awq_search_joint",
 )
 STAGES = ("act_stats", "scale_table", "search_operand", "search_gemm", "loss_reduce", "quantize_pack",
           "weight_t", "clip_gram", "clip_operand", "clip_loss")
@@ -78,6 +79,8 @@ _version = _sig("awq_version", I, [])
 _clip_ws = _sig("awq_clip_search_workspace_size", SZ, [I64, I64, I64, I, I, I])
 _clip = _sig("awq_clip_search", I, [P, P, P, I64, I64, I64, P, I, I, I, P, P, P, P, SZ, P, P])
 _pack_clip = _sig("awq_quantize_pack_clip", I, [P, P, P, I64, I64, I, I, P, P, P])
+_joint_ws = _sig("awq_search_joint_workspace_size", SZ, [I64, I64, P, I, I, I, I, I])
+_joint = _sig("awq_search_joint", I, [P, P, P, I, P, I64, I64, P, I, I, I, I, P, P, P, P, P, SZ, P, P])
 
 
 class AwqError(RuntimeError):
@@ -242,6 +245,46 @@ def quantize_pack_clip(W: torch.Tensor, s: torch.Tensor, clip: torch.Tensor, bit
     sc = torch.empty(D_in // group, D_out, dtype=torch.float32, device=W.device)
     _check(_pack_clip(_ptr(W), _ptr(s), _ptr(clip), D_in, D_out, bits, group, _ptr(packed), _ptr(sc), _stream()))
     return packed, sc
+
+
+@dataclass
+class JointResult:
+    L: torch.Tensor             # [n_alpha] fp64 joint loss
+    L_layers: torch.Tensor      # [n_layers, n_alpha] fp64
+    alpha_star: torch.Tensor    # [1] fp32
+    alpha_idx: torch.Tensor     # [1] int32
+    status: torch.Tensor
+
+
+def search_joint(X: torch.Tensor, Ws: Sequence[torch.Tensor], a: torch.Tensor, alpha_grid: Sequence[float],
+                 bits: int = 4, group: int = 128, workspace: Optional[Workspace] = None, check_status: bool = True,
+                 loss_form: int = LOSS_ERROR) -> JointResult:
+    """One scale vector for several linears that share X: ``awq_search_joint``."""
+    X = _dev(X, torch.bfloat16, "X")
+    Ws = [_dev(W, torch.float32, "W") for W in Ws]
+    a = _dev(a, torch.float32, "a")
+    N, D_in = X.shape
+    nl = len(Ws)
+    ptrs = (ctypes.c_void_p * nl)(*[W.data_ptr() for W in Ws])
+    douts = (ctypes.c_int64 * nl)(*[W.shape[1] for W in Ws])
+    A = len(alpha_grid)
+    grid = (ctypes.c_float * A)(*[float(v) for v in alpha_grid])
+    dev = X.device
+    L = torch.empty(A, dtype=torch.float64, device=dev)
+    Ll = torch.empty(nl, A, dtype=torch.float64, device=dev)
+    astar = torch.empty(1, dtype=torch.float32, device=dev)
+    aidx = torch.empty(1, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    nbytes = int(_joint_ws(N, D_in, douts, nl, A, bits, group, loss_form))
+    if nbytes == 0:
+        raise AwqError(AWQ_EINVAL, _last_error().decode(errors="replace"))
+    ws = (workspace or _default_ws).get(nbytes, dev)
+    _check(_joint(_ptr(X), ptrs, douts, nl, _ptr(a), N, D_in, grid, A, bits, group, loss_form, _ptr(L), _ptr(Ll),
+                  _ptr(astar), _ptr(aidx), _ptr(ws), ws.numel(), _ptr(status), _stream()))
+    res = JointResult(L, Ll, astar, aidx, status)
+    if check_status:
+        check_device_status(status)
+    return res
 
 
 def check_device_status(status: torch.Tensor) -> None:

@@ -658,4 +658,84 @@ int awq_quantize_pack_clip(const float* W, const float* s, const float* clip, in
   return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "quantize_pack kernel (clipped)");
 }
 
+// ---------------------------------------------------------------- joint search over shared-input linears
+static int check_joint(const int64_t* D_outs, int n_layers, int64_t* Dsum) {
+  if (!D_outs) return fail(AWQ_EINVAL, "D_outs is NULL");
+  if (n_layers < 1 || n_layers > awq::kMaxJointLayers)
+    return fail(AWQ_EUNSUPPORTED, "n_layers = %d: need 1..%d", n_layers, awq::kMaxJointLayers);
+  int64_t s = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    if (D_outs[l] < 4 || D_outs[l] % 4)
+      return fail(AWQ_EINVAL, "D_outs[%d] = %lld: need a multiple of 4, at least 4", l, (long long)D_outs[l]);
+    s += D_outs[l];
+  }
+  *Dsum = s;
+  return AWQ_OK;
+}
+
+size_t awq_search_joint_workspace_size(int64_t N, int64_t D_in, const int64_t* D_outs, int n_layers, int n_alpha,
+                                       int bits, int group, int loss_form) {
+  int64_t Dsum = 0;
+  if (check_joint(D_outs, n_layers, &Dsum) != AWQ_OK) return 0;
+  const size_t base = awq_search_workspace_size(N, D_in, Dsum, n_alpha, bits, group, loss_form);
+  if (base == 0) return 0;
+  return base + round_up(static_cast<size_t>(D_in) * Dsum * 4, 256) +
+         round_up(static_cast<size_t>(n_alpha) * Dsum * 8, 256);
+}
+
+int awq_search_joint(const void* X, const float* const* Ws, const int64_t* D_outs, int n_layers, const float* a,
+                     int64_t N, int64_t D_in, const float* alpha_grid, int n_alpha, int bits, int group,
+                     int loss_form, double* L, double* L_layers, float* alpha_star, int32_t* alpha_idx,
+                     void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  int64_t Dsum = 0;
+  AWQ_TRY(check_joint(D_outs, n_layers, &Dsum));
+  if (!Ws) return fail(AWQ_EINVAL, "Ws is NULL");
+  for (int l = 0; l < n_layers; ++l) {
+    int rc = check_ptr(Ws[l], "Ws[l]", 16);
+    if (rc != AWQ_OK) return fail(rc, "layer %d: %s", l, g_last_error.c_str());
+  }
+  // The shapes and pointers of the joint layer; W is checked per layer above.
+  AWQ_TRY(check_search_args(X, Ws[0], a, N, D_in, Dsum, alpha_grid, n_alpha, bits, group, loss_form, L, nullptr,
+                            alpha_star, alpha_idx));
+  if (L_layers) AWQ_TRY(check_ptr(L_layers, "L_layers", 8));
+  int sms = 0;
+  AWQ_TRY(device_info(&sms));
+  const SearchLayout lay = search_layout(N, D_in, Dsum, n_alpha, group, loss_form, sms);
+  const size_t w_off = lay.total;
+  const size_t lc_off = w_off + round_up(static_cast<size_t>(D_in) * Dsum * 4, 256);
+  const size_t need = lc_off + round_up(static_cast<size_t>(n_alpha) * Dsum * 8, 256);
+  if (!workspace) return fail(AWQ_EWORKSPACE, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(AWQ_EALIGN, "workspace is not 256-byte aligned");
+  if (workspace_bytes < need) return fail(AWQ_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+  if (status && !aligned(status, 4)) return fail(AWQ_EALIGN, "status is not 4-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* Wcat = reinterpret_cast<float*>(ws + w_off);
+  double* Lcol = reinterpret_cast<double*>(ws + lc_off);
+  int32_t* st_word = status ? status : reinterpret_cast<int32_t*>(ws + lay.status);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(st_word, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(status)");
+  // The layers side by side: [D_in][sum of D_out].  L is a sum over output
+  // columns, so the search of the joint matrix gives sum_l L_l(alpha).
+  awq::Segments seg{};
+  int64_t off = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    seg.off[l] = off;
+    e = cudaMemcpy2DAsync(Wcat + off, static_cast<size_t>(Dsum) * 4, Ws[l], static_cast<size_t>(D_outs[l]) * 4,
+                          static_cast<size_t>(D_outs[l]) * 4, static_cast<size_t>(D_in), cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaMemcpy2DAsync(joint weights)");
+    off += D_outs[l];
+  }
+  seg.off[n_layers] = off;
+  awq::AlphaList al{};
+  for (int i = 0; i < n_alpha; ++i) al.v[i] = alpha_grid[i];
+  AWQ_TRY(search_one(X, Wcat, a, N, D_in, Dsum, al, n_alpha, bits, group, loss_form, L, Lcol, alpha_star, alpha_idx,
+                     ws, st_word, st, sms));
+  if (L_layers) {
+    e = awq::launch_segment_sums(Lcol, n_alpha, Dsum, seg, n_layers, L_layers, st);
+    if (e != cudaSuccess) return fail_cuda(e, "per-layer loss sums");
+  }
+  return AWQ_OK;
+}
+
 }  // extern "C"

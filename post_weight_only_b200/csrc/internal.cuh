@@ -54,6 +54,14 @@ cudaError_t launch_loss_reduce(const float* partial, int A, int H, int64_t D_out
                                int nblk, const AlphaList& alphas, double* L, float* alpha_star, int* alpha_idx,
                                cudaStream_t st);
 int loss_reduce_blocks(int64_t D_out);
+// Column ranges [off[l], off[l+1]) of the layers of a joint search.
+constexpr int kMaxJointLayers = 16;
+struct Segments {
+  int64_t off[kMaxJointLayers + 1];
+};
+// out [n_seg][A]: the sums of L_col [A][D] over each range, in a fixed order.
+cudaError_t launch_segment_sums(const double* L_col, int A, int64_t D, const Segments& seg, int n_seg, double* out,
+                                cudaStream_t st);
 
 // ---- search.cu
 struct SearchShape {

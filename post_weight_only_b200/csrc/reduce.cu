@@ -56,7 +56,34 @@ __global__ void loss_final_kernel(const double* __restrict__ blk, int A, int nbl
   }
 }
 
+// Per-layer losses of a joint search: L_layer[l][a] = sum of L_col[a][n] over
+// the layer's column range [off[l], off[l+1]), each thread a strided share in
+// ascending order, then a fixed binary tree.
+__global__ void __launch_bounds__(kThreads)
+    segment_sums_kernel(const double* __restrict__ L_col, int64_t D, Segments seg, double* __restrict__ out) {
+  __shared__ double red[kThreads];
+  const int a = blockIdx.x, l = blockIdx.y;
+  const int A = gridDim.x;
+  double acc = 0.0;
+  for (int64_t n = seg.off[l] + threadIdx.x; n < seg.off[l + 1]; n += kThreads)
+    acc += L_col[static_cast<int64_t>(a) * D + n];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = kThreads / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) out[static_cast<int64_t>(l) * A + a] = red[0];
+}
+
 }  // namespace
+
+cudaError_t launch_segment_sums(const double* L_col, int A, int64_t D, const Segments& seg, int n_seg, double* out,
+                                cudaStream_t st) {
+  segment_sums_kernel<<<dim3(static_cast<unsigned>(A), static_cast<unsigned>(n_seg)), kThreads, 0, st>>>(L_col, D,
+                                                                                                         seg, out);
+  return cudaGetLastError();
+}
 
 int loss_reduce_blocks(int64_t D_out) { return static_cast<int>((D_out + kThreads - 1) / kThreads); }
 

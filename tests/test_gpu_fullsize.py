@@ -146,3 +146,23 @@ def test_sweep_4096x11008_n16k(awq, bits, group):
     for li, spec in enumerate(wl.layers):
         X = synth.make_x(spec.N, spec.D_in, spec.x)
         _check_layer_path(awq, X, W, alphas, bits, group, "error", _sample_cols(W.shape[1], 2, seed=20 + li))
+
+
+def test_llama70b_qkv_joint(awq):
+    """q/k/v of the 70B-shaped block share one input, hence one scale vector:
+    the joint loss is the sum of the layers' losses, each of which matches a
+    separate search of that layer."""
+    wl = synth.workload("llama70b_block")
+    alphas = synth.alpha_grid(wl.n_intervals).tolist()
+    bits, group = wl.quant[0]
+    specs = wl.layers[:3]
+    X = synth.make_x(specs[0].N, specs[0].D_in, specs[0].x).cuda()
+    Ws = [synth.make_w(s.D_in, s.D_out, s.w_std, s.w_seed).cuda() for s in specs]
+    a = awq.act_stats(X)
+    r = awq.search_joint(X, Ws, a, alphas, bits, group)
+    L, per = r.L.cpu().numpy(), r.L_layers.cpu().numpy()
+    assert np.allclose(per.sum(axis=0), L, rtol=1e-12)
+    assert int(r.alpha_idx.item()) == int(np.argmin(L))
+    for l, W in enumerate(Ws):
+        single = awq.search(X, W, a, alphas, bits, group).L.cpu().numpy()
+        assert np.allclose(per[l], single, rtol=1e-6)

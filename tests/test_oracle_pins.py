@@ -269,3 +269,27 @@ def test_outlier_channels_pull_alpha_up():
     alphas = synth.alpha_grid(20).numpy()
     L, best = oracle.search(X, W, a, alphas, 4, 128)
     assert best > 0 and L[best] < L[0]
+
+
+# ------------------------------------------------------------------ joint search of shared-input linears
+def test_joint_search_one_layer_is_the_search():
+    X, W = synth.layer_inputs(synth.small_layer(32, 256, 24, seed=41))
+    a = oracle.act_stats(X).astype(np.float32)
+    alphas = synth.alpha_grid(10).numpy()
+    L, best, per = oracle.search_joint(X, [W], a, alphas, 4, 128)
+    L1, b1 = oracle.search(X, W, a, alphas, 4, 128)
+    assert np.array_equal(L, L1) and best == b1 and np.array_equal(per[0], L1)
+
+
+def test_joint_search_equals_search_of_side_by_side_weights():
+    """A layer's loss is a sum over its output columns, so the joint loss of
+    q/k/v-like layers is the loss of their weights side by side."""
+    X, W1 = synth.layer_inputs(synth.small_layer(32, 256, 24, seed=42))
+    W2 = synth.make_w(256, 16, 0.02, 7)
+    W3 = synth.make_w(256, 8, 0.03, 8)
+    a = oracle.act_stats(X).astype(np.float32)
+    alphas = synth.alpha_grid(10).numpy()
+    L, best, per = oracle.search_joint(X, [W1, W2, W3], a, alphas, 4, 128)
+    Lc, bc = oracle.search(X, torch.cat([W1, W2, W3], dim=1), a, alphas, 4, 128)
+    assert np.allclose(L, Lc, rtol=1e-12) and best == bc
+    assert np.allclose(per.sum(axis=0), L, rtol=0)
