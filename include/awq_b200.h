@@ -251,6 +251,21 @@ AWQ_API int awq_quantize_pack_clip(const float* W, const float* s, const float* 
                                    int bits, int group, uint32_t* packed, float* scales, void* stream);
 
 /*
+ * Final quantise + pack with options (the pack of awq_quantize_pack and
+ * awq_quantize_pack_clip):
+ *   clip    [D_in/group][D_out] fp32 clip ratios, or NULL for none
+ *   flags   AWQ_PACK_DELTA_FP16: delta is rounded to FP16 (round to nearest
+ *           even; mudrobot.github.io AWQ notes, "analysing the quantisation
+ *           error": delta stored in FP16) before the codes are formed, codes
+ *           are clamped to +-qmax, and `scales` receives FP16 values
+ *           ([D_in/group][D_out] uint16 bit patterns).  Without the flag
+ *           `scales` is [D_in/group][D_out] fp32, as in awq_quantize_pack.
+ */
+#define AWQ_PACK_DELTA_FP16 1
+AWQ_API int awq_quantize_pack_ex(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out,
+                                 int bits, int group, int flags, uint32_t* packed, void* scales, void* stream);
+
+/*
  * The layer's reference output Y = X bf16(W) computed by the search's own
  * tensor-core GEMM (the X W term of the loss, concept page flow step 4c), fp32.
  *   Y          [N][D_out] fp32 output

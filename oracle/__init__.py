@@ -55,6 +55,8 @@ def _load():
         lib.oracle_quantize.restype = None
         lib.oracle_quantize_clip.argtypes = [P, P, P, I64, I64, I, I, P, P]
         lib.oracle_quantize_clip.restype = None
+        lib.oracle_quantize_ex.argtypes = [P, P, P, I64, I64, I, I, I, P, P]
+        lib.oracle_quantize_ex.restype = None
         lib.oracle_clip_loss.argtypes = [P, P, P, I64, I64, I64, P, I, I, I, P, I64, P, P]
         lib.oracle_clip_loss.restype = None
         lib.oracle_pack.argtypes = [P, I64, I64, I, P]
@@ -114,22 +116,24 @@ def scales(a, alpha: float) -> np.ndarray:
     return s
 
 
-def quantize(W, s, bits: int, group: int, clip=None) -> Tuple[np.ndarray, np.ndarray]:
+def quantize(W, s, bits: int, group: int, clip=None, delta16: bool = False) -> Tuple[np.ndarray, np.ndarray]:
     """Codes q [D_in, D_out] (int8) and deltas [D_in/group, D_out] (fp32) of
     diag(s).W.  compassingai.com concept page, "quantisation math".  clip:
     optional [D_in/group, D_out] fp32 clip ratios (the group maximum is
-    replaced by fl32(clip * max) before delta is formed)."""
+    replaced by fl32(clip * max) before delta is formed).  delta16: delta is
+    rounded to FP16 (mudrobot.github.io notes: delta stored in FP16) and the
+    codes use that value; the returned deltas are then FP16-representable."""
     W = _f32(W)
     D_in, D_out = W.shape
     s = None if s is None else _f32(s)
     q = np.empty((D_in, D_out), dtype=np.int8)
     d = np.empty((D_in // group, D_out), dtype=np.float32)
-    if clip is None:
-        _load().oracle_quantize(_ptr(W), _ptr(s), D_in, D_out, bits, group, _ptr(q), _ptr(d))
-    else:
+    c = None
+    if clip is not None:
         c = _f32(clip)
         assert c.shape == (D_in // group, D_out)
-        _load().oracle_quantize_clip(_ptr(W), _ptr(s), _ptr(c), D_in, D_out, bits, group, _ptr(q), _ptr(d))
+    _load().oracle_quantize_ex(_ptr(W), _ptr(s), _ptr(c), D_in, D_out, bits, group, int(bool(delta16)), _ptr(q),
+                               _ptr(d))
     return q, d
 
 

@@ -96,6 +96,27 @@ void oracle_scales(const float *a, int64_t D, float alpha, float *s)
     }
 }
 
+/* Round a finite fp32 value to the nearest IEEE binary16 value (ties to
+ * even), returned as a float: 11 significant bits in the normal range
+ * (|x| >= 2^-14), a fixed step of 2^-24 below it, infinity from 65520 up
+ * ([P2] "analysing the quantisation error": delta stored in FP16). */
+static float round_to_fp16(float x)
+{
+    double ax = fabs((double)x);
+    if (ax >= 65520.0)
+        return x > 0 ? INFINITY : -INFINITY;
+    if (ax == 0.0)
+        return x;
+    int e;
+    frexp(ax, &e);                 /* ax = f * 2^e, f in [0.5, 1): the binade is 2^(e-1) */
+    int ulp_exp = (e - 1) - 10;    /* 10 fraction bits */
+    if (ulp_exp < -24)
+        ulp_exp = -24;             /* subnormal step */
+    const double ulp = ldexp(1.0, ulp_exp);
+    const double r = nearbyint(ax / ulp) * ulp;   /* exact scaling; round half to even */
+    return (float)(x < 0 ? -r : r);
+}
+
 /* [P1] "quantisation math", steps 1-3, applied to one group of one column of
  * W' = diag(s) W ([P1] flow step 4a):
  *   w'_k  = fl32(s_k * w_k)
@@ -107,7 +128,7 @@ void oracle_scales(const float *a, int64_t D, float alpha, float *s)
  * delta is formed, and the clamp then bounds the codes of the clipped weights.
  * clip = 1 leaves m unchanged (fl32(1 * m) = m). */
 static void quantize_group(const float *W, const float *s, int64_t D_out, int64_t n,
-                           int64_t k0, int group, int bits, float clip, int8_t *q, float *delta)
+                           int64_t k0, int group, int bits, float clip, int delta16, int8_t *q, float *delta)
 {
     const int qmax = (1 << (bits - 1)) - 1;
     float m = 0.0f;
@@ -119,7 +140,9 @@ static void quantize_group(const float *W, const float *s, int64_t D_out, int64_
             m = am;
     }
     m = clip * m;
-    const float d = m / (float)qmax;
+    float d = m / (float)qmax;
+    if (delta16)
+        d = round_to_fp16(d);      /* the exported FP16 delta, which the codes then use */
     *delta = d;
     for (int k = 0; k < group; ++k) {
         int code = 0;
@@ -140,15 +163,16 @@ static void quantize_group(const float *W, const float *s, int64_t D_out, int64_
 
 /* Quantise every (group, column) of diag(s) W.  q: [D_in][D_out] codes in
  * [-qmax, qmax]; delta: [D_in/group][D_out].  clip: [D_in/group][D_out] clip
- * ratios, or NULL for none. */
-void oracle_quantize_clip(const float *W, const float *s, const float *clip, int64_t D_in, int64_t D_out,
-                          int bits, int group, int8_t *q, float *delta)
+ * ratios, or NULL for none.  delta16: delta is rounded to FP16 before the
+ * codes are formed (the exported scale format). */
+void oracle_quantize_ex(const float *W, const float *s, const float *clip, int64_t D_in, int64_t D_out,
+                        int bits, int group, int delta16, int8_t *q, float *delta)
 {
     int8_t *col = (int8_t *)malloc((size_t)group);
     for (int64_t n = 0; n < D_out; ++n) {
         for (int64_t g = 0; g < D_in / group; ++g) {
-            quantize_group(W, s, D_out, n, g * group, group, bits, clip ? clip[g * D_out + n] : 1.0f, col,
-                           &delta[g * D_out + n]);
+            quantize_group(W, s, D_out, n, g * group, group, bits, clip ? clip[g * D_out + n] : 1.0f, delta16,
+                           col, &delta[g * D_out + n]);
             for (int k = 0; k < group; ++k)
                 q[(g * group + k) * D_out + n] = col[k];
         }
@@ -156,10 +180,16 @@ void oracle_quantize_clip(const float *W, const float *s, const float *clip, int
     free(col);
 }
 
+void oracle_quantize_clip(const float *W, const float *s, const float *clip, int64_t D_in, int64_t D_out,
+                          int bits, int group, int8_t *q, float *delta)
+{
+    oracle_quantize_ex(W, s, clip, D_in, D_out, bits, group, 0, q, delta);
+}
+
 void oracle_quantize(const float *W, const float *s, int64_t D_in, int64_t D_out,
                      int bits, int group, int8_t *q, float *delta)
 {
-    oracle_quantize_clip(W, s, NULL, D_in, D_out, bits, group, q, delta);
+    oracle_quantize_ex(W, s, NULL, D_in, D_out, bits, group, 0, q, delta);
 }
 
 /* Pack codes: word (k8, n) holds rows 8*k8 .. 8*k8+7 of column n, row 8*k8+i in
@@ -194,7 +224,7 @@ static double column_loss(const double *Xd, const float *W, const float *s,
         const int64_t k0 = g * group;
         if (quantize) {
             float d;
-            quantize_group(W, s, D_out, n, k0, group, bits, 1.0f, qcol, &d);
+            quantize_group(W, s, D_out, n, k0, group, bits, 1.0f, 0, qcol, &d);
             for (int k = 0; k < group; ++k) {
                 double sk = s ? (double)s[k0 + k] : 1.0;
                 e[k0 + k] = (double)qcol[k] * (double)d / sk - (double)W[(k0 + k) * D_out + n];
@@ -364,7 +394,7 @@ void oracle_clip_loss(const uint16_t *X, const float *W, const float *s, int64_t
                 int ibest = 0;
                 for (int i = 0; i < n_clip; ++i) {
                     float d;
-                    quantize_group(W, s, D_out, n, k0, group, bits, clip[i], qg, &d);
+                    quantize_group(W, s, D_out, n, k0, group, bits, clip[i], 0, qg, &d);
                     for (int k = 0; k < group; ++k) {
                         double sk = s ? (double)s[k0 + k] : 1.0;
                         e[k] = (double)qg[k] * (double)d / sk - (double)W[(k0 + k) * D_out + n];

@@ -29,7 +29,7 @@ EXPORTS = (
     "awq_layer_output_workspace_size", "awq_layer_output", "awq_selftest_wait_timeout",
     "awq_get_last_error", "awq_version", "awq_profile_enable", "awq_profile_reset", "awq_profile_read",
     "awq_search_noalloc", "awq_clip_search_workspace_size", "awq_clip_search", "awq_quantize_pack_clip",
-    "awq_search_joint_workspace_size", "awq_search_joint",
+    "awq_search_joint_workspace_size", "awq_search_joint", "awq_quantize_pack_ex",
 )
 STAGES = ("act_stats", "scale_table", "search_operand", "search_gemm", "loss_reduce", "quantize_pack",
           "weight_t", "clip_gram", "clip_operand", "clip_loss")
@@ -80,6 +80,8 @@ _clip_ws = _sig("awq_clip_search_workspace_size", SZ, [I64, I64, I64, I, I, I])
 _clip = _sig("awq_clip_search", I, [P, P, P, I64, I64, I64, P, I, I, I, P, P, P, P, SZ, P, P])
 _pack_clip = _sig("awq_quantize_pack_clip", I, [P, P, P, I64, I64, I, I, P, P, P])
 _joint_ws = _sig("awq_search_joint_workspace_size", SZ, [I64, I64, P, I, I, I, I, I])
+_pack_ex = _sig("awq_quantize_pack_ex", I, [P, P, P, I64, I64, I, I, I, P, P, P])
+PACK_DELTA_FP16 = 1
 _joint = _sig("awq_search_joint", I, [P, P, P, I, P, I64, I64, P, I, I, I, I, P, P, P, P, P, SZ, P, P])
 
 
@@ -231,6 +233,23 @@ def clip_search(X: torch.Tensor, W: torch.Tensor, s: torch.Tensor, clip_grid: Se
     if check_status:
         check_device_status(status)
     return res
+
+
+def quantize_pack_ex(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int = 128,
+                     clip: Optional[torch.Tensor] = None, delta_fp16: bool = False):
+    """``awq_quantize_pack_ex``: the final pack with optional clip ratios and
+    FP16 deltas.  Returns (packed int32 view [D_in/8, D_out], scales
+    [D_in/group, D_out] as float16 when delta_fp16 else float32)."""
+    W = _dev(W, torch.float32, "W")
+    s = _dev(s, torch.float32, "s")
+    if clip is not None:
+        clip = _dev(clip, torch.float32, "clip")
+    D_in, D_out = W.shape
+    packed = torch.empty(D_in // 8, D_out, dtype=torch.int32, device=W.device)
+    sc = torch.empty(D_in // group, D_out, dtype=torch.float16 if delta_fp16 else torch.float32, device=W.device)
+    _check(_pack_ex(_ptr(W), _ptr(s), _ptr(clip), D_in, D_out, bits, group, PACK_DELTA_FP16 if delta_fp16 else 0,
+                    _ptr(packed), _ptr(sc), _stream()))
+    return packed, sc
 
 
 def quantize_pack_clip(W: torch.Tensor, s: torch.Tensor, clip: torch.Tensor, bits: int = 4, group: int = 128):

@@ -409,23 +409,7 @@ int awq_search_batched(const awq_layer* layers, int n_layers, const float* alpha
 
 int awq_quantize_pack(const float* W, const float* s, int64_t D_in, int64_t D_out, int bits, int group,
                       uint32_t* packed, float* scales, void* stream) {
-  AWQ_TRY(check_quant_args(bits, group));
-  if (D_in < group || D_in > kMaxDin || D_in % group)
-    return fail(AWQ_EINVAL, "D_in = %lld: need a positive multiple of group = %d", (long long)D_in, group);
-  if (D_out < 1 || D_out > kMaxDim) return fail(AWQ_EINVAL, "D_out = %lld out of range", (long long)D_out);
-  AWQ_TRY(check_ptr(W, "W", 16));
-  AWQ_TRY(check_ptr(s, "s", 16));
-  AWQ_TRY(check_ptr(packed, "packed", 16));
-  AWQ_TRY(check_ptr(scales, "scales", 16));
-  int sms = 0;
-  AWQ_TRY(device_info(&sms));
-  cudaError_t e;
-  {
-    StageTimer t(AWQ_STAGE_QUANTIZE_PACK, static_cast<cudaStream_t>(stream));
-    e = awq::launch_quantize_pack(W, s, nullptr, D_in, D_out, bits, group, packed, scales, sms,
-                                   static_cast<cudaStream_t>(stream));
-  }
-  return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "quantize_pack kernel");
+  return awq_quantize_pack_ex(W, s, nullptr, D_in, D_out, bits, group, 0, packed, scales, stream);
 }
 
 // ---------------------------------------------------------------- weight-clipping search
@@ -638,13 +622,20 @@ int awq_clip_search(const void* X, const float* W, const float* s, int64_t N, in
 
 int awq_quantize_pack_clip(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out, int bits,
                            int group, uint32_t* packed, float* scales, void* stream) {
+  if (!clip) return fail(AWQ_EINVAL, "clip is NULL");
+  return awq_quantize_pack_ex(W, s, clip, D_in, D_out, bits, group, 0, packed, scales, stream);
+}
+
+int awq_quantize_pack_ex(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out, int bits,
+                         int group, int flags, uint32_t* packed, void* scales, void* stream) {
   AWQ_TRY(check_quant_args(bits, group));
+  if (flags & ~AWQ_PACK_DELTA_FP16) return fail(AWQ_EINVAL, "flags = %#x: unknown bits", flags);
   if (D_in < group || D_in > kMaxDin || D_in % group)
     return fail(AWQ_EINVAL, "D_in = %lld: need a positive multiple of group = %d", (long long)D_in, group);
   if (D_out < 1 || D_out > kMaxDim) return fail(AWQ_EINVAL, "D_out = %lld out of range", (long long)D_out);
   AWQ_TRY(check_ptr(W, "W", 16));
   AWQ_TRY(check_ptr(s, "s", 16));
-  AWQ_TRY(check_ptr(clip, "clip", 4));
+  if (clip) AWQ_TRY(check_ptr(clip, "clip", 4));
   AWQ_TRY(check_ptr(packed, "packed", 16));
   AWQ_TRY(check_ptr(scales, "scales", 16));
   int sms = 0;
@@ -652,10 +643,10 @@ int awq_quantize_pack_clip(const float* W, const float* s, const float* clip, in
   cudaError_t e;
   {
     StageTimer t(AWQ_STAGE_QUANTIZE_PACK, static_cast<cudaStream_t>(stream));
-    e = awq::launch_quantize_pack(W, s, clip, D_in, D_out, bits, group, packed, scales, sms,
-                                  static_cast<cudaStream_t>(stream));
+    e = awq::launch_quantize_pack(W, s, clip, D_in, D_out, bits, group, (flags & AWQ_PACK_DELTA_FP16) != 0, packed,
+                                  scales, sms, static_cast<cudaStream_t>(stream));
   }
-  return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "quantize_pack kernel (clipped)");
+  return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "quantize_pack kernel");
 }
 
 // ---------------------------------------------------------------- joint search over shared-input linears

@@ -293,3 +293,40 @@ def test_joint_search_equals_search_of_side_by_side_weights():
     Lc, bc = oracle.search(X, torch.cat([W1, W2, W3], dim=1), a, alphas, 4, 128)
     assert np.allclose(L, Lc, rtol=1e-12) and best == bc
     assert np.allclose(per.sum(axis=0), L, rtol=0)
+
+
+# ------------------------------------------------------------------ FP16 delta export
+def test_delta16_is_the_ieee_half_rounding_of_delta():
+    """delta16 = the IEEE binary16 round-to-nearest-even of the fp32 delta,
+    checked against numpy's float16 conversion (an independent routine)."""
+    X, W = synth.layer_inputs(synth.small_layer(8, 512, 96, seed=51))
+    s = oracle.scales(oracle.act_stats(X).astype(np.float32), 0.5)
+    _, d32 = oracle.quantize(W, s, 4, 128)
+    _, d16 = oracle.quantize(W, s, 4, 128, delta16=True)
+    assert np.array_equal(d16, d32.astype(np.float16).astype(np.float32))
+    # tiny and huge magnitudes: subnormal halves and the overflow threshold
+    Wt = np.zeros((32, 6), np.float32)
+    Wt[0] = [7e-8, 3e-6, 1.0, 6.5e4 * 7, 1e6, -2.5e-7]
+    _, dt = oracle.quantize(Wt, None, 4, 32, delta16=True)
+    _, dt32 = oracle.quantize(Wt, None, 4, 32)
+    with np.errstate(over="ignore"):               # 1e6 / 7 overflows FP16 to infinity on both sides
+        assert np.array_equal(dt, dt32.astype(np.float16).astype(np.float32))
+
+
+def test_delta16_codes_round_with_the_half_delta():
+    """With delta16 the codes are those of the FP16 delta: every unclamped
+    code is within half a step of w'/delta16, and groups whose fp32 delta is
+    already an FP16 value (powers of two) keep the plain codes."""
+    X, W = synth.layer_inputs(synth.small_layer(8, 256, 64, seed=52))
+    s = oracle.scales(oracle.act_stats(X).astype(np.float32), 0.4)
+    q, d = oracle.quantize(W, s, 4, 64, delta16=True)
+    wp = s[:, None].astype(np.float64) * W.numpy().astype(np.float64)
+    y = wp / np.repeat(d, 64, axis=0).astype(np.float64)
+    inside = np.abs(q) < 7
+    assert np.all(np.abs(y[inside] - q[inside]) <= 0.5 + 1e-6)
+    assert np.abs(q).max() <= 7
+    Wp = np.zeros((32, 3), np.float32)
+    Wp[:, 0] = np.linspace(-7, 7, 32)            # max 7 -> delta 1
+    Wp[:, 1] = np.linspace(-0.875, 0.5, 32)      # max 0.875 -> delta 0.125
+    Wp[:, 2] = np.linspace(-14, 3, 32)           # max 14 -> delta 2
+    assert np.array_equal(oracle.quantize(Wp, None, 4, 32, delta16=True)[0], oracle.quantize(Wp, None, 4, 32)[0])
