@@ -57,6 +57,8 @@ def _load():
         lib.oracle_quantize_clip.restype = None
         lib.oracle_quantize_ex.argtypes = [P, P, P, I64, I64, I, I, I, P, P]
         lib.oracle_quantize_ex.restype = None
+        lib.oracle_w4a16.argtypes = [P, P, P, P, I64, I64, I64, I, I, P]
+        lib.oracle_w4a16.restype = None
         lib.oracle_clip_loss.argtypes = [P, P, P, I64, I64, I64, P, I, I, I, P, I64, P, P]
         lib.oracle_clip_loss.restype = None
         lib.oracle_pack.argtypes = [P, I64, I64, I, P]
@@ -230,4 +232,19 @@ def search_joint(X, Ws, a, alphas, bits: int, group: int):
     L = per.sum(axis=0)
     best = int(np.flatnonzero(L == L.min())[0])
     return L, best, per
+
+
+def w4a16(X, s, packed, scales, bits: int, group: int) -> np.ndarray:
+    """Y = X diag(1/s) Dequant(W_q) in fp64 from the packed words and the
+    per-group deltas (compassingai.com concept page, "inference-time
+    equivalent")."""
+    Xb = _as_bf16_bits(X)
+    s = _f32(s)
+    packed = np.ascontiguousarray(packed).view(np.uint32)
+    scales = _f32(scales)
+    N, D_in = Xb.shape
+    D_out = packed.shape[1]
+    Y = np.empty((N, D_out), dtype=np.float64)
+    _load().oracle_w4a16(_ptr(Xb), _ptr(s), _ptr(packed), _ptr(scales), N, D_in, D_out, bits, group, _ptr(Y))
+    return Y
 

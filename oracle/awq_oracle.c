@@ -422,3 +422,39 @@ void oracle_clip_loss(const uint16_t *X, const float *W, const float *s, int64_t
     }
     free(Xd);
 }
+
+/* The quantised layer applied to activations ([P1] "inference-time
+ * equivalent": W_quantized = Quantize(diag(s*) W) with s* kept as metadata and
+ * 1/s* folded into the input; [P2] "searching the optimal scale": the output
+ * Q(W diag(s)) (diag(s)^-1 X)):
+ *   Y[t][n] = sum_k x_tk / s_k * (u_kn - 2^(b-1)) * delta_{k/group, n}
+ * with u the offset-binary nibble of row k, column n of the packed words
+ * (row 8*k8+i in bits 4i..4i+3 of word (k8, n)).  fp64 throughout. */
+void oracle_w4a16(const uint16_t *X, const float *s, const uint32_t *packed, const float *scales, int64_t N,
+                  int64_t D_in, int64_t D_out, int bits, int group, double *Y)
+{
+    const int off = 1 << (bits - 1);
+    double *wd = (double *)malloc((size_t)(D_in * D_out) * sizeof(double));
+    for (int64_t k = 0; k < D_in; ++k)
+        for (int64_t n = 0; n < D_out; ++n) {
+            const uint32_t word = packed[(k / 8) * D_out + n];
+            const int u = (int)((word >> (4 * (k % 8))) & 0xFu);
+            wd[k * D_out + n] = (double)(u - off) * (double)scales[(k / group) * D_out + n] / (double)s[k];
+        }
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < N; ++t) {
+        for (int64_t n = 0; n < D_out; ++n)
+            Y[t * D_out + n] = 0.0;
+        for (int64_t k = 0; k < D_in; ++k) {
+            const double x = bf16_bits_to_double(X[t * D_in + k]);
+            if (x == 0.0)
+                continue;
+            const double *wr = wd + k * D_out;
+            double *yr = Y + t * D_out;
+            for (int64_t n = 0; n < D_out; ++n)
+                yr[n] += x * wr[n];
+        }
+    }
+    free(wd);
+}
+

@@ -330,3 +330,31 @@ def test_delta16_codes_round_with_the_half_delta():
     Wp[:, 1] = np.linspace(-0.875, 0.5, 32)      # max 0.875 -> delta 0.125
     Wp[:, 2] = np.linspace(-14, 3, 32)           # max 14 -> delta 2
     assert np.array_equal(oracle.quantize(Wp, None, 4, 32, delta16=True)[0], oracle.quantize(Wp, None, 4, 32)[0])
+
+
+# ------------------------------------------------------------------ the quantised layer (W4A16 consumer)
+def test_w4a16_exact_on_representable_weights():
+    """Weights that are integer multiples of a power-of-two delta, with s = 1,
+    quantise exactly, so the layer output is X W (numpy matmul)."""
+    rng = np.random.default_rng(61)
+    D_in, D_out, N = 128, 24, 5
+    codes = rng.integers(-7, 8, size=(D_in, D_out))
+    codes[0] = 7                                      # every group reaches qmax: delta = 0.25 exactly
+    W = (codes * 0.25).astype(np.float32)
+    X = torch.randn(N, D_in, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    q, d = oracle.quantize(W, None, 4, 128)
+    assert np.all(d == 0.25) and np.array_equal(q, codes)
+    Y = oracle.w4a16(X, np.ones(D_in, np.float32), oracle.pack(q, 4), d, 4, 128)
+    assert np.allclose(Y, X.double().numpy() @ W.astype(np.float64), rtol=1e-12, atol=1e-12)
+
+
+def test_w4a16_is_the_dequantised_search_operand():
+    """With scales s the output is X S^-1 Q(S W): the same weights the search's
+    loss dequantises, checked with a numpy matmul on the oracle's codes."""
+    X, W = synth.layer_inputs(synth.small_layer(6, 256, 40, seed=62))
+    s = oracle.scales(oracle.act_stats(X).astype(np.float32), 0.5)
+    for bits, group in ((4, 128), (3, 64), (2, 32)):
+        q, d = oracle.quantize(W, s, bits, group)
+        w_hat = q * np.repeat(d, group, axis=0).astype(np.float64) / s.astype(np.float64)[:, None]
+        Y = oracle.w4a16(X, s, oracle.pack(q, bits), d, bits, group)
+        assert np.allclose(Y, X.double().numpy() @ w_hat, rtol=1e-12, atol=1e-12)
