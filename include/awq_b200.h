@@ -266,6 +266,24 @@ AWQ_API int awq_quantize_pack_ex(const float* W, const float* s, const float* cl
                                  int bits, int group, int flags, uint32_t* packed, void* scales, void* stream);
 
 /*
+ * The quantised layer applied to activations, the consumer of the pack
+ * format (compassingai.com AWQ concept page, "inference-time equivalent":
+ * the INT4 weights with s* kept as metadata and 1/s* folded into the input):
+ *     Y[t][n] = sum_k x_tk / s_k * (u_kn - 2^(bits-1)) * scales[k/group][n]
+ * with u the offset-binary codes of `packed` (the layout of
+ * awq_quantize_pack).  The weights are dequantised into shared memory as
+ * bf16(q * fl(delta / s_k)) (one rounding each) and multiplied on the tensor
+ * cores with fp32 accumulation; at small N the K dimension is split over a
+ * cluster of CTAs whose partial sums fold in a fixed order.
+ *   X       [N][D_in] bf16;  s [D_in] fp32 (s*);  packed [D_in/8][D_out] uint32
+ *   scales  [D_in/group][D_out] fp32;  bits 2..4;  group 32, 64 or 128
+ *   Y       [N][D_out] fp32 output
+ *   status  [1] int32 device status word (required), as for awq_search
+ */
+AWQ_API int awq_w4a16_gemm(const void* X, const float* s, const uint32_t* packed, const float* scales, int64_t N,
+                           int64_t D_in, int64_t D_out, int bits, int group, float* Y, int32_t* status, void* stream);
+
+/*
  * The layer's reference output Y = X bf16(W) computed by the search's own
  * tensor-core GEMM (the X W term of the loss, concept page flow step 4c), fp32.
  *   Y          [N][D_out] fp32 output
@@ -328,7 +346,8 @@ enum {
   AWQ_STAGE_CLIP_GRAM = 7,     /* awq_clip_search: X^T and the group Gram blocks X_g^T X_g */
   AWQ_STAGE_CLIP_OPERAND = 8,  /* awq_clip_search: bf16 operand per clip ratio */
   AWQ_STAGE_CLIP_LOSS = 9,     /* awq_clip_search: e^T H_g e per (ratio, group, column), argmin */
-  AWQ_NUM_STAGES = 10
+  AWQ_STAGE_W4A16 = 10,        /* awq_w4a16_gemm */
+  AWQ_NUM_STAGES = 11
 };
 AWQ_API int awq_profile_enable(int on);
 AWQ_API int awq_profile_reset(void);

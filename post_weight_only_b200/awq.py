@@ -29,10 +29,10 @@ EXPORTS = (
     "awq_layer_output_workspace_size", "awq_layer_output", "awq_selftest_wait_timeout",
     "awq_get_last_error", "awq_version", "awq_profile_enable", "awq_profile_reset", "awq_profile_read",
     "awq_search_noalloc", "awq_clip_search_workspace_size", "awq_clip_search", "awq_quantize_pack_clip",
-    "awq_search_joint_workspace_size", "awq_search_joint", "awq_quantize_pack_ex",
+    "awq_search_joint_workspace_size", "awq_search_joint", "awq_quantize_pack_ex", "awq_w4a16_gemm",
 )
 STAGES = ("act_stats", "scale_table", "search_operand", "search_gemm", "loss_reduce", "quantize_pack",
-          "weight_t", "clip_gram", "clip_operand", "clip_loss")
+          "weight_t", "clip_gram", "clip_operand", "clip_loss", "w4a16")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -82,6 +82,7 @@ _pack_clip = _sig("awq_quantize_pack_clip", I, [P, P, P, I64, I64, I, I, P, P, P
 _joint_ws = _sig("awq_search_joint_workspace_size", SZ, [I64, I64, P, I, I, I, I, I])
 _pack_ex = _sig("awq_quantize_pack_ex", I, [P, P, P, I64, I64, I, I, I, P, P, P])
 PACK_DELTA_FP16 = 1
+_w4a16 = _sig("awq_w4a16_gemm", I, [P, P, P, P, I64, I64, I64, I, I, P, P, P])
 _joint = _sig("awq_search_joint", I, [P, P, P, I, P, I64, I64, P, I, I, I, I, P, P, P, P, P, SZ, P, P])
 
 
@@ -250,6 +251,26 @@ def quantize_pack_ex(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int
     _check(_pack_ex(_ptr(W), _ptr(s), _ptr(clip), D_in, D_out, bits, group, PACK_DELTA_FP16 if delta_fp16 else 0,
                     _ptr(packed), _ptr(sc), _stream()))
     return packed, sc
+
+
+def w4a16_gemm(X: torch.Tensor, s: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, bits: int = 4,
+               group: int = 128, check_status: bool = True) -> torch.Tensor:
+    """Y = X diag(1/s) Dequant(packed, scales), fp32: ``awq_w4a16_gemm``."""
+    X = _dev(X, torch.bfloat16, "X")
+    s = _dev(s, torch.float32, "s")
+    if packed.dtype not in (torch.int32, torch.uint32):
+        raise ValueError("packed must hold 32-bit words")
+    packed = packed.contiguous()
+    scales = _dev(scales, torch.float32, "scales")
+    N, D_in = X.shape
+    D_out = packed.shape[1]
+    Y = torch.empty(N, D_out, dtype=torch.float32, device=X.device)
+    status = torch.zeros(1, dtype=torch.int32, device=X.device)
+    _check(_w4a16(_ptr(X), _ptr(s), _ptr(packed), _ptr(scales), N, D_in, D_out, bits, group, _ptr(Y), _ptr(status),
+                  _stream()))
+    if check_status:
+        check_device_status(status)
+    return Y
 
 
 def quantize_pack_clip(W: torch.Tensor, s: torch.Tensor, clip: torch.Tensor, bits: int = 4, group: int = 128):

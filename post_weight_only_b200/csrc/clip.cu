@@ -35,17 +35,6 @@ namespace {
 enum ClipSite { kSiteGramFull = 16, kSiteGramEmpty, kSiteGramAcc, kSiteLossAFull, kSiteLossAEmpty, kSiteLossHFull,
                 kSiteLossHEmpty, kSiteLossAccFull, kSiteLossAccEmpty };
 
-// ---------------------------------------------------------------- helpers
-__device__ __forceinline__ void mma_ss_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                           uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // ---------------------------------------------------------------- transpose, reciprocal
 __global__ void __launch_bounds__(256)
     xt_kernel(const uint16_t* __restrict__ X, int64_t N, int64_t D, int64_t Np, uint16_t* __restrict__ XT) {
@@ -139,7 +128,7 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         const uint64_t desc = sw128_kmajor_desc(smem_u32(smem + s * kGramTile));
 #pragma unroll
-        for (int j = 0; j < 4; ++j) mma_ss_f16(tbase, desc + 2 * j, desc + 2 * j, idesc, (kb | j) != 0 ? 1u : 0u);
+        for (int j = 0; j < 4; ++j) mma_ss_f16_cta(tbase, desc + 2 * j, desc + 2 * j, idesc, (kb | j) != 0 ? 1u : 0u);
         mma_commit(&empty[s]);
       }
       aborted = !ok;
@@ -326,7 +315,7 @@ __global__ void __launch_bounds__(kLossThreads, 1)
             const uint64_t bdesc = sw128_kmajor_desc(smem_u32(h_sm + kb * (G * 64 * 2)));
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              mma_ss_f16(tbase + b * G, adesc + 2 * j, bdesc + 2 * j, idesc, (kb | j) != 0 ? 1u : 0u);
+              mma_ss_f16_cta(tbase + b * G, adesc + 2 * j, bdesc + 2 * j, idesc, (kb | j) != 0 ? 1u : 0u);
           }
           mma_commit(&acc_full[b]);
         }

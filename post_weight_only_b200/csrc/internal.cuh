@@ -106,6 +106,14 @@ int launch_clip_loss(const uint16_t* op, const uint16_t* Hb, int64_t D_in, int64
                      const AlphaList& clips, int n_clip, float* clip_out, int* idx_out, float* loss_out, int num_sms,
                      int* status, uint64_t timeout_ns, cudaStream_t st, cudaError_t* cerr, const char** what);
 
+// ---- w4a16.cu (the quantised layer applied to activations)
+// Y [N][D_out] fp32 = X diag(1/s) Dequant(packed, scales), tcgen05 with the
+// weights dequantised into shared memory; split K over a cluster when the
+// output has few tiles.
+int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const float* scales, int64_t N, int64_t D_in,
+                 int64_t D_out, int bits, int group, float* Y, int num_sms, int* status, uint64_t timeout_ns,
+                 cudaStream_t st, cudaError_t* cerr, const char** what);
+
 // Self-test of the bounded wait: one CTA waits on an mbarrier that nothing
 // arrives at, gives up after timeout_ns and records the timeout in *status.
 cudaError_t launch_wait_timeout_selftest(int* status, uint64_t timeout_ns, cudaStream_t st);
