@@ -53,6 +53,7 @@ def parse_args():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clip", action="store_true", help="skip timing the weight-clipping search")
+    ap.add_argument("--no-w4a16", action="store_true", help="skip timing the W4A16 consumer kernel")
     ap.add_argument("--no-at-scale", action="store_true",
                     help="skip timing the statistic and pack kernels on the 70B block's largest operands")
     ap.add_argument("--loss-form", choices=("error", "reference"), default="error")
@@ -453,6 +454,36 @@ def run_ours(args):
             "frac_clipped": float((cr.idx > 0).float().mean().item()),
         }
 
+    # ---------------- the W4A16 consumer of the pack format (not part of the step)
+    w4_info = None
+    if not args.no_w4a16:
+        g4 = torch.Generator(device=dev).manual_seed(4321 + rank)
+        w4_info = {}
+        for name, (Dk, Dn, Ns) in (("down_proj_28672x8192", (28672, 8192, (1, 16))),
+                                    ("attn_proj_4096x4096", (4096, 4096, (1, 16, 4096)))):
+            packed_q = torch.randint(-2 ** 31, 2 ** 31 - 1, (Dk // 8, Dn), generator=g4, device=dev,
+                                     dtype=torch.int64).to(torch.int32)
+            scales_q = torch.rand(Dk // group, Dn, generator=g4, device=dev) * 0.01 + 1e-3
+            s_q = torch.rand(Dk, generator=g4, device=dev) + 0.5
+            weights = rotating(packed_q)
+            w_bytes = Dk * Dn // 2 + (Dk // group) * Dn * 4
+            for Nq in Ns:
+                Xq = torch.randn(Nq, Dk, generator=g4, device=dev).to(torch.bfloat16)
+                ws_q = torch.empty(awq.w4a16_workspace_size(Nq, Dk, Dn), dtype=torch.uint8, device=dev)
+                ms = loop_ms(lambda pk: awq.w4a16_gemm(Xq, s_q, pk, scales_q, bits, group, check_status=False,
+                                                       workspace=ws_q), weights, reps=20)
+                # algorithmic bytes: packed words, deltas, X and s read once, Y
+                # written once (the scaled copy of X in the workspace is not counted)
+                nbytes = w_bytes + Nq * Dk * 2 + Nq * Dn * 4 + Dk * 4
+                gbs = nbytes / (ms / 1e3) / 1e9
+                tf = 2.0 * Nq * Dk * Dn / (ms / 1e3) / 1e12
+                w4_info[f"{name}_N{Nq}"] = {
+                    "ms": ms, "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
+                    "frac_hbm": gbs / float(load_peaks()[0]["hbm_gbs"]), "tflops": tf,
+                    "frac_bf16": tf / float(load_peaks()[0]["bf16_tflops"])}
+            del weights, packed_q
+        torch.cuda.empty_cache()
+
     def hbm(stage, nbytes):
         ms, n = prof[stage]
         if n == 0:
@@ -486,6 +517,7 @@ def run_ours(args):
                         "search_operand": hbm("search_operand", operand_bytes)},
         "hbm_kernels_at_scale": at_scale or None,
         "clip_search": clip_info,
+        "w4a16": w4_info,
         "kernels": kernels,
         "e2e": {"value": A * world / (e2e_per_step / 1e3), "unit": UNIT, "ms_per_step": e2e_per_step,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

@@ -24,9 +24,8 @@
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
  *     only enqueue work; they are asynchronous with respect to the host and
  *     do not synchronise.  Scratch space comes from a caller-provided
- *     workspace whose size is queried; the one exception is awq_act_stats,
- *     which takes a small stream-ordered scratch from the device's default
- *     memory pool (see there).  The library calls no other allocator.
+ *     workspace whose size is queried (or, for awq_search_noalloc, a fixed
+ *     array inside the library).  The library calls no allocator.
  *   - The return value is an awq_status.  A non-OK status from argument
  *     checking is returned before any work is enqueued; awq_get_last_error()
  *     then describes it.  Errors found on the device (a wait that timed out)
@@ -88,11 +87,8 @@ enum { AWQ_LOSS_ERROR = 0, AWQ_LOSS_REFERENCE = 1 };
  *   stat  AWQ_STAT_MEAN: a_j = (sum_i |X_ij|) / N, summed in fp32 in a fixed
  *         order (bit-reproducible); AWQ_STAT_MAX: a_j = max_i |X_ij| (exact)
  *   a     [D_in] fp32 output
- * When the rows are split over several CTAs (the usual case: the work is cut
- * into about one CTA per SM), the per-CTA partial rows go to a scratch of at
- * most (number of SMs) x 1024 floats (about 0.6 MB on B200) taken with
- * cudaMallocAsync and released with cudaFreeAsync on `stream` (capturable in
- * a CUDA graph); a failure of that allocation returns AWQ_ECUDA.
+ * The rows are split over the two CTAs of a cluster pair, which fold their
+ * partial rows through distributed shared memory: no scratch is used.
  */
 AWQ_API int awq_act_stats(const void* X, int64_t N, int64_t D_in, int stat, float* a, void* stream);
 
@@ -268,20 +264,30 @@ AWQ_API int awq_quantize_pack_ex(const float* W, const float* s, const float* cl
 /*
  * The quantised layer applied to activations, the consumer of the pack
  * format (compassingai.com AWQ concept page, "inference-time equivalent":
- * the INT4 weights with s* kept as metadata and 1/s* folded into the input):
+ * the INT4 weights with s* kept as metadata and 1/s* folded into the input;
+ * AWQ paper, TinyChat section, "on-the-fly weight dequantization"):
  *     Y[t][n] = sum_k x_tk / s_k * (u_kn - 2^(bits-1)) * scales[k/group][n]
  * with u the offset-binary codes of `packed` (the layout of
- * awq_quantize_pack).  The weights are dequantised into shared memory as
- * bf16(q * fl(delta / s_k)) (one rounding each) and multiplied on the tensor
- * cores with fp32 accumulation; at small N the K dimension is split over a
- * cluster of CTAs whose partial sums fold in a fixed order.
- *   X       [N][D_in] bf16;  s [D_in] fp32 (s*);  packed [D_in/8][D_out] uint32
- *   scales  [D_in/group][D_out] fp32;  bits 2..4;  group 32, 64 or 128
- *   Y       [N][D_out] fp32 output
- *   status  [1] int32 device status word (required), as for awq_search
+ * awq_quantize_pack).  Two launches on `stream`: X' = bf16(X / s) into the
+ * workspace, then a tensor-core GEMM that dequantises the weights into
+ * shared memory as bf16((u - 2^(bits-1)) * bf16(delta)) (one rounding of the
+ * product) and accumulates in fp32.  For N <= 64 the k blocks of all output
+ * tiles are shared out evenly over the CTAs (stream-K); a tile split between
+ * CTAs is summed from partial tiles in the workspace in a fixed order, so
+ * the result is deterministic.
+ *   X         [N][D_in] bf16;  s [D_in] fp32 (s*);  packed [D_in/8][D_out] uint32
+ *   scales    [D_in/group][D_out] fp32;  bits 2..4;  group 32, 64 or 128
+ *   D_out     a multiple of 4 (the rows of packed words are read by TMA)
+ *   Y         [N][D_out] fp32 output
+ *   workspace at least awq_w4a16_workspace_size(N, D_in, D_out) bytes: the
+ *             scaled activations (N x D_in bf16) and, for N <= 64, room for
+ *             the partial tiles.  No device is needed to compute the size.
+ *   status    [1] int32 device status word (required), as for awq_search
  */
+AWQ_API size_t awq_w4a16_workspace_size(int64_t N, int64_t D_in, int64_t D_out);
 AWQ_API int awq_w4a16_gemm(const void* X, const float* s, const uint32_t* packed, const float* scales, int64_t N,
-                           int64_t D_in, int64_t D_out, int bits, int group, float* Y, int32_t* status, void* stream);
+                           int64_t D_in, int64_t D_out, int bits, int group, float* Y, void* workspace,
+                           size_t workspace_bytes, int32_t* status, void* stream);
 
 /*
  * The layer's reference output Y = X bf16(W) computed by the search's own

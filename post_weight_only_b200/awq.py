@@ -30,6 +30,7 @@ EXPORTS = (
     "awq_get_last_error", "awq_version", "awq_profile_enable", "awq_profile_reset", "awq_profile_read",
     "awq_search_noalloc", "awq_clip_search_workspace_size", "awq_clip_search", "awq_quantize_pack_clip",
     "awq_search_joint_workspace_size", "awq_search_joint", "awq_quantize_pack_ex", "awq_w4a16_gemm",
+    "awq_w4a16_workspace_size",
 )
 STAGES = ("act_stats", "scale_table", "search_operand", "search_gemm", "loss_reduce", "quantize_pack",
           "weight_t", "clip_gram", "clip_operand", "clip_loss", "w4a16")
@@ -82,7 +83,8 @@ _pack_clip = _sig("awq_quantize_pack_clip", I, [P, P, P, I64, I64, I, I, P, P, P
 _joint_ws = _sig("awq_search_joint_workspace_size", SZ, [I64, I64, P, I, I, I, I, I])
 _pack_ex = _sig("awq_quantize_pack_ex", I, [P, P, P, I64, I64, I, I, I, P, P, P])
 PACK_DELTA_FP16 = 1
-_w4a16 = _sig("awq_w4a16_gemm", I, [P, P, P, P, I64, I64, I64, I, I, P, P, P])
+_w4a16 = _sig("awq_w4a16_gemm", I, [P, P, P, P, I64, I64, I64, I, I, P, P, SZ, P, P])
+_w4a16_ws = _sig("awq_w4a16_workspace_size", SZ, [I64, I64, I64])
 _joint = _sig("awq_search_joint", I, [P, P, P, I, P, I64, I64, P, I, I, I, I, P, P, P, P, P, SZ, P, P])
 
 
@@ -254,8 +256,11 @@ def quantize_pack_ex(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int
 
 
 def w4a16_gemm(X: torch.Tensor, s: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, bits: int = 4,
-               group: int = 128, check_status: bool = True) -> torch.Tensor:
-    """Y = X diag(1/s) Dequant(packed, scales), fp32: ``awq_w4a16_gemm``."""
+               group: int = 128, check_status: bool = True,
+               workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y = X diag(1/s) Dequant(packed, scales), fp32: ``awq_w4a16_gemm``.
+    ``workspace`` (uint8, at least ``w4a16_workspace_size(N, D_in, D_out)`` bytes)
+    is allocated per call when not given."""
     X = _dev(X, torch.bfloat16, "X")
     s = _dev(s, torch.float32, "s")
     if packed.dtype not in (torch.int32, torch.uint32):
@@ -266,11 +271,18 @@ def w4a16_gemm(X: torch.Tensor, s: torch.Tensor, packed: torch.Tensor, scales: t
     D_out = packed.shape[1]
     Y = torch.empty(N, D_out, dtype=torch.float32, device=X.device)
     status = torch.zeros(1, dtype=torch.int32, device=X.device)
-    _check(_w4a16(_ptr(X), _ptr(s), _ptr(packed), _ptr(scales), N, D_in, D_out, bits, group, _ptr(Y), _ptr(status),
-                  _stream()))
+    nbytes = _w4a16_ws(N, D_in, D_out)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=X.device)
+    _check(_w4a16(_ptr(X), _ptr(s), _ptr(packed), _ptr(scales), N, D_in, D_out, bits, group, _ptr(Y),
+                  _ptr(workspace), workspace.numel(), _ptr(status), _stream()))
     if check_status:
         check_device_status(status)
     return Y
+
+
+def w4a16_workspace_size(N: int, D_in: int, D_out: int) -> int:
+    return int(_w4a16_ws(N, D_in, D_out))
 
 
 def quantize_pack_clip(W: torch.Tensor, s: torch.Tensor, clip: torch.Tensor, bits: int = 4, group: int = 128):

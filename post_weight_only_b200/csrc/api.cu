@@ -729,18 +729,30 @@ int awq_search_joint(const void* X, const float* const* Ws, const int64_t* D_out
   return AWQ_OK;
 }
 
+size_t awq_w4a16_workspace_size(int64_t N, int64_t D_in, int64_t D_out) {
+  if (N < 1 || D_in < 1 || D_out < 1) return 0;
+  return awq::w4a16_scratch_bytes(N, D_in, D_out) + 256;
+}
+
 int awq_w4a16_gemm(const void* X, const float* s, const uint32_t* packed, const float* scales, int64_t N,
-                   int64_t D_in, int64_t D_out, int bits, int group, float* Y, int32_t* status, void* stream) {
+                   int64_t D_in, int64_t D_out, int bits, int group, float* Y, void* workspace,
+                   size_t workspace_bytes, int32_t* status, void* stream) {
   if (N < 1 || N > kMaxDim) return fail(AWQ_EINVAL, "N = %lld: need 1 <= N <= 2^24", (long long)N);
   AWQ_TRY(check_quant_args(bits, group));
   if (D_in < group || D_in > kMaxDin || D_in % group)
     return fail(AWQ_EINVAL, "D_in = %lld: need a positive multiple of group = %d", (long long)D_in, group);
-  if (D_out < 1 || D_out > kMaxDim) return fail(AWQ_EINVAL, "D_out = %lld out of range", (long long)D_out);
+  if (D_out < 4 || D_out > kMaxDim || D_out % 4)
+    return fail(AWQ_EINVAL, "D_out = %lld: need a positive multiple of 4 (rows of packed words are read by TMA)",
+                (long long)D_out);
   AWQ_TRY(check_ptr(X, "X", 16));
-  AWQ_TRY(check_ptr(s, "s", 4));
-  AWQ_TRY(check_ptr(packed, "packed", 4));
-  AWQ_TRY(check_ptr(scales, "scales", 4));
+  AWQ_TRY(check_ptr(s, "s", 16));
+  AWQ_TRY(check_ptr(packed, "packed", 16));
+  AWQ_TRY(check_ptr(scales, "scales", 16));
   AWQ_TRY(check_ptr(Y, "Y", 4));
+  if (!workspace) return fail(AWQ_EWORKSPACE, "workspace is NULL");
+  const size_t need = awq_w4a16_workspace_size(N, D_in, D_out);
+  if (workspace_bytes < need) return fail(AWQ_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+  void* xs = reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(workspace) + 255) & ~uintptr_t(255));
   if (!status) return fail(AWQ_EINVAL, "status is NULL");
   AWQ_TRY(check_ptr(status, "status", 4));
   int sms = 0;
@@ -752,8 +764,8 @@ int awq_w4a16_gemm(const void* X, const float* s, const uint32_t* packed, const 
   int rc;
   {
     StageTimer t(AWQ_STAGE_W4A16, st);
-    rc = awq::launch_w4a16(X, s, packed, scales, N, D_in, D_out, bits, group, Y, sms, status, timeout_ns(), st, &e,
-                           &what);
+    rc = awq::launch_w4a16(X, s, packed, scales, N, D_in, D_out, bits, group, Y, xs, sms, status, timeout_ns(), st,
+                           &e, &what);
   }
   if (rc != AWQ_OK) return e != cudaSuccess ? fail_cuda(e, what) : fail(rc, "%s failed", what);
   return AWQ_OK;

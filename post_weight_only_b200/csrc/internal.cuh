@@ -19,8 +19,7 @@ struct AlphaList {
 };
 
 // ---- act_stats.cu
-// Uses a stream-ordered scratch of at most about num_sms x 1024 floats (from
-// the device's default memory pool) when the rows are split over CTAs.
+// No scratch: the row split folds through distributed shared memory.
 cudaError_t launch_act_stats(const uint16_t* X, int64_t N, int64_t D, int stat, float* a, int num_sms,
                              cudaStream_t st);
 
@@ -90,6 +89,12 @@ int launch_search(const SearchShape& sh, const SearchBuffers& b, int grid, uint6
 // `rows` rows, `planes` planes (0: a 2-D map); box box_inner x box_rows.
 bool make_bf16_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t planes,
                    uint32_t box_inner, uint32_t box_rows);
+// 3-D bf16 map (128-byte swizzle) with byte strides of dimensions 1 and 2.
+bool make_bf16_map_3d(CUtensorMap* m, const void* base, const uint64_t dims[3], const uint64_t strides[2],
+                      const uint32_t box[3]);
+// Unswizzled TMA map over rows of `inner` 4-byte elements (fp32 or uint32).
+bool make_word_map(CUtensorMap* m, const void* base, bool is_float, uint64_t inner, uint64_t rows,
+                   uint32_t box_inner, uint32_t box_rows);
 
 // ---- clip.cu (the weight-clipping search)
 // XT [D][Np] = X^T, tokens padded with zeros to Np (a multiple of 8).
@@ -108,11 +113,14 @@ int launch_clip_loss(const uint16_t* op, const uint16_t* Hb, int64_t D_in, int64
 
 // ---- w4a16.cu (the quantised layer applied to activations)
 // Y [N][D_out] fp32 = X diag(1/s) Dequant(packed, scales), tcgen05 with the
-// weights dequantised into shared memory; split K over a cluster when the
-// output has few tiles.
+// weights dequantised into shared memory; stream-K over the k blocks when
+// the token tile is small.  ws: scratch of w4a16_scratch_bytes(N, D_in, D_out)
+// bytes, 256-byte aligned (scaled activations, stream-K partial tiles).
+// D_out must be a multiple of 4.
+size_t w4a16_scratch_bytes(int64_t N, int64_t D_in, int64_t D_out);
 int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const float* scales, int64_t N, int64_t D_in,
-                 int64_t D_out, int bits, int group, float* Y, int num_sms, int* status, uint64_t timeout_ns,
-                 cudaStream_t st, cudaError_t* cerr, const char** what);
+                 int64_t D_out, int bits, int group, float* Y, void* ws, int num_sms, int* status,
+                 uint64_t timeout_ns, cudaStream_t st, cudaError_t* cerr, const char** what);
 
 // Self-test of the bounded wait: one CTA waits on an mbarrier that nothing
 // arrives at, gives up after timeout_ns and records the timeout in *status.

@@ -496,6 +496,36 @@ bool make_bf16_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t ro
   return r == CUDA_SUCCESS;
 }
 
+// A 3-D bf16 map with explicit byte strides for dimensions 1 and 2 (any
+// order of strides; each a multiple of 16 bytes), 128-byte swizzle.
+bool make_bf16_map_3d(CUtensorMap* m, const void* base, const uint64_t dims[3], const uint64_t strides[2],
+                      const uint32_t box[3]) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const uint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// An unswizzled TMA map over a row-major 2-D array of 4-byte elements
+// (uint32 or fp32): `inner` contiguous elements per row, `rows` rows, box
+// box_inner x box_rows.
+bool make_word_map(CUtensorMap* m, const void* base, bool is_float, uint64_t inner, uint64_t rows,
+                   uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t dims[2] = {inner, rows};
+  const uint64_t str[1] = {inner * 4};
+  const uint32_t box[2] = {box_inner, box_rows};
+  const uint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, is_float ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT32, 2,
+                  const_cast<void*>(base), dims, str, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int search_token_tiles(int N) { return (N + kBN - 1) / kBN; }
 
 int search_partial_rows(int N) { return 2 * search_token_tiles(N); }

@@ -2,103 +2,208 @@
 //     Y = X diag(1/s) Dequant(W_q),   Dequant(W_q)[k][n] = (u_kn - 2^(b-1)) delta_{k/G, n},
 // straight from the packed offset-binary words of awq_quantize_pack
 // (compassingai.com AWQ concept page, "inference-time equivalent": the INT4
-// weights with s* kept as metadata and 1/s* folded into the input).
+// weights with s* kept as metadata and 1/s* folded into the input; AWQ paper,
+// TinyChat section, "on-the-fly weight dequantization": the integers are
+// turned into 16-bit floats inside the GEMM's main loop).
 //
-// tcgen05 GEMM (cta_group::1): D[n][t] = sum_k A[n][k] B[t][k] with
-//   A  the dequantised weight tile (M = 128 output columns, 64 k per stage,
-//      K-major bf16, 128-byte swizzle), produced in shared memory by the
-//      producer warps: A[n][k] = bf16(q_kn * fl(delta * (1/s_k))), one
-//      rounding per weight (the search's reference-form operand);
-//   B  the X tile (N = Nt tokens, Nt a multiple of 16 up to 256), by TMA.
-// A thread of the producer warps owns one output column: per stage it loads
-// the column's eight packed words (coalesced across the columns) and turns
-// each into one 16-byte chunk of its row of A.
+// Two launches:
+//   1. scale_x: X' = bf16(X / s) into scratch, rows padded with zeros to a
+//      multiple of 64 columns (so that a k block never crosses a row), each
+//      run of 8 columns stored in the order 0,4,1,5,2,6,3,7.  A packed word holds rows 8j..8j+7 as
+//      nibbles 0..7; one mask-and-OR of (word >> 4i) with 0x000F000F |
+//      0x43004300 gives the bf16 pair {128 + u_{8j+i}, 128 + u_{8j+i+4}}
+//      (exact), so with that order of X' the pairs go straight into the
+//      K-major A tile (the same reason the paper's GPU packing interleaves
+//      the weights; the permutation sits on the activation side here so
+//      that the pack format keeps its natural order).
+//   2. the GEMM (tcgen05, cta_group::1): D[n][t] = sum_k A[n][k] X'[t][k]
+//      with A the dequantised weight tile, 128 output columns x 64 k per
+//      k block, bf16((u - 2^(b-1)) * bf16(delta)): the subtraction is exact
+//      and the product is rounded once.
 //
-// Split K: with few output tiles (small N), a cluster of KS CTAs shares one
-// tile, each CTA a contiguous range of k blocks; the partial tiles fold
-// through distributed shared memory in rank order (deterministic).
+// A stage holds KPS consecutive k blocks of one unit: the X' planes
+// [KPS][Nt][64] (one 3-D box, 128-byte swizzle), the packed words
+// [8 KPS][128] (one TMA box) and their scale rows (one box).  On B200 a
+// thread that issues TMA loads and waits for them streams at a rate set by
+// the number of loads it keeps going rather than their size, so the small
+// token tiles (memory-bound) take KPS = 4 (a 16 KiB box of packed words) and
+// two issuing warps that fill alternate stages; large token tiles take
+// KPS = 1 (the X' box alone is 32 KiB) and one issuing warp.
 //
-// Roles (192 threads): warp 0 TMA of X, warp 1 TMEM allocation and MMA issue
-// (lane 0), warps 2-5 producers and then the epilogue (warp w owns TMEM lane
-// quarter w % 4 = columns 32 (w % 4) .. + 31 of the tile).  Every mbarrier
-// wait is bounded.
-#include <cooperative_groups.h>
+// Roles (480 threads):
+//   warps 0-1   TMA issue (lane 0).
+//   warp 2      TMEM allocation and MMA issue (lane 0) into one of two
+//               accumulators, so that a unit's epilogue overlaps the next
+//               unit's main loop.
+//   warps 3-10  dequantisers: thread (n, h) owns column n of the tile and
+//               half h of each k block; it reads its 4 words per k block from
+//               the stage (conflict-free, the words of a k8 row are
+//               contiguous over n) and writes chunks 4h..4h+3 of row n of
+//               the A tile.
+//   warps 11-14 epilogue: TMEM lanes 32 (w % 4) .. + 31 -> Y.
+// Work: a unit is a 128-column x Nt-token output tile of KBS = ceil(KB /
+// KPS) stage steps.  Large N: units are dealt out to a persistent grid,
+// whole.  N <= 64: stream-K -- the units x KBS steps are cut into equal
+// contiguous shares, one per CTA, so that every SM streams the same number
+// of packed bytes.  A unit split between CTAs is summed from partial tiles
+// in the workspace by the CTA that finishes it last (an atomic count per
+// unit), always in CTA order: the result does not depend on timing.  Every
+// mbarrier wait is bounded.
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
 #include "internal.cuh"
 #include "ptx.cuh"
 
-namespace cg = cooperative_groups;
-
 namespace awq {
 namespace {
 
-constexpr int kW4Threads = 192;
-constexpr int kW4ABytes = 128 * 64 * 2;          // one A stage
-constexpr int kW4MaxFoldTokens = 64;             // split K only for token tiles up to this
+constexpr int kW4Threads = 480;
+constexpr int kW4TmaWarps = 2;
+constexpr int kW4MmaWarp = 2;
+constexpr int kW4DqWarp0 = 3;
+constexpr int kW4DqWarps = 8;
+constexpr int kW4EpiWarp0 = kW4DqWarp0 + kW4DqWarps;   // 11
+constexpr int kW4ABytes = 128 * 64 * 2;          // one dequantised A tile
+constexpr int kW4PkBytes = 8 * 128 * 4;          // the packed words of one k block
+constexpr int kW4MaxStreamTokens = 64;           // stream-K for token tiles up to this
+constexpr int kW4MaxStages = 16;
+constexpr int kW4MaxGrid = 512;                  // bounds the partial-tile workspace
+constexpr uint32_t kW4SleepNs = 20000;           // suspend hint of the waits
 
-enum W4Site { kSiteW4XEmpty = 40, kSiteW4XFull, kSiteW4AEmpty, kSiteW4AFull, kSiteW4Acc };
+enum W4Site {
+  kSiteW4WEmpty = 40, kSiteW4WFull, kSiteW4AEmpty, kSiteW4AFull, kSiteW4AccEmpty, kSiteW4AccFull, kSiteW4Done
+};
 
 struct W4Params {
-  const uint32_t* packed;   // [D_in/8][D_out]
-  const float* scales;      // [D_in/G][D_out]
-  const float* s;           // [D_in]
   float* Y;                 // [N][D_out]
-  int64_t N, D_in, D_out;
-  int bits, Nt, KB, KS, n_tiles, stages;
+  float* partial;           // stream-K: [grid][2][N][128] partial tiles
+  int* count;               // stream-K: [units] contributions received (zeroed by scale_x)
+  int64_t N, D_out;
+  int off;                  // 2^(bits-1)
+  int Nt, KB, kps, KBS, n_tiles, units;
+  int stream;               // 1: stream-K over units x KBS steps, `chunk` steps per CTA
+  int issuers;              // TMA warps that fill alternate stages (1 or 2)
+  int64_t chunk, total;
+  int stages, a_stages, stage_bytes, scale_rows, tcols;
   int* status;
   unsigned long long timeout_ns;
 };
+
+// The segments of work of CTA c, in order: (unit, first step, end step).
+struct SegCursor {
+  int64_t f, f1;
+};
+__device__ __forceinline__ SegCursor seg_begin(const W4Params& p, int c) {
+  if (p.stream) {
+    const int64_t f0 = c * p.chunk;
+    return {f0, f0 + p.chunk < p.total ? f0 + p.chunk : p.total};
+  }
+  return {c, p.units};
+}
+__device__ __forceinline__ bool seg_next(SegCursor& cur, const W4Params& p, int& u, int& ka, int& kb) {
+  if (cur.f >= cur.f1) return false;
+  if (p.stream) {
+    u = static_cast<int>(cur.f / p.KBS);
+    ka = static_cast<int>(cur.f - static_cast<int64_t>(u) * p.KBS);
+    const int64_t left = cur.f1 - cur.f;
+    kb = left < p.KBS - ka ? ka + static_cast<int>(left) : p.KBS;
+    cur.f += kb - ka;
+  } else {
+    u = static_cast<int>(cur.f);
+    ka = 0;
+    kb = p.KBS;
+    cur.f += gridDim.x;
+  }
+  return true;
+}
+
+// ------------------------------------------------------------ X' = X / s
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t h) { return __uint_as_float(h << 16); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
+// One thread per run of 8 columns of X' [N][P8 * 8]; runs j >= D8 are the zero pad.
+__global__ void __launch_bounds__(256) scale_x_kernel(const uint4* __restrict__ X, const float4* __restrict__ s,
+                                                      int64_t total, int64_t D8, int64_t P8, uint4* __restrict__ Xs,
+                                                      int* count, int n_count) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_count; i += gridDim.x * blockDim.x) count[i] = 0;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / P8, j = i - t * P8;
+    if (j >= D8) {
+      Xs[i] = make_uint4(0u, 0u, 0u, 0u);
+      continue;
+    }
+    const uint4 xv = X[t * D8 + j];
+    const float4 s0 = __ldg(s + 2 * j), s1 = __ldg(s + 2 * j + 1);
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t h = (e & 1) ? (xw[e >> 1] >> 16) : (xw[e >> 1] & 0xFFFFu);
+      v[e] = __fdiv_rn(bf16_bits_to_float(h), sv[e]);
+    }
+    Xs[i] = make_uint4(pack_bf16(v[0], v[4]), pack_bf16(v[1], v[5]), pack_bf16(v[2], v[6]), pack_bf16(v[3], v[7]));
+  }
+}
+
+// ------------------------------------------------------------ the GEMM
+__device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t u) { return *reinterpret_cast<__nv_bfloat162*>(&u); }
+__device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
+
 template <int G>
 __global__ void __launch_bounds__(kW4Threads, 1)
-    w4a16_kernel(const __grid_constant__ CUtensorMap tmX, const W4Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int S = p.stages;
-  const int b_bytes = p.Nt * 64 * 2;
-  uint8_t* a_sm = smem;                                        // [S] x 16 KiB
-  uint8_t* b_sm = a_sm + S * kW4ABytes;                        // [S] x Nt*128 B
-  float* r_sm = reinterpret_cast<float*>(b_sm + S * b_bytes);  // [4 producer warps][64] 1/s of a stage's k
-  float* fold = r_sm + 4 * 64;                                 // [Nt][128] (split K)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(fold + (p.KS > 1 ? p.Nt * 128 : 0));
-  uint64_t* x_full = bars;
-  uint64_t* x_empty = x_full + S;
-  uint64_t* a_full = x_empty + S;
-  uint64_t* a_empty = a_full + S;
-  uint64_t* acc_full = a_empty + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+    w4a16_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
+                 const __grid_constant__ CUtensorMap tmS, const W4Params p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  // 1024-byte aligned base (128-byte swizzle atoms), derived by pointer
+  // arithmetic on the shared array so that accesses stay in the shared space.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int S = p.stages, AS = p.a_stages, KPS = p.kps;
+  const int xs_bytes = KPS * p.Nt * 128;          // the X' planes of a stage
+  const int pk_bytes = KPS * kW4PkBytes;
+  uint8_t* a_sm = smem + S * p.stage_bytes;       // [AS] x 16 KiB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(a_sm + AS * kW4ABytes);
+  uint64_t* w_full = bars;
+  uint64_t* w_empty = w_full + S;
+  uint64_t* a_full = w_empty + S;
+  uint64_t* a_empty = a_full + AS;
+  uint64_t* acc_full = a_empty + AS;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* done = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* epi_state = abort_flag + 1;      // [0] an epilogue warp failed, [1] this CTA folds the unit
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int ks = p.KS > 1 ? static_cast<int>(cluster.block_rank()) : 0;
-  const int tile = blockIdx.x / p.KS;
-  const int n_tile = tile % p.n_tiles, t_tile = tile / p.n_tiles;
-  const int64_t n0 = static_cast<int64_t>(n_tile) * 128, t0 = static_cast<int64_t>(t_tile) * p.Nt;
-  const int kb0 = static_cast<int>(static_cast<int64_t>(p.KB) * ks / p.KS);
-  const int kb1 = static_cast<int>(static_cast<int64_t>(p.KB) * (ks + 1) / p.KS);
-  const int tcols = p.Nt <= 32 ? 32 : (p.Nt <= 64 ? 64 : (p.Nt <= 128 ? 128 : 256));
+  const int c = blockIdx.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&x_full[s], 1);
-      mbar_init(&x_empty[s], 1);
-      mbar_init(&a_full[s], 4);
+      mbar_init(&w_full[s], 1);
+      mbar_init(&w_empty[s], kW4DqWarps + 1);      // the dequantiser warps + the MMA commit
+    }
+    for (int s = 0; s < AS; ++s) {
+      mbar_init(&a_full[s], kW4DqWarps);
       mbar_init(&a_empty[s], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(done, 1);
     *abort_flag = 0;
+    epi_state[0] = 0;
+    epi_state[1] = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, tcols);
+  if (warp == kW4MmaWarp) {
+    tmem_alloc(tmem_slot, 2 * p.tcols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -108,137 +213,263 @@ __global__ void __launch_bounds__(kW4Threads, 1)
   const uint64_t tmo = p.timeout_ns;
   bool aborted = false;
 
-  if (warp == 0) {
-    // ---------------------------------------------------------- TMA of X
-    if (lane == 0) {
-      int last[8] = {-1, -1, -1, -1, -1, -1, -1, -1};
-      for (int kb = kb0; kb < kb1; ++kb) {
-        const int i = kb - kb0, s = i % S, r = i / S;
-        if (!wait_bounded(&x_empty[s], (r & 1) ^ 1, abort_flag, p.status, kSiteW4XEmpty, tmo)) {
-          aborted = true;
-          break;
+  if (warp < kW4TmaWarps) {
+    // ---------------------------------------------------------- TMA: warp w fills the stages of step index = w mod issuers
+    if (lane == 0 && warp < p.issuers) {
+      const uint32_t tx = static_cast<uint32_t>(xs_bytes + pk_bytes + p.scale_rows * 128 * 4);
+      const int step = p.issuers;
+      int s = warp;                 // this warp's next stage slot (S is a multiple of `step`)
+      uint32_t ph = 0;
+      uint32_t i = 0, fills = 0;    // step counter of the CTA, fills issued by this warp
+      bool ok = true;
+      SegCursor cur = seg_begin(p, c);
+      int u, ka, kb1;
+      while (ok && seg_next(cur, p, u, ka, kb1)) {
+        const int n0 = (u % p.n_tiles) * 128, t0 = (u / p.n_tiles) * p.Nt;
+        for (int st = ka; st < kb1; ++st, ++i) {
+          if (static_cast<int>(i % static_cast<uint32_t>(step)) != warp) continue;
+          if (!wait_bounded_sleep(&w_empty[s], ph ^ 1, abort_flag, p.status, kSiteW4WEmpty, tmo, kW4SleepNs)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sp = smem + s * p.stage_bytes;
+          const int kb = st * KPS;
+          mbar_arrive_expect_tx(&w_full[s], tx);
+          tma_load_3d(sp, &tmX, &w_full[s], 0, t0, kb);
+          tma_load_2d(sp + xs_bytes, &tmP, &w_full[s], n0, kb * 8);
+          tma_load_2d(sp + xs_bytes + pk_bytes, &tmS, &w_full[s], n0, (kb * 64) / G);
+          ++fills;
+          s += step;
+          if (s >= S) {
+            s -= S;
+            ph ^= 1;
+          }
         }
-        mbar_arrive_expect_tx(&x_full[s], static_cast<uint32_t>(b_bytes));
-        tma_load_2d(b_sm + s * b_bytes, &tmX, &x_full[s], kb * 64, static_cast<int>(t0));
-        last[s] = r;
       }
+      aborted = !ok;
+      // Every fill issued has landed before the CTA may exit (matters only
+      // when another role gave up early): fill j of this warp used slot
+      // (warp + step j) mod S in phase ((warp + step j) / S) & 1.
       volatile int no_abort = 0;
-      for (int s = 0; s < S; ++s)
-        if (last[s] >= 0) wait_bounded(&x_full[s], last[s] & 1, &no_abort, p.status, kSiteW4XFull, tmo);
+      const uint32_t per_round = static_cast<uint32_t>(S / step);
+      for (uint32_t j = fills > per_round ? fills - per_round : 0; j < fills; ++j) {
+        const uint32_t q = static_cast<uint32_t>(warp) + static_cast<uint32_t>(step) * j;
+        wait_bounded(&w_full[q % S], (q / S) & 1, &no_abort, p.status, kSiteW4WFull, tmo);
+      }
     }
-  } else if (warp == 1) {
+  } else if (warp == kW4MmaWarp) {
     // ---------------------------------------------------------- MMA issue
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, p.Nt);
+      int s = 0, sa = 0, b = 0;
+      uint32_t ph = 0, pha = 0, phb = 0;
       bool ok = true;
-      for (int kb = kb0; kb < kb1; ++kb) {
-        const int i = kb - kb0, s = i % S, r = i / S;
-        if (!wait_bounded(&a_full[s], r & 1, abort_flag, p.status, kSiteW4AFull, tmo) ||
-            !wait_bounded(&x_full[s], r & 1, abort_flag, p.status, kSiteW4XFull, tmo)) {
+      SegCursor cur = seg_begin(p, c);
+      int u, ka, kb1;
+      const uint32_t idesc = idesc_bf16_f32(128, p.Nt);
+      while (ok && seg_next(cur, p, u, ka, kb1)) {
+        if (!wait_bounded_sleep(&acc_empty[b], phb ^ 1, abort_flag, p.status, kSiteW4AccEmpty, tmo, kW4SleepNs)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t adesc = sw128_kmajor_desc(smem_u32(a_sm + s * kW4ABytes));
-        const uint64_t bdesc = sw128_kmajor_desc(smem_u32(b_sm + s * b_bytes));
+        const uint32_t d_tmem = tbase + static_cast<uint32_t>(b * p.tcols);
+        for (int st = ka; st < kb1 && ok; ++st) {
+          if (!wait_bounded_sleep(&w_full[s], ph, abort_flag, p.status, kSiteW4WFull, tmo, kW4SleepNs)) {
+            ok = false;
+            break;
+          }
+          for (int j = 0; j < KPS; ++j) {
+            if (!wait_bounded_sleep(&a_full[sa], pha, abort_flag, p.status, kSiteW4AFull, tmo, kW4SleepNs)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t adesc = sw128_kmajor_desc(smem_u32(a_sm + sa * kW4ABytes));
+            const uint64_t bdesc = sw128_kmajor_desc(smem_u32(smem + s * p.stage_bytes + j * p.Nt * 128));
 #pragma unroll
-        for (int j = 0; j < 4; ++j) mma_ss_f16_cta(tbase, adesc + 2 * j, bdesc + 2 * j, idesc, (i | j) != 0 ? 1u : 0u);
-        mma_commit(&a_empty[s]);
-        mma_commit(&x_empty[s]);
+            for (int k = 0; k < 4; ++k)
+              mma_ss_f16_cta(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (st > ka || j > 0 || k > 0) ? 1u : 0u);
+            mma_commit(&a_empty[sa]);
+            if (++sa == AS) {
+              sa = 0;
+              pha ^= 1;
+            }
+          }
+          if (!ok) break;
+          mma_commit(&w_empty[s]);     // the MMAs read X' from the stage
+          if (++s == S) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[b]);
+        b ^= 1;
+        if (b == 0) phb ^= 1;
       }
       aborted = !ok;
-      mma_commit(acc_full);       // arrives once every MMA issued above has completed
+      mma_commit(done);            // arrives once every MMA issued above has completed
       volatile int no_abort = 0;
-      wait_bounded(acc_full, 0, &no_abort, p.status, kSiteW4Acc, tmo);
+      wait_bounded(done, 0, &no_abort, p.status, kSiteW4Done, tmo);
     }
     __syncwarp();
-  } else {
-    // ---------------------------------------------------------- producers, then the epilogue
-    const int q = warp & 3;
-    const int n = q * 32 + lane;                  // column in the tile
-    const int64_t nn = n0 + n;
-    const bool valid = nn < p.D_out;
-    const float off = static_cast<float>(1 << (p.bits - 1));
+  } else if (warp < kW4EpiWarp0) {
+    // ---------------------------------------------------------- dequantisers
+    const int n = (warp & 3) * 32 + lane;
+    const int h = (warp - kW4DqWarp0) >> 2;       // half of each k block: chunks 4h..4h+3
+    const uint32_t bias_bits = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(128.0f + p.off)));
+    const __nv_bfloat162 bias = as_bf162(bias_bits | (bias_bits << 16));     // 128 + off, exact
+    const int swz = n & 7;
+    int s = 0, sa = 0;
+    uint32_t ph = 0, pha = 0;
     bool ok = true;
-    for (int kb = kb0; kb < kb1 && ok; ++kb) {
-      const int i = kb - kb0, s = i % S, r = i / S;
-      const bool got = wait_bounded(&a_empty[s], (r & 1) ^ 1, abort_flag, p.status, kSiteW4AEmpty, tmo);
-      if (!__all_sync(0xffffffffu, got)) {
-        ok = false;
-        break;
-      }
-      const int64_t k0 = static_cast<int64_t>(kb) * 64;
-      // 1/s of the stage's 64 rows (zero past D_in), each warp its own copy
-      float* rs = r_sm + q * 64;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int64_t k = k0 + lane + 32 * h;
-        rs[lane + 32 * h] = k < p.D_in ? __frcp_rn(__ldg(p.s + k)) : 0.0f;
-      }
-      __syncwarp();
-      uint4* arow = reinterpret_cast<uint4*>(a_sm + s * kW4ABytes + (n >> 3) * 1024 + (n & 7) * 128);
-#pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        const int64_t k8 = k0 / 8 + w;
-        uint4 chunk = make_uint4(0u, 0u, 0u, 0u);
-        if (valid && k8 * 8 < p.D_in) {
-          const uint32_t word = __ldg(p.packed + k8 * p.D_out + nn);
-          const float delta = __ldg(p.scales + ((k8 * 8) / G) * p.D_out + nn);
-          float v[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float qv = static_cast<float>((word >> (4 * e)) & 0xFu) - off;        // exact small integer
-            v[e] = __fmul_rn(qv, __fmul_rn(delta, rs[w * 8 + e]));
-          }
-          chunk = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
-                             pack_bf16(v[6], v[7]));
+    SegCursor cur = seg_begin(p, c);
+    int u, ka, kb1;
+    while (ok && seg_next(cur, p, u, ka, kb1)) {
+      for (int st = ka; st < kb1 && ok; ++st) {
+        const bool got = wait_bounded_sleep(&w_full[s], ph, abort_flag, p.status, kSiteW4WFull, tmo, kW4SleepNs);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
         }
-        arow[w ^ (n & 7)] = chunk;                 // 16-byte chunk w of row n, 128-byte swizzle
-      }
-      fence_proxy_async_smem();
-      __syncwarp();                                // also: every lane is done with rs before it is rewritten
-      if (lane == 0) mbar_arrive(&a_full[s]);
-    }
-    // ---------------------------------------------------------- epilogue
-    if (ok) {
-      const bool got = wait_bounded(acc_full, 0, abort_flag, p.status, kSiteW4Acc, tmo);
-      ok = __all_sync(0xffffffffu, got);
-    }
-    if (ok) {
-      tc_fence_after();
-      const uint32_t lane_addr = tbase + (static_cast<uint32_t>(q * 32) << 16);
-      for (int c = 0; c < p.Nt; c += 16) {
-        uint32_t v[16];
-        tmem_ld16(lane_addr + c, v);
-        tmem_wait_ld();
-        if (p.KS > 1) {
+        const uint8_t* sp = smem + s * p.stage_bytes;
+        const int kb0 = st * KPS;
+        const int row0 = (kb0 * 64) / G;           // first scale row of the stage
+        for (int j = 0; j < KPS; ++j) {
+          const bool got_a = wait_bounded_sleep(&a_empty[sa], pha ^ 1, abort_flag, p.status, kSiteW4AEmpty, tmo,
+                                                kW4SleepNs);
+          if (!__all_sync(0xffffffffu, got_a)) {
+            ok = false;
+            break;
+          }
+          const uint32_t* pk = reinterpret_cast<const uint32_t*>(sp + xs_bytes) + (8 * j + 4 * h) * 128 + n;
+          uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) fold[(c + e) * 128 + n] = __uint_as_float(v[e]);
-        } else if (valid) {
+          for (int i = 0; i < 4; ++i) w[i] = pk[i * 128];
+          const int srow = ((kb0 + j) * 64 + 32 * h) / G - row0;
+          const float* sc = reinterpret_cast<const float*>(sp + xs_bytes + pk_bytes) + srow * 128 + n;
+          const __nv_bfloat162 d2 = __float2bfloat162_rn(sc[0]);
+          uint32_t o[16];                           // chunks 4h..4h+3 of row n: 16 bf16 pairs
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (t0 + c + e < p.N) p.Y[(t0 + c + e) * p.D_out + nn] = __uint_as_float(v[e]);
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t pair = ((w[i] >> (4 * q)) & 0x000F000Fu) | 0x43004300u;   // {128 + u_q, 128 + u_{q+4}}
+              o[4 * i + q] = as_u32(__hmul2(__hsub2(as_bf162(pair), bias), d2));
+            }
+          uint4* arow = reinterpret_cast<uint4*>(a_sm + sa * kW4ABytes + (n >> 3) * 1024 + (n & 7) * 128);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)   // chunk 4h+i of row n, 128-byte swizzle
+            arow[(4 * h + i) ^ swz] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[sa]);
+          if (++sa == AS) {
+            sa = 0;
+            pha ^= 1;
+          }
+        }
+        if (!ok) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&w_empty[s]);
+        if (++s == S) {
+          s = 0;
+          ph ^= 1;
         }
       }
     }
     aborted = !ok;
-  }
-  if (p.KS > 1) {
-    // The K split folds in rank order: CTA ks writes tokens t with t % KS == ks.
-    cluster.sync();
-    if (warp >= 2 && !aborted) {
-      const int n = (warp & 3) * 32 + lane;
-      const int64_t nn = n0 + n;
-      if (nn < p.D_out) {
-        for (int t = ks; t < p.Nt; t += p.KS) {
-          if (t0 + t >= p.N) break;
-          float acc = 0.0f;
-          for (int rk = 0; rk < p.KS; ++rk) acc += cluster.map_shared_rank(fold, rk)[t * 128 + n];
-          p.Y[(t0 + t) * p.D_out + nn] = acc;
+  } else {
+    // ---------------------------------------------------------- epilogue
+    // All four warps walk the same segments and meet at the same named
+    // barriers; a warp that failed keeps walking (doing no work) so that the
+    // barrier counts always match.
+    const int q = warp & 3;
+    const int n = q * 32 + lane;
+    const uint32_t lane_q = static_cast<uint32_t>(q * 32) << 16;
+    int b = 0;
+    uint32_t phb = 0;
+    bool ok = true;
+    bool first_seg = true;
+    SegCursor cur = seg_begin(p, c);
+    int u, ka, kb1;
+    while (seg_next(cur, p, u, ka, kb1)) {
+      const bool whole = ka == 0 && kb1 == p.KBS;
+      const int64_t nn = static_cast<int64_t>(u % p.n_tiles) * 128 + n;
+      const int64_t t0 = static_cast<int64_t>(u / p.n_tiles) * p.Nt;
+      const int slot = first_seg ? 0 : 1;
+      float* part = p.partial + ((static_cast<int64_t>(c) * 2 + slot) * p.N) * 128 + n;
+      const bool got = ok && wait_bounded_sleep(&acc_full[b], phb, abort_flag, p.status, kSiteW4AccFull, tmo,
+                                                 kW4SleepNs);
+      ok = __all_sync(0xffffffffu, got);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t lane_addr = tbase + static_cast<uint32_t>(b * p.tcols) + lane_q;
+        for (int cc = 0; cc < p.Nt; cc += 16) {
+          uint32_t v[16];
+          tmem_ld16(lane_addr + cc, v);
+          tmem_wait_ld();
+          if (whole) {
+            if (nn < p.D_out) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                if (t0 + cc + e < p.N) p.Y[(t0 + cc + e) * p.D_out + nn] = __uint_as_float(v[e]);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              if (cc + e < p.N) part[(cc + e) * 128] = __uint_as_float(v[e]);     // stream-K: one token tile
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
+      }
+      b ^= 1;
+      if (b == 0) phb ^= 1;
+      if (!whole) {
+        // Publish the partial tile; the last of the unit's contributors sums
+        // them all in CTA order.
+        if (!ok && lane == 0) epi_state[0] = 1;
+        __threadfence();
+        named_barrier(1, 128);
+        if (warp == kW4EpiWarp0 && lane == 0) {
+          int fold = 0;
+          if (epi_state[0] == 0) {
+            const int64_t first = static_cast<int64_t>(u) * p.KBS / p.chunk;
+            const int64_t last = (static_cast<int64_t>(u + 1) * p.KBS - 1) / p.chunk;
+            const int old = atomicAdd(&p.count[u], 1);
+            fold = old == static_cast<int>(last - first);
+            if (fold) __threadfence();
+          }
+          epi_state[1] = fold;
+        }
+        named_barrier(1, 128);
+        if (epi_state[1] && nn < p.D_out) {
+          const int64_t first = static_cast<int64_t>(u) * p.KBS / p.chunk;
+          const int64_t last = (static_cast<int64_t>(u + 1) * p.KBS - 1) / p.chunk;
+          // eight token rows at a time, so that eight loads per contributor are in flight
+          for (int t0r = 0; t0r < p.N; t0r += 8) {
+            float acc[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+            for (int64_t cp = first; cp <= last; ++cp) {
+              // CTA cp holds unit u in slot 0 unless u is not its first unit
+              const int sl = (cp == first && (cp * p.chunk) / p.KBS != u) ? 1 : 0;
+              const float* src = p.partial + ((cp * 2 + sl) * p.N + t0r) * 128 + n;
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                if (t0r + e < p.N) acc[e] += __ldcg(src + e * 128);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if (t0r + e < p.N) p.Y[(t0r + e) * p.D_out + nn] = acc[e];
+          }
         }
       }
+      first_seg = false;
     }
-    cluster.sync();
+    aborted = !ok;
   }
   if (aborted || *abort_flag) {
     const uint64_t tstart = globaltimer_ns();
@@ -247,52 +478,91 @@ __global__ void __launch_bounds__(kW4Threads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tbase, tcols);
+  if (warp == kW4MmaWarp) tmem_dealloc(tbase, 2 * p.tcols);
 }
 
 }  // namespace
 
+namespace {
+
+struct W4Layout {
+  size_t xs, count, partial, total;
+};
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+int w4_token_tile(int64_t N) { return N >= 256 ? 256 : static_cast<int>((N + 15) / 16 * 16); }
+
+W4Layout w4_layout(int64_t N, int64_t D_in, int64_t D_out) {
+  W4Layout l;
+  const int Nt = w4_token_tile(N);
+  const int64_t units = ((D_out + 127) / 128) * ((N + Nt - 1) / Nt);
+  l.xs = 0;
+  const int64_t Dp = (D_in + 63) / 64 * 64;     // X' rows padded to whole k blocks
+  l.count = round256(static_cast<size_t>(N) * static_cast<size_t>(Dp) * 2);
+  l.partial = l.count + round256(static_cast<size_t>(units) * 4);
+  const size_t part = Nt <= kW4MaxStreamTokens ? static_cast<size_t>(kW4MaxGrid) * 2 * N * 128 * 4 : 0;
+  l.total = l.partial + part;
+  return l;
+}
+
+}  // namespace
+
+size_t w4a16_scratch_bytes(int64_t N, int64_t D_in, int64_t D_out) { return w4_layout(N, D_in, D_out).total; }
+
 int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const float* scales, int64_t N, int64_t D_in,
-                 int64_t D_out, int bits, int group, float* Y, int num_sms, int* status, uint64_t timeout_ns,
-                 cudaStream_t st, cudaError_t* cerr, const char** what) {
+                 int64_t D_out, int bits, int group, float* Y, void* ws, int num_sms, int* status,
+                 uint64_t timeout_ns, cudaStream_t st, cudaError_t* cerr, const char** what) {
   *cerr = cudaSuccess;
-  const int Nt = N >= 256 ? 256 : static_cast<int>((N + 15) / 16 * 16);
+  const W4Layout lay = w4_layout(N, D_in, D_out);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  void* xs = wsb + lay.xs;
+  int* count = reinterpret_cast<int*>(wsb + lay.count);
+  float* partial = reinterpret_cast<float*>(wsb + lay.partial);
+
+  const int Nt = w4_token_tile(N);
   const int n_tiles = static_cast<int>((D_out + 127) / 128);
   const int t_tiles = static_cast<int>((N + Nt - 1) / Nt);
   const int KB = static_cast<int>((D_in + 63) / 64);
-  const long long tiles = static_cast<long long>(n_tiles) * t_tiles;
-  int KS = 1;
-  if (Nt <= kW4MaxFoldTokens && tiles < num_sms) {
-    long long k = num_sms / tiles;
-    if (k > 8) k = 8;
-    if (k > KB) k = KB;
-    KS = static_cast<int>(k < 1 ? 1 : k);
+  const int units = n_tiles * t_tiles;
+  const bool stream = Nt <= kW4MaxStreamTokens;
+
+  // 1. X' = X / s, rows padded to KB * 64 columns, columns permuted within
+  //    runs of 8; clears the unit counts
+  const int64_t Dp = static_cast<int64_t>(KB) * 64;
+  {
+    const int64_t total = N * (Dp / 8);
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > static_cast<int64_t>(num_sms) * 16) blocks = static_cast<int64_t>(num_sms) * 16;
+    scale_x_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        static_cast<const uint4*>(X), reinterpret_cast<const float4*>(s), total, D_in / 8, Dp / 8,
+        static_cast<uint4*>(xs), count, stream ? units : 0);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      *cerr = e;
+      *what = "scale_x_kernel launch";
+      return kECuda;
+    }
   }
-  const int stages = Nt > 128 ? 3 : 4;
-  CUtensorMap mX;
-  if (!make_bf16_map(&mX, X, static_cast<uint64_t>(D_in), static_cast<uint64_t>(N), 0, 64,
-                     static_cast<uint32_t>(Nt))) {
-    *what = "tensor map for X";
-    return kECuda;
-  }
-  W4Params p;
-  p.packed = packed;
-  p.scales = scales;
-  p.s = s;
-  p.Y = Y;
-  p.N = N;
-  p.D_in = D_in;
-  p.D_out = D_out;
-  p.bits = bits;
-  p.Nt = Nt;
-  p.KB = KB;
-  p.KS = KS;
-  p.n_tiles = n_tiles;
-  p.stages = stages;
-  p.status = status;
-  p.timeout_ns = timeout_ns;
-  const int smem = 1024 + stages * (kW4ABytes + Nt * 128) + 4 * 64 * 4 + (KS > 1 ? Nt * 128 * 4 : 0) + 256;
-  void (*kern)(CUtensorMap, W4Params) = nullptr;
+  // 2. the GEMM
+  const int tcols = Nt <= 32 ? 32 : (Nt <= 64 ? 64 : (Nt <= 128 ? 128 : 256));
+  // k blocks per stage: fat stages, two issuing warps for the memory-bound small token tiles
+  const int kps = Nt <= 32 ? 4 : (Nt <= 64 ? 2 : 1);
+  const int issuers = kps > 1 ? 2 : 1;
+  const int KBS = (KB + kps - 1) / kps;
+  const int scale_rows = kps * 64 >= group ? kps * 64 / group : 1;
+  const int stage_bytes = (kps * Nt * 128 + kps * kW4PkBytes + scale_rows * 512 + 1023) / 1024 * 1024;
+  // One CTA per SM; its shared memory goes to deep rings.
+  const int budget = 220 * 1024;
+  const int a_stages = Nt <= 32 ? 4 : 3;
+  const int fixed = a_stages * kW4ABytes + 1024 + 512;   // alignment slack, barriers
+  int stages = (budget - fixed) / stage_bytes;
+  if (stages > kW4MaxStages) stages = kW4MaxStages;
+  stages -= stages % issuers;                    // each issuing warp owns every issuers-th stage
+  if (stages < 2) stages = 2;
+  const int smem = fixed + stages * stage_bytes;
+
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, W4Params) = nullptr;
   switch (group) {
     case 32: kern = w4a16_kernel<32>; break;
     case 64: kern = w4a16_kernel<64>; break;
@@ -302,21 +572,63 @@ int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const fl
       return kEUnsupported;
   }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(tiles * KS));
-    cfg.blockDim = dim3(kW4Threads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = KS;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, mX, p);
+  if (e != cudaSuccess) {
+    *cerr = e;
+    *what = "w4a16_kernel attributes";
+    return kECuda;
   }
+  int64_t slots = num_sms;
+  if (slots > kW4MaxGrid) slots = kW4MaxGrid;
+
+  // X' as [KB][N][64]: dimension 1 (tokens) has stride Dp, dimension 2
+  // (k blocks) stride 64 elements; one box = the X' planes of a stage.
+  CUtensorMap mX, mP, mS;
+  const uint64_t xdims[3] = {64, static_cast<uint64_t>(N), static_cast<uint64_t>(KB)};
+  const uint64_t xstr[2] = {static_cast<uint64_t>(Dp) * 2, 128};
+  const uint32_t xbox[3] = {64, static_cast<uint32_t>(Nt), static_cast<uint32_t>(kps)};
+  if (!make_bf16_map_3d(&mX, xs, xdims, xstr, xbox) ||
+      !make_word_map(&mP, packed, false, static_cast<uint64_t>(D_out), static_cast<uint64_t>(D_in / 8), 128,
+                     static_cast<uint32_t>(8 * kps)) ||
+      !make_word_map(&mS, scales, true, static_cast<uint64_t>(D_out), static_cast<uint64_t>(D_in / group), 128,
+                     static_cast<uint32_t>(scale_rows))) {
+    *what = "tensor maps for the W4A16 GEMM";
+    return kECuda;
+  }
+  W4Params p;
+  p.Y = Y;
+  p.partial = partial;
+  p.count = count;
+  p.N = N;
+  p.D_out = D_out;
+  p.off = 1 << (bits - 1);
+  p.Nt = Nt;
+  p.KB = KB;
+  p.kps = kps;
+  p.KBS = KBS;
+  p.n_tiles = n_tiles;
+  p.units = units;
+  p.stream = stream ? 1 : 0;
+  p.issuers = issuers;
+  p.total = static_cast<int64_t>(units) * KBS;
+  p.stages = stages;
+  p.a_stages = a_stages;
+  p.stage_bytes = stage_bytes;
+  p.scale_rows = scale_rows;
+  p.tcols = tcols;
+  p.status = status;
+  p.timeout_ns = timeout_ns;
+  int64_t grid;
+  if (stream) {
+    // equal shares of the units x KBS stage steps, one per CTA slot
+    const int64_t want = p.total < slots ? p.total : slots;
+    p.chunk = (p.total + want - 1) / want;
+    grid = (p.total + p.chunk - 1) / p.chunk;
+  } else {
+    p.chunk = KBS;
+    grid = units < slots ? units : slots;
+  }
+  kern<<<static_cast<unsigned>(grid), kW4Threads, smem, st>>>(mX, mP, mS, p);
+  e = cudaGetLastError();
   if (e != cudaSuccess) {
     *cerr = e;
     *what = "w4a16_kernel launch";

@@ -115,6 +115,31 @@ def test_argument_checks_without_gpu(lib):
     assert q(fake, fake, 200, 64, 4, 128, fake, fake, None) == 1
     assert q(fake, fake, 256, 64, 6, 128, fake, fake, None) == 3
 
+    g = lib.awq_w4a16_gemm
+    SZ = ctypes.c_size_t
+    g.argtypes = [P, P, P, P, I64, I64, I64, I, I, P, P, SZ, P, P]
+    g.restype = I
+    gws = lib.awq_w4a16_workspace_size
+    gws.argtypes = [I64, I64, I64]
+    gws.restype = SZ
+    assert gws(16, 4096, 4096) >= 16 * 4096 * 2            # the scaled activations, bf16
+    gargs = dict(X=fake, s=fake, P=fake, sc=fake, N=16, D_in=256, D_out=64, bits=4, group=128, Y=fake, ws=fake,
+                 wsb=gws(16, 256, 64), st=fake, stream=None)
+
+    def gcall(**kw):
+        d = dict(gargs, **kw)
+        return g(d["X"], d["s"], d["P"], d["sc"], d["N"], d["D_in"], d["D_out"], d["bits"], d["group"], d["Y"],
+                 d["ws"], d["wsb"], d["st"], d["stream"])
+
+    assert gcall(D_out=66) == 1                           # rows of packed words must be 16-byte multiples
+    assert gcall(N=0) == 1
+    assert gcall(group=256) == 3
+    assert gcall(D_in=192) == 1
+    assert gcall(s=fake + 4) == 2                          # s is read as float4
+    assert gcall(ws=None) == 4
+    assert gcall(wsb=gws(16, 256, 64) - 1) == 4
+    assert gcall(st=None) == 1                             # the status word is required
+
     t = lib.awq_selftest_wait_timeout
     t.argtypes = [P, I64, P]
     t.restype = I

@@ -2,10 +2,15 @@
 applied to activations) against the oracle, on codes packed by the library
 itself.
 
-Tolerance, from the arithmetic: each dequantised weight q * delta / s_k is
-rounded to bf16 once (relative error at most 2^-8, modelled as independent
-and uniform), X is exact, accumulation is fp32.  Per output
-    |Y_gpu - Y| <= 6 sqrt(sum_k x_tk^2 w_kn^2 U^2 / 3) + 1e-5 sum_k |x_tk w_kn|.
+Tolerance, from the arithmetic of the CUDA path: x_tk / s_k is rounded to
+bf16 once, each weight q * bf16(delta) is rounded to bf16 once (relative
+errors at most 2^-9 each, modelled as independent and uniform; the model
+allows uniform errors up to U = 2^-8 per term, which covers both), and delta
+is rounded to bf16 once per (group, column): a relative error of at most
+2^-9 shared by the whole group, bounded deterministically.  Accumulation is
+fp32.  Per output
+    |Y_gpu - Y| <= 6 sqrt(sum_k x_tk^2 w_kn^2 U^2 / 3)
+                   + 2^-9 sum_g |sum_{k in g} x_tk w_kn| + 1e-5 sum_k |x_tk w_kn|.
 """
 import numpy as np
 import pytest
@@ -27,6 +32,18 @@ def awq():
     return mod
 
 
+def _bound(x, w_hat, group):
+    """x [N][D_in] fp64, w_hat [D_in][D_out] the exact dequantised weights
+    (with 1/s)."""
+    G = w_hat.shape[0] // group
+    per_group = np.zeros((x.shape[0], w_hat.shape[1]))
+    for g in range(G):
+        sl = slice(g * group, (g + 1) * group)
+        per_group += np.abs(x[:, sl] @ w_hat[sl])
+    return (6.0 * np.sqrt((x ** 2) @ (w_hat ** 2) * U * U / 3.0) + 2.0 ** -9 * per_group
+            + 1e-5 * (np.abs(x) @ np.abs(w_hat)))
+
+
 def _case(awq, N, D_in, D_out, bits, group, seed):
     X, W = synth.layer_inputs(synth.small_layer(max(N, 8), D_in, D_out, seed=seed))
     X = X[:N].contiguous()
@@ -40,8 +57,7 @@ def _case(awq, N, D_in, D_out, bits, group, seed):
     Y_or = oracle.w4a16(X, s, p_np, sc_np, bits, group)
     q, d = oracle.quantize(W, s, bits, group)
     w_hat = q * np.repeat(d, group, axis=0).astype(np.float64) / s.astype(np.float64)[:, None]
-    x = X.double().numpy()
-    bound = 6.0 * np.sqrt((x ** 2) @ (w_hat ** 2) * U * U / 3.0) + 1e-5 * (np.abs(x) @ np.abs(w_hat))
+    bound = _bound(X.double().numpy(), w_hat, group)
     return Y, Y_or, bound
 
 
@@ -52,6 +68,13 @@ def _case(awq, N, D_in, D_out, bits, group, seed):
     (37, 384, 132, 3, 64),
     (300, 1024, 260, 4, 128),     # two token tiles of 256, no split
     (64, 256, 128, 2, 128),
+    (33, 4160, 1024, 4, 32),      # D_in % 64 == 32 (a half k block), two groups per k block, split K
+    (1000, 512, 4096, 4, 64),     # 128 units of (128 columns x 256 tokens): more units than one per CTA
+    (17, 8192, 2048, 3, 128),     # Nt = 32, 16 column tiles: stream-K, shares inside one unit
+    (8, 256, 65536, 4, 128),      # 512 units of 4 k blocks: a CTA's share spans whole units + partial ends
+    (32, 2048, 640, 4, 64),       # the largest 4-k-block-stage token tile (Nt = 32), group 64
+    (33, 2048, 640, 4, 128),      # the smallest 2-k-block-stage token tile (Nt = 48)
+    (3, 1056, 96, 2, 32),         # group 32 (two groups per k block), 2-bit, D_in not a multiple of 256
 ])
 def test_w4a16_against_oracle(awq, N, D_in, D_out, bits, group):
     Y, Y_or, bound = _case(awq, N, D_in, D_out, bits, group, seed=N + D_in)
@@ -62,3 +85,35 @@ def test_w4a16_reproducible(awq):
     Y1, _, _ = _case(awq, 3, 1024, 512, 4, 128, seed=1)
     Y2, _, _ = _case(awq, 3, 1024, 512, 4, 128, seed=1)
     assert np.array_equal(Y1, Y2)
+
+
+def test_w4a16_decode_full_size(awq):
+    """A 70B-class down projection (D_in 28672, D_out 8192) at one token: the
+    stream-K decode configuration that is timed; sampled columns checked
+    against the oracle's definition."""
+    N, D_in, D_out, bits, group = 1, 28672, 8192, 4, 128
+    g = torch.Generator().manual_seed(11)
+    X = (torch.randn(N, D_in, generator=g) * 0.5).to(torch.bfloat16)
+    s = torch.rand(D_in, generator=g) + 0.5
+    packed = torch.randint(-2 ** 31, 2 ** 31 - 1, (D_in // 8, D_out), generator=g, dtype=torch.int64).to(torch.int32)
+    scales = torch.rand(D_in // group, D_out, generator=g) * 0.01 + 1e-3
+    Y = awq.w4a16_gemm(X.cuda(), s.cuda(), packed.cuda(), scales.cuda(), bits, group).cpu().numpy()
+    cols = np.random.default_rng(0).choice(D_out, size=64, replace=False)
+    p_np = packed.numpy().view(np.uint32)[:, cols]
+    sc_np = scales.numpy()[:, cols]
+    Y_or = oracle.w4a16(X, s.numpy(), np.ascontiguousarray(p_np), np.ascontiguousarray(sc_np), bits, group)
+    k = np.arange(D_in)
+    u = (p_np[k // 8] >> (4 * (k % 8))[:, None]) & 0xF
+    w_hat = (u.astype(np.float64) - 8) * np.repeat(sc_np, group, axis=0).astype(np.float64) / \
+        s.numpy().astype(np.float64)[:, None]
+    bound = _bound(X.double().numpy(), w_hat, group)
+    assert np.all(np.abs(Y[:, cols] - Y_or) <= bound), np.max(np.abs(Y[:, cols] - Y_or) / bound)
+
+
+def test_w4a16_rejects_unaligned_columns(awq):
+    X = torch.zeros(4, 128, dtype=torch.bfloat16, device="cuda")
+    s = torch.ones(128, device="cuda")
+    packed = torch.zeros(16, 6, dtype=torch.int32, device="cuda")
+    scales = torch.ones(1, 6, device="cuda")
+    with pytest.raises(awq.AwqError):
+        awq.w4a16_gemm(X, s, packed, scales, 4, 128)
