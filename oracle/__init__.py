@@ -24,6 +24,11 @@ _LIB = os.path.join(_HERE, "liboracle_awq.so")
 STAT_MEAN = 0
 STAT_MAX = 1
 
+# quantiser modes: delta = max / (2^(b-1) - 1), codes in +-(2^(b-1) - 1); or
+# delta = max / 2^(b-1), codes in [-2^(b-1), 2^(b-1) - 1]
+QMODE_SYMMETRIC = 0
+QMODE_POW2 = 1
+
 _lib = None
 
 
@@ -67,6 +72,16 @@ def _load():
         lib.oracle_loss_cols.restype = None
         lib.oracle_search.argtypes = [P, P, P, I64, I64, I64, P, I, I, I, P, I64, P, P]
         lib.oracle_search.restype = I
+        lib.oracle_quantize_mode.argtypes = [P, P, P, I64, I64, I, I, I, I, P, P]
+        lib.oracle_quantize_mode.restype = None
+        lib.oracle_weight_mean.argtypes = [P, I64, I64, P]
+        lib.oracle_weight_mean.restype = None
+        lib.oracle_scales_balanced.argtypes = [P, P, I64, F, P]
+        lib.oracle_scales_balanced.restype = None
+        lib.oracle_loss_cols_mode.argtypes = [P, P, P, I64, I64, I64, I, I, I, I, P, I64, P]
+        lib.oracle_loss_cols_mode.restype = None
+        lib.oracle_search_mode.argtypes = [P, P, P, P, I64, I64, I64, P, I, I, I, I, P, I64, P, P]
+        lib.oracle_search_mode.restype = I
         lib.oracle_literal_loss.argtypes = [P, P, P, I64, I64, I64, I, I]
         lib.oracle_literal_loss.restype = ctypes.c_longdouble
         lib.oracle_num_threads.argtypes = []
@@ -109,22 +124,40 @@ def act_stats(X, stat: int = STAT_MEAN) -> np.ndarray:
     return a
 
 
-def scales(a, alpha: float) -> np.ndarray:
+def scales(a, alpha: float, w_mean=None) -> np.ndarray:
     """s_j = a_j^alpha (floored), fp32.  compassingai.com concept page, flow
-    step 3."""
+    step 3.  With w_mean: the balanced scale s_j = a_j^alpha /
+    w_mean_j^(1 - alpha) (zhihu AWQ/GPTQ/SmoothQuant comparison, "the scale
+    per channel"), both statistics floored."""
     a = _f32(a)
     s = np.empty_like(a)
-    _load().oracle_scales(_ptr(a), a.shape[0], float(alpha), _ptr(s))
+    if w_mean is None:
+        _load().oracle_scales(_ptr(a), a.shape[0], float(alpha), _ptr(s))
+    else:
+        b = _f32(w_mean)
+        _load().oracle_scales_balanced(_ptr(a), _ptr(b), a.shape[0], float(alpha), _ptr(s))
     return s
 
 
-def quantize(W, s, bits: int, group: int, clip=None, delta16: bool = False) -> Tuple[np.ndarray, np.ndarray]:
+def weight_mean(W) -> np.ndarray:
+    """w_mean_j = mean_n |W_jn| over input channel j's row (fp64 sum, one fp32
+    rounding): the weight statistic of the balanced scale."""
+    W = _f32(W)
+    out = np.empty(W.shape[0], dtype=np.float32)
+    _load().oracle_weight_mean(_ptr(W), W.shape[0], W.shape[1], _ptr(out))
+    return out
+
+
+def quantize(W, s, bits: int, group: int, clip=None, delta16: bool = False,
+             qmode: int = QMODE_SYMMETRIC) -> Tuple[np.ndarray, np.ndarray]:
     """Codes q [D_in, D_out] (int8) and deltas [D_in/group, D_out] (fp32) of
     diag(s).W.  compassingai.com concept page, "quantisation math".  clip:
     optional [D_in/group, D_out] fp32 clip ratios (the group maximum is
     replaced by fl32(clip * max) before delta is formed).  delta16: delta is
     rounded to FP16 (mudrobot.github.io notes: delta stored in FP16) and the
-    codes use that value; the returned deltas are then FP16-representable."""
+    codes use that value; the returned deltas are then FP16-representable.
+    qmode QMODE_POW2: delta = max / 2^(b-1) (mudrobot.github.io notes,
+    "analysing the quantisation error"), codes clamped to [-2^(b-1), 2^(b-1) - 1]."""
     W = _f32(W)
     D_in, D_out = W.shape
     s = None if s is None else _f32(s)
@@ -134,8 +167,8 @@ def quantize(W, s, bits: int, group: int, clip=None, delta16: bool = False) -> T
     if clip is not None:
         c = _f32(clip)
         assert c.shape == (D_in // group, D_out)
-    _load().oracle_quantize_ex(_ptr(W), _ptr(s), _ptr(c), D_in, D_out, bits, group, int(bool(delta16)), _ptr(q),
-                               _ptr(d))
+    _load().oracle_quantize_mode(_ptr(W), _ptr(s), _ptr(c), D_in, D_out, bits, group, int(bool(delta16)),
+                                 int(qmode), _ptr(q), _ptr(d))
     return q, d
 
 
@@ -173,7 +206,7 @@ def pack(q: np.ndarray, bits: int) -> np.ndarray:
 
 
 def loss_cols(X, W, s, bits: int, group: int, cols: Optional[Sequence[int]] = None,
-              quantize_w: bool = True) -> np.ndarray:
+              quantize_w: bool = True, qmode: int = QMODE_SYMMETRIC) -> np.ndarray:
     """Per-column share of ||X S^-1 Q(S W) - X W||^2 (fp64) for one scale
     vector.  compassingai.com concept page, flow step 4c."""
     Xb = _as_bf16_bits(X)
@@ -184,17 +217,19 @@ def loss_cols(X, W, s, bits: int, group: int, cols: Optional[Sequence[int]] = No
     c = None if cols is None else np.ascontiguousarray(cols, dtype=np.int64)
     nc = D_out if c is None else c.shape[0]
     out = np.empty(nc, dtype=np.float64)
-    _load().oracle_loss_cols(_ptr(Xb), _ptr(W), _ptr(s), N, D_in, D_out, bits, group,
-                             1 if quantize_w else 0, _ptr(c), 0 if c is None else nc, _ptr(out))
+    _load().oracle_loss_cols_mode(_ptr(Xb), _ptr(W), _ptr(s), N, D_in, D_out, bits, group,
+                                  1 if quantize_w else 0, int(qmode), _ptr(c), 0 if c is None else nc, _ptr(out))
     return out
 
 
 def search(X, W, a, alphas, bits: int, group: int, cols: Optional[Sequence[int]] = None,
-           want_cols: bool = False):
+           want_cols: bool = False, qmode: int = QMODE_SYMMETRIC, w_mean=None):
     """Grid search over alpha: returns (L [n_alpha] fp64, best index[, L_col]).
 
     compassingai.com concept page, flow steps 3-5; mudrobot.github.io notes,
-    "searching the optimal scale" (alpha* = argmin L(s_X^alpha) on [0, 1])."""
+    "searching the optimal scale" (alpha* = argmin L(s_X^alpha) on [0, 1]).
+    qmode selects the quantiser (see quantize); w_mean switches to the
+    balanced scale (see scales)."""
     Xb = _as_bf16_bits(X)
     W = _f32(W)
     a = _f32(a)
@@ -205,8 +240,9 @@ def search(X, W, a, alphas, bits: int, group: int, cols: Optional[Sequence[int]]
     nc = D_out if c is None else c.shape[0]
     L = np.empty(al.shape[0], dtype=np.float64)
     Lc = np.empty((al.shape[0], nc), dtype=np.float64) if want_cols else None
-    best = _load().oracle_search(_ptr(Xb), _ptr(W), _ptr(a), N, D_in, D_out, _ptr(al), al.shape[0],
-                                 bits, group, _ptr(c), 0 if c is None else nc, _ptr(L), _ptr(Lc))
+    b = None if w_mean is None else _f32(w_mean)
+    best = _load().oracle_search_mode(_ptr(Xb), _ptr(W), _ptr(a), _ptr(b), N, D_in, D_out, _ptr(al), al.shape[0],
+                                      bits, group, int(qmode), _ptr(c), 0 if c is None else nc, _ptr(L), _ptr(Lc))
     if want_cols:
         return L, int(best), Lc
     return L, int(best)

@@ -96,6 +96,39 @@ void oracle_scales(const float *a, int64_t D, float alpha, float *s)
     }
 }
 
+/* The weight statistic of the balanced scale ([P3] "the scale per channel":
+ * s_j = mean|X_j|^alpha / mean|W_j|^(1-alpha)): w_mean_j = (sum_n |W_jn|) / D_out
+ * over input channel j's row of W, summed in fp64, rounded to fp32 once. */
+void oracle_weight_mean(const float *W, int64_t D_in, int64_t D_out, float *w_mean)
+{
+    for (int64_t j = 0; j < D_in; ++j) {
+        double acc = 0.0;
+        for (int64_t n = 0; n < D_out; ++n)
+            acc += fabs((double)W[j * D_out + n]);
+        w_mean[j] = (float)(acc / (double)D_out);
+    }
+}
+
+/* The balanced scale s_j = a_j^alpha / b_j^(1-alpha) ([P3], same passage), with
+ * a and b each floored as in oracle_scales (1e-6 of its maximum; all zero ->
+ * 1).  Computed in fp64, rounded to fp32 once. */
+void oracle_scales_balanced(const float *a, const float *b, int64_t D, float alpha, float *s)
+{
+    float amax = 0.0f, bmax = 0.0f;
+    for (int64_t j = 0; j < D; ++j) {
+        if (a[j] > amax)
+            amax = a[j];
+        if (b[j] > bmax)
+            bmax = b[j];
+    }
+    const float afl = 1e-6f * amax, bfl = 1e-6f * bmax;
+    for (int64_t j = 0; j < D; ++j) {
+        const float aj = amax == 0.0f ? 1.0f : (a[j] > afl ? a[j] : afl);
+        const float bj = bmax == 0.0f ? 1.0f : (b[j] > bfl ? b[j] : bfl);
+        s[j] = (float)(pow((double)aj, (double)alpha) / pow((double)bj, 1.0 - (double)alpha));
+    }
+}
+
 /* Round a finite fp32 value to the nearest IEEE binary16 value (ties to
  * even), returned as a float: 11 significant bits in the normal range
  * (|x| >= 2^-14), a fixed step of 2^-24 below it, infinity from 65520 up
@@ -128,9 +161,14 @@ static float round_to_fp16(float x)
  * delta is formed, and the clamp then bounds the codes of the clipped weights.
  * clip = 1 leaves m unchanged (fl32(1 * m) = m). */
 static void quantize_group(const float *W, const float *s, int64_t D_out, int64_t n,
-                           int64_t k0, int group, int bits, float clip, int delta16, int8_t *q, float *delta)
+                           int64_t k0, int group, int bits, float clip, int delta16, int qmode, int8_t *q,
+                           float *delta)
 {
     const int qmax = (1 << (bits - 1)) - 1;
+    /* qmode 1 ([P2] "analysing the quantisation error"): delta = max / 2^(b-1)
+     * (an exact power-of-two scaling), codes clamped to [-2^(b-1), 2^(b-1) - 1]
+     * so that they fit b bits (the passage gives no clamp; +max would be 2^(b-1)). */
+    const int qlo = qmode == 1 ? -(qmax + 1) : -qmax;
     float m = 0.0f;
     for (int k = 0; k < group; ++k) {
         float w = W[(k0 + k) * D_out + n];
@@ -140,7 +178,7 @@ static void quantize_group(const float *W, const float *s, int64_t D_out, int64_
             m = am;
     }
     m = clip * m;
-    float d = m / (float)qmax;
+    float d = qmode == 1 ? ldexpf(m, -(bits - 1)) : m / (float)qmax;
     if (delta16)
         d = round_to_fp16(d);      /* the exported FP16 delta, which the codes then use */
     *delta = d;
@@ -153,8 +191,8 @@ static void quantize_group(const float *W, const float *s, int64_t D_out, int64_
             float r = nearbyintf(t); /* round half to even in the default mode */
             if (r > (float)qmax)
                 r = (float)qmax;
-            if (r < (float)-qmax)
-                r = (float)-qmax;
+            if (r < (float)qlo)
+                r = (float)qlo;
             code = (int)r;
         }
         q[k] = (int8_t)code;
@@ -165,19 +203,25 @@ static void quantize_group(const float *W, const float *s, int64_t D_out, int64_
  * [-qmax, qmax]; delta: [D_in/group][D_out].  clip: [D_in/group][D_out] clip
  * ratios, or NULL for none.  delta16: delta is rounded to FP16 before the
  * codes are formed (the exported scale format). */
-void oracle_quantize_ex(const float *W, const float *s, const float *clip, int64_t D_in, int64_t D_out,
-                        int bits, int group, int delta16, int8_t *q, float *delta)
+void oracle_quantize_mode(const float *W, const float *s, const float *clip, int64_t D_in, int64_t D_out,
+                          int bits, int group, int delta16, int qmode, int8_t *q, float *delta)
 {
     int8_t *col = (int8_t *)malloc((size_t)group);
     for (int64_t n = 0; n < D_out; ++n) {
         for (int64_t g = 0; g < D_in / group; ++g) {
             quantize_group(W, s, D_out, n, g * group, group, bits, clip ? clip[g * D_out + n] : 1.0f, delta16,
-                           col, &delta[g * D_out + n]);
+                           qmode, col, &delta[g * D_out + n]);
             for (int k = 0; k < group; ++k)
                 q[(g * group + k) * D_out + n] = col[k];
         }
     }
     free(col);
+}
+
+void oracle_quantize_ex(const float *W, const float *s, const float *clip, int64_t D_in, int64_t D_out,
+                        int bits, int group, int delta16, int8_t *q, float *delta)
+{
+    oracle_quantize_mode(W, s, clip, D_in, D_out, bits, group, delta16, 0, q, delta);
 }
 
 void oracle_quantize_clip(const float *W, const float *s, const float *clip, int64_t D_in, int64_t D_out,
@@ -218,13 +262,13 @@ void oracle_pack(const int8_t *q, int64_t D_in, int64_t D_out, int bits, uint32_
  * cancellation check. */
 static double column_loss(const double *Xd, const float *W, const float *s,
                           int64_t N, int64_t D_in, int64_t D_out, int64_t n,
-                          int bits, int group, int quantize, double *e, int8_t *qcol)
+                          int bits, int group, int quantize, int qmode, double *e, int8_t *qcol)
 {
     for (int64_t g = 0; g < D_in / group; ++g) {
         const int64_t k0 = g * group;
         if (quantize) {
             float d;
-            quantize_group(W, s, D_out, n, k0, group, bits, 1.0f, 0, qcol, &d);
+            quantize_group(W, s, D_out, n, k0, group, bits, 1.0f, 0, qmode, qcol, &d);
             for (int k = 0; k < group; ++k) {
                 double sk = s ? (double)s[k0 + k] : 1.0;
                 e[k0 + k] = (double)qcol[k] * (double)d / sk - (double)W[(k0 + k) * D_out + n];
@@ -259,9 +303,9 @@ static double *x_to_double(const uint16_t *X, int64_t N, int64_t D_in)
 
 /* Per-column losses for one scale vector s (NULL = all ones).  cols == NULL
  * means every column; otherwise L_col[c] is the loss of column cols[c]. */
-void oracle_loss_cols(const uint16_t *X, const float *W, const float *s,
-                      int64_t N, int64_t D_in, int64_t D_out, int bits, int group,
-                      int quantize, const int64_t *cols, int64_t ncols, double *L_col)
+void oracle_loss_cols_mode(const uint16_t *X, const float *W, const float *s,
+                           int64_t N, int64_t D_in, int64_t D_out, int bits, int group,
+                           int quantize, int qmode, const int64_t *cols, int64_t ncols, double *L_col)
 {
     double *Xd = x_to_double(X, N, D_in);
     const int64_t nc = cols ? ncols : D_out;
@@ -272,12 +316,19 @@ void oracle_loss_cols(const uint16_t *X, const float *W, const float *s,
 #pragma omp for schedule(dynamic, 1)
         for (int64_t c = 0; c < nc; ++c) {
             int64_t n = cols ? cols[c] : c;
-            L_col[c] = column_loss(Xd, W, s, N, D_in, D_out, n, bits, group, quantize, e, qcol);
+            L_col[c] = column_loss(Xd, W, s, N, D_in, D_out, n, bits, group, quantize, qmode, e, qcol);
         }
         free(e);
         free(qcol);
     }
     free(Xd);
+}
+
+void oracle_loss_cols(const uint16_t *X, const float *W, const float *s,
+                      int64_t N, int64_t D_in, int64_t D_out, int bits, int group,
+                      int quantize, const int64_t *cols, int64_t ncols, double *L_col)
+{
+    oracle_loss_cols_mode(X, W, s, N, D_in, D_out, bits, group, quantize, 0, cols, ncols, L_col);
 }
 
 /* [P1] flow steps 3-5 for one layer: for every alpha on the grid, s = a^alpha,
@@ -286,18 +337,23 @@ void oracle_loss_cols(const uint16_t *X, const float *W, const float *s,
  * L: [n_alpha]; L_col: [n_alpha][ncols] (may be NULL); restricted to the
  * columns in cols when cols != NULL (L then sums those columns only).
  * Returns the argmin index. */
-int oracle_search(const uint16_t *X, const float *W, const float *a,
-                  int64_t N, int64_t D_in, int64_t D_out,
-                  const float *alphas, int n_alpha, int bits, int group,
-                  const int64_t *cols, int64_t ncols, double *L, double *L_col)
+/* As oracle_search, with the quantiser mode (qmode, see quantize_group) and
+ * the balanced scale when b != NULL (s = a^alpha / b^(1-alpha), [P3]). */
+int oracle_search_mode(const uint16_t *X, const float *W, const float *a, const float *b,
+                       int64_t N, int64_t D_in, int64_t D_out,
+                       const float *alphas, int n_alpha, int bits, int group, int qmode,
+                       const int64_t *cols, int64_t ncols, double *L, double *L_col)
 {
     const int64_t nc = cols ? ncols : D_out;
     float *s = (float *)malloc((size_t)D_in * sizeof(float));
     double *lc = (double *)malloc((size_t)nc * sizeof(double));
     int best = 0;
     for (int ai = 0; ai < n_alpha; ++ai) {
-        oracle_scales(a, D_in, alphas[ai], s);
-        oracle_loss_cols(X, W, s, N, D_in, D_out, bits, group, 1, cols, ncols, lc);
+        if (b)
+            oracle_scales_balanced(a, b, D_in, alphas[ai], s);
+        else
+            oracle_scales(a, D_in, alphas[ai], s);
+        oracle_loss_cols_mode(X, W, s, N, D_in, D_out, bits, group, 1, qmode, cols, ncols, lc);
         double sum = 0.0;
         for (int64_t c = 0; c < nc; ++c) {
             sum += lc[c];
@@ -311,6 +367,14 @@ int oracle_search(const uint16_t *X, const float *W, const float *a,
     free(lc);
     free(s);
     return best;
+}
+
+int oracle_search(const uint16_t *X, const float *W, const float *a,
+                  int64_t N, int64_t D_in, int64_t D_out,
+                  const float *alphas, int n_alpha, int bits, int group,
+                  const int64_t *cols, int64_t ncols, double *L, double *L_col)
+{
+    return oracle_search_mode(X, W, a, NULL, N, D_in, D_out, alphas, n_alpha, bits, group, 0, cols, ncols, L, L_col);
 }
 
 /* The literal two-product form of [P1] flow step 4c for tiny layers:
@@ -394,7 +458,7 @@ void oracle_clip_loss(const uint16_t *X, const float *W, const float *s, int64_t
                 int ibest = 0;
                 for (int i = 0; i < n_clip; ++i) {
                     float d;
-                    quantize_group(W, s, D_out, n, k0, group, bits, clip[i], 0, qg, &d);
+                    quantize_group(W, s, D_out, n, k0, group, bits, clip[i], 0, 0, qg, &d);
                     for (int k = 0; k < group; ++k) {
                         double sk = s ? (double)s[k0 + k] : 1.0;
                         e[k] = (double)qg[k] * (double)d / sk - (double)W[(k0 + k) * D_out + n];

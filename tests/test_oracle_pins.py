@@ -9,6 +9,7 @@ invariance; sign symmetry), bounds (|q| <= qmax, |error| <= delta / 2), a
 library check of the loss (numpy fp64 matmul) and brute force on tiny layers.
 """
 import json
+import math
 import os
 
 import numpy as np
@@ -358,3 +359,95 @@ def test_w4a16_is_the_dequantised_search_operand():
         w_hat = q * np.repeat(d, group, axis=0).astype(np.float64) / s.astype(np.float64)[:, None]
         Y = oracle.w4a16(X, s, oracle.pack(q, bits), d, bits, group)
         assert np.allclose(Y, X.double().numpy() @ w_hat, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- quantiser with delta = max / 2^(b-1)
+# (mudrobot.github.io notes, "analysing the quantisation error": Q(w) = delta *
+# Round(w / delta), delta = max|w| / 2^(N-1); codes clamped to N bits.)
+
+def test_pow2_quantiser_worked_example():
+    # one group of 4 in one column: max |w| = 1 -> delta = 1/8;
+    # 0.5 -> 4, -1 -> -8, 0.26 -> round(2.08) = 2, 0.74 -> round(5.92) = 6
+    W = np.array([[0.5], [-1.0], [0.26], [0.74]], dtype=np.float32)
+    q, d = oracle.quantize(W, None, 4, 4, qmode=oracle.QMODE_POW2)
+    assert d[0, 0] == np.float32(0.125)
+    assert q[:, 0].tolist() == [4, -8, 2, 6]
+
+
+def test_pow2_quantiser_clamps_the_positive_maximum():
+    # +max maps to 2^(b-1) = 8, one past the largest 4-bit code: clamped to 7
+    W = np.array([[1.0], [-0.5], [0.25], [0.0]], dtype=np.float32)
+    q, d = oracle.quantize(W, None, 4, 4, qmode=oracle.QMODE_POW2)
+    assert d[0, 0] == np.float32(0.125) and q[:, 0].tolist() == [7, -4, 2, 0]
+    q3, d3 = oracle.quantize(W, None, 3, 4, qmode=oracle.QMODE_POW2)
+    assert d3[0, 0] == np.float32(0.25) and q3[:, 0].tolist() == [3, -2, 1, 0]
+
+
+def test_pow2_quantiser_brute_force():
+    rng = np.random.default_rng(5)
+    W = (rng.standard_normal((64, 6)) * np.exp(rng.standard_normal((64, 1)))).astype(np.float32)
+    s = (rng.random(64) + 0.5).astype(np.float32)
+    for bits in (2, 3, 4):
+        q, d = oracle.quantize(W, s, bits, 32, qmode=oracle.QMODE_POW2)
+        lo, hi = -(1 << (bits - 1)), (1 << (bits - 1)) - 1
+        for g in range(2):
+            for n in range(6):
+                wp = (s[32 * g:32 * g + 32] * W[32 * g:32 * g + 32, n]).astype(np.float32)
+                m = np.max(np.abs(wp))
+                assert d[g, n] * (1 << (bits - 1)) == m          # exact power-of-two scaling
+                for k in range(32):
+                    t = float(np.float32(wp[k] / d[g, n]))
+                    cand = np.arange(lo, hi + 1)
+                    err = np.abs(cand - t)
+                    best = cand[err == err.min()]
+                    want = best[0] if len(best) == 1 else best[best % 2 == 0][0]   # ties to even
+                    assert q[32 * g + k, n] == want
+
+
+def test_pow2_quantiser_search_differs_from_symmetric():
+    X, W = synth.layer_inputs(synth.small_layer(64, 128, 16, seed=3))
+    a = oracle.act_stats(X).astype(np.float32)
+    grid = np.array([0.0, 0.5], np.float32)
+    L0, _ = oracle.search(X, W, a, grid, 4, 64)
+    L1, _ = oracle.search(X, W, a, grid, 4, 64, qmode=oracle.QMODE_POW2)
+    assert np.all(L0 > 0) and np.all(L1 > 0) and not np.allclose(L0, L1)
+    # the search's loss is the column losses of the same quantiser
+    s = oracle.scales(a, 0.5)
+    assert np.isclose(L1[1], oracle.loss_cols(X, W, s, 4, 64, qmode=oracle.QMODE_POW2).sum(), rtol=1e-12)
+
+
+# ---------------------------------------------------------------- balanced scale
+# (zhihu AWQ/GPTQ/SmoothQuant comparison: s_j = mean|X_j|^alpha / mean|W_j|^(1-alpha))
+
+def test_weight_mean_closed_form():
+    rng = np.random.default_rng(8)
+    W = rng.standard_normal((40, 300)).astype(np.float32)
+    want = np.array([math.fsum(np.abs(W[j]).astype(np.float64)) / 300 for j in range(40)], dtype=np.float32)
+    assert np.allclose(oracle.weight_mean(W), want, rtol=2e-7, atol=0)
+
+
+def test_balanced_scale_closed_forms():
+    rng = np.random.default_rng(9)
+    a = (rng.random(50) + 0.1).astype(np.float32)
+    b = (rng.random(50) + 0.1).astype(np.float32)
+    # alpha = 1: the plain activation scale; alpha = 0: 1 / b; alpha = 1/2: sqrt(a / b)
+    assert np.array_equal(oracle.scales(a, 1.0, w_mean=b), oracle.scales(a, 1.0))
+    assert np.array_equal(oracle.scales(a, 0.0, w_mean=b), (1.0 / b.astype(np.float64)).astype(np.float32))
+    half = np.sqrt(a.astype(np.float64) / b.astype(np.float64)).astype(np.float32)
+    assert np.allclose(oracle.scales(a, 0.5, w_mean=b), half, rtol=1e-7, atol=0)
+
+
+def test_balanced_scale_floors_a_zero_weight_row():
+    a = np.array([1.0, 2.0, 4.0], dtype=np.float32)
+    b = np.array([0.0, 1.0, 2.0], dtype=np.float32)
+    s = oracle.scales(a, 0.0, w_mean=b)
+    assert np.isfinite(s).all() and s[0] == np.float32(1.0 / np.float32(1e-6 * np.float32(2.0)))
+
+
+def test_balanced_search_with_unit_weight_means_is_the_plain_search():
+    X, W = synth.layer_inputs(synth.small_layer(48, 128, 12, seed=4))
+    a = oracle.act_stats(X).astype(np.float32)
+    grid = np.array([0.0, 0.25, 0.5, 1.0], np.float32)
+    L0, b0 = oracle.search(X, W, a, grid, 4, 64)
+    L1, b1 = oracle.search(X, W, a, grid, 4, 64, w_mean=np.ones(128, np.float32))
+    assert np.array_equal(L0, L1) and b0 == b1
