@@ -106,6 +106,26 @@ AWQ_API int awq_scales(const float* a, int64_t D_in, float alpha, float* s, void
 AWQ_API int awq_scales_dev(const float* a, int64_t D_in, const float* alpha_dev, float* s, void* stream);
 
 /*
+ * The weight statistic of the balanced scale (zhihu AWQ/GPTQ/SmoothQuant
+ * comparison, the per-channel scale s_j = mean|X_j|^alpha / mean|W_j|^(1-alpha)):
+ *     w_mean[j] = (sum_n |W[j][n]|) / D_out,
+ * summed in fp64 (a fixed order), rounded to fp32 once.
+ *   W       [D_in][D_out] fp32, 16-byte aligned;  w_mean [D_in] fp32 output
+ */
+AWQ_API int awq_weight_mean(const float* W, int64_t D_in, int64_t D_out, float* w_mean, void* stream);
+
+/*
+ * Scale vector with an optional weight statistic: s_j = a_j^alpha when w_mean
+ * is NULL (as awq_scales), else the balanced s_j = a_j^alpha / w_mean_j^(1-alpha).
+ * Both statistics are floored at 1e-6 of their maximum.  The powers are taken
+ * in fp64, and the result is rounded to fp32 once.  alpha_dev (device, may be
+ * NULL) overrides alpha (HOST, 0 <= alpha <= 1), e.g. the alpha_star of
+ * awq_search_ex.
+ */
+AWQ_API int awq_scales_ex(const float* a, const float* w_mean, int64_t D_in, float alpha, const float* alpha_dev,
+                          float* s, void* stream);
+
+/*
  * Bytes of workspace awq_search needs for this shape on the current device
  * (0 if the arguments are invalid).
  */
@@ -143,6 +163,34 @@ AWQ_API int awq_search(const void* X, const float* W, const float* a, int64_t N,
                        const float* alpha_grid, int n_alpha, int bits, int group, int loss_form, double* L,
                        double* L_col, float* alpha_star, int32_t* alpha_idx, void* workspace, size_t workspace_bytes,
                        int32_t* status, void* stream);
+
+/*
+ * Quantiser and scale variants of the search (NEXT f2):
+ *   quantizer  AWQ_QUANT_SYMMETRIC: delta = max|w'| / (2^(b-1)-1), codes in
+ *              +-(2^(b-1)-1) (as awq_search);
+ *              AWQ_QUANT_DELTA_POW2 (mudrobot.github.io notes, "analysing the
+ *              quantisation error"): delta = max|w'| / 2^(b-1), codes clamped to
+ *              [-2^(b-1), 2^(b-1)-1] (the passage gives no clamp; +max would
+ *              need b+1 bits).  Pack with AWQ_PACK_DELTA_POW2.
+ *   w_mean     NULL, or [D_in] device fp32 (awq_weight_mean): the candidate
+ *              scales are the balanced a^alpha / w_mean^(1-alpha); recover s*
+ *              with awq_scales_ex.
+ */
+#define AWQ_QUANT_SYMMETRIC 0
+#define AWQ_QUANT_DELTA_POW2 1
+typedef struct {
+  int quantizer;
+  const float* w_mean;
+} awq_search_options;
+
+/*
+ * awq_search with options (NULL = awq_search).  Same arguments, outputs,
+ * workspace size (awq_search_workspace_size) and errors.
+ */
+AWQ_API int awq_search_ex(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
+                          const float* alpha_grid, int n_alpha, int bits, int group, int loss_form,
+                          const awq_search_options* options, double* L, double* L_col, float* alpha_star,
+                          int32_t* alpha_idx, void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
 
 /* One layer of a batched search (see awq_search for the meaning of each field). */
 typedef struct {
@@ -258,6 +306,11 @@ AWQ_API int awq_quantize_pack_clip(const float* W, const float* s, const float* 
  *           `scales` is [D_in/group][D_out] fp32, as in awq_quantize_pack.
  */
 #define AWQ_PACK_DELTA_FP16 1
+/*   AWQ_PACK_DELTA_POW2: delta = max / 2^(b-1) (with any clip ratio applied
+ *           to max first), codes clamped to [-2^(b-1), 2^(b-1)-1]; the
+ *           quantiser of awq_search_ex's AWQ_QUANT_DELTA_POW2.  Combines with
+ *           AWQ_PACK_DELTA_FP16 (the power-of-two delta then rounded to FP16). */
+#define AWQ_PACK_DELTA_POW2 2
 AWQ_API int awq_quantize_pack_ex(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out,
                                  int bits, int group, int flags, uint32_t* packed, void* scales, void* stream);
 

@@ -30,7 +30,7 @@ EXPORTS = (
     "awq_get_last_error", "awq_version", "awq_profile_enable", "awq_profile_reset", "awq_profile_read",
     "awq_search_noalloc", "awq_clip_search_workspace_size", "awq_clip_search", "awq_quantize_pack_clip",
     "awq_search_joint_workspace_size", "awq_search_joint", "awq_quantize_pack_ex", "awq_w4a16_gemm",
-    "awq_w4a16_workspace_size",
+    "awq_w4a16_workspace_size", "awq_search_ex", "awq_weight_mean", "awq_scales_ex",
 )
 STAGES = ("act_stats", "scale_table", "search_operand", "search_gemm", "loss_reduce", "quantize_pack",
           "weight_t", "clip_gram", "clip_operand", "clip_loss", "w4a16")
@@ -64,8 +64,21 @@ def _sig(name, res, args):
 _act_stats = _sig("awq_act_stats", I, [P, I64, I64, I, P, P])
 _scales = _sig("awq_scales", I, [P, I64, F, P, P])
 _scales_dev = _sig("awq_scales_dev", I, [P, I64, P, P, P])
+_scales_ex = _sig("awq_scales_ex", I, [P, P, I64, F, P, P, P])
+_weight_mean = _sig("awq_weight_mean", I, [P, I64, I64, P, P])
 _search_ws = _sig("awq_search_workspace_size", SZ, [I64, I64, I64, I, I, I, I])
 _search = _sig("awq_search", I, [P, P, P, I64, I64, I64, P, I, I, I, I, P, P, P, P, P, SZ, P, P])
+
+
+class AwqSearchOptions(ctypes.Structure):
+    _fields_ = [("quantizer", ctypes.c_int), ("w_mean", P)]
+
+
+QUANT_SYMMETRIC = 0
+QUANT_DELTA_POW2 = 1
+PACK_DELTA_POW2 = 2
+_search_ex = _sig("awq_search_ex", I, [P, P, P, I64, I64, I64, P, I, I, I, I, ctypes.POINTER(AwqSearchOptions), P, P,
+                                       P, P, P, SZ, P, P])
 _batched_ws = _sig("awq_search_batched_workspace_size", SZ, [ctypes.POINTER(AwqLayer), I, I, I, I, I])
 _batched = _sig("awq_search_batched", I, [ctypes.POINTER(AwqLayer), I, P, I, I, I, I, P, SZ, P, P])
 _pack = _sig("awq_quantize_pack", I, [P, P, I64, I64, I, I, P, P, P])
@@ -128,11 +141,29 @@ def act_stats(X: torch.Tensor, stat: int = STAT_MEAN) -> torch.Tensor:
     return a
 
 
-def scales(a: torch.Tensor, alpha) -> torch.Tensor:
+def weight_mean(W: torch.Tensor) -> torch.Tensor:
+    """w_mean[j] = mean_n |W[j][n]|: ``awq_weight_mean`` (the weight statistic
+    of the balanced scale)."""
+    W = _dev(W, torch.float32, "W")
+    out = torch.empty(W.shape[0], dtype=torch.float32, device=W.device)
+    _check(_weight_mean(_ptr(W), W.shape[0], W.shape[1], _ptr(out), _stream()))
+    return out
+
+
+def scales(a: torch.Tensor, alpha, w_mean: Optional[torch.Tensor] = None) -> torch.Tensor:
     """s = a^alpha (floored): ``awq_scales`` for a host alpha, ``awq_scales_dev``
-    when alpha is a one-element CUDA tensor."""
+    when alpha is a one-element CUDA tensor; with w_mean the balanced
+    a^alpha / w_mean^(1 - alpha) (``awq_scales_ex``)."""
     a = _dev(a, torch.float32, "a")
     s = torch.empty_like(a)
+    if w_mean is not None:
+        b = _dev(w_mean, torch.float32, "w_mean")
+        if isinstance(alpha, torch.Tensor):
+            al = _dev(alpha.reshape(1), torch.float32, "alpha")
+            _check(_scales_ex(_ptr(a), _ptr(b), a.numel(), 0.0, _ptr(al), _ptr(s), _stream()))
+        else:
+            _check(_scales_ex(_ptr(a), _ptr(b), a.numel(), float(alpha), None, _ptr(s), _stream()))
+        return s
     if isinstance(alpha, torch.Tensor):
         al = _dev(alpha.reshape(1), torch.float32, "alpha")
         _check(_scales_dev(_ptr(a), a.numel(), _ptr(al), _ptr(s), _stream()))
@@ -176,8 +207,10 @@ _default_ws = Workspace()
 
 def search(X: torch.Tensor, W: torch.Tensor, a: torch.Tensor, alpha_grid: Sequence[float], bits: int = 4,
            group: int = 128, want_cols: bool = False, workspace: Optional[Workspace] = None,
-           check_status: bool = True, loss_form: int = LOSS_ERROR) -> SearchResult:
-    """Grid search over alpha for one layer: ``awq_search``."""
+           check_status: bool = True, loss_form: int = LOSS_ERROR, quantizer: int = QUANT_SYMMETRIC,
+           w_mean: Optional[torch.Tensor] = None) -> SearchResult:
+    """Grid search over alpha for one layer: ``awq_search``, or
+    ``awq_search_ex`` with a quantiser variant or the balanced scale."""
     X = _dev(X, torch.bfloat16, "X")
     W = _dev(W, torch.float32, "W")
     a = _dev(a, torch.float32, "a")
@@ -193,8 +226,15 @@ def search(X: torch.Tensor, W: torch.Tensor, a: torch.Tensor, alpha_grid: Sequen
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     nbytes = search_workspace_size(N, D_in, D_out, A, bits, group, loss_form)
     ws = (workspace or _default_ws).get(nbytes, dev)
-    _check(_search(_ptr(X), _ptr(W), _ptr(a), N, D_in, D_out, grid, A, bits, group, loss_form, _ptr(L), _ptr(Lc),
-                   _ptr(astar), _ptr(aidx), _ptr(ws), ws.numel(), _ptr(status), _stream()))
+    if quantizer == QUANT_SYMMETRIC and w_mean is None:
+        _check(_search(_ptr(X), _ptr(W), _ptr(a), N, D_in, D_out, grid, A, bits, group, loss_form, _ptr(L), _ptr(Lc),
+                       _ptr(astar), _ptr(aidx), _ptr(ws), ws.numel(), _ptr(status), _stream()))
+    else:
+        b = None if w_mean is None else _dev(w_mean, torch.float32, "w_mean")
+        opts = AwqSearchOptions(int(quantizer), _ptr(b))
+        _check(_search_ex(_ptr(X), _ptr(W), _ptr(a), N, D_in, D_out, grid, A, bits, group, loss_form,
+                          ctypes.byref(opts), _ptr(L), _ptr(Lc), _ptr(astar), _ptr(aidx), _ptr(ws), ws.numel(),
+                          _ptr(status), _stream()))
     res = SearchResult(L, astar, aidx, Lc, status)
     if check_status:
         check_device_status(status)
@@ -239,7 +279,7 @@ def clip_search(X: torch.Tensor, W: torch.Tensor, s: torch.Tensor, clip_grid: Se
 
 
 def quantize_pack_ex(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int = 128,
-                     clip: Optional[torch.Tensor] = None, delta_fp16: bool = False):
+                     clip: Optional[torch.Tensor] = None, delta_fp16: bool = False, delta_pow2: bool = False):
     """``awq_quantize_pack_ex``: the final pack with optional clip ratios and
     FP16 deltas.  Returns (packed int32 view [D_in/8, D_out], scales
     [D_in/group, D_out] as float16 when delta_fp16 else float32)."""
@@ -250,8 +290,8 @@ def quantize_pack_ex(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int
     D_in, D_out = W.shape
     packed = torch.empty(D_in // 8, D_out, dtype=torch.int32, device=W.device)
     sc = torch.empty(D_in // group, D_out, dtype=torch.float16 if delta_fp16 else torch.float32, device=W.device)
-    _check(_pack_ex(_ptr(W), _ptr(s), _ptr(clip), D_in, D_out, bits, group, PACK_DELTA_FP16 if delta_fp16 else 0,
-                    _ptr(packed), _ptr(sc), _stream()))
+    flags = (PACK_DELTA_FP16 if delta_fp16 else 0) | (PACK_DELTA_POW2 if delta_pow2 else 0)
+    _check(_pack_ex(_ptr(W), _ptr(s), _ptr(clip), D_in, D_out, bits, group, flags, _ptr(packed), _ptr(sc), _stream()))
     return packed, sc
 
 

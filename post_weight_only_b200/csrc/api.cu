@@ -177,12 +177,18 @@ void prof_collect() {
     if (_rc != AWQ_OK) return _rc; \
   } while (0)
 
+// Quantiser and scale variants of the search (awq_search_ex).
+struct SearchOpts {
+  int qmode = awq::kQuantSymmetric;
+  const float* w_mean = nullptr;    // balanced scale a^alpha / w_mean^(1 - alpha) when set
+};
+
 // The search for one layer with a workspace already checked; does not reset
 // the status word.
 int search_one(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
                const awq::AlphaList& alphas, int A, int bits, int group, int form, double* L, double* L_col,
                float* alpha_star, int32_t* alpha_idx, uint8_t* ws, int32_t* status, cudaStream_t st,
-               int num_sms) {
+               int num_sms, const SearchOpts& opts = SearchOpts()) {
   const SearchLayout lay = search_layout(N, D_in, D_out, A, group, form, num_sms);
   float* s_tab = reinterpret_cast<float*>(ws + lay.s_tab);
   float* r_tab = reinterpret_cast<float*>(ws + lay.r_tab);
@@ -195,12 +201,12 @@ int search_one(const void* X, const float* W, const float* a, int64_t N, int64_t
   cudaError_t e;
   {
     StageTimer t(AWQ_STAGE_SCALE_TABLE, st);
-    e = awq::launch_scale_table(a, D_in, alphas, nullptr, A, s_tab, r_tab, st);
+    e = awq::launch_scale_table(a, opts.w_mean, D_in, alphas, nullptr, A, s_tab, r_tab, st);
   }
   if (e != cudaSuccess) return fail_cuda(e, "scale table kernel");
   {
     StageTimer t(AWQ_STAGE_SEARCH_OPERAND, st);
-    e = awq::launch_search_operand(W, s_tab, r_tab, D_in, D_out, A, bits, group, form, op, st);
+    e = awq::launch_search_operand(W, s_tab, r_tab, D_in, D_out, A, bits, group, form, opts.qmode, op, st);
   }
   if (e != cudaSuccess) return fail_cuda(e, "search operand kernel");
   if (wt) {
@@ -295,10 +301,12 @@ int awq_act_stats(const void* X, int64_t N, int64_t D_in, int stat, float* a, vo
   return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "act_stats kernel");
 }
 
-static int scales_common(const float* a, int64_t D_in, float alpha, const float* alpha_dev, float* s, void* stream) {
+static int scales_common(const float* a, const float* w_mean, int64_t D_in, float alpha, const float* alpha_dev,
+                         float* s, void* stream) {
   if (D_in < 1 || D_in > kMaxDim) return fail(AWQ_EINVAL, "D_in = %lld out of range", (long long)D_in);
   AWQ_TRY(check_ptr(a, "a", 4));
   AWQ_TRY(check_ptr(s, "s", 4));
+  if (w_mean) AWQ_TRY(check_ptr(w_mean, "w_mean", 4));
   int sms = 0;
   AWQ_TRY(device_info(&sms));
   awq::AlphaList al{};
@@ -306,18 +314,36 @@ static int scales_common(const float* a, int64_t D_in, float alpha, const float*
   cudaError_t e;
   {
     StageTimer t(AWQ_STAGE_SCALE_TABLE, static_cast<cudaStream_t>(stream));
-    e = awq::launch_scale_table(a, D_in, al, alpha_dev, 1, s, nullptr, static_cast<cudaStream_t>(stream));
+    e = awq::launch_scale_table(a, w_mean, D_in, al, alpha_dev, 1, s, nullptr, static_cast<cudaStream_t>(stream));
   }
   return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "scale table kernel");
 }
 
 int awq_scales(const float* a, int64_t D_in, float alpha, float* s, void* stream) {
-  return scales_common(a, D_in, alpha, nullptr, s, stream);
+  return scales_common(a, nullptr, D_in, alpha, nullptr, s, stream);
 }
 
 int awq_scales_dev(const float* a, int64_t D_in, const float* alpha_dev, float* s, void* stream) {
   AWQ_TRY(check_ptr(alpha_dev, "alpha_dev", 4));
-  return scales_common(a, D_in, 0.0f, alpha_dev, s, stream);
+  return scales_common(a, nullptr, D_in, 0.0f, alpha_dev, s, stream);
+}
+
+int awq_scales_ex(const float* a, const float* w_mean, int64_t D_in, float alpha, const float* alpha_dev, float* s,
+                  void* stream) {
+  if (alpha_dev) AWQ_TRY(check_ptr(alpha_dev, "alpha_dev", 4));
+  if (!alpha_dev && !(alpha >= 0.0f && alpha <= 1.0f)) return fail(AWQ_EINVAL, "alpha = %g: need 0 <= alpha <= 1", alpha);
+  return scales_common(a, w_mean, D_in, alpha, alpha_dev, s, stream);
+}
+
+int awq_weight_mean(const float* W, int64_t D_in, int64_t D_out, float* w_mean, void* stream) {
+  if (D_in < 1 || D_in > kMaxDim || D_out < 1 || D_out > kMaxDim)
+    return fail(AWQ_EINVAL, "D_in = %lld, D_out = %lld out of range", (long long)D_in, (long long)D_out);
+  AWQ_TRY(check_ptr(W, "W", 16));
+  AWQ_TRY(check_ptr(w_mean, "w_mean", 4));
+  int sms = 0;
+  AWQ_TRY(device_info(&sms));
+  cudaError_t e = awq::launch_weight_mean(W, D_in, D_out, w_mean, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "weight mean kernel");
 }
 
 size_t awq_search_workspace_size(int64_t N, int64_t D_in, int64_t D_out, int n_alpha, int bits, int group,
@@ -330,10 +356,10 @@ size_t awq_search_workspace_size(int64_t N, int64_t D_in, int64_t D_out, int n_a
   return search_layout(N, D_in, D_out, n_alpha, group, loss_form, sms).total;
 }
 
-int awq_search(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
-               const float* alpha_grid, int n_alpha, int bits, int group, int loss_form, double* L, double* L_col,
-               float* alpha_star, int32_t* alpha_idx, void* workspace, size_t workspace_bytes, int32_t* status,
-               void* stream) {
+static int search_impl(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
+                       const float* alpha_grid, int n_alpha, int bits, int group, int loss_form, double* L,
+                       double* L_col, float* alpha_star, int32_t* alpha_idx, void* workspace, size_t workspace_bytes,
+                       int32_t* status, void* stream, const SearchOpts& opts) {
   AWQ_TRY(check_search_args(X, W, a, N, D_in, D_out, alpha_grid, n_alpha, bits, group, loss_form, L, L_col,
                             alpha_star, alpha_idx));
   int sms = 0;
@@ -352,7 +378,31 @@ int awq_search(const void* X, const float* W, const float* a, int64_t N, int64_t
   awq::AlphaList al{};
   for (int i = 0; i < n_alpha; ++i) al.v[i] = alpha_grid[i];
   return search_one(X, W, a, N, D_in, D_out, al, n_alpha, bits, group, loss_form, L, L_col, alpha_star, alpha_idx,
-                    ws, st_word, st, sms);
+                    ws, st_word, st, sms, opts);
+}
+
+int awq_search(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
+               const float* alpha_grid, int n_alpha, int bits, int group, int loss_form, double* L, double* L_col,
+               float* alpha_star, int32_t* alpha_idx, void* workspace, size_t workspace_bytes, int32_t* status,
+               void* stream) {
+  return search_impl(X, W, a, N, D_in, D_out, alpha_grid, n_alpha, bits, group, loss_form, L, L_col, alpha_star,
+                     alpha_idx, workspace, workspace_bytes, status, stream, SearchOpts());
+}
+
+int awq_search_ex(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
+                  const float* alpha_grid, int n_alpha, int bits, int group, int loss_form,
+                  const awq_search_options* options, double* L, double* L_col, float* alpha_star,
+                  int32_t* alpha_idx, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  SearchOpts o;
+  if (options) {
+    if (options->quantizer != AWQ_QUANT_SYMMETRIC && options->quantizer != AWQ_QUANT_DELTA_POW2)
+      return fail(AWQ_EINVAL, "quantizer = %d: need AWQ_QUANT_SYMMETRIC or AWQ_QUANT_DELTA_POW2", options->quantizer);
+    if (options->w_mean) AWQ_TRY(check_ptr(options->w_mean, "w_mean", 4));
+    o.qmode = options->quantizer == AWQ_QUANT_DELTA_POW2 ? awq::kQuantPow2 : awq::kQuantSymmetric;
+    o.w_mean = options->w_mean;
+  }
+  return search_impl(X, W, a, N, D_in, D_out, alpha_grid, n_alpha, bits, group, loss_form, L, L_col, alpha_star,
+                     alpha_idx, workspace, workspace_bytes, status, stream, o);
 }
 
 size_t awq_search_batched_workspace_size(const awq_layer* layers, int n_layers, int n_alpha, int bits, int group,
@@ -629,7 +679,7 @@ int awq_quantize_pack_clip(const float* W, const float* s, const float* clip, in
 int awq_quantize_pack_ex(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out, int bits,
                          int group, int flags, uint32_t* packed, void* scales, void* stream) {
   AWQ_TRY(check_quant_args(bits, group));
-  if (flags & ~AWQ_PACK_DELTA_FP16) return fail(AWQ_EINVAL, "flags = %#x: unknown bits", flags);
+  if (flags & ~(AWQ_PACK_DELTA_FP16 | AWQ_PACK_DELTA_POW2)) return fail(AWQ_EINVAL, "flags = %#x: unknown bits", flags);
   if (D_in < group || D_in > kMaxDin || D_in % group)
     return fail(AWQ_EINVAL, "D_in = %lld: need a positive multiple of group = %d", (long long)D_in, group);
   if (D_out < 1 || D_out > kMaxDim) return fail(AWQ_EINVAL, "D_out = %lld out of range", (long long)D_out);
@@ -643,7 +693,8 @@ int awq_quantize_pack_ex(const float* W, const float* s, const float* clip, int6
   cudaError_t e;
   {
     StageTimer t(AWQ_STAGE_QUANTIZE_PACK, static_cast<cudaStream_t>(stream));
-    e = awq::launch_quantize_pack(W, s, clip, D_in, D_out, bits, group, (flags & AWQ_PACK_DELTA_FP16) != 0, packed,
+    e = awq::launch_quantize_pack(W, s, clip, D_in, D_out, bits, group, (flags & AWQ_PACK_DELTA_FP16) != 0,
+                                  (flags & AWQ_PACK_DELTA_POW2) ? awq::kQuantPow2 : awq::kQuantSymmetric, packed,
                                   scales, sms, static_cast<cudaStream_t>(stream));
   }
   return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "quantize_pack kernel");

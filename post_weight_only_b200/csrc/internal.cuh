@@ -10,6 +10,11 @@ namespace awq {
 
 constexpr int kMaxAlpha = 64;
 
+// Quantisers: delta = max / (2^(b-1) - 1), codes +-(2^(b-1) - 1); or the
+// power-of-two delta = max / 2^(b-1), codes [-2^(b-1), 2^(b-1) - 1].
+constexpr int kQuantSymmetric = 0;
+constexpr int kQuantPow2 = 1;
+
 // Loss forms of the search (see search.cu).
 constexpr int kFormError = 0;        // L = ||X E||^2 with E = S^-1 Q(S W) - W as the MMA operand
 constexpr int kFormReference = 1;    // L = ||X S^-1 Q(S W) - X W||^2, reference output subtracted
@@ -26,14 +31,17 @@ cudaError_t launch_act_stats(const uint16_t* X, int64_t N, int64_t D, int stat, 
 // ---- scales.cu
 // s_tab [A][D] (may be null), r_tab [A][D] = fl32(1 / s) (may be null).
 // alpha_dev != null: a single alpha read from device memory (A must be 1).
-cudaError_t launch_scale_table(const float* a, int64_t D, const AlphaList& alphas, const float* alpha_dev, int A,
-                               float* s_tab, float* r_tab, cudaStream_t st);
+// b != null: the balanced scale a^alpha / b^(1 - alpha).
+cudaError_t launch_scale_table(const float* a, const float* b, int64_t D, const AlphaList& alphas,
+                               const float* alpha_dev, int A, float* s_tab, float* r_tab, cudaStream_t st);
+// b [D_in] = mean_n |W[j][n]| (fp64 sums, one rounding).
+cudaError_t launch_weight_mean(const float* W, int64_t D_in, int64_t D_out, float* b, cudaStream_t st);
 
 // ---- quant.cu
 // The search's A operand for every alpha, bf16 [A][D_out][D_in]: error form
 // (S^-1 Q(S W) - W)^T, reference form (S^-1 Q(S W))^T.  See quant.cu.
 cudaError_t launch_search_operand(const float* W, const float* s_tab, const float* r_tab, int64_t D_in,
-                                  int64_t D_out, int A, int bits, int group, int form, uint16_t* op,
+                                  int64_t D_out, int A, int bits, int group, int form, int qmode, uint16_t* op,
                                   cudaStream_t st);
 // The clipping search's operand for every clip ratio c of `clips`, bf16
 // [n_clip][D_out][D_in]: (S^-1 Q_c(S W) - W)^T with the group maximum scaled
@@ -47,8 +55,8 @@ cudaError_t launch_weight_t(const float* W, int64_t D_in, int64_t D_out, uint16_
 // clip [D_in/group][D_out] (may be null) scales each group maximum; delta16:
 // delta rounded to FP16 before the codes, scales stored as FP16 (else fp32).
 cudaError_t launch_quantize_pack(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out,
-                                 int bits, int group, bool delta16, uint32_t* packed, void* scales, int num_sms,
-                                 cudaStream_t st);
+                                 int bits, int group, bool delta16, int qmode, uint32_t* packed, void* scales,
+                                 int num_sms, cudaStream_t st);
 
 // ---- reduce.cu
 cudaError_t launch_loss_reduce(const float* partial, int A, int H, int64_t D_out, double* L_col, double* blk,

@@ -29,13 +29,15 @@ def activations64(X):
     return x, (x ** 2).sum(axis=0)
 
 
-def rounding_bound(X, W, a, alpha, bits, group, form="error", cols=None, k_sigma=6.0, x64=None):
+def rounding_bound(X, W, a, alpha, bits, group, form="error", cols=None, k_sigma=6.0, x64=None,
+                   qmode=0, w_mean=None):
     """Per-column bound on |L_gpu - L| for the columns `cols` (all if None).
     Only those columns of W are quantised and expanded: the quantiser works
-    column by column.  x64 = activations64(X) may be passed to save its cost."""
-    s = oracle.scales(a, alpha).astype(np.float64)
+    column by column.  x64 = activations64(X) may be passed to save its cost.
+    qmode / w_mean: the quantiser and scale variants (see oracle.search)."""
+    s = oracle.scales(a, alpha, w_mean=w_mean).astype(np.float64)
     Wc = W if cols is None else W[:, np.asarray(cols)].contiguous()
-    q, d = oracle.quantize(Wc, s.astype(np.float32), bits, group)
+    q, d = oracle.quantize(Wc, s.astype(np.float32), bits, group, qmode=qmode)
     w = Wc.numpy().astype(np.float64)
     step = np.repeat(d, group, axis=0).astype(np.float64) / s[:, None]      # delta / s_k
     w_hat = q.astype(np.float64) * step

@@ -140,6 +140,36 @@ def test_argument_checks_without_gpu(lib):
     assert gcall(wsb=gws(16, 256, 64) - 1) == 4
     assert gcall(st=None) == 1                             # the status word is required
 
+    class Opts(ctypes.Structure):
+        _fields_ = [("quantizer", ctypes.c_int), ("w_mean", ctypes.c_void_p)]
+
+    x = lib.awq_search_ex
+    x.argtypes = [P, P, P, I64, I64, I64, P, I, I, I, I, ctypes.POINTER(Opts), P, P, P, P, P, ctypes.c_size_t, P, P]
+    x.restype = I
+
+    def xcall(opts, **kw):
+        d = dict(args, **kw)
+        return x(d["X"], d["W"], d["a"], d["N"], d["D_in"], d["D_out"], d["grid"], d["A"], d["bits"], d["group"],
+                 d["form"], opts, d["L"], d["Lc"], d["astar"], d["aidx"], d["ws"], d["wsb"], d["st"], d["stream"])
+
+    assert xcall(ctypes.byref(Opts(2, None))) == 1           # unknown quantiser
+    assert xcall(ctypes.byref(Opts(1, fake + 2))) == 2       # misaligned weight means
+    assert xcall(ctypes.byref(Opts(1, None)), bits=5) == 3   # the common checks still apply
+    wm = lib.awq_weight_mean
+    wm.argtypes = [P, I64, I64, P, P]
+    wm.restype = I
+    assert wm(fake, 0, 16, fake, None) == 1
+    assert wm(fake + 4, 16, 16, fake, None) == 2
+    se = lib.awq_scales_ex
+    se.argtypes = [P, P, I64, ctypes.c_float, P, P, P]
+    se.restype = I
+    assert se(fake, fake, 16, 1.5, None, fake, None) == 1    # alpha outside [0, 1]
+    assert se(fake, fake + 2, 16, 0.5, None, fake, None) == 2
+    pe = lib.awq_quantize_pack_ex
+    pe.argtypes = [P, P, P, I64, I64, I, I, I, P, P, P]
+    pe.restype = I
+    assert pe(fake, fake, None, 256, 64, 4, 128, 4, fake, fake, None) == 1   # unknown flag bit
+
     t = lib.awq_selftest_wait_timeout
     t.argtypes = [P, I64, P]
     t.restype = I

@@ -1,0 +1,165 @@
+"""GPU parity of the quantiser and scale variants of the search (NEXT f2)
+against the CPU oracle, through the C ABI.
+
+  * the power-of-two delta (mudrobot.github.io AWQ notes, "analysing the
+    quantisation error": delta = max|w| / 2^(b-1), codes clamped to b bits):
+    the final pack bit-exact (codes, packed words, deltas) on both pack
+    kernels, alone and with clip ratios and FP16 deltas; the search's losses
+    within the arithmetic's bound and relative 1e-2, alpha* by the contract's
+    rule;
+  * the balanced scale (zhihu AWQ/GPTQ/SmoothQuant comparison, the
+    per-channel scale s_j = mean|X_j|^alpha / mean|W_j|^(1-alpha)): the weight
+    statistic within relative 1e-6 (fp64 sums in another order), the scales
+    within one fp32 ulp (fp64 powers from two math libraries), the search as
+    above with the GPU's weight statistic given to both sides.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_bounds import check_alpha, rounding_bound
+from post_weight_only_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+L_RTOL = 1e-2
+
+
+@pytest.fixture(scope="module")
+def awq():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from post_weight_only_b200 import awq as mod
+    return mod
+
+
+def _layer(N, D_in, D_out, seed=0):
+    return synth.layer_inputs(synth.small_layer(N, D_in, D_out, seed=seed))
+
+
+def _ulps(x, y):
+    xi = x.astype(np.float32).view(np.int32).astype(np.int64)
+    yi = y.astype(np.float32).view(np.int32).astype(np.int64)
+    return np.abs(xi - yi)
+
+
+# ---------------------------------------------------------------- power-of-two delta
+@pytest.mark.parametrize("bits,group,D_in,D_out,delta16,clip", [
+    (4, 128, 512, 256, False, False),     # tiled pack kernel
+    (3, 64, 384, 200, False, False),
+    (2, 32, 96, 36, False, False),
+    (4, 128, 256, 203, False, False),     # D_out % 4 != 0: the untiled kernel
+    (4, 64, 256, 128, True, False),       # with FP16 deltas
+    (4, 128, 256, 131, True, True),       # FP16 deltas and clip ratios, untiled
+    (4, 128, 512, 128, False, True),      # clip ratios, tiled
+])
+def test_pack_pow2_bit_exact(awq, bits, group, D_in, D_out, delta16, clip):
+    X, W = _layer(16, D_in, D_out, seed=D_in + D_out)
+    s = oracle.scales(oracle.act_stats(X).astype(np.float32), 0.4)
+    c = None
+    if clip:
+        rng = np.random.default_rng(D_out)
+        c = synth.clip_grid(20).numpy()[rng.integers(0, 21, size=(D_in // group, D_out))]
+    packed, sc = awq.quantize_pack_ex(W.cuda(), torch.from_numpy(s).cuda(), bits, group,
+                                      clip=None if c is None else torch.from_numpy(c).cuda(),
+                                      delta_fp16=delta16, delta_pow2=True)
+    q, d = oracle.quantize(W, s, bits, group, clip=c, delta16=delta16, qmode=oracle.QMODE_POW2)
+    assert q.min() >= -(1 << (bits - 1)) and q.max() <= (1 << (bits - 1)) - 1
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), oracle.pack(q, bits))
+    got = sc.cpu().numpy()
+    assert np.array_equal(got.astype(np.float32) if delta16 else got, d)
+
+
+def test_pack_pow2_codes_reach_both_ends(awq):
+    """The largest magnitude of a group sits at code 2^(b-1) - 1 when
+    positive and at -2^(b-1) when negative."""
+    W = torch.zeros(128, 8)
+    W[3, :4] = 1.0
+    W[5, 4:] = -1.0
+    W[7, :] = 0.3
+    s = torch.ones(128)
+    packed, sc = awq.quantize_pack_ex(W.cuda(), s.cuda(), 4, 128, delta_pow2=True)
+    q, d = oracle.quantize(W, s.numpy(), 4, 128, qmode=oracle.QMODE_POW2)
+    assert q[3, :4].tolist() == [7] * 4 and q[5, 4:].tolist() == [-8] * 4
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), oracle.pack(q, 4))
+
+
+@pytest.mark.parametrize("form", ("error", "reference"))
+@pytest.mark.parametrize("N,D_in,D_out,bits,group", [
+    (300, 512, 200, 4, 128),
+    (97, 96, 132, 2, 32),
+    (64, 256, 128, 3, 64),
+])
+def test_search_pow2_against_oracle(awq, form, N, D_in, D_out, bits, group):
+    X, W = _layer(N, D_in, D_out, seed=N + D_out)
+    a = oracle.act_stats(X).astype(np.float32)
+    alphas = synth.alpha_grid(20).numpy()
+    lf = awq.LOSS_ERROR if form == "error" else awq.LOSS_REFERENCE
+    res = awq.search(X.cuda(), W.cuda(), torch.from_numpy(a).cuda(), alphas.tolist(), bits, group, loss_form=lf,
+                     quantizer=awq.QUANT_DELTA_POW2)
+    L_gpu = res.L.cpu().numpy()
+    L_or, best = oracle.search(X, W, a, alphas, bits, group, qmode=oracle.QMODE_POW2)
+    for i, al in enumerate(alphas):
+        bound = rounding_bound(X, W, a, al, bits, group, form, qmode=oracle.QMODE_POW2).sum()
+        err = abs(L_gpu[i] - L_or[i])
+        assert err <= bound, (al, L_gpu[i], L_or[i], bound)
+        if form == "error":
+            assert err <= L_RTOL * L_or[i], (al, err / L_or[i])
+    check_alpha(L_or, best, int(res.alpha_idx.item()))
+
+
+# ---------------------------------------------------------------- balanced scale
+@pytest.mark.parametrize("D_in,D_out", [(512, 256), (4096, 4096), (96, 36), (1, 8)])
+def test_weight_mean(awq, D_in, D_out):
+    rng = np.random.default_rng(D_in)
+    W = (rng.standard_normal((D_in, D_out)) * np.exp(rng.standard_normal((D_in, 1)))).astype(np.float32)
+    b = awq.weight_mean(torch.from_numpy(W).cuda()).cpu().numpy()
+    assert np.allclose(b, oracle.weight_mean(W), rtol=1e-6, atol=0)
+
+
+@pytest.mark.parametrize("alpha", [0.0, 0.3, 0.5, 1.0])
+def test_balanced_scales(awq, alpha):
+    rng = np.random.default_rng(3)
+    a = (rng.random(1000) + 0.01).astype(np.float32)
+    b = (rng.random(1000) + 0.01).astype(np.float32)
+    a[7] = 0.0
+    b[9] = 0.0                                            # both floors
+    s_gpu = awq.scales(torch.from_numpy(a).cuda(), alpha, w_mean=torch.from_numpy(b).cuda()).cpu().numpy()
+    s_or = oracle.scales(a, alpha, w_mean=b)
+    assert np.all(_ulps(s_gpu, s_or) <= 1), np.max(_ulps(s_gpu, s_or))
+    assert np.mean(s_gpu == s_or) > 0.999
+    # the device-alpha form gives the same values
+    s_dev = awq.scales(torch.from_numpy(a).cuda(), torch.tensor([alpha], device="cuda"),
+                       w_mean=torch.from_numpy(b).cuda()).cpu().numpy()
+    assert np.array_equal(s_dev, s_gpu)
+
+
+@pytest.mark.parametrize("form", ("error", "reference"))
+@pytest.mark.parametrize("N,D_in,D_out,bits,group", [
+    (300, 512, 200, 4, 128),
+    (130, 256, 64, 4, 64),
+])
+def test_search_balanced_against_oracle(awq, form, N, D_in, D_out, bits, group):
+    X, W = _layer(N, D_in, D_out, seed=N + 3 * D_out)
+    a = oracle.act_stats(X).astype(np.float32)
+    b_dev = awq.weight_mean(W.cuda())
+    b = b_dev.cpu().numpy()
+    alphas = synth.alpha_grid(20).numpy()
+    lf = awq.LOSS_ERROR if form == "error" else awq.LOSS_REFERENCE
+    res = awq.search(X.cuda(), W.cuda(), torch.from_numpy(a).cuda(), alphas.tolist(), bits, group, loss_form=lf,
+                     w_mean=b_dev)
+    L_gpu = res.L.cpu().numpy()
+    L_or, best = oracle.search(X, W, a, alphas, bits, group, w_mean=b)
+    for i, al in enumerate(alphas):
+        bound = rounding_bound(X, W, a, al, bits, group, form, w_mean=b).sum()
+        err = abs(L_gpu[i] - L_or[i])
+        assert err <= bound, (al, L_gpu[i], L_or[i], bound)
+        if form == "error":
+            assert err <= L_RTOL * L_or[i], (al, err / L_or[i])
+    check_alpha(L_or, best, int(res.alpha_idx.item()))
+    # s* on the device from alpha* and the pack bit-exact for it
+    s_star = awq.scales(torch.from_numpy(a).cuda(), res.alpha_star, w_mean=b_dev)
+    packed, sc = awq.quantize_pack(W.cuda(), s_star, bits, group)
+    q, d = oracle.quantize(W, s_star.cpu().numpy(), bits, group)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), oracle.pack(q, bits))
