@@ -33,7 +33,7 @@
  *   - Inputs are assumed finite; NaN or Inf inputs give unspecified (but
  *     memory-safe) results.
  *   - Supported bit widths are 2, 3 and 4 (codes are stored as 4-bit
- *     offset-binary values); group sizes are 32, 64 and 128.
+ *     offset-binary values); group sizes are 32, 64, 128 and 256.
  */
 #ifndef AWQ_B200_H
 #define AWQ_B200_H
@@ -145,7 +145,7 @@ AWQ_API size_t awq_search_workspace_size(int64_t N, int64_t D_in, int64_t D_out,
  * order.
  *   X           [N][D_in] bf16;  W [D_in][D_out] fp32;  a [D_in] fp32
  *   alpha_grid  HOST array of n_alpha fp32 values, 1 <= n_alpha <= 64
- *   bits        2, 3 or 4;  group 32, 64 or 128;  D_in % group == 0,
+ *   bits        2, 3 or 4;  group 32, 64, 128 or 256;  D_in % group == 0,
  *               D_in <= 2^20, D_out % 4 == 0, D_out <= 2^24, 1 <= N <= 2^24
  *   loss_form   AWQ_LOSS_ERROR or AWQ_LOSS_REFERENCE
  *   L           [n_alpha] fp64 output (device)
@@ -329,7 +329,7 @@ AWQ_API int awq_quantize_pack_ex(const float* W, const float* s, const float* cl
  * CTAs is summed from partial tiles in the workspace in a fixed order, so
  * the result is deterministic.
  *   X         [N][D_in] bf16;  s [D_in] fp32 (s*);  packed [D_in/8][D_out] uint32
- *   scales    [D_in/group][D_out] fp32;  bits 2..4;  group 32, 64 or 128
+ *   scales    [D_in/group][D_out] fp32;  bits 2..4;  group 32, 64, 128 or 256
  *   D_out     a multiple of 4 (the rows of packed words are read by TMA)
  *   Y         [N][D_out] fp32 output
  *   workspace at least awq_w4a16_workspace_size(N, D_in, D_out) bytes: the

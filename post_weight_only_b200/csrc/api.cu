@@ -104,8 +104,8 @@ int check_form(int form) {
 
 int check_quant_args(int bits, int group) {
   if (bits < 2 || bits > 4) return fail(AWQ_EUNSUPPORTED, "bits = %d: supported bit widths are 2, 3 and 4", bits);
-  if (group != 32 && group != 64 && group != 128)
-    return fail(AWQ_EUNSUPPORTED, "group = %d: supported group sizes are 32, 64 and 128", group);
+  if (group != 32 && group != 64 && group != 128 && group != 256)
+    return fail(AWQ_EUNSUPPORTED, "group = %d: supported group sizes are 32, 64, 128 and 256", group);
   return AWQ_OK;
 }
 

@@ -567,6 +567,7 @@ int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const fl
     case 32: kern = w4a16_kernel<32>; break;
     case 64: kern = w4a16_kernel<64>; break;
     case 128: kern = w4a16_kernel<128>; break;
+    case 256: kern = w4a16_kernel<256>; break;
     default:
       *what = "group";
       return kEUnsupported;

@@ -72,6 +72,8 @@ def test_argument_checks_without_gpu(lib):
     assert call(bits=5) == 3
     assert call(bits=1) == 3
     assert call(group=96) == 3
+    assert call(group=512) == 3
+    assert call(group=256, D_in=384) == 1                 # not a multiple of group 256
     assert call(D_in=192) == 1                            # not a multiple of group 128
     assert call(A=0) == 3
     assert call(A=65) == 3
@@ -133,7 +135,7 @@ def test_argument_checks_without_gpu(lib):
 
     assert gcall(D_out=66) == 1                           # rows of packed words must be 16-byte multiples
     assert gcall(N=0) == 1
-    assert gcall(group=256) == 3
+    assert gcall(group=512) == 3
     assert gcall(D_in=192) == 1
     assert gcall(s=fake + 4) == 2                          # s is read as float4
     assert gcall(ws=None) == 4

@@ -95,7 +95,7 @@ def test_scales_from_device_alpha(awq):
 
 
 # ------------------------------------------------------------------ quantise + pack
-@pytest.mark.parametrize("bits,group", [(4, 128), (4, 64), (3, 128), (2, 32), (3, 32)])
+@pytest.mark.parametrize("bits,group", [(4, 128), (4, 64), (3, 128), (2, 32), (3, 32), (4, 256)])
 @pytest.mark.parametrize("D_in,D_out", [(256, 200), (1024, 4096)])
 def test_quantize_pack_bit_exact(awq, bits, group, D_in, D_out):
     X, W = _layer(32, D_in, D_out, seed=D_out + bits)
@@ -114,6 +114,8 @@ def test_quantize_pack_bit_exact(awq, bits, group, D_in, D_out):
     (4, 32, 96, 200),      # the last 128-row tile reaches past D_in
     (3, 64, 192, 132),     # same, two groups per tile
     (4, 64, 320, 4100),    # ragged last column tile
+    (4, 256, 768, 132),    # group 256: the untiled kernel, 64 rows per thread
+    (3, 256, 256, 7),
 ])
 def test_quantize_pack_ragged(awq, bits, group, D_in, D_out):
     X, W = _layer(16, D_in, D_out, seed=D_in + D_out)
@@ -193,6 +195,7 @@ def _search_both(awq, X, W, bits, group, alphas, cols=None, form="error"):
     (97, 96, 132, 2, 32, 8),         # D_in not a multiple of 64; two groups per stage
     (1, 512, 1024, 4, 128, 20),      # a single token
     (700, 384, 4, 4, 128, 20),       # four output columns (one ragged tile)
+    (300, 768, 200, 4, 256, 20),     # group 256 (16 threads per column in the pre-pass)
 ])
 def test_search_small(awq, form, N, D_in, D_out, bits, group, n_int):
     """Every alpha within the arithmetic's own bound; within relative 1e-2 of

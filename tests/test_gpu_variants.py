@@ -53,6 +53,7 @@ def _ulps(x, y):
     (4, 64, 256, 128, True, False),       # with FP16 deltas
     (4, 128, 256, 131, True, True),       # FP16 deltas and clip ratios, untiled
     (4, 128, 512, 128, False, True),      # clip ratios, tiled
+    (4, 256, 512, 96, True, False),       # group 256 (untiled) with FP16 deltas
 ])
 def test_pack_pow2_bit_exact(awq, bits, group, D_in, D_out, delta16, clip):
     X, W = _layer(16, D_in, D_out, seed=D_in + D_out)

@@ -72,6 +72,8 @@ def _case(awq, N, D_in, D_out, bits, group, seed):
     (1000, 512, 4096, 4, 64),     # 128 units of (128 columns x 256 tokens): more units than one per CTA
     (17, 8192, 2048, 3, 128),     # Nt = 32, 16 column tiles: stream-K, shares inside one unit
     (8, 256, 65536, 4, 128),      # 512 units of 4 k blocks: a CTA's share spans whole units + partial ends
+    (5, 1024, 200, 4, 256),       # group 256: one delta row per 4-k-block stage
+    (300, 768, 256, 4, 256),      # group 256, large token tile (one k block per stage)
     (32, 2048, 640, 4, 64),       # the largest 4-k-block-stage token tile (Nt = 32), group 64
     (33, 2048, 640, 4, 128),      # the smallest 2-k-block-stage token tile (Nt = 48)
     (3, 1056, 96, 2, 32),         # group 32 (two groups per k block), 2-bit, D_in not a multiple of 256
