@@ -66,6 +66,8 @@ def _load():
         lib.oracle_w4a16.restype = None
         lib.oracle_clip_loss.argtypes = [P, P, P, I64, I64, I64, P, I, I, I, P, I64, P, P]
         lib.oracle_clip_loss.restype = None
+        lib.oracle_pack3.argtypes = [P, I64, I64, P]
+        lib.oracle_pack3.restype = None
         lib.oracle_pack.argtypes = [P, I64, I64, I, P]
         lib.oracle_pack.restype = None
         lib.oracle_loss_cols.argtypes = [P, P, P, I64, I64, I64, I, I, I, P, I64, P]
@@ -202,6 +204,17 @@ def pack(q: np.ndarray, bits: int) -> np.ndarray:
     D_in, D_out = q.shape
     out = np.empty((D_in // 8, D_out), dtype=np.uint32)
     _load().oracle_pack(_ptr(q), D_in, D_out, bits, _ptr(out))
+    return out
+
+
+def pack3(q: np.ndarray) -> np.ndarray:
+    """Dense 3-bit packing of codes in [-4, 3]: words [D_in/32 * 3][D_out]
+    (uint32), code i of rows 32j..32j+31 at bits 3i..3i+2 of the 96-bit string
+    made of words 3j, 3j+1, 3j+2 (little-endian), as u = q + 4."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    D_in, D_out = q.shape
+    out = np.empty((D_in // 32 * 3, D_out), dtype=np.uint32)
+    _load().oracle_pack3(_ptr(q), D_in, D_out, _ptr(out))
     return out
 
 

@@ -254,6 +254,28 @@ void oracle_pack(const int8_t *q, int64_t D_in, int64_t D_out, int bits, uint32_
     }
 }
 
+/* Dense 3-bit packing (NEXT f2): the 32 codes of rows 32j .. 32j+31 of column
+ * n as one 96-bit little-endian string, code i (u = q + 4) at bits 3i .. 3i+2,
+ * stored as words (3j, n), (3j+1, n), (3j+2, n) holding bits 0-31, 32-63 and
+ * 64-95.  Codes 10 and 21 straddle two words.  D_in % 32 == 0. */
+void oracle_pack3(const int8_t *q, int64_t D_in, int64_t D_out, uint32_t *packed)
+{
+    for (int64_t j = 0; j < D_in / 32; ++j) {
+        for (int64_t n = 0; n < D_out; ++n) {
+            uint32_t w[3] = {0u, 0u, 0u};
+            for (int i = 0; i < 32; ++i) {
+                const uint32_t u = (uint32_t)((int)q[(32 * j + i) * D_out + n] + 4) & 7u;
+                for (int b = 0; b < 3; ++b) {
+                    const int bit = 3 * i + b;
+                    w[bit / 32] |= ((u >> b) & 1u) << (bit % 32);
+                }
+            }
+            for (int t = 0; t < 3; ++t)
+                packed[(3 * j + t) * D_out + n] = w[t];
+        }
+    }
+}
+
 /* [P1] flow step 4c for a set of output columns:
  *   L_n = sum_i ( sum_k x_ik * e_kn )^2,   e_kn = q_kn * delta_gn / s_k - w_kn
  * which is column n's share of ||X S^-1 Q(S W) - X W||^2 (exact algebra: the

@@ -451,3 +451,34 @@ def test_balanced_search_with_unit_weight_means_is_the_plain_search():
     L0, b0 = oracle.search(X, W, a, grid, 4, 64)
     L1, b1 = oracle.search(X, W, a, grid, 4, 64, w_mean=np.ones(128, np.float32))
     assert np.array_equal(L0, L1) and b0 == b1
+
+
+# ---------------------------------------------------------------- dense 3-bit packing
+
+def test_pack3_worked_example():
+    # codes 0..31 of one column: u_i = q_i + 4 with q_i = (i % 8) - 4, i.e. u_i = i % 8;
+    # the 96-bit string is sum_i u_i 2^(3i); read it back 3 bits at a time
+    q = ((np.arange(32) % 8) - 4).astype(np.int8).reshape(32, 1)
+    w = oracle.pack3(q)
+    assert w.shape == (3, 1)
+    big = int(w[0, 0]) | (int(w[1, 0]) << 32) | (int(w[2, 0]) << 64)
+    assert big == sum((i % 8) << (3 * i) for i in range(32))
+    # code 10 straddles words 0 and 1 (bits 30..32), code 21 words 1 and 2 (bits 63..65)
+    assert (int(w[0, 0]) >> 30) | ((int(w[1, 0]) & 1) << 2) == 10 % 8
+    assert (int(w[1, 0]) >> 31) | ((int(w[2, 0]) & 3) << 1) == 21 % 8
+
+
+def test_pack3_round_trip_random():
+    rng = np.random.default_rng(12)
+    q = rng.integers(-4, 4, size=(96, 7)).astype(np.int8)
+    w = oracle.pack3(q)
+    for j in range(3):
+        for n in range(7):
+            big = int(w[3 * j, n]) | (int(w[3 * j + 1, n]) << 32) | (int(w[3 * j + 2, n]) << 64)
+            got = [((big >> (3 * i)) & 7) - 4 for i in range(32)]
+            assert got == q[32 * j:32 * j + 32, n].tolist()
+
+
+def test_pack3_is_three_quarters_of_the_nibble_format():
+    q = np.zeros((256, 5), np.int8)
+    assert oracle.pack3(q).size * 4 == oracle.pack(q, 3).size * 3
