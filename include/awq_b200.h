@@ -311,6 +311,14 @@ AWQ_API int awq_quantize_pack_clip(const float* W, const float* s, const float* 
  *           quantiser of awq_search_ex's AWQ_QUANT_DELTA_POW2.  Combines with
  *           AWQ_PACK_DELTA_FP16 (the power-of-two delta then rounded to FP16). */
 #define AWQ_PACK_DELTA_POW2 2
+/*   AWQ_PACK_DENSE3 (bits = 3 only): codes stored densely, 32 rows of a
+ *           column in three words: `packed` is [D_in/32 * 3][D_out] uint32,
+ *           word (3j + t, n) holding bits 32t..32t+31 of the 96-bit
+ *           little-endian string whose bits 3i..3i+2 are row 32j + i's
+ *           u = q + 4 (codes 10 and 21 straddle two words).  With D_out % 4 != 0
+ *           it needs group 128 or 256 (AWQ_EUNSUPPORTED otherwise).
+ *           awq_w4a16_gemm reads the 4-bit container layout only. */
+#define AWQ_PACK_DENSE3 4
 AWQ_API int awq_quantize_pack_ex(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out,
                                  int bits, int group, int flags, uint32_t* packed, void* scales, void* stream);
 

@@ -77,6 +77,7 @@ class AwqSearchOptions(ctypes.Structure):
 QUANT_SYMMETRIC = 0
 QUANT_DELTA_POW2 = 1
 PACK_DELTA_POW2 = 2
+PACK_DENSE3 = 4
 _search_ex = _sig("awq_search_ex", I, [P, P, P, I64, I64, I64, P, I, I, I, I, ctypes.POINTER(AwqSearchOptions), P, P,
                                        P, P, P, SZ, P, P])
 _batched_ws = _sig("awq_search_batched_workspace_size", SZ, [ctypes.POINTER(AwqLayer), I, I, I, I, I])
@@ -279,7 +280,8 @@ def clip_search(X: torch.Tensor, W: torch.Tensor, s: torch.Tensor, clip_grid: Se
 
 
 def quantize_pack_ex(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int = 128,
-                     clip: Optional[torch.Tensor] = None, delta_fp16: bool = False, delta_pow2: bool = False):
+                     clip: Optional[torch.Tensor] = None, delta_fp16: bool = False, delta_pow2: bool = False,
+                     dense3: bool = False):
     """``awq_quantize_pack_ex``: the final pack with optional clip ratios and
     FP16 deltas.  Returns (packed int32 view [D_in/8, D_out], scales
     [D_in/group, D_out] as float16 when delta_fp16 else float32)."""
@@ -288,9 +290,11 @@ def quantize_pack_ex(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int
     if clip is not None:
         clip = _dev(clip, torch.float32, "clip")
     D_in, D_out = W.shape
-    packed = torch.empty(D_in // 8, D_out, dtype=torch.int32, device=W.device)
+    rows = D_in // 32 * 3 if dense3 else D_in // 8
+    packed = torch.empty(rows, D_out, dtype=torch.int32, device=W.device)
     sc = torch.empty(D_in // group, D_out, dtype=torch.float16 if delta_fp16 else torch.float32, device=W.device)
-    flags = (PACK_DELTA_FP16 if delta_fp16 else 0) | (PACK_DELTA_POW2 if delta_pow2 else 0)
+    flags = ((PACK_DELTA_FP16 if delta_fp16 else 0) | (PACK_DELTA_POW2 if delta_pow2 else 0)
+             | (PACK_DENSE3 if dense3 else 0))
     _check(_pack_ex(_ptr(W), _ptr(s), _ptr(clip), D_in, D_out, bits, group, flags, _ptr(packed), _ptr(sc), _stream()))
     return packed, sc
 

@@ -679,10 +679,14 @@ int awq_quantize_pack_clip(const float* W, const float* s, const float* clip, in
 int awq_quantize_pack_ex(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out, int bits,
                          int group, int flags, uint32_t* packed, void* scales, void* stream) {
   AWQ_TRY(check_quant_args(bits, group));
-  if (flags & ~(AWQ_PACK_DELTA_FP16 | AWQ_PACK_DELTA_POW2)) return fail(AWQ_EINVAL, "flags = %#x: unknown bits", flags);
+  if (flags & ~(AWQ_PACK_DELTA_FP16 | AWQ_PACK_DELTA_POW2 | AWQ_PACK_DENSE3))
+    return fail(AWQ_EINVAL, "flags = %#x: unknown bits", flags);
+  if ((flags & AWQ_PACK_DENSE3) && bits != 3) return fail(AWQ_EINVAL, "AWQ_PACK_DENSE3 needs bits = 3 (bits = %d)", bits);
   if (D_in < group || D_in > kMaxDin || D_in % group)
     return fail(AWQ_EINVAL, "D_in = %lld: need a positive multiple of group = %d", (long long)D_in, group);
   if (D_out < 1 || D_out > kMaxDim) return fail(AWQ_EINVAL, "D_out = %lld out of range", (long long)D_out);
+  if ((flags & AWQ_PACK_DENSE3) && D_out % 4 && group < 128)
+    return fail(AWQ_EUNSUPPORTED, "AWQ_PACK_DENSE3 with D_out %% 4 != 0 needs group 128 or 256 (group = %d)", group);
   AWQ_TRY(check_ptr(W, "W", 16));
   AWQ_TRY(check_ptr(s, "s", 16));
   if (clip) AWQ_TRY(check_ptr(clip, "clip", 4));
@@ -694,8 +698,9 @@ int awq_quantize_pack_ex(const float* W, const float* s, const float* clip, int6
   {
     StageTimer t(AWQ_STAGE_QUANTIZE_PACK, static_cast<cudaStream_t>(stream));
     e = awq::launch_quantize_pack(W, s, clip, D_in, D_out, bits, group, (flags & AWQ_PACK_DELTA_FP16) != 0,
-                                  (flags & AWQ_PACK_DELTA_POW2) ? awq::kQuantPow2 : awq::kQuantSymmetric, packed,
-                                  scales, sms, static_cast<cudaStream_t>(stream));
+                                  (flags & AWQ_PACK_DELTA_POW2) ? awq::kQuantPow2 : awq::kQuantSymmetric,
+                                  (flags & AWQ_PACK_DENSE3) != 0, packed, scales, sms,
+                                  static_cast<cudaStream_t>(stream));
   }
   return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "quantize_pack kernel");
 }

@@ -54,9 +54,10 @@ cudaError_t launch_weight_t(const float* W, int64_t D_in, int64_t D_out, uint16_
 // Final quantise + pack for one given scale vector s (natural nibble order);
 // clip [D_in/group][D_out] (may be null) scales each group maximum; delta16:
 // delta rounded to FP16 before the codes, scales stored as FP16 (else fp32).
+// dense3: 3-bit codes as 96-bit strings of 32 rows (words [D_in/32*3][D_out]).
 cudaError_t launch_quantize_pack(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out,
-                                 int bits, int group, bool delta16, int qmode, uint32_t* packed, void* scales,
-                                 int num_sms, cudaStream_t st);
+                                 int bits, int group, bool delta16, int qmode, bool dense3, uint32_t* packed,
+                                 void* scales, int num_sms, cudaStream_t st);
 
 // ---- reduce.cu
 cudaError_t launch_loss_reduce(const float* partial, int A, int H, int64_t D_out, double* L_col, double* blk,

@@ -170,7 +170,9 @@ def test_argument_checks_without_gpu(lib):
     pe = lib.awq_quantize_pack_ex
     pe.argtypes = [P, P, P, I64, I64, I, I, I, P, P, P]
     pe.restype = I
-    assert pe(fake, fake, None, 256, 64, 4, 128, 4, fake, fake, None) == 1   # unknown flag bit
+    assert pe(fake, fake, None, 256, 64, 4, 128, 8, fake, fake, None) == 1   # unknown flag bit
+    assert pe(fake, fake, None, 256, 64, 4, 128, 4, fake, fake, None) == 1   # dense packing needs 3-bit codes
+    assert pe(fake, fake, None, 256, 66, 3, 64, 4, fake, fake, None) == 3    # dense, D_out % 4 != 0, group 64
 
     t = lib.awq_selftest_wait_timeout
     t.argtypes = [P, I64, P]

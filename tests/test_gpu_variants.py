@@ -164,3 +164,46 @@ def test_search_balanced_against_oracle(awq, form, N, D_in, D_out, bits, group):
     packed, sc = awq.quantize_pack(W.cuda(), s_star, bits, group)
     q, d = oracle.quantize(W, s_star.cpu().numpy(), bits, group)
     assert np.array_equal(packed.cpu().numpy().view(np.uint32), oracle.pack(q, bits))
+
+
+# ---------------------------------------------------------------- dense 3-bit packing
+@pytest.mark.parametrize("group,D_in,D_out,pow2,clip", [
+    (128, 512, 256, False, False),     # tiled kernel
+    (64, 384, 200, False, False),
+    (32, 96, 36, True, False),         # tiled, power-of-two delta (codes reach -4)
+    (128, 256, 203, False, False),     # untiled (D_out % 4 != 0), one string per thread
+    (256, 512, 131, True, False),      # untiled, group 256: two strings per thread
+    (128, 512, 128, False, True),      # clip ratios, tiled
+])
+def test_pack_dense3_bit_exact(awq, group, D_in, D_out, pow2, clip):
+    X, W = _layer(16, D_in, D_out, seed=7 * D_in + D_out)
+    s = oracle.scales(oracle.act_stats(X).astype(np.float32), 0.45)
+    c = None
+    if clip:
+        rng = np.random.default_rng(D_in)
+        c = synth.clip_grid(20).numpy()[rng.integers(0, 21, size=(D_in // group, D_out))]
+    packed, sc = awq.quantize_pack_ex(W.cuda(), torch.from_numpy(s).cuda(), 3, group,
+                                      clip=None if c is None else torch.from_numpy(c).cuda(), delta_pow2=pow2,
+                                      dense3=True)
+    q, d = oracle.quantize(W, s, 3, group, clip=c, qmode=oracle.QMODE_POW2 if pow2 else oracle.QMODE_SYMMETRIC)
+    assert packed.shape == (D_in // 32 * 3, D_out)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), oracle.pack3(q))
+    assert np.array_equal(sc.cpu().numpy(), d)
+
+
+def test_pack_dense3_zero_group(awq):
+    W = torch.zeros(128, 8)
+    W[:, 4:] = torch.linspace(-1, 1, 128)[:, None]
+    s = torch.ones(128)
+    packed, _ = awq.quantize_pack_ex(W.cuda(), s.cuda(), 3, 128, dense3=True)
+    q, _ = oracle.quantize(W, s.numpy(), 3, 128)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), oracle.pack3(q))
+
+
+def test_pack_dense3_unsupported_combination(awq):
+    W = torch.zeros(64, 6, device="cuda")
+    s = torch.ones(64, device="cuda")
+    with pytest.raises(awq.AwqError):
+        awq.quantize_pack_ex(W, s, 3, 32, dense3=True)     # D_out % 4 != 0 with a group below 128
+    with pytest.raises(awq.AwqError):
+        awq.quantize_pack_ex(torch.zeros(64, 8, device="cuda"), s, 4, 32, dense3=True)   # 4-bit codes
