@@ -175,17 +175,28 @@ AWQ_API int awq_search(const void* X, const float* W, const float* a, int64_t N,
  *   w_mean     NULL, or [D_in] device fp32 (awq_weight_mean): the candidate
  *              scales are the balanced a^alpha / w_mean^(1-alpha); recover s*
  *              with awq_scales_ex.
+ *   gram_form  nonzero: evaluate L(alpha) = sum_n e_n^T H e_n with H = X^T X
+ *              (the Gram form of the loss, NEXT f4): H is formed once
+ *              (tensor cores, fp32, rounded to bf16), then each alpha costs
+ *              2 D_in^2 D_out flops instead of 2 N D_in D_out, which is cheaper
+ *              when N > D_in.  Error form only.  The workspace is
+ *              awq_search_ex_workspace_size(...).
  */
 #define AWQ_QUANT_SYMMETRIC 0
 #define AWQ_QUANT_DELTA_POW2 1
 typedef struct {
   int quantizer;
   const float* w_mean;
+  int gram_form;
 } awq_search_options;
 
+/* Bytes of workspace awq_search_ex needs with these options (0 if invalid). */
+AWQ_API size_t awq_search_ex_workspace_size(int64_t N, int64_t D_in, int64_t D_out, int n_alpha, int bits, int group,
+                                            int loss_form, const awq_search_options* options);
+
 /*
- * awq_search with options (NULL = awq_search).  Same arguments, outputs,
- * workspace size (awq_search_workspace_size) and errors.
+ * awq_search with options (NULL = awq_search).  Same arguments, outputs and
+ * errors; workspace awq_search_ex_workspace_size(...) bytes.
  */
 AWQ_API int awq_search_ex(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
                           const float* alpha_grid, int n_alpha, int bits, int group, int loss_form,

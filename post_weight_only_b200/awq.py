@@ -30,7 +30,7 @@ EXPORTS = (
     "awq_get_last_error", "awq_version", "awq_profile_enable", "awq_profile_reset", "awq_profile_read",
     "awq_search_noalloc", "awq_clip_search_workspace_size", "awq_clip_search", "awq_quantize_pack_clip",
     "awq_search_joint_workspace_size", "awq_search_joint", "awq_quantize_pack_ex", "awq_w4a16_gemm",
-    "awq_w4a16_workspace_size", "awq_search_ex", "awq_weight_mean", "awq_scales_ex",
+    "awq_w4a16_workspace_size", "awq_search_ex", "awq_weight_mean", "awq_scales_ex", "awq_search_ex_workspace_size",
 )
 STAGES = ("act_stats", "scale_table", "search_operand", "search_gemm", "loss_reduce", "quantize_pack",
           "weight_t", "clip_gram", "clip_operand", "clip_loss", "w4a16")
@@ -71,13 +71,15 @@ _search = _sig("awq_search", I, [P, P, P, I64, I64, I64, P, I, I, I, I, P, P, P,
 
 
 class AwqSearchOptions(ctypes.Structure):
-    _fields_ = [("quantizer", ctypes.c_int), ("w_mean", P)]
+    _fields_ = [("quantizer", ctypes.c_int), ("w_mean", P), ("gram_form", ctypes.c_int)]
 
 
 QUANT_SYMMETRIC = 0
 QUANT_DELTA_POW2 = 1
 PACK_DELTA_POW2 = 2
 PACK_DENSE3 = 4
+_search_ex_ws = _sig("awq_search_ex_workspace_size", SZ, [I64, I64, I64, I, I, I, I,
+                                                          ctypes.POINTER(AwqSearchOptions)])
 _search_ex = _sig("awq_search_ex", I, [P, P, P, I64, I64, I64, P, I, I, I, I, ctypes.POINTER(AwqSearchOptions), P, P,
                                        P, P, P, SZ, P, P])
 _batched_ws = _sig("awq_search_batched_workspace_size", SZ, [ctypes.POINTER(AwqLayer), I, I, I, I, I])
@@ -209,9 +211,10 @@ _default_ws = Workspace()
 def search(X: torch.Tensor, W: torch.Tensor, a: torch.Tensor, alpha_grid: Sequence[float], bits: int = 4,
            group: int = 128, want_cols: bool = False, workspace: Optional[Workspace] = None,
            check_status: bool = True, loss_form: int = LOSS_ERROR, quantizer: int = QUANT_SYMMETRIC,
-           w_mean: Optional[torch.Tensor] = None) -> SearchResult:
+           w_mean: Optional[torch.Tensor] = None, gram: bool = False) -> SearchResult:
     """Grid search over alpha for one layer: ``awq_search``, or
-    ``awq_search_ex`` with a quantiser variant or the balanced scale."""
+    ``awq_search_ex`` with a quantiser variant, the balanced scale or the
+    Gram form of the loss."""
     X = _dev(X, torch.bfloat16, "X")
     W = _dev(W, torch.float32, "W")
     a = _dev(a, torch.float32, "a")
@@ -225,14 +228,18 @@ def search(X: torch.Tensor, W: torch.Tensor, a: torch.Tensor, alpha_grid: Sequen
     astar = torch.empty(1, dtype=torch.float32, device=dev)
     aidx = torch.empty(1, dtype=torch.int32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    nbytes = search_workspace_size(N, D_in, D_out, A, bits, group, loss_form)
+    plain = quantizer == QUANT_SYMMETRIC and w_mean is None and not gram
+    b = None if w_mean is None else _dev(w_mean, torch.float32, "w_mean")
+    opts = AwqSearchOptions(int(quantizer), _ptr(b), 1 if gram else 0)
+    nbytes = (search_workspace_size(N, D_in, D_out, A, bits, group, loss_form) if plain
+              else int(_search_ex_ws(N, D_in, D_out, A, bits, group, loss_form, ctypes.byref(opts))))
+    if nbytes == 0:
+        raise AwqError(AWQ_EINVAL, "awq_search_ex_workspace_size: invalid arguments")
     ws = (workspace or _default_ws).get(nbytes, dev)
-    if quantizer == QUANT_SYMMETRIC and w_mean is None:
+    if plain:
         _check(_search(_ptr(X), _ptr(W), _ptr(a), N, D_in, D_out, grid, A, bits, group, loss_form, _ptr(L), _ptr(Lc),
                        _ptr(astar), _ptr(aidx), _ptr(ws), ws.numel(), _ptr(status), _stream()))
     else:
-        b = None if w_mean is None else _dev(w_mean, torch.float32, "w_mean")
-        opts = AwqSearchOptions(int(quantizer), _ptr(b))
         _check(_search_ex(_ptr(X), _ptr(W), _ptr(a), N, D_in, D_out, grid, A, bits, group, loss_form,
                           ctypes.byref(opts), _ptr(L), _ptr(Lc), _ptr(astar), _ptr(aidx), _ptr(ws), ws.numel(),
                           _ptr(status), _stream()))

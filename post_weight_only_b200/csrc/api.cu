@@ -181,7 +181,34 @@ void prof_collect() {
 struct SearchOpts {
   int qmode = awq::kQuantSymmetric;
   const float* w_mean = nullptr;    // balanced scale a^alpha / w_mean^(1 - alpha) when set
+  bool gram = false;                // L = sum_n e_n^T (X^T X) e_n (error form only)
 };
+
+// Workspace of the Gram form: X^T (tokens padded to 8), H = X^T X in fp32 and
+// in bf16, then the search's own layout for D_in "tokens" (the rows of H).
+struct GramLayout {
+  int64_t Np;
+  size_t xt, hf, hb, search, total;
+  SearchLayout sl;
+};
+
+GramLayout gram_layout(int64_t N, int64_t D_in, int64_t D_out, int A, int group, int num_sms) {
+  GramLayout g{};
+  g.Np = (N + 7) / 8 * 8;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += round_up(bytes, 256);
+    return o;
+  };
+  g.xt = take(static_cast<size_t>(D_in) * g.Np * 2);
+  g.hf = take(static_cast<size_t>(D_in) * D_in * 4);
+  g.hb = take(static_cast<size_t>(D_in) * D_in * 2);
+  g.sl = search_layout(D_in, D_in, D_out, A, group, awq::kFormGram, num_sms);
+  g.search = take(g.sl.total);
+  g.total = off;
+  return g;
+}
 
 // The search for one layer with a workspace already checked; does not reset
 // the status word.
@@ -206,7 +233,8 @@ int search_one(const void* X, const float* W, const float* a, int64_t N, int64_t
   if (e != cudaSuccess) return fail_cuda(e, "scale table kernel");
   {
     StageTimer t(AWQ_STAGE_SEARCH_OPERAND, st);
-    e = awq::launch_search_operand(W, s_tab, r_tab, D_in, D_out, A, bits, group, form, opts.qmode, op, st);
+    const int op_form = form == awq::kFormGram ? awq::kFormError : form;   // the Gram form reads E = S^-1 Q(SW) - W
+    e = awq::launch_search_operand(W, s_tab, r_tab, D_in, D_out, A, bits, group, op_form, opts.qmode, op, st);
   }
   if (e != cudaSuccess) return fail_cuda(e, "search operand kernel");
   if (wt) {
@@ -364,6 +392,45 @@ static int search_impl(const void* X, const float* W, const float* a, int64_t N,
                             alpha_star, alpha_idx));
   int sms = 0;
   AWQ_TRY(device_info(&sms));
+  if (opts.gram) {
+    // L(alpha) = sum_n e_n^T H e_n with H = X^T X (Gram form): H once, then the
+    // search GEMM over the D_in rows of H instead of the N tokens of X.
+    if (loss_form != AWQ_LOSS_ERROR) return fail(AWQ_EINVAL, "the Gram form evaluates the error form only");
+    const GramLayout gl = gram_layout(N, D_in, D_out, n_alpha, group, sms);
+    if (!workspace) return fail(AWQ_EWORKSPACE, "workspace is NULL");
+    if (!aligned(workspace, 256)) return fail(AWQ_EALIGN, "workspace is not 256-byte aligned");
+    if (workspace_bytes < gl.total)
+      return fail(AWQ_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, gl.total);
+    if (status && !aligned(status, 4)) return fail(AWQ_EALIGN, "status is not 4-byte aligned");
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* sws = ws + gl.search;
+    int32_t* st_word = status ? status : reinterpret_cast<int32_t*>(sws + gl.sl.status);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(st_word, 0, sizeof(int32_t), st);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(status)");
+    uint16_t* xt = reinterpret_cast<uint16_t*>(ws + gl.xt);
+    float* hf = reinterpret_cast<float*>(ws + gl.hf);
+    uint16_t* hb = reinterpret_cast<uint16_t*>(ws + gl.hb);
+    {
+      StageTimer t(AWQ_STAGE_CLIP_GRAM, st);
+      e = awq::launch_xt(static_cast<const uint16_t*>(X), N, D_in, gl.Np, xt, st);
+      if (e != cudaSuccess) return fail_cuda(e, "transpose of X");
+      // H = X^T X by the search GEMM in its output-only mode: "tokens" are the
+      // D_in rows of X^T, the reduction runs over the (padded) tokens of X.
+      awq::SearchShape shH{static_cast<int>(D_in), static_cast<int>(gl.Np), static_cast<int>(D_in), 0, 4, 128,
+                           AWQ_LOSS_REFERENCE};
+      awq::SearchBuffers bH{xt, xt, nullptr, nullptr, nullptr, hf, st_word};
+      const char* what = "search kernel (Gram matrix)";
+      const int rc = awq::launch_search(shH, bH, awq::search_grid_size(shH, sms), timeout_ns(), st, &e, &what);
+      if (rc != AWQ_OK) return e != cudaSuccess ? fail_cuda(e, what) : fail(rc, "%s failed", what);
+      e = awq::launch_to_bf16(hf, D_in * D_in, hb, st);
+      if (e != cudaSuccess) return fail_cuda(e, "bf16 rounding of the Gram matrix");
+    }
+    awq::AlphaList al{};
+    for (int i = 0; i < n_alpha; ++i) al.v[i] = alpha_grid[i];
+    return search_one(hb, W, a, D_in, D_in, D_out, al, n_alpha, bits, group, awq::kFormGram, L, L_col, alpha_star,
+                      alpha_idx, sws, st_word, st, sms, opts);
+  }
   const SearchLayout lay = search_layout(N, D_in, D_out, n_alpha, group, loss_form, sms);
   if (!workspace) return fail(AWQ_EWORKSPACE, "workspace is NULL");
   if (!aligned(workspace, 256)) return fail(AWQ_EALIGN, "workspace is not 256-byte aligned");
@@ -400,9 +467,20 @@ int awq_search_ex(const void* X, const float* W, const float* a, int64_t N, int6
     if (options->w_mean) AWQ_TRY(check_ptr(options->w_mean, "w_mean", 4));
     o.qmode = options->quantizer == AWQ_QUANT_DELTA_POW2 ? awq::kQuantPow2 : awq::kQuantSymmetric;
     o.w_mean = options->w_mean;
+    o.gram = options->gram_form != 0;
   }
   return search_impl(X, W, a, N, D_in, D_out, alpha_grid, n_alpha, bits, group, loss_form, L, L_col, alpha_star,
                      alpha_idx, workspace, workspace_bytes, status, stream, o);
+}
+
+size_t awq_search_ex_workspace_size(int64_t N, int64_t D_in, int64_t D_out, int n_alpha, int bits, int group,
+                                    int loss_form, const awq_search_options* options) {
+  if (!options || !options->gram_form) return awq_search_workspace_size(N, D_in, D_out, n_alpha, bits, group, loss_form);
+  if (check_layer_shape(N, D_in, D_out) != AWQ_OK || check_quant_args(bits, group) != AWQ_OK) return 0;
+  if (loss_form != AWQ_LOSS_ERROR || D_in % group || n_alpha < 1 || n_alpha > AWQ_MAX_ALPHA) return 0;
+  int sms = 0;
+  if (device_info(&sms) != AWQ_OK) return 0;
+  return gram_layout(N, D_in, D_out, n_alpha, group, sms).total;
 }
 
 size_t awq_search_batched_workspace_size(const awq_layer* layers, int n_layers, int n_alpha, int bits, int group,

@@ -408,6 +408,24 @@ cudaError_t launch_xt(const uint16_t* X, int64_t N, int64_t D, int64_t Np, uint1
   return cudaGetLastError();
 }
 
+namespace {
+// dst [n] bf16 = round-to-nearest of src [n] fp32 (the Gram matrix as the
+// search GEMM's operand).
+__global__ void __launch_bounds__(256) to_bf16_kernel(const float* __restrict__ src, int64_t n,
+                                                      uint16_t* __restrict__ dst) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    dst[i] = __bfloat16_as_ushort(__float2bfloat16_rn(src[i]));
+}
+}  // namespace
+
+cudaError_t launch_to_bf16(const float* src, int64_t n, uint16_t* dst, cudaStream_t st) {
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  to_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(src, n, dst);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_recip(const float* s, int64_t D, float* r, cudaStream_t st) {
   recip_kernel<<<static_cast<unsigned>((D + 255) / 256), 256, 0, st>>>(s, D, r);
   return cudaGetLastError();

@@ -18,6 +18,7 @@ constexpr int kQuantPow2 = 1;
 // Loss forms of the search (see search.cu).
 constexpr int kFormError = 0;        // L = ||X E||^2 with E = S^-1 Q(S W) - W as the MMA operand
 constexpr int kFormReference = 1;    // L = ||X S^-1 Q(S W) - X W||^2, reference output subtracted
+constexpr int kFormGram = 2;         // L = sum_n e_n^T H e_n with H = X^T X given in place of X (N = D_in)
 
 struct AlphaList {
   float v[kMaxAlpha];
@@ -110,6 +111,8 @@ bool make_word_map(CUtensorMap* m, const void* base, bool is_float, uint64_t inn
 cudaError_t launch_xt(const uint16_t* X, int64_t N, int64_t D, int64_t Np, uint16_t* XT, cudaStream_t st);
 // r = 1 / s (IEEE).
 cudaError_t launch_recip(const float* s, int64_t D, float* r, cudaStream_t st);
+// dst [n] = bf16(src [n]), round to nearest even.
+cudaError_t launch_to_bf16(const float* src, int64_t n, uint16_t* dst, cudaStream_t st);
 // Hb [D_in/group][group][group] bf16: the diagonal Gram blocks X_g^T X_g.
 int launch_gram(const uint16_t* XT, int64_t D_in, int64_t Np, int group, uint16_t* Hb, int* status,
                 uint64_t timeout_ns, cudaStream_t st, cudaError_t* cerr, const char** what);

@@ -88,6 +88,7 @@ enum Site { kSiteTmaEmpty = 1, kSiteMmaAccEmpty, kSiteMmaFull, kSiteEpiAccFull, 
 struct Params {
   int N, D_in, D_out, A;
   int Tt, Wt, U, KB, H, gemm_only, weight_minor;
+  const uint16_t* op;         // Gram form: the operand E [A][D_out][D_in], read by the epilogue
   float* yref;
   float* partial;
   float* y_out;
@@ -357,6 +358,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
           }
           if (n < p.D_out) p.partial[(static_cast<size_t>(pass) * p.H + hrow) * p.D_out + n] = s0 + s1;
+        } else if (kForm == kFormGram) {
+          // "Tokens" are rows t of H = X^T X: the accumulator holds (H e_n)_t
+          // for this warp's 128 rows; the partial is sum_t e_nt (H e_n)_t, with
+          // e_n read back from the operand (bf16, row n contiguous in t).
+          const int t0 = tt * kBN + h * kHalfN;
+          const bool col_ok = n < p.D_out;
+          const uint16_t* erow = p.op + (static_cast<size_t>(pass) * p.D_out + (col_ok ? n : 0)) * p.D_in;
+          float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll 1
+          for (int c2 = 0; c2 < kHalfN / 64; ++c2) {
+            uint32_t v[2][32];
+            tmem_ld32(acc + c2 * 64, v[0]);
+            tmem_ld32(acc + c2 * 64 + 32, v[1]);
+            uint4 ev[8];                                 // e_n at rows t0 + 64 c2 .. + 63
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int t = t0 + c2 * 64 + 8 * j;
+              ev[j] = (col_ok && t < p.D_in) ? __ldg(reinterpret_cast<const uint4*>(erow + t))
+                                             : make_uint4(0u, 0u, 0u, 0u);
+            }
+            tmem_wait_ld();
+            if (c2 == kHalfN / 64 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive_cluster(release);
+            }
+            const uint32_t* ew = reinterpret_cast<const uint32_t*>(ev);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {               // bf16 pairs: rows 2e, 2e+1 of each 32-row half
+              s0 = fmaf(__uint_as_float(ew[e] << 16), __uint_as_float(v[0][2 * e]), s0);
+              s0 = fmaf(__uint_as_float(ew[e] & 0xFFFF0000u), __uint_as_float(v[0][2 * e + 1]), s0);
+              s1 = fmaf(__uint_as_float(ew[16 + e] << 16), __uint_as_float(v[1][2 * e]), s1);
+              s1 = fmaf(__uint_as_float(ew[16 + e] & 0xFFFF0000u), __uint_as_float(v[1][2 * e + 1]), s1);
+            }
+          }
+          if (col_ok) p.partial[(static_cast<size_t>(pass) * p.H + hrow) * p.D_out + n] = s0 + s1;
         } else if (ref) {
 #pragma unroll 1
           for (int c = 0; c < kHalfN / 32; ++c) {
@@ -586,14 +623,16 @@ int launch_search(const SearchShape& sh, const SearchBuffers& b, int grid, uint6
     const double op_per_alpha = 2.0 * sh.D_in * static_cast<double>(sh.D_out);
     p.weight_minor = (!gemm_only && x_bytes > op_per_alpha) ? 1 : 0;
   }
+  p.op = b.op;
   p.yref = b.yref;
   p.partial = b.partial;
   p.y_out = b.y_out;
   p.status = b.status;
   p.timeout_ns = timeout_ns;
 
-  cudaError_t e = form == kFormError ? launch_form<kFormError>(grid, mX, mWt, mOp, p, st)
-                                     : launch_form<kFormReference>(grid, mX, mWt, mOp, p, st);
+  cudaError_t e = form == kFormError  ? launch_form<kFormError>(grid, mX, mWt, mOp, p, st)
+                  : form == kFormGram ? launch_form<kFormGram>(grid, mX, mWt, mOp, p, st)
+                                      : launch_form<kFormReference>(grid, mX, mWt, mOp, p, st);
   if (e != cudaSuccess) {
     *cerr = e;
     *what = "search_kernel launch";

@@ -143,7 +143,7 @@ def test_argument_checks_without_gpu(lib):
     assert gcall(st=None) == 1                             # the status word is required
 
     class Opts(ctypes.Structure):
-        _fields_ = [("quantizer", ctypes.c_int), ("w_mean", ctypes.c_void_p)]
+        _fields_ = [("quantizer", ctypes.c_int), ("w_mean", ctypes.c_void_p), ("gram_form", ctypes.c_int)]
 
     x = lib.awq_search_ex
     x.argtypes = [P, P, P, I64, I64, I64, P, I, I, I, I, ctypes.POINTER(Opts), P, P, P, P, P, ctypes.c_size_t, P, P]
@@ -154,9 +154,13 @@ def test_argument_checks_without_gpu(lib):
         return x(d["X"], d["W"], d["a"], d["N"], d["D_in"], d["D_out"], d["grid"], d["A"], d["bits"], d["group"],
                  d["form"], opts, d["L"], d["Lc"], d["astar"], d["aidx"], d["ws"], d["wsb"], d["st"], d["stream"])
 
-    assert xcall(ctypes.byref(Opts(2, None))) == 1           # unknown quantiser
-    assert xcall(ctypes.byref(Opts(1, fake + 2))) == 2       # misaligned weight means
-    assert xcall(ctypes.byref(Opts(1, None)), bits=5) == 3   # the common checks still apply
+    assert xcall(ctypes.byref(Opts(2, None, 0))) == 1        # unknown quantiser
+    assert xcall(ctypes.byref(Opts(1, fake + 2, 0))) == 2    # misaligned weight means
+    assert xcall(ctypes.byref(Opts(1, None, 0)), bits=5) == 3   # the common checks still apply
+    xws = lib.awq_search_ex_workspace_size
+    xws.argtypes = [I64, I64, I64, I, I, I, I, ctypes.POINTER(Opts)]
+    xws.restype = ctypes.c_size_t
+    assert xws(64, 256, 64, 3, 4, 128, 1, ctypes.byref(Opts(0, None, 1))) == 0   # Gram form: error form only
     wm = lib.awq_weight_mean
     wm.argtypes = [P, I64, I64, P, P]
     wm.restype = I
