@@ -53,6 +53,7 @@ def parse_args():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clip", action="store_true", help="skip timing the weight-clipping search")
+    ap.add_argument("--no-gram", action="store_true", help="skip timing the Gram form of the search")
     ap.add_argument("--no-w4a16", action="store_true", help="skip timing the W4A16 consumer kernel")
     ap.add_argument("--no-at-scale", action="store_true",
                     help="skip timing the statistic and pack kernels on the 70B block's largest operands")
@@ -454,6 +455,47 @@ def run_ours(args):
             "frac_clipped": float((cr.idx > 0).float().mean().item()),
         }
 
+    # ---------------- the Gram form of the search on the 16384-token sweep layer
+    # (not part of the step): L(alpha) = sum_n e_n^T (X^T X) e_n against the
+    # direct ||X E||^2, one call each on the same layer and 41-point grid.
+    gram_info = None
+    if not args.no_gram:
+        gspec = synth.workload("sweep_4096x11008_n16k").layers[1]
+        Xg_cpu, Wg_cpu = synth.layer_inputs(gspec)
+        Xg, Wg = Xg_cpu.to(dev), Wg_cpu.to(dev)
+        ag = awq.act_stats(Xg)
+        ggrid = synth.alpha_grid(40).tolist()
+        gws = awq.Workspace()
+        gram_info = {"layer": f"{gspec.name} (N={gspec.N}, D_in={gspec.D_in}, D_out={gspec.D_out}), 41 alphas, 4-bit g128"}
+        results = {}
+        for mode in ("direct", "gram"):
+            use_gram = mode == "gram"
+            awq.search(Xg, Wg, ag, ggrid, bits, group, workspace=gws, gram=use_gram)
+            torch.cuda.synchronize()
+            times = []
+            for _ in range(3):
+                flush.zero_()
+                flush_sink.add_(flush.amax())
+                ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                ea.record()
+                rr = awq.search(Xg, Wg, ag, ggrid, bits, group, workspace=gws, gram=use_gram, check_status=False)
+                eb.record()
+                times.append((ea, eb))
+            torch.cuda.synchronize()
+            awq.check_device_status(rr.status)
+            ms = sum(a_.elapsed_time(b_) for a_, b_ in times) / len(times)
+            results[mode] = rr
+            gemm_flops = 2.0 * (gspec.D_in if use_gram else gspec.N) * gspec.D_in * gspec.D_out * len(ggrid)
+            gram_info[mode] = {"ms_per_call": ms, "gemm_flops": gemm_flops,
+                               "alpha_star": float(rr.alpha_star.item()),
+                               "direct_equivalent_tflops": 2.0 * gspec.N * gspec.D_in * gspec.D_out * len(ggrid)
+                                                           / (ms / 1e3) / 1e12}
+        Ld, Lg = results["direct"].L.cpu(), results["gram"].L.cpu()
+        gram_info["speedup"] = gram_info["direct"]["ms_per_call"] / gram_info["gram"]["ms_per_call"]
+        gram_info["max_rel_diff_L"] = float(((Lg - Ld).abs() / Ld).max().item())
+        del Xg, Wg, gws, results
+        torch.cuda.empty_cache()
+
     # ---------------- the W4A16 consumer of the pack format (not part of the step)
     # Each call is timed as one node group of a CUDA graph of 20 calls (its
     # host cost is not measured, so small decode shapes are not host-bound);
@@ -543,6 +585,7 @@ def run_ours(args):
                         "search_operand": hbm("search_operand", operand_bytes)},
         "hbm_kernels_at_scale": at_scale or None,
         "clip_search": clip_info,
+        "gram_search": gram_info,
         "w4a16": w4_info,
         "kernels": kernels,
         "e2e": {"value": A * world / (e2e_per_step / 1e3), "unit": UNIT, "ms_per_step": e2e_per_step,
