@@ -28,6 +28,7 @@ STAT_MAX = 1
 # delta = max / 2^(b-1), codes in [-2^(b-1), 2^(b-1) - 1]
 QMODE_SYMMETRIC = 0
 QMODE_POW2 = 1
+QMODE_ASYMMETRIC = 2     # MinMax with a zero point: codes u in [0, 2^b - 1], w ~ (u - z) delta
 
 _lib = None
 
@@ -76,6 +77,8 @@ def _load():
         lib.oracle_search.restype = I
         lib.oracle_quantize_mode.argtypes = [P, P, P, I64, I64, I, I, I, I, P, P]
         lib.oracle_quantize_mode.restype = None
+        lib.oracle_quantize_asym.argtypes = [P, P, I64, I64, I, I, I, P, P, P]
+        lib.oracle_quantize_asym.restype = None
         lib.oracle_weight_mean.argtypes = [P, I64, I64, P]
         lib.oracle_weight_mean.restype = None
         lib.oracle_scales_balanced.argtypes = [P, P, I64, F, P]
@@ -172,6 +175,30 @@ def quantize(W, s, bits: int, group: int, clip=None, delta16: bool = False,
     _load().oracle_quantize_mode(_ptr(W), _ptr(s), _ptr(c), D_in, D_out, bits, group, int(bool(delta16)),
                                  int(qmode), _ptr(q), _ptr(d))
     return q, d
+
+
+def quantize_asym(W, s, bits: int, group: int, delta16: bool = False):
+    """The asymmetric (MinMax, zero-point) quantiser of diag(s).W (concept
+    page, "the AWQ mechanism": absmax or MinMax; symmetric or asymmetric).
+    Returns (signed codes q = u - z [D_in, D_out] int8, deltas
+    [D_in/group, D_out] fp32, zero points z [D_in/group, D_out] uint8); the
+    stored codes are u = q + z in [0, 2^b - 1]."""
+    W = _f32(W)
+    D_in, D_out = W.shape
+    s = None if s is None else _f32(s)
+    q = np.empty((D_in, D_out), dtype=np.int8)
+    d = np.empty((D_in // group, D_out), dtype=np.float32)
+    z = np.empty((D_in // group, D_out), dtype=np.uint8)
+    _load().oracle_quantize_asym(_ptr(W), _ptr(s), D_in, D_out, bits, group, int(bool(delta16)), _ptr(q), _ptr(d),
+                                 _ptr(z))
+    return q, d, z
+
+
+def pack_unsigned(u: np.ndarray) -> np.ndarray:
+    """Nibble packing of unsigned codes u in [0, 15] (natural order, no
+    offset): the layout of pack() with u in place of q + 2^(b-1)."""
+    u = np.asarray(u, dtype=np.int16)
+    return pack((u - 8).astype(np.int8), 4)
 
 
 def clip_search(X, W, s, clip_grid, bits: int, group: int, cols: Optional[Sequence[int]] = None,

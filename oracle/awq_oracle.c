@@ -160,10 +160,68 @@ static float round_to_fp16(float x)
  * quantisation MSE): the group maximum m is replaced by fl32(clip * m) before
  * delta is formed, and the clamp then bounds the codes of the clipped weights.
  * clip = 1 leaves m unchanged (fl32(1 * m) = m). */
+/* qmode 2, the asymmetric (MinMax, zero-point) quantiser ([P1] "the AWQ
+ * mechanism": absmax or MinMax uniform quantisation; "symmetric or asymmetric
+ * both work"), with the plainest textbook reading of MinMax:
+ *   lo = min(0, min_k w'_k),  hi = max(0, max_k w'_k)   (zero stays exact)
+ *   delta = fl32(fl32(hi - lo) / (2^b - 1))
+ *   z = clamp(round(fl32(-lo / delta)), 0, 2^b - 1)
+ *   u_k = clamp(round(fl32(w'_k / delta)) + z, 0, 2^b - 1)
+ * and the dequantised weight is (u_k - z) delta.  q receives the signed code
+ * u_k - z (so that every loss below reads q * delta), *zero the point z.
+ * An all-zero group has delta = 0, z = 0 and codes 0. */
+static void quantize_group_asym(const float *W, const float *s, int64_t D_out, int64_t n, int64_t k0, int group,
+                                int bits, int delta16, int8_t *q, float *delta, uint8_t *zero)
+{
+    const int umax = (1 << bits) - 1;
+    float lo = 0.0f, hi = 0.0f;
+    for (int k = 0; k < group; ++k) {
+        float w = W[(k0 + k) * D_out + n];
+        float wp = s ? s[k0 + k] * w : w;
+        if (wp < lo)
+            lo = wp;
+        if (wp > hi)
+            hi = wp;
+    }
+    float d = (hi - lo) / (float)umax;
+    if (delta16)
+        d = round_to_fp16(d);
+    *delta = d;
+    int z = 0;
+    if (d != 0.0f) {
+        float zr = nearbyintf(-lo / d);
+        if (zr < 0.0f)
+            zr = 0.0f;
+        if (zr > (float)umax)
+            zr = (float)umax;
+        z = (int)zr;
+    }
+    *zero = (uint8_t)z;
+    for (int k = 0; k < group; ++k) {
+        int code = 0;
+        if (d != 0.0f) {
+            float w = W[(k0 + k) * D_out + n];
+            float wp = s ? s[k0 + k] * w : w;
+            float r = nearbyintf(wp / d) + (float)z;
+            if (r < 0.0f)
+                r = 0.0f;
+            if (r > (float)umax)
+                r = (float)umax;
+            code = (int)r - z;
+        }
+        q[k] = (int8_t)code;
+    }
+}
+
 static void quantize_group(const float *W, const float *s, int64_t D_out, int64_t n,
                            int64_t k0, int group, int bits, float clip, int delta16, int qmode, int8_t *q,
                            float *delta)
 {
+    if (qmode == 2) {
+        uint8_t zdummy;
+        quantize_group_asym(W, s, D_out, n, k0, group, bits, delta16, q, delta, &zdummy);
+        return;
+    }
     const int qmax = (1 << (bits - 1)) - 1;
     /* qmode 1 ([P2] "analysing the quantisation error"): delta = max / 2^(b-1)
      * (an exact power-of-two scaling), codes clamped to [-2^(b-1), 2^(b-1) - 1]
@@ -211,6 +269,23 @@ void oracle_quantize_mode(const float *W, const float *s, const float *clip, int
         for (int64_t g = 0; g < D_in / group; ++g) {
             quantize_group(W, s, D_out, n, g * group, group, bits, clip ? clip[g * D_out + n] : 1.0f, delta16,
                            qmode, col, &delta[g * D_out + n]);
+            for (int k = 0; k < group; ++k)
+                q[(g * group + k) * D_out + n] = col[k];
+        }
+    }
+    free(col);
+}
+
+/* The asymmetric quantiser over every (group, column): q [D_in][D_out] signed
+ * codes u - z, delta and zeros [D_in/group][D_out]. */
+void oracle_quantize_asym(const float *W, const float *s, int64_t D_in, int64_t D_out, int bits, int group,
+                          int delta16, int8_t *q, float *delta, uint8_t *zeros)
+{
+    int8_t *col = (int8_t *)malloc((size_t)group);
+    for (int64_t n = 0; n < D_out; ++n) {
+        for (int64_t g = 0; g < D_in / group; ++g) {
+            quantize_group_asym(W, s, D_out, n, g * group, group, bits, delta16, col, &delta[g * D_out + n],
+                                &zeros[g * D_out + n]);
             for (int k = 0; k < group; ++k)
                 q[(g * group + k) * D_out + n] = col[k];
         }

@@ -482,3 +482,74 @@ def test_pack3_round_trip_random():
 def test_pack3_is_three_quarters_of_the_nibble_format():
     q = np.zeros((256, 5), np.int8)
     assert oracle.pack3(q).size * 4 == oracle.pack(q, 3).size * 3
+
+
+# ---------------------------------------------------------------- asymmetric (MinMax, zero-point) quantiser
+# (compassingai.com concept page, "the AWQ mechanism": absmax or MinMax; "symmetric or
+# asymmetric both work".  Range [min(0, min w'), max(0, max w')], delta = range / (2^b - 1),
+# z = round(-lo / delta), u = clamp(round(w' / delta) + z, 0, 2^b - 1), w ~ (u - z) delta.)
+
+def test_asym_worked_example():
+    W = np.array([[0.5], [-1.0], [0.26], [0.74]], dtype=np.float32)
+    q, d, z = oracle.quantize_asym(W, None, 4, 4)
+    rng_ = np.float32(np.float32(0.74) - np.float32(-1.0))
+    assert d[0, 0] == np.float32(rng_ / np.float32(15.0))              # 1.74 / 15 = 0.116
+    assert z[0, 0] == 9                                                # round(1 / 0.116) = round(8.62)
+    assert q[:, 0].tolist() == [4, -9, 2, 6]                           # u = 13, 0, 11, 15
+
+
+def test_asym_one_sided_groups():
+    pos = np.array([[0.0], [0.3], [1.5], [0.75]], dtype=np.float32)   # lo = 0: z = 0, max -> 15
+    q, d, z = oracle.quantize_asym(pos, None, 4, 4)
+    assert z[0, 0] == 0 and q[:, 0].tolist() == [0, 3, 15, 8] and d[0, 0] == np.float32(np.float32(1.5) / 15)
+    neg = -pos                                                          # hi = 0: z = 15, min -> u = 0
+    q, d, z = oracle.quantize_asym(neg, None, 4, 4)
+    assert z[0, 0] == 15 and (q[:, 0] + 15).tolist() == [15, 12, 0, 7]
+
+
+def test_asym_brute_force_and_invariants():
+    rng = np.random.default_rng(21)
+    W = (rng.standard_normal((64, 5)) + rng.normal(0, 1, (1, 5))).astype(np.float32)
+    W[5, 2] = 0.0
+    s = (rng.random(64) + 0.5).astype(np.float32)
+    for bits in (2, 3, 4):
+        q, d, z = oracle.quantize_asym(W, s, bits, 32)
+        umax = (1 << bits) - 1
+        for g in range(2):
+            for n in range(5):
+                wp = (s[32 * g:32 * g + 32] * W[32 * g:32 * g + 32, n]).astype(np.float32)
+                lo, hi = min(np.float32(0), wp.min()), max(np.float32(0), wp.max())
+                assert d[g, n] == np.float32(np.float32(hi - lo) / np.float32(umax))
+                assert 0 <= z[g, n] <= umax
+                for k in range(32):
+                    u = int(q[32 * g + k, n]) + int(z[g, n])
+                    assert 0 <= u <= umax
+                    t = float(np.float32(wp[k] / d[g, n]))
+                    cand = np.arange(umax + 1) - int(z[g, n])            # signed codes reachable
+                    err = np.abs(cand - t)
+                    best = cand[err == err.min()]
+                    want = best[0] if len(best) == 1 else best[best % 2 == 0][0]   # ties to even
+                    assert q[32 * g + k, n] == want
+        # an exact zero stays exactly zero
+        assert q[5, 2] == 0
+
+
+def test_asym_search_uses_the_quantiser():
+    X, W = synth.layer_inputs(synth.small_layer(64, 128, 16, seed=6))
+    a = oracle.act_stats(X).astype(np.float32)
+    grid = np.array([0.0, 0.5], np.float32)
+    L2, _ = oracle.search(X, W, a, grid, 4, 64, qmode=oracle.QMODE_ASYMMETRIC)
+    s = oracle.scales(a, 0.5)
+    q, d, z = oracle.quantize_asym(W, s, 4, 64)
+    e = q.astype(np.float64) * np.repeat(d, 64, axis=0) / s.astype(np.float64)[:, None] - W.numpy()
+    x = X.float().numpy().astype(np.float64)
+    assert np.isclose(L2[1], ((x @ e) ** 2).sum(), rtol=1e-10)
+    # the asymmetric grid is finer for one-signed groups: a lower loss than the symmetric one here
+    L0, _ = oracle.search(X, W, a, grid, 4, 64)
+    assert np.all(L2 > 0) and not np.allclose(L0, L2)
+
+
+def test_pack_unsigned_layout():
+    u = (np.arange(16) % 16).astype(np.int16).reshape(16, 1)
+    w = oracle.pack_unsigned(u)
+    assert w.shape == (2, 1) and int(w[0, 0]) == 0x76543210 and int(w[1, 0]) == 0xFEDCBA98
