@@ -172,6 +172,13 @@ AWQ_API int awq_search(const void* X, const float* W, const float* a, int64_t N,
  *              quantisation error"): delta = max|w'| / 2^(b-1), codes clamped to
  *              [-2^(b-1), 2^(b-1)-1] (the passage gives no clamp; +max would
  *              need b+1 bits).  Pack with AWQ_PACK_DELTA_POW2.
+ *              AWQ_QUANT_ASYMMETRIC (compassingai.com AWQ concept page, "the
+ *              AWQ mechanism": MinMax uniform quantisation, symmetric or
+ *              asymmetric): lo = min(0, min w'), hi = max(0, max w'),
+ *              delta = (hi - lo) / (2^b - 1), zero point
+ *              z = clamp(rne(-lo / delta), 0, 2^b - 1), codes
+ *              q = clamp(rne(w' / delta), -z, 2^b - 1 - z); the dequantised
+ *              weight is q delta.  Pack with awq_quantize_pack_zp.
  *   w_mean     NULL, or [D_in] device fp32 (awq_weight_mean): the candidate
  *              scales are the balanced a^alpha / w_mean^(1-alpha); recover s*
  *              with awq_scales_ex.
@@ -184,6 +191,7 @@ AWQ_API int awq_search(const void* X, const float* W, const float* a, int64_t N,
  */
 #define AWQ_QUANT_SYMMETRIC 0
 #define AWQ_QUANT_DELTA_POW2 1
+#define AWQ_QUANT_ASYMMETRIC 2
 typedef struct {
   int quantizer;
   const float* w_mean;
@@ -332,6 +340,22 @@ AWQ_API int awq_quantize_pack_clip(const float* W, const float* s, const float* 
 #define AWQ_PACK_DENSE3 4
 AWQ_API int awq_quantize_pack_ex(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out,
                                  int bits, int group, int flags, uint32_t* packed, void* scales, void* stream);
+
+/*
+ * Final quantise + pack with the asymmetric quantiser (AWQ_QUANT_ASYMMETRIC
+ * above): the codes stored are u = q + z in [0, 2^b - 1] in the layout of
+ * awq_quantize_pack (nibbles) or, with AWQ_PACK_DENSE3, the dense 3-bit
+ * layout; the dequantised weight is (u - z) * scales[g][n].
+ *   flags   AWQ_PACK_DELTA_FP16 and/or AWQ_PACK_DENSE3 (AWQ_PACK_DELTA_POW2
+ *           is rejected with AWQ_EINVAL).  With AWQ_PACK_DELTA_FP16 delta is
+ *           rounded to FP16 before z and the codes are formed.
+ *   zeros   [D_in/group][D_out] uint8 output: z (device).
+ * No clip ratio (the clipping search is symmetric).  An all-zero group has
+ * delta = 0, z = 0 and codes 0.  Errors as awq_quantize_pack_ex.
+ * awq_w4a16_gemm reads symmetric codes only.
+ */
+AWQ_API int awq_quantize_pack_zp(const float* W, const float* s, int64_t D_in, int64_t D_out, int bits, int group,
+                                 int flags, uint32_t* packed, void* scales, uint8_t* zeros, void* stream);
 
 /*
  * The quantised layer applied to activations, the consumer of the pack

@@ -31,6 +31,7 @@ EXPORTS = (
     "awq_search_noalloc", "awq_clip_search_workspace_size", "awq_clip_search", "awq_quantize_pack_clip",
     "awq_search_joint_workspace_size", "awq_search_joint", "awq_quantize_pack_ex", "awq_w4a16_gemm",
     "awq_w4a16_workspace_size", "awq_search_ex", "awq_weight_mean", "awq_scales_ex", "awq_search_ex_workspace_size",
+    "awq_quantize_pack_zp",
 )
 STAGES = ("act_stats", "scale_table", "search_operand", "search_gemm", "loss_reduce", "quantize_pack",
           "weight_t", "clip_gram", "clip_operand", "clip_loss", "w4a16")
@@ -76,6 +77,7 @@ class AwqSearchOptions(ctypes.Structure):
 
 QUANT_SYMMETRIC = 0
 QUANT_DELTA_POW2 = 1
+QUANT_ASYMMETRIC = 2
 PACK_DELTA_POW2 = 2
 PACK_DENSE3 = 4
 _search_ex_ws = _sig("awq_search_ex_workspace_size", SZ, [I64, I64, I64, I, I, I, I,
@@ -98,6 +100,7 @@ _clip = _sig("awq_clip_search", I, [P, P, P, I64, I64, I64, P, I, I, I, P, P, P,
 _pack_clip = _sig("awq_quantize_pack_clip", I, [P, P, P, I64, I64, I, I, P, P, P])
 _joint_ws = _sig("awq_search_joint_workspace_size", SZ, [I64, I64, P, I, I, I, I, I])
 _pack_ex = _sig("awq_quantize_pack_ex", I, [P, P, P, I64, I64, I, I, I, P, P, P])
+_pack_zp = _sig("awq_quantize_pack_zp", I, [P, P, I64, I64, I, I, I, P, P, P, P])
 PACK_DELTA_FP16 = 1
 _w4a16 = _sig("awq_w4a16_gemm", I, [P, P, P, P, I64, I64, I64, I, I, P, P, SZ, P, P])
 _w4a16_ws = _sig("awq_w4a16_workspace_size", SZ, [I64, I64, I64])
@@ -304,6 +307,23 @@ def quantize_pack_ex(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int
              | (PACK_DENSE3 if dense3 else 0))
     _check(_pack_ex(_ptr(W), _ptr(s), _ptr(clip), D_in, D_out, bits, group, flags, _ptr(packed), _ptr(sc), _stream()))
     return packed, sc
+
+
+def quantize_pack_zp(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int = 128,
+                     delta_fp16: bool = False, dense3: bool = False):
+    """``awq_quantize_pack_zp``: the final pack with the asymmetric quantiser.
+    Returns (packed int32 view, scales, zeros uint8 [D_in/group, D_out]); the
+    codes are u = q + z."""
+    W = _dev(W, torch.float32, "W")
+    s = _dev(s, torch.float32, "s")
+    D_in, D_out = W.shape
+    rows = D_in // 32 * 3 if dense3 else D_in // 8
+    packed = torch.empty(rows, D_out, dtype=torch.int32, device=W.device)
+    sc = torch.empty(D_in // group, D_out, dtype=torch.float16 if delta_fp16 else torch.float32, device=W.device)
+    zeros = torch.empty(D_in // group, D_out, dtype=torch.uint8, device=W.device)
+    flags = (PACK_DELTA_FP16 if delta_fp16 else 0) | (PACK_DENSE3 if dense3 else 0)
+    _check(_pack_zp(_ptr(W), _ptr(s), D_in, D_out, bits, group, flags, _ptr(packed), _ptr(sc), _ptr(zeros), _stream()))
+    return packed, sc, zeros
 
 
 def w4a16_gemm(X: torch.Tensor, s: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, bits: int = 4,

@@ -462,10 +462,15 @@ int awq_search_ex(const void* X, const float* W, const float* a, int64_t N, int6
                   int32_t* alpha_idx, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
   SearchOpts o;
   if (options) {
-    if (options->quantizer != AWQ_QUANT_SYMMETRIC && options->quantizer != AWQ_QUANT_DELTA_POW2)
-      return fail(AWQ_EINVAL, "quantizer = %d: need AWQ_QUANT_SYMMETRIC or AWQ_QUANT_DELTA_POW2", options->quantizer);
+    switch (options->quantizer) {
+      case AWQ_QUANT_SYMMETRIC: o.qmode = awq::kQuantSymmetric; break;
+      case AWQ_QUANT_DELTA_POW2: o.qmode = awq::kQuantPow2; break;
+      case AWQ_QUANT_ASYMMETRIC: o.qmode = awq::kQuantAsymmetric; break;
+      default:
+        return fail(AWQ_EINVAL, "quantizer = %d: need AWQ_QUANT_SYMMETRIC, AWQ_QUANT_DELTA_POW2 or AWQ_QUANT_ASYMMETRIC",
+                    options->quantizer);
+    }
     if (options->w_mean) AWQ_TRY(check_ptr(options->w_mean, "w_mean", 4));
-    o.qmode = options->quantizer == AWQ_QUANT_DELTA_POW2 ? awq::kQuantPow2 : awq::kQuantSymmetric;
     o.w_mean = options->w_mean;
     o.gram = options->gram_form != 0;
   }
@@ -754,8 +759,9 @@ int awq_quantize_pack_clip(const float* W, const float* s, const float* clip, in
   return awq_quantize_pack_ex(W, s, clip, D_in, D_out, bits, group, 0, packed, scales, stream);
 }
 
-int awq_quantize_pack_ex(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out, int bits,
-                         int group, int flags, uint32_t* packed, void* scales, void* stream) {
+static int quantize_pack_impl(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out,
+                              int bits, int group, int flags, int qmode, uint32_t* packed, void* scales,
+                              uint8_t* zeros, void* stream) {
   AWQ_TRY(check_quant_args(bits, group));
   if (flags & ~(AWQ_PACK_DELTA_FP16 | AWQ_PACK_DELTA_POW2 | AWQ_PACK_DENSE3))
     return fail(AWQ_EINVAL, "flags = %#x: unknown bits", flags);
@@ -770,17 +776,31 @@ int awq_quantize_pack_ex(const float* W, const float* s, const float* clip, int6
   if (clip) AWQ_TRY(check_ptr(clip, "clip", 4));
   AWQ_TRY(check_ptr(packed, "packed", 16));
   AWQ_TRY(check_ptr(scales, "scales", 16));
+  if (qmode == awq::kQuantAsymmetric) AWQ_TRY(check_ptr(zeros, "zeros", 1));
   int sms = 0;
   AWQ_TRY(device_info(&sms));
   cudaError_t e;
   {
     StageTimer t(AWQ_STAGE_QUANTIZE_PACK, static_cast<cudaStream_t>(stream));
-    e = awq::launch_quantize_pack(W, s, clip, D_in, D_out, bits, group, (flags & AWQ_PACK_DELTA_FP16) != 0,
-                                  (flags & AWQ_PACK_DELTA_POW2) ? awq::kQuantPow2 : awq::kQuantSymmetric,
-                                  (flags & AWQ_PACK_DENSE3) != 0, packed, scales, sms,
+    e = awq::launch_quantize_pack(W, s, clip, D_in, D_out, bits, group, (flags & AWQ_PACK_DELTA_FP16) != 0, qmode,
+                                  (flags & AWQ_PACK_DENSE3) != 0, packed, scales, zeros, sms,
                                   static_cast<cudaStream_t>(stream));
   }
   return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "quantize_pack kernel");
+}
+
+int awq_quantize_pack_ex(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out, int bits,
+                         int group, int flags, uint32_t* packed, void* scales, void* stream) {
+  return quantize_pack_impl(W, s, clip, D_in, D_out, bits, group, flags,
+                            (flags & AWQ_PACK_DELTA_POW2) ? awq::kQuantPow2 : awq::kQuantSymmetric, packed, scales,
+                            nullptr, stream);
+}
+
+int awq_quantize_pack_zp(const float* W, const float* s, int64_t D_in, int64_t D_out, int bits, int group, int flags,
+                         uint32_t* packed, void* scales, uint8_t* zeros, void* stream) {
+  if (flags & AWQ_PACK_DELTA_POW2) return fail(AWQ_EINVAL, "AWQ_PACK_DELTA_POW2 does not apply to the asymmetric quantiser");
+  return quantize_pack_impl(W, s, nullptr, D_in, D_out, bits, group, flags, awq::kQuantAsymmetric, packed, scales,
+                            zeros, stream);
 }
 
 // ---------------------------------------------------------------- joint search over shared-input linears

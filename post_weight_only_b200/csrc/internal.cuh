@@ -10,10 +10,13 @@ namespace awq {
 
 constexpr int kMaxAlpha = 64;
 
-// Quantisers: delta = max / (2^(b-1) - 1), codes +-(2^(b-1) - 1); or the
-// power-of-two delta = max / 2^(b-1), codes [-2^(b-1), 2^(b-1) - 1].
+// Quantisers: delta = max / (2^(b-1) - 1), codes +-(2^(b-1) - 1); the
+// power-of-two delta = max / 2^(b-1), codes [-2^(b-1), 2^(b-1) - 1]; or the
+// asymmetric MinMax delta = (hi - lo) / (2^b - 1) with zero point z, codes
+// [-z, 2^b - 1 - z] (stored as u = q + z).
 constexpr int kQuantSymmetric = 0;
 constexpr int kQuantPow2 = 1;
+constexpr int kQuantAsymmetric = 2;
 
 // Loss forms of the search (see search.cu).
 constexpr int kFormError = 0;        // L = ||X E||^2 with E = S^-1 Q(S W) - W as the MMA operand
@@ -56,9 +59,10 @@ cudaError_t launch_weight_t(const float* W, int64_t D_in, int64_t D_out, uint16_
 // clip [D_in/group][D_out] (may be null) scales each group maximum; delta16:
 // delta rounded to FP16 before the codes, scales stored as FP16 (else fp32).
 // dense3: 3-bit codes as 96-bit strings of 32 rows (words [D_in/32*3][D_out]).
+// qmode kQuantAsymmetric: zeros [D_in/group][D_out] receives z (clip must be null).
 cudaError_t launch_quantize_pack(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out,
                                  int bits, int group, bool delta16, int qmode, bool dense3, uint32_t* packed,
-                                 void* scales, int num_sms, cudaStream_t st);
+                                 void* scales, uint8_t* zeros, int num_sms, cudaStream_t st);
 
 // ---- reduce.cu
 cudaError_t launch_loss_reduce(const float* partial, int A, int H, int64_t D_out, double* L_col, double* blk,

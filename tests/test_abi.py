@@ -154,7 +154,7 @@ def test_argument_checks_without_gpu(lib):
         return x(d["X"], d["W"], d["a"], d["N"], d["D_in"], d["D_out"], d["grid"], d["A"], d["bits"], d["group"],
                  d["form"], opts, d["L"], d["Lc"], d["astar"], d["aidx"], d["ws"], d["wsb"], d["st"], d["stream"])
 
-    assert xcall(ctypes.byref(Opts(2, None, 0))) == 1        # unknown quantiser
+    assert xcall(ctypes.byref(Opts(3, None, 0))) == 1        # unknown quantiser
     assert xcall(ctypes.byref(Opts(1, fake + 2, 0))) == 2    # misaligned weight means
     assert xcall(ctypes.byref(Opts(1, None, 0)), bits=5) == 3   # the common checks still apply
     xws = lib.awq_search_ex_workspace_size
@@ -177,6 +177,13 @@ def test_argument_checks_without_gpu(lib):
     assert pe(fake, fake, None, 256, 64, 4, 128, 8, fake, fake, None) == 1   # unknown flag bit
     assert pe(fake, fake, None, 256, 64, 4, 128, 4, fake, fake, None) == 1   # dense packing needs 3-bit codes
     assert pe(fake, fake, None, 256, 66, 3, 64, 4, fake, fake, None) == 3    # dense, D_out % 4 != 0, group 64
+    zp = lib.awq_quantize_pack_zp
+    zp.argtypes = [P, P, I64, I64, I, I, I, P, P, P, P]
+    zp.restype = I
+    assert zp(fake, fake, 256, 64, 4, 128, 2, fake, fake, fake, None) == 1     # no power-of-two delta
+    assert zp(fake, fake, 256, 64, 4, 128, 0, fake, fake, None, None) == 1     # zeros is required
+    assert zp(fake, fake, 256, 64, 4, 128, 4, fake, fake, fake, None) == 1     # dense needs 3-bit codes
+    assert zp(fake, fake, 250, 64, 4, 128, 0, fake, fake, fake, None) == 1     # D_in % group != 0
 
     t = lib.awq_selftest_wait_timeout
     t.argtypes = [P, I64, P]

@@ -31,9 +31,9 @@ def awq():
     return mod
 
 
-def _gram_bound(X, W, a, alpha, bits, group):
+def _gram_bound(X, W, a, alpha, bits, group, qmode=oracle.QMODE_SYMMETRIC):
     s = oracle.scales(a, alpha)
-    q, d = oracle.quantize(W, s, bits, group)
+    q, d = oracle.quantize(W, s, bits, group, qmode=qmode)
     w = W.numpy().astype(np.float64)
     e = q.astype(np.float64) * np.repeat(d, group, axis=0).astype(np.float64) / s.astype(np.float64)[:, None] - w
     x = X.float().numpy().astype(np.float64)
@@ -62,6 +62,26 @@ def test_gram_search_against_oracle(awq, N, D_in, D_out, bits, group):
         assert err <= bound, (al, L_gpu[i], L_or[i], bound)
         assert err <= 1e-2 * L_or[i], (al, err / L_or[i])
     assert np.allclose(res.L_col.cpu().numpy().sum(axis=1), L_gpu, rtol=1e-9)
+    check_alpha(L_or, best, int(res.alpha_idx.item()))
+
+
+def test_gram_search_asymmetric(awq):
+    """The Gram form with the asymmetric quantiser's operand."""
+    N, D_in, D_out, bits, group = 900, 256, 136, 4, 64
+    qm = oracle.QMODE_ASYMMETRIC
+    X, W = synth.layer_inputs(synth.small_layer(N, D_in, D_out, seed=77))
+    a = oracle.act_stats(X).astype(np.float32)
+    alphas = synth.alpha_grid(10).numpy()
+    res = awq.search(X.cuda(), W.cuda(), torch.from_numpy(a).cuda(), alphas.tolist(), bits, group, gram=True,
+                     quantizer=awq.QUANT_ASYMMETRIC)
+    L_gpu = res.L.cpu().numpy()
+    L_or, best = oracle.search(X, W, a, alphas, bits, group, qmode=qm)
+    for i, al in enumerate(alphas):
+        bound = (rounding_bound(X, W, a, al, bits, group, "error", qmode=qm).sum()
+                 + _gram_bound(X, W, a, al, bits, group, qmode=qm).sum())
+        err = abs(L_gpu[i] - L_or[i])
+        assert err <= bound, (al, L_gpu[i], L_or[i], bound)
+        assert err <= 1e-2 * L_or[i], (al, err / L_or[i])
     check_alpha(L_or, best, int(res.alpha_idx.item()))
 
 

@@ -11,7 +11,12 @@ against the CPU oracle, through the C ABI.
     per-channel scale s_j = mean|X_j|^alpha / mean|W_j|^(1-alpha)): the weight
     statistic within relative 1e-6 (fp64 sums in another order), the scales
     within one fp32 ulp (fp64 powers from two math libraries), the search as
-    above with the GPU's weight statistic given to both sides.
+    above with the GPU's weight statistic given to both sides;
+  * the asymmetric quantiser (compassingai.com AWQ concept page, "the AWQ
+    mechanism": MinMax with a zero point): the zero-point pack bit-exact
+    (codes, packed words in both layouts, deltas, zero points) on both pack
+    kernels, including one-sided, all-zero and clamped groups; the search as
+    above.
 """
 import numpy as np
 import pytest
@@ -207,3 +212,103 @@ def test_pack_dense3_unsupported_combination(awq):
         awq.quantize_pack_ex(W, s, 3, 32, dense3=True)     # D_out % 4 != 0 with a group below 128
     with pytest.raises(awq.AwqError):
         awq.quantize_pack_ex(torch.zeros(64, 8, device="cuda"), s, 4, 32, dense3=True)   # 4-bit codes
+
+
+# ---------------------------------------------------------------- asymmetric (MinMax, zero point)
+def _check_zp(awq, W, s, bits, group, delta16=False, dense3=False):
+    packed, sc, z = awq.quantize_pack_zp(W.cuda(), torch.from_numpy(s).cuda(), bits, group, delta_fp16=delta16,
+                                         dense3=dense3)
+    q, d, z_or = oracle.quantize_asym(W, s, bits, group, delta16=delta16)
+    u = q.astype(np.int16) + np.repeat(z_or, group, axis=0).astype(np.int16)
+    assert u.min() >= 0 and u.max() <= (1 << bits) - 1
+    want = oracle.pack3((u - 4).astype(np.int8)) if dense3 else oracle.pack_unsigned(u)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), want)
+    assert np.array_equal(z.cpu().numpy(), z_or)
+    got = sc.cpu().numpy()
+    assert np.array_equal(got.astype(np.float32) if delta16 else got, d)
+    return q, d, z_or
+
+
+@pytest.mark.parametrize("bits,group,D_in,D_out,delta16,dense3", [
+    (4, 128, 512, 256, False, False),     # tiled pack kernel
+    (3, 64, 384, 200, False, False),
+    (2, 32, 96, 36, False, False),
+    (4, 128, 256, 203, False, False),     # D_out % 4 != 0: the untiled kernel
+    (4, 64, 256, 128, True, False),       # FP16 deltas (z formed from the rounded delta)
+    (4, 256, 512, 96, True, False),       # group 256 (untiled) with FP16 deltas
+    (3, 128, 512, 128, False, True),      # dense 3-bit, tiled
+    (3, 32, 128, 64, False, True),        # dense 3-bit, group 32 (one string per group)
+    (3, 256, 512, 131, True, True),       # dense 3-bit, untiled, FP16 deltas
+])
+def test_pack_asym_bit_exact(awq, bits, group, D_in, D_out, delta16, dense3):
+    X, W = _layer(16, D_in, D_out, seed=D_in + 7 * D_out)
+    s = oracle.scales(oracle.act_stats(X).astype(np.float32), 0.6)
+    _check_zp(awq, W, s, bits, group, delta16, dense3)
+
+
+@pytest.mark.parametrize("dense3", [False, True])
+def test_pack_asym_special_groups(awq, dense3):
+    """One-sided groups (z = 0 and z = 2^b - 1), an all-zero group (delta = 0,
+    z = 0, codes 0), shifted columns, and a group whose top code is clamped:
+    lo = -3.5, hi = 11.5 give delta = 1, z = rne(3.5) = 4 and rne(11.5) = 12
+    above 2^b - 1 - z = 11 (4 bits)."""
+    bits = 3 if dense3 else 4
+    rng = np.random.default_rng(5)
+    W = rng.standard_normal((256, 64)).astype(np.float32)
+    W[:128, 0:8] = np.abs(W[:128, 0:8])          # non-negative groups
+    W[:128, 8:16] = -np.abs(W[:128, 8:16])       # non-positive groups
+    W[:128, 16:20] = 0.0                         # all-zero groups
+    W[:, 20:40] += 3.0                           # mostly positive, lo = 0 in many groups
+    W[128:, 40:44] = 0.25
+    W[128, 40:44] = -3.5
+    W[129, 40:44] = 11.5
+    s = np.ones(256, dtype=np.float32)
+    q, d, z = _check_zp(awq, torch.from_numpy(W), s, bits, 128, dense3=dense3)
+    umax = (1 << bits) - 1
+    assert np.all(z[0, 0:8] == 0) and np.all(z[0, 8:16] == umax)
+    assert np.all(d[0, 16:20] == 0) and np.all(z[0, 16:20] == 0) and np.all(q[:128, 16:20] == 0)
+    if bits == 4:
+        assert np.all(d[1, 40:44] == 1.0) and np.all(z[1, 40:44] == 4)
+        assert np.all(q[129, 40:44] == 11) and np.all(q[128, 40:44] == -4)
+
+
+@pytest.mark.parametrize("form", ("error", "reference"))
+@pytest.mark.parametrize("N,D_in,D_out,bits,group", [
+    (300, 512, 200, 4, 128),
+    (97, 96, 132, 2, 32),
+    (64, 256, 128, 3, 64),
+    (40, 512, 96, 4, 256),
+])
+def test_search_asym_against_oracle(awq, form, N, D_in, D_out, bits, group):
+    X, W = _layer(N, D_in, D_out, seed=N + 5 * D_out)
+    a = oracle.act_stats(X).astype(np.float32)
+    alphas = synth.alpha_grid(20).numpy()
+    lf = awq.LOSS_ERROR if form == "error" else awq.LOSS_REFERENCE
+    res = awq.search(X.cuda(), W.cuda(), torch.from_numpy(a).cuda(), alphas.tolist(), bits, group, loss_form=lf,
+                     quantizer=awq.QUANT_ASYMMETRIC)
+    L_gpu = res.L.cpu().numpy()
+    L_or, best = oracle.search(X, W, a, alphas, bits, group, qmode=oracle.QMODE_ASYMMETRIC)
+    for i, al in enumerate(alphas):
+        bound = rounding_bound(X, W, a, al, bits, group, form, qmode=oracle.QMODE_ASYMMETRIC).sum()
+        err = abs(L_gpu[i] - L_or[i])
+        assert err <= bound, (al, L_gpu[i], L_or[i], bound)
+        if form == "error":
+            assert err <= L_RTOL * L_or[i], (al, err / L_or[i])
+    check_alpha(L_or, best, int(res.alpha_idx.item()))
+
+
+def test_search_asym_below_symmetric(awq):
+    """On weights with a non-zero mean per column the asymmetric grid fits the
+    groups' ranges better: its losses lie below the symmetric ones (a
+    property of the two quantisers, checked on the oracle's own losses too)."""
+    X, W = _layer(256, 512, 128, seed=9)
+    W = W + 0.05
+    a = torch.from_numpy(oracle.act_stats(X).astype(np.float32)).cuda()
+    grid = synth.alpha_grid(10).tolist()
+    L_sym = awq.search(X.cuda(), W.cuda(), a, grid, 4, 128).L.cpu().numpy()
+    L_asym = awq.search(X.cuda(), W.cuda(), a, grid, 4, 128, quantizer=awq.QUANT_ASYMMETRIC).L.cpu().numpy()
+    assert np.all(L_asym < L_sym)
+    Lo_sym, _ = oracle.search(X, W, a.cpu().numpy(), np.asarray(grid, dtype=np.float32), 4, 128)
+    Lo_asym, _ = oracle.search(X, W, a.cpu().numpy(), np.asarray(grid, dtype=np.float32), 4, 128,
+                               qmode=oracle.QMODE_ASYMMETRIC)
+    assert np.all(Lo_asym < Lo_sym)
