@@ -524,12 +524,13 @@ def run_ours(args):
     w4_info = None
     if not args.no_w4a16:
         g4 = torch.Generator(device=dev).manual_seed(4321 + rank)
-        w4_info = {"timing": "CUDA graph of 20 calls (pre-pass + GEMM + status clear), weights rotated over "
-                             "copies > 256 MiB; synthetic packed words and deltas",
+        w4_info = {"timing": "CUDA graph of 20 calls (status clear, then N <= 4: GEMV + split reduce, else "
+                             "pre-pass + GEMM), weights rotated over copies > 256 MiB; synthetic packed words "
+                             "and deltas",
                    "algorithmic_bytes": "packed words + fp32 deltas + X (bf16) + s + Y (fp32), each once"}
         hbm_peak = float(load_peaks()[0]["hbm_gbs"])
         bf16_peak = float(load_peaks()[0]["bf16_tflops"])
-        for name, (Dk, Dn, Ns) in (("down_proj_28672x8192", (28672, 8192, (1, 16))),
+        for name, (Dk, Dn, Ns) in (("down_proj_28672x8192", (28672, 8192, (1, 4, 16))),
                                     ("attn_proj_4096x4096", (4096, 4096, (1, 16, 4096))),
                                     ("square_8192x8192", (8192, 8192, (4096,)))):
             packed_q = torch.randint(-2 ** 31, 2 ** 31 - 1, (Dk // 8, Dn), generator=g4, device=dev,
@@ -547,7 +548,7 @@ def run_ours(args):
                 gbs = nbytes / (ms / 1e3) / 1e9
                 tf = 2.0 * Nq * Dk * Dn / (ms / 1e3) / 1e12
                 w4_info[f"{name}_N{Nq}"] = {
-                    "ms": ms, "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "frac_hbm": gbs / hbm_peak,
+                    "path": "cuda-core GEMV" if Nq <= 4 else "tcgen05 GEMM", "ms": ms, "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "frac_hbm": gbs / hbm_peak,
                     "tflops": tf, "frac_bf16": tf / bf16_peak}
             del weights, packed_q
         torch.cuda.empty_cache()

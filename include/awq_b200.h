@@ -364,20 +364,24 @@ AWQ_API int awq_quantize_pack_zp(const float* W, const float* s, int64_t D_in, i
  * AWQ paper, TinyChat section, "on-the-fly weight dequantization"):
  *     Y[t][n] = sum_k x_tk / s_k * (u_kn - 2^(bits-1)) * scales[k/group][n]
  * with u the offset-binary codes of `packed` (the layout of
- * awq_quantize_pack).  Two launches on `stream`: X' = bf16(X / s) into the
- * workspace, then a tensor-core GEMM that dequantises the weights into
- * shared memory as bf16((u - 2^(bits-1)) * bf16(delta)) (one rounding of the
- * product) and accumulates in fp32.  For N <= 64 the k blocks of all output
- * tiles are shared out evenly over the CTAs (stream-K); a tile split between
- * CTAs is summed from partial tiles in the workspace in a fixed order, so
+ * awq_quantize_pack).  N <= 4 (decode): a CUDA-core GEMV in fp32 (x / s
+ * rounded once, exact integer weights, delta applied per 8 rows), split over
+ * k with the split partials summed in a fixed order by a second launch.
+ * N > 4: two launches on `stream`, X' = bf16(X / s) into the workspace, then
+ * a tensor-core GEMM that dequantises the weights into shared memory as
+ * bf16((u - 2^(bits-1)) * bf16(delta)) (one rounding of the product) and
+ * accumulates in fp32.  For N <= 64 the k blocks of all output tiles are
+ * shared out evenly over the CTAs (stream-K); a tile split between CTAs is
+ * summed from partial tiles in the workspace in a fixed order.  Either way
  * the result is deterministic.
  *   X         [N][D_in] bf16;  s [D_in] fp32 (s*);  packed [D_in/8][D_out] uint32
  *   scales    [D_in/group][D_out] fp32;  bits 2..4;  group 32, 64, 128 or 256
  *   D_out     a multiple of 4 (the rows of packed words are read by TMA)
  *   Y         [N][D_out] fp32 output
- *   workspace at least awq_w4a16_workspace_size(N, D_in, D_out) bytes: the
- *             scaled activations (N x D_in bf16) and, for N <= 64, room for
- *             the partial tiles.  No device is needed to compute the size.
+ *   workspace at least awq_w4a16_workspace_size(N, D_in, D_out) bytes: for
+ *             N <= 4 the split partials (up to 32 x N x D_out fp32); else
+ *             the scaled activations (N x D_in bf16) and, for N <= 64, room
+ *             for the partial tiles.  No device is needed to compute the size.
  *   status    [1] int32 device status word (required), as for awq_search
  */
 AWQ_API size_t awq_w4a16_workspace_size(int64_t N, int64_t D_in, int64_t D_out);

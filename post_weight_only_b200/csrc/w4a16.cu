@@ -41,6 +41,11 @@
 //               contiguous over n) and writes chunks 4h..4h+3 of row n of
 //               the A tile.
 //   warps 11-14 epilogue: TMEM lanes 32 (w % 4) .. + 31 -> Y.
+// Decode (N <= 4 tokens) takes a CUDA-core GEMV instead (see
+// w4a16_gemv_kernel): there the work is a stream of packed words with a few
+// FMAs per weight, bound by HBM, and a tensor-core tile of 16+ tokens would
+// sit mostly idle.
+//
 // Work: a unit is a 128-column x Nt-token output tile of KBS = ceil(KB /
 // KPS) stage steps.  Large N: units are dealt out to a persistent grid,
 // whole.  N <= 64: stream-K -- the units x KBS steps are cut into equal
@@ -481,6 +486,172 @@ __global__ void __launch_bounds__(kW4Threads, 1)
   if (warp == kW4MmaWarp) tmem_dealloc(tbase, 2 * p.tcols);
 }
 
+// ------------------------------------------------------------ decode: the GEMV
+// Y[t][n] = sum_k x~_tk * 16^(k%4) (u_kn - off) * delta_{k/G, n} on CUDA cores
+// for N <= 4 tokens, fp32 throughout (x / s rounded once, IEEE division; no
+// bf16 roundings of the weights).
+//
+// Dequantisation without integer-to-float conversions: for nibble i < 4 of a
+// word (bits 4i..4i+3), (w & (0xF << 4i)) | 0x4B000000 is the float
+// 2^23 + 16^i u exactly (the nibble lies in the mantissa), and subtracting
+// 2^23 + 16^i off leaves 16^i (u - off) exactly; nibbles 4..7 are the same
+// after w >> 16.  The factor 16^i is folded into the activation side,
+// x~_k = (x_k / s_k) 16^-(k % 4) (an exact power-of-two scaling), so every
+// product x~ * 16^i (u - off) equals x' (u - off).  Per word: one shift,
+// eight mask-ORs, four paired subtractions and four paired FMAs per token.
+//
+// Work: CTA (column tile, split) owns 128 columns (lane l: columns 4l..4l+3,
+// one 16-byte load per k8 row) and a contiguous range of k8 rows, which its 8
+// warps take in turn (warp w: rows w, w + 8, ...).  x~ of the range is
+// staged in shared memory in chunks of kGvChunk8 rows; each row's 8 values
+// are a warp-wide broadcast.  The warps' sums are added in warp order, and
+// with several splits the partial rows [split][N][D_out] are summed in split
+// order by gemv_reduce_kernel: the result does not depend on timing.  No
+// waits between CTAs.
+constexpr int kGvThreads = 256;
+constexpr int kGvCols = 128;
+constexpr int kGvChunk8 = 128;                   // k8 rows of x~ staged at a time
+constexpr int kGvUnroll = 4;                     // k8 rows in flight per warp (2 for 3-4 tokens)
+constexpr int kGvMaxSplit = 32;
+constexpr int kGvMaxTokens = 4;
+
+__device__ __forceinline__ float nib(uint32_t w, uint32_t mask) { return __uint_as_float((w & mask) | 0x4B000000u); }
+
+template <int NT>
+__global__ void __launch_bounds__(kGvThreads, NT == 1 ? 3 : 2) w4a16_gemv_kernel(const uint4* __restrict__ X,
+                                                                const float4* __restrict__ s,
+                                                                const uint4* __restrict__ packed,
+                                                                const float4* __restrict__ scales, int64_t D_in,
+                                                                int64_t D_out, int gshift, int off, int R8,
+                                                                float* __restrict__ out) {
+  constexpr int U = NT <= 2 ? kGvUnroll : kGvUnroll / 2;     // fits two CTAs per SM at 3-4 tokens
+  __shared__ __align__(16) float xt[NT * kGvChunk8 * 8];       // x~ [NT][chunk rows * 8]
+  __shared__ __align__(16) float red[8 * NT * kGvCols];         // per-warp sums
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t rows8 = D_in / 8;
+  const int64_t D4 = D_out / 4;
+  const int64_t rb = static_cast<int64_t>(blockIdx.y) * R8;      // first k8 row of this split
+  const int64_t re = rb + R8 < rows8 ? rb + R8 : rows8;
+  const int64_t n4 = static_cast<int64_t>(blockIdx.x) * (kGvCols / 4) + lane;   // column quad
+  const bool valid = n4 < D4;
+  const float fo = static_cast<float>(off);
+  const float2 bias01 = make_float2(-(8388608.0f + fo), -(8388608.0f + 16.0f * fo));
+  const float2 bias23 = make_float2(-(8388608.0f + 256.0f * fo), -(8388608.0f + 4096.0f * fo));
+  float2 tot[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tot[t][c] = make_float2(0.0f, 0.0f);
+
+  for (int64_t cb = rb; cb < re; cb += kGvChunk8) {
+    const int nr = static_cast<int>(re - cb < kGvChunk8 ? re - cb : kGvChunk8);
+    if (cb != rb) __syncthreads();                 // the previous chunk's x~ is no longer read
+    for (int i = threadIdx.x; i < NT * nr; i += kGvThreads) {
+      const int t = i / nr, r = i - t * nr;
+      const uint4 xv = X[t * rows8 + cb + r];
+      const float4 s0 = __ldg(s + 2 * (cb + r)), s1 = __ldg(s + 2 * (cb + r) + 1);
+      float4 lo, hi;
+      lo.x = __fdiv_rn(bf16_bits_to_float(xv.x & 0xFFFFu), s0.x);
+      lo.y = __fmul_rn(__fdiv_rn(bf16_bits_to_float(xv.x >> 16), s0.y), 0.0625f);
+      lo.z = __fmul_rn(__fdiv_rn(bf16_bits_to_float(xv.y & 0xFFFFu), s0.z), 0.00390625f);
+      lo.w = __fmul_rn(__fdiv_rn(bf16_bits_to_float(xv.y >> 16), s0.w), 0.000244140625f);
+      hi.x = __fdiv_rn(bf16_bits_to_float(xv.z & 0xFFFFu), s1.x);
+      hi.y = __fmul_rn(__fdiv_rn(bf16_bits_to_float(xv.z >> 16), s1.y), 0.0625f);
+      hi.z = __fmul_rn(__fdiv_rn(bf16_bits_to_float(xv.w & 0xFFFFu), s1.z), 0.00390625f);
+      hi.w = __fmul_rn(__fdiv_rn(bf16_bits_to_float(xv.w >> 16), s1.w), 0.000244140625f);
+      float4* dst = reinterpret_cast<float4*>(xt + (t * kGvChunk8 + r) * 8);
+      dst[0] = lo;
+      dst[1] = hi;
+    }
+    __syncthreads();
+    if (valid) {
+      for (int r = warp; r < nr; r += 8 * U) {
+        uint4 pw[U];
+        float4 d[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int rr = r + 8 * u;
+          if (rr < nr) {
+            pw[u] = __ldcs(packed + (cb + rr) * D4 + n4);
+            d[u] = __ldg(scales + (((cb + rr) * 8) >> gshift) * D4 + n4);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int rr = r + 8 * u;
+          if (rr >= nr) break;                       // uniform over the warp
+          float4 xa[NT], xb[NT];
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            const float4* src = reinterpret_cast<const float4*>(xt + (t * kGvChunk8 + rr) * 8);
+            xa[t] = src[0];
+            xb[t] = src[1];
+          }
+          const uint32_t wv[4] = {pw[u].x, pw[u].y, pw[u].z, pw[u].w};
+          const float dv[4] = {d[u].x, d[u].y, d[u].z, d[u].w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t w = wv[c], wh = w >> 16;
+            const float2 v01 = __fadd2_rn(make_float2(nib(w, 0xFu), nib(w, 0xF0u)), bias01);
+            const float2 v23 = __fadd2_rn(make_float2(nib(w, 0xF00u), nib(w, 0xF000u)), bias23);
+            const float2 v45 = __fadd2_rn(make_float2(nib(wh, 0xFu), nib(wh, 0xF0u)), bias01);
+            const float2 v67 = __fadd2_rn(make_float2(nib(wh, 0xF00u), nib(wh, 0xF000u)), bias23);
+            const float2 d2 = make_float2(dv[c], dv[c]);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+              float2 a = __fmul2_rn(v01, make_float2(xa[t].x, xa[t].y));
+              a = __ffma2_rn(v23, make_float2(xa[t].z, xa[t].w), a);
+              a = __ffma2_rn(v45, make_float2(xb[t].x, xb[t].y), a);
+              a = __ffma2_rn(v67, make_float2(xb[t].z, xb[t].w), a);
+              tot[t][c] = __ffma2_rn(a, d2, tot[t][c]);
+            }
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+    reinterpret_cast<float4*>(red)[(warp * NT + t) * (kGvCols / 4) + lane] =
+        make_float4(tot[t][0].x + tot[t][0].y, tot[t][1].x + tot[t][1].y, tot[t][2].x + tot[t][2].y,
+                    tot[t][3].x + tot[t][3].y);
+  __syncthreads();
+  if (threadIdx.x < NT * 32) {
+    const int t = threadIdx.x >> 5, q = threadIdx.x & 31;
+    const int64_t m4 = static_cast<int64_t>(blockIdx.x) * (kGvCols / 4) + q;
+    if (m4 < D4) {
+      const float4* rv = reinterpret_cast<const float4*>(red);
+      float4 a = rv[t * (kGvCols / 4) + q];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) {
+        const float4 b = rv[(w * NT + t) * (kGvCols / 4) + q];
+        a.x += b.x;
+        a.y += b.y;
+        a.z += b.z;
+        a.w += b.w;
+      }
+      reinterpret_cast<float4*>(out)[(static_cast<int64_t>(blockIdx.y) * NT + t) * D4 + m4] = a;
+    }
+  }
+}
+
+// Y = sum over splits of the partial rows, in split order.
+__global__ void __launch_bounds__(256) gemv_reduce_kernel(const float4* __restrict__ part, int splits, int64_t n4,
+                                                          float4* __restrict__ Y) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float4 a = part[i];
+    for (int k = 1; k < splits; ++k) {
+      const float4 b = part[k * n4 + i];
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    Y[i] = a;
+  }
+}
+
 }  // namespace
 
 namespace {
@@ -495,6 +666,11 @@ int w4_token_tile(int64_t N) { return N >= 256 ? 256 : static_cast<int>((N + 15)
 
 W4Layout w4_layout(int64_t N, int64_t D_in, int64_t D_out) {
   W4Layout l;
+  if (N <= kGvMaxTokens) {                        // the GEMV: partial rows of up to kGvMaxSplit splits
+    l.xs = l.count = l.partial = 0;
+    l.total = round256(static_cast<size_t>(kGvMaxSplit) * N * D_out * 4);
+    return l;
+  }
   const int Nt = w4_token_tile(N);
   const int64_t units = ((D_out + 127) / 128) * ((N + Nt - 1) / Nt);
   l.xs = 0;
@@ -506,6 +682,63 @@ W4Layout w4_layout(int64_t N, int64_t D_in, int64_t D_out) {
   return l;
 }
 
+template <int NT>
+cudaError_t launch_gemv_nt(dim3 grid, cudaStream_t st, const void* X, const float* s, const uint32_t* packed,
+                           const float* scales, int64_t D_in, int64_t D_out, int gshift, int off, int R8, float* out) {
+  w4a16_gemv_kernel<NT><<<grid, kGvThreads, 0, st>>>(
+      static_cast<const uint4*>(X), reinterpret_cast<const float4*>(s), reinterpret_cast<const uint4*>(packed),
+      reinterpret_cast<const float4*>(scales), D_in, D_out, gshift, off, R8, out);
+  return cudaGetLastError();
+}
+
+int launch_w4a16_gemv(const void* X, const float* s, const uint32_t* packed, const float* scales, int64_t N,
+                      int64_t D_in, int64_t D_out, int bits, int group, float* Y, void* ws, int num_sms,
+                      cudaStream_t st, cudaError_t* cerr, const char** what) {
+  const int64_t rows8 = D_in / 8;
+  const int64_t tiles = (D_out + kGvCols - 1) / kGvCols;
+  // About eight CTAs per SM over column tiles x splits; at least 8 k8 rows
+  // (one per warp) per split.
+  int64_t splits = (static_cast<int64_t>(num_sms > 0 ? num_sms : 1) * 8 + tiles / 2) / tiles;
+  if (splits > rows8 / 8) splits = rows8 / 8;
+  if (splits > kGvMaxSplit) splits = kGvMaxSplit;
+  if (splits < 1) splits = 1;
+  int64_t R8 = (rows8 + splits - 1) / splits;
+  R8 = (R8 + 7) / 8 * 8;
+  splits = (rows8 + R8 - 1) / R8;
+  const int gshift = group == 32 ? 5 : group == 64 ? 6 : group == 128 ? 7 : 8;
+  const int off = 1 << (bits - 1);
+  float* out = splits == 1 ? Y : static_cast<float*>(ws);
+  const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(splits));
+  cudaError_t e;
+  switch (N) {
+    case 1: e = launch_gemv_nt<1>(grid, st, X, s, packed, scales, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
+    case 2: e = launch_gemv_nt<2>(grid, st, X, s, packed, scales, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
+    case 3: e = launch_gemv_nt<3>(grid, st, X, s, packed, scales, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
+    case 4: e = launch_gemv_nt<4>(grid, st, X, s, packed, scales, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
+    default: *what = "gemv token count"; return kEUnsupported;
+  }
+  if (e != cudaSuccess) {
+    *cerr = e;
+    *what = "w4a16_gemv_kernel launch";
+    return kECuda;
+  }
+  if (splits > 1) {
+    const int64_t n4 = N * D_out / 4;
+    int64_t blocks = (n4 + 255) / 256;
+    if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
+    gemv_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(static_cast<const float4*>(ws),
+                                                                     static_cast<int>(splits), n4,
+                                                                     reinterpret_cast<float4*>(Y));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      *cerr = e;
+      *what = "gemv_reduce_kernel launch";
+      return kECuda;
+    }
+  }
+  return kOk;
+}
+
 }  // namespace
 
 size_t w4a16_scratch_bytes(int64_t N, int64_t D_in, int64_t D_out) { return w4_layout(N, D_in, D_out).total; }
@@ -514,6 +747,8 @@ int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const fl
                  int64_t D_out, int bits, int group, float* Y, void* ws, int num_sms, int* status,
                  uint64_t timeout_ns, cudaStream_t st, cudaError_t* cerr, const char** what) {
   *cerr = cudaSuccess;
+  if (N <= kGvMaxTokens)
+    return launch_w4a16_gemv(X, s, packed, scales, N, D_in, D_out, bits, group, Y, ws, num_sms, st, cerr, what);
   const W4Layout lay = w4_layout(N, D_in, D_out);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   void* xs = wsb + lay.xs;

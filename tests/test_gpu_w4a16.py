@@ -2,7 +2,12 @@
 applied to activations) against the oracle, on codes packed by the library
 itself.
 
-Tolerance, from the arithmetic of the CUDA path: x_tk / s_k is rounded to
+Two CUDA paths: N <= 4 tokens run the CUDA-core GEMV (fp32 throughout: x / s
+rounded once to fp32, exact integer weights, delta applied per k8 row); more
+tokens run the tensor-core GEMM.  The bound below, derived for the GEMM,
+covers the GEMV's smaller errors too.
+
+Tolerance, from the arithmetic of the tensor-core path: x_tk / s_k is rounded to
 bf16 once, each weight q * bf16(delta) is rounded to bf16 once (relative
 errors at most 2^-9 each, modelled as independent and uniform; the model
 allows uniform errors up to U = 2^-8 per term, which covers both), and delta
@@ -62,7 +67,12 @@ def _case(awq, N, D_in, D_out, bits, group, seed):
 
 
 @pytest.mark.parametrize("N,D_in,D_out,bits,group", [
-    (1, 4096, 4096, 4, 128),      # one decode token: split K over a cluster
+    (1, 4096, 4096, 4, 128),      # one decode token: the GEMV, split K
+    (2, 512, 200, 4, 128),        # GEMV: ragged second column tile
+    (4, 1024, 132, 3, 64),        # GEMV at its largest token count
+    (1, 32, 4, 4, 32),            # GEMV: one group, four k8 rows (fewer than the warps), one column quad
+    (2, 2048, 256, 4, 256),       # GEMV, group 256
+    (3, 256, 1000, 2, 32),        # GEMV, 2-bit, group 32
     (5, 512, 200, 4, 128),        # ragged columns, a few tokens
     (16, 96, 36, 4, 32),          # D_in not a multiple of 64: a half k block
     (37, 384, 132, 3, 64),
@@ -89,12 +99,17 @@ def test_w4a16_reproducible(awq):
     assert np.array_equal(Y1, Y2)
 
 
-def test_w4a16_decode_full_size(awq):
-    """A 70B-class down projection (D_in 28672, D_out 8192) at one token: the
-    stream-K decode configuration that is timed; sampled columns checked
-    against the oracle's definition."""
-    N, D_in, D_out, bits, group = 1, 28672, 8192, 4, 128
-    g = torch.Generator().manual_seed(11)
+@pytest.mark.parametrize("N,D_in,D_out", [
+    (1, 28672, 8192),     # the timed decode configuration (split K, two x~ chunks per split)
+    (4, 28672, 8192),
+    (2, 8192, 32768),     # few splits, long splits: two x~ chunks each
+])
+def test_w4a16_decode_full_size(awq, N, D_in, D_out):
+    """A 70B-class down projection (D_in 28672, D_out 8192) at one and four
+    tokens, the GEMV configuration that is timed, and a wide layer; sampled
+    columns checked against the oracle's definition."""
+    bits, group = 4, 128
+    g = torch.Generator().manual_seed(11 + N)
     X = (torch.randn(N, D_in, generator=g) * 0.5).to(torch.bfloat16)
     s = torch.rand(D_in, generator=g) + 0.5
     packed = torch.randint(-2 ** 31, 2 ** 31 - 1, (D_in // 8, D_out), generator=g, dtype=torch.int64).to(torch.int32)
