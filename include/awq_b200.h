@@ -365,7 +365,7 @@ AWQ_API int awq_quantize_pack_zp(const float* W, const float* s, int64_t D_in, i
  *     Y[t][n] = sum_k x_tk / s_k * (u_kn - 2^(bits-1)) * scales[k/group][n]
  * with u the offset-binary codes of `packed` (the layout of
  * awq_quantize_pack).  N <= 4 (decode): a CUDA-core GEMV in fp32 (x / s
- * rounded once, exact integer weights, delta applied per 8 rows), split over
+ * rounded once, exact integer weights, delta applied once per group), split over
  * k with the split partials summed in a fixed order by a second launch.
  * N > 4: two launches on `stream`, X' = bf16(X / s) into the workspace, then
  * a tensor-core GEMM that dequantises the weights into shared memory as

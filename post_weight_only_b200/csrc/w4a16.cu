@@ -489,7 +489,7 @@ __global__ void __launch_bounds__(kW4Threads, 1)
 // ------------------------------------------------------------ decode: the GEMV
 // Y[t][n] = sum_k x~_tk * 16^(k%4) (u_kn - off) * delta_{k/G, n} on CUDA cores
 // for N <= 4 tokens, fp32 throughout (x / s rounded once, IEEE division; no
-// bf16 roundings of the weights).
+// bf16 roundings of the weights; delta applied once per group).
 //
 // Dequantisation without integer-to-float conversions: for nibble i < 4 of a
 // word (bits 4i..4i+3), (w & (0xF << 4i)) | 0x4B000000 is the float
@@ -501,8 +501,8 @@ __global__ void __launch_bounds__(kW4Threads, 1)
 // eight mask-ORs, four paired subtractions and four paired FMAs per token.
 //
 // Work: CTA (column tile, split) owns 128 columns (lane l: columns 4l..4l+3,
-// one 16-byte load per k8 row) and a contiguous range of k8 rows, which its 8
-// warps take in turn (warp w: rows w, w + 8, ...).  x~ of the range is
+// one 16-byte load per k8 row) and a contiguous range of k8 rows, cut into
+// eight contiguous runs, one per warp.  x~ of the range is
 // staged in shared memory in chunks of kGvChunk8 rows; each row's 8 values
 // are a warp-wide broadcast.  The warps' sums are added in warp order, and
 // with several splits the partial rows [split][N][D_out] are summed in split
@@ -565,21 +565,45 @@ __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 3 : 2) w4a16_gemv_kernel
     }
     __syncthreads();
     if (valid) {
-      for (int r = warp; r < nr; r += 8 * U) {
-        uint4 pw[U];
-        float4 d[U];
+      // warp w: the contiguous rows [w q, min((w + 1) q, nr)) of the chunk,
+      // q = ceil(nr / 8); products are summed per quantisation group and
+      // delta is applied once per group (and at the end of the range).
+      const int q = (nr + 7) >> 3;
+      const int r0 = warp * q, r1 = r0 + q < nr ? r0 + q : nr;
+      float2 acc[NT][4];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int rr = r + 8 * u;
-          if (rr < nr) {
-            pw[u] = __ldcs(packed + (cb + rr) * D4 + n4);
-            d[u] = __ldg(scales + (((cb + rr) * 8) >> gshift) * D4 + n4);
-          }
+      for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[t][c] = make_float2(0.0f, 0.0f);
+      int64_t g_cur = -1;                          // the group acc belongs to
+      float4 dcur = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      auto flush = [&]() {
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          tot[t][0] = __ffma2_rn(acc[t][0], make_float2(dcur.x, dcur.x), tot[t][0]);
+          tot[t][1] = __ffma2_rn(acc[t][1], make_float2(dcur.y, dcur.y), tot[t][1]);
+          tot[t][2] = __ffma2_rn(acc[t][2], make_float2(dcur.z, dcur.z), tot[t][2]);
+          tot[t][3] = __ffma2_rn(acc[t][3], make_float2(dcur.w, dcur.w), tot[t][3]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[t][c] = make_float2(0.0f, 0.0f);
         }
+      };
+      for (int r = r0; r < r1; r += U) {
+        const uint4* pp = packed + (cb + r) * D4 + n4;
+        uint4 pw[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (r + u < r1) pw[u] = __ldcs(pp + u * D4);
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-          const int rr = r + 8 * u;
-          if (rr >= nr) break;                       // uniform over the warp
+          const int rr = r + u;
+          if (rr >= r1) break;                       // uniform over the warp
+          const int64_t g = ((cb + rr) * 8) >> gshift;
+          if (g != g_cur) {                          // uniform over the warp
+            if (g_cur >= 0) flush();
+            dcur = __ldg(scales + g * D4 + n4);      // used at the group's flush
+            g_cur = g;
+          }
           float4 xa[NT], xb[NT];
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
@@ -588,7 +612,6 @@ __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 3 : 2) w4a16_gemv_kernel
             xb[t] = src[1];
           }
           const uint32_t wv[4] = {pw[u].x, pw[u].y, pw[u].z, pw[u].w};
-          const float dv[4] = {d[u].x, d[u].y, d[u].z, d[u].w};
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const uint32_t w = wv[c], wh = w >> 16;
@@ -596,18 +619,17 @@ __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 3 : 2) w4a16_gemv_kernel
             const float2 v23 = __fadd2_rn(make_float2(nib(w, 0xF00u), nib(w, 0xF000u)), bias23);
             const float2 v45 = __fadd2_rn(make_float2(nib(wh, 0xFu), nib(wh, 0xF0u)), bias01);
             const float2 v67 = __fadd2_rn(make_float2(nib(wh, 0xF00u), nib(wh, 0xF000u)), bias23);
-            const float2 d2 = make_float2(dv[c], dv[c]);
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
-              float2 a = __fmul2_rn(v01, make_float2(xa[t].x, xa[t].y));
-              a = __ffma2_rn(v23, make_float2(xa[t].z, xa[t].w), a);
-              a = __ffma2_rn(v45, make_float2(xb[t].x, xb[t].y), a);
-              a = __ffma2_rn(v67, make_float2(xb[t].z, xb[t].w), a);
-              tot[t][c] = __ffma2_rn(a, d2, tot[t][c]);
+              float2 a2 = __ffma2_rn(v01, make_float2(xa[t].x, xa[t].y), acc[t][c]);
+              a2 = __ffma2_rn(v23, make_float2(xa[t].z, xa[t].w), a2);
+              a2 = __ffma2_rn(v45, make_float2(xb[t].x, xb[t].y), a2);
+              acc[t][c] = __ffma2_rn(v67, make_float2(xb[t].z, xb[t].w), a2);
             }
           }
         }
       }
+      if (g_cur >= 0) flush();
     }
   }
 #pragma unroll
