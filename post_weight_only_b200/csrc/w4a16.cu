@@ -86,6 +86,8 @@ struct W4Params {
   int* count;               // stream-K: [units] contributions received (zeroed by scale_x)
   int64_t N, D_out;
   int off;                  // 2^(bits-1)
+  uint32_t magic;           // 0x43004300, passed at run time so that it lives in a register and each
+                            // mask-and-OR is one three-input logic op (an op takes one immediate)
   int Nt, KB, kps, KBS, n_tiles, units;
   int stream;               // 1: stream-K over units x KBS steps, `chunk` steps per CTA
   int issuers;              // TMA warps that fill alternate stages (1 or 2)
@@ -323,6 +325,7 @@ __global__ void __launch_bounds__(kW4Threads, 1)
     const int n = (warp & 3) * 32 + lane;
     const int h = (warp - kW4DqWarp0) >> 2;       // half of each k block: chunks 4h..4h+3
     const uint32_t bias_bits = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(128.0f + p.off)));
+    const uint32_t magic = p.magic;
     const __nv_bfloat162 bias = as_bf162(bias_bits | (bias_bits << 16));     // 128 + off, exact
     const int swz = n & 7;
     int s = 0, sa = 0;
@@ -359,7 +362,7 @@ __global__ void __launch_bounds__(kW4Threads, 1)
           for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const uint32_t pair = ((w[i] >> (4 * q)) & 0x000F000Fu) | 0x43004300u;   // {128 + u_q, 128 + u_{q+4}}
+              const uint32_t pair = ((w[i] >> (4 * q)) & 0x000F000Fu) | magic;   // {128 + u_q, 128 + u_{q+4}}
               o[4 * i + q] = as_u32(__hmul2(__hsub2(as_bf162(pair), bias), d2));
             }
           uint4* arow = reinterpret_cast<uint4*>(a_sm + sa * kW4ABytes + (n >> 3) * 1024 + (n & 7) * 128);
@@ -515,15 +518,19 @@ constexpr int kGvUnroll = 4;                     // k8 rows in flight per warp (
 constexpr int kGvMaxSplit = 32;
 constexpr int kGvMaxTokens = 4;
 
-__device__ __forceinline__ float nib(uint32_t w, uint32_t mask) { return __uint_as_float((w & mask) | 0x4B000000u); }
+// magic = 0x4B000000 (2^23), a kernel argument so that it sits in a register
+// and (w & mask) | magic is one three-input logic op.
+__device__ __forceinline__ float nib(uint32_t w, uint32_t mask, uint32_t magic) {
+  return __uint_as_float((w & mask) | magic);
+}
 
 template <int NT>
 __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 3 : 2) w4a16_gemv_kernel(const uint4* __restrict__ X,
                                                                 const float4* __restrict__ s,
                                                                 const uint4* __restrict__ packed,
                                                                 const float4* __restrict__ scales, int64_t D_in,
-                                                                int64_t D_out, int gshift, int off, int R8,
-                                                                float* __restrict__ out) {
+                                                                int64_t D_out, int gshift, int off,
+                                                                uint32_t magic, int R8, float* __restrict__ out) {
   constexpr int U = NT <= 2 ? kGvUnroll : kGvUnroll / 2;     // fits two CTAs per SM at 3-4 tokens
   __shared__ __align__(16) float xt[NT * kGvChunk8 * 8];       // x~ [NT][chunk rows * 8]
   __shared__ __align__(16) float red[8 * NT * kGvCols];         // per-warp sums
@@ -615,10 +622,10 @@ __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 3 : 2) w4a16_gemv_kernel
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const uint32_t w = wv[c], wh = w >> 16;
-            const float2 v01 = __fadd2_rn(make_float2(nib(w, 0xFu), nib(w, 0xF0u)), bias01);
-            const float2 v23 = __fadd2_rn(make_float2(nib(w, 0xF00u), nib(w, 0xF000u)), bias23);
-            const float2 v45 = __fadd2_rn(make_float2(nib(wh, 0xFu), nib(wh, 0xF0u)), bias01);
-            const float2 v67 = __fadd2_rn(make_float2(nib(wh, 0xF00u), nib(wh, 0xF000u)), bias23);
+            const float2 v01 = __fadd2_rn(make_float2(nib(w, 0xFu, magic), nib(w, 0xF0u, magic)), bias01);
+            const float2 v23 = __fadd2_rn(make_float2(nib(w, 0xF00u, magic), nib(w, 0xF000u, magic)), bias23);
+            const float2 v45 = __fadd2_rn(make_float2(nib(wh, 0xFu, magic), nib(wh, 0xF0u, magic)), bias01);
+            const float2 v67 = __fadd2_rn(make_float2(nib(wh, 0xF00u, magic), nib(wh, 0xF000u, magic)), bias23);
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
               float2 a2 = __ffma2_rn(v01, make_float2(xa[t].x, xa[t].y), acc[t][c]);
@@ -709,7 +716,7 @@ cudaError_t launch_gemv_nt(dim3 grid, cudaStream_t st, const void* X, const floa
                            const float* scales, int64_t D_in, int64_t D_out, int gshift, int off, int R8, float* out) {
   w4a16_gemv_kernel<NT><<<grid, kGvThreads, 0, st>>>(
       static_cast<const uint4*>(X), reinterpret_cast<const float4*>(s), reinterpret_cast<const uint4*>(packed),
-      reinterpret_cast<const float4*>(scales), D_in, D_out, gshift, off, R8, out);
+      reinterpret_cast<const float4*>(scales), D_in, D_out, gshift, off, 0x4B000000u, R8, out);
   return cudaGetLastError();
 }
 
@@ -859,6 +866,7 @@ int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const fl
   p.N = N;
   p.D_out = D_out;
   p.off = 1 << (bits - 1);
+  p.magic = 0x43004300u;
   p.Nt = Nt;
   p.KB = KB;
   p.kps = kps;
