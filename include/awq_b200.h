@@ -377,7 +377,7 @@ AWQ_API int awq_quantize_pack_zp(const float* W, const float* s, int64_t D_in, i
  *   X         [N][D_in] bf16;  s [D_in] fp32 (s*);  packed [D_in/8][D_out] uint32
  *   scales    [D_in/group][D_out] fp32;  bits 2..4;  group 32, 64, 128 or 256
  *   D_out     a multiple of 4 (the rows of packed words are read by TMA)
- *   Y         [N][D_out] fp32 output
+ *   Y         [N][D_out] fp32 output, 4-byte aligned
  *   workspace at least awq_w4a16_workspace_size(N, D_in, D_out) bytes: for
  *             N <= 4 the split partials (up to 32 x N x D_out fp32); else
  *             the scaled activations (N x D_in bf16) and, for N <= 64, room

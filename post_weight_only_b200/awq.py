@@ -328,10 +328,11 @@ def quantize_pack_zp(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int
 
 def w4a16_gemm(X: torch.Tensor, s: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, bits: int = 4,
                group: int = 128, check_status: bool = True,
-               workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+               workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Y = X diag(1/s) Dequant(packed, scales), fp32: ``awq_w4a16_gemm``.
     ``workspace`` (uint8, at least ``w4a16_workspace_size(N, D_in, D_out)`` bytes)
-    is allocated per call when not given."""
+    is allocated per call when not given; ``out`` (contiguous fp32 [N, D_out]
+    on the same device) receives Y when given."""
     X = _dev(X, torch.bfloat16, "X")
     s = _dev(s, torch.float32, "s")
     if packed.dtype not in (torch.int32, torch.uint32):
@@ -340,7 +341,13 @@ def w4a16_gemm(X: torch.Tensor, s: torch.Tensor, packed: torch.Tensor, scales: t
     scales = _dev(scales, torch.float32, "scales")
     N, D_in = X.shape
     D_out = packed.shape[1]
-    Y = torch.empty(N, D_out, dtype=torch.float32, device=X.device)
+    if out is None:
+        Y = torch.empty(N, D_out, dtype=torch.float32, device=X.device)
+    else:
+        if out.dtype != torch.float32 or out.device != X.device or tuple(out.shape) != (N, D_out) \
+                or not out.is_contiguous():
+            raise ValueError("out must be a contiguous float32 [N, D_out] tensor on X's device")
+        Y = out
     status = torch.zeros(1, dtype=torch.int32, device=X.device)
     nbytes = _w4a16_ws(N, D_in, D_out)
     if workspace is None or workspace.numel() < nbytes:

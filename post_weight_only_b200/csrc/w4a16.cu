@@ -664,9 +664,10 @@ __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 3 : 2) w4a16_gemv_kernel
   }
 }
 
-// Y = sum over splits of the partial rows, in split order.
+// Y = sum over splits of the partial rows, in split order.  y16: Y is 16-byte
+// aligned (else four scalar stores; the API asks only 4-byte alignment of Y).
 __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float4* __restrict__ part, int splits, int64_t n4,
-                                                          float4* __restrict__ Y) {
+                                                          float* __restrict__ Y, int y16) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     float4 a = part[i];
@@ -677,7 +678,14 @@ __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float4* __restri
       a.z += b.z;
       a.w += b.w;
     }
-    Y[i] = a;
+    if (y16) {
+      reinterpret_cast<float4*>(Y)[i] = a;
+    } else {
+      Y[4 * i] = a.x;
+      Y[4 * i + 1] = a.y;
+      Y[4 * i + 2] = a.z;
+      Y[4 * i + 3] = a.w;
+    }
   }
 }
 
@@ -736,7 +744,10 @@ int launch_w4a16_gemv(const void* X, const float* s, const uint32_t* packed, con
   splits = (rows8 + R8 - 1) / R8;
   const int gshift = group == 32 ? 5 : group == 64 ? 6 : group == 128 ? 7 : 8;
   const int off = 1 << (bits - 1);
-  float* out = splits == 1 ? Y : static_cast<float*>(ws);
+  // The GEMV stores 16-byte rows: straight into Y when there is one split and
+  // Y is 16-byte aligned, else into the workspace for gemv_reduce_kernel.
+  const bool y16 = (reinterpret_cast<uintptr_t>(Y) & 15u) == 0;
+  float* out = splits == 1 && y16 ? Y : static_cast<float*>(ws);
   const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(splits));
   cudaError_t e;
   switch (N) {
@@ -751,13 +762,12 @@ int launch_w4a16_gemv(const void* X, const float* s, const uint32_t* packed, con
     *what = "w4a16_gemv_kernel launch";
     return kECuda;
   }
-  if (splits > 1) {
+  if (out != Y) {
     const int64_t n4 = N * D_out / 4;
     int64_t blocks = (n4 + 255) / 256;
     if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
     gemv_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(static_cast<const float4*>(ws),
-                                                                     static_cast<int>(splits), n4,
-                                                                     reinterpret_cast<float4*>(Y));
+                                                                     static_cast<int>(splits), n4, Y, y16 ? 1 : 0);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
       *cerr = e;

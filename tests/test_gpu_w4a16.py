@@ -127,6 +127,23 @@ def test_w4a16_decode_full_size(awq, N, D_in, D_out):
     assert np.all(np.abs(Y[:, cols] - Y_or) <= bound), np.max(np.abs(Y[:, cols] - Y_or) / bound)
 
 
+@pytest.mark.parametrize("N,D_in,D_out", [(1, 4096, 512), (2, 64, 128), (8, 1024, 256)])
+def test_w4a16_output_only_4_byte_aligned(awq, N, D_in, D_out):
+    """Y may be 4-byte aligned only (the ABI's requirement): the GEMV then
+    goes through the workspace and stores scalars; the values are those of an
+    aligned Y, bit for bit (the same sums in the same order)."""
+    X, W = synth.layer_inputs(synth.small_layer(max(N, 8), D_in, D_out, seed=3))
+    X = X[:N].contiguous().cuda()
+    s = torch.from_numpy(oracle.scales(oracle.act_stats(X.cpu()).astype(np.float32), 0.5)).cuda()
+    packed, sc = awq.quantize_pack(W.cuda(), s, 4, 64)
+    Y_ref = awq.w4a16_gemm(X, s, packed, sc, 4, 64)
+    buf = torch.full((N * D_out + 1,), float("nan"), device="cuda")
+    Y_off = buf[1:].view(N, D_out)                    # 4 bytes past a 256-byte-aligned allocation
+    assert Y_off.data_ptr() % 16 == 4
+    awq.w4a16_gemm(X, s, packed, sc, 4, 64, out=Y_off)
+    assert torch.equal(Y_off, Y_ref)
+
+
 def test_w4a16_rejects_unaligned_columns(awq):
     X = torch.zeros(4, 128, dtype=torch.bfloat16, device="cuda")
     s = torch.ones(128, device="cuda")
