@@ -65,6 +65,8 @@ def _load():
         lib.oracle_quantize_ex.restype = None
         lib.oracle_w4a16.argtypes = [P, P, P, P, I64, I64, I64, I, I, P]
         lib.oracle_w4a16.restype = None
+        lib.oracle_w4a16_zp.argtypes = [P, P, P, P, P, I64, I64, I64, I, P]
+        lib.oracle_w4a16_zp.restype = None
         lib.oracle_clip_loss.argtypes = [P, P, P, I64, I64, I64, P, I, I, I, P, I64, P, P]
         lib.oracle_clip_loss.restype = None
         lib.oracle_pack3.argtypes = [P, I64, I64, P]
@@ -322,5 +324,22 @@ def w4a16(X, s, packed, scales, bits: int, group: int) -> np.ndarray:
     D_out = packed.shape[1]
     Y = np.empty((N, D_out), dtype=np.float64)
     _load().oracle_w4a16(_ptr(Xb), _ptr(s), _ptr(packed), _ptr(scales), N, D_in, D_out, bits, group, _ptr(Y))
+    return Y
+
+
+def w4a16_zp(X, s, packed, scales, zeros, group: int) -> np.ndarray:
+    """Y = X diag(1/s) Dequant(W_q) in fp64 from asymmetric codes: the stored
+    u = q + z of quantize_asym, packed by pack_unsigned, minus each group's
+    zero point z, times its delta."""
+    Xb = _as_bf16_bits(X)
+    s = _f32(s)
+    packed = np.ascontiguousarray(packed).view(np.uint32)
+    scales = _f32(scales)
+    zeros = np.ascontiguousarray(zeros, dtype=np.uint8)
+    N, D_in = Xb.shape
+    D_out = packed.shape[1]
+    Y = np.empty((N, D_out), dtype=np.float64)
+    _load().oracle_w4a16_zp(_ptr(Xb), _ptr(s), _ptr(packed), _ptr(scales), _ptr(zeros), N, D_in, D_out, group,
+                            _ptr(Y))
     return Y
 

@@ -619,3 +619,36 @@ void oracle_w4a16(const uint16_t *X, const float *s, const uint32_t *packed, con
     free(wd);
 }
 
+/* The layer applied to activations from asymmetric (zero-point) codes (the
+ * stored u = q + z of the MinMax quantiser): as oracle_w4a16 with each
+ * group's zero point in place of 2^(b-1),
+ *   Y[t][n] = sum_k x_tk / s_k * (u_kn - z_{k/group, n}) * delta_{k/group, n},
+ * zeros [D_in/group][D_out] uint8.  fp64 throughout. */
+void oracle_w4a16_zp(const uint16_t *X, const float *s, const uint32_t *packed, const float *scales,
+                     const uint8_t *zeros, int64_t N, int64_t D_in, int64_t D_out, int group, double *Y)
+{
+    double *wd = (double *)malloc((size_t)(D_in * D_out) * sizeof(double));
+    for (int64_t k = 0; k < D_in; ++k)
+        for (int64_t n = 0; n < D_out; ++n) {
+            const uint32_t word = packed[(k / 8) * D_out + n];
+            const int u = (int)((word >> (4 * (k % 8))) & 0xFu);
+            const int z = (int)zeros[(k / group) * D_out + n];
+            wd[k * D_out + n] = (double)(u - z) * (double)scales[(k / group) * D_out + n] / (double)s[k];
+        }
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < N; ++t) {
+        for (int64_t n = 0; n < D_out; ++n)
+            Y[t * D_out + n] = 0.0;
+        for (int64_t k = 0; k < D_in; ++k) {
+            const double x = bf16_bits_to_double(X[t * D_in + k]);
+            if (x == 0.0)
+                continue;
+            const double *wr = wd + k * D_out;
+            double *yr = Y + t * D_out;
+            for (int64_t n = 0; n < D_out; ++n)
+                yr[n] += x * wr[n];
+        }
+    }
+    free(wd);
+}
+

@@ -553,3 +553,43 @@ def test_pack_unsigned_layout():
     u = (np.arange(16) % 16).astype(np.int16).reshape(16, 1)
     w = oracle.pack_unsigned(u)
     assert w.shape == (2, 1) and int(w[0, 0]) == 0x76543210 and int(w[1, 0]) == 0xFEDCBA98
+
+
+# ---------------------------------------------------------------- W4A16 from asymmetric (zero-point) codes
+def test_w4a16_zp_closed_form():
+    """One group of 32 rows, x = 1, s = 1, codes u_k = k mod 16, zero point 3,
+    delta 0.5: Y = 0.5 (sum_k u_k - 32 * 3) = 0.5 (2 * 120 - 96) = 72."""
+    u = (np.arange(32) % 16).reshape(32, 1)
+    packed = oracle.pack_unsigned(u)
+    X = torch.ones(1, 32).to(torch.bfloat16)
+    Y = oracle.w4a16_zp(X, np.ones(32, np.float32), packed, np.full((1, 1), 0.5, np.float32),
+                        np.full((1, 1), 3, np.uint8), 32)
+    assert Y.shape == (1, 1) and Y[0, 0] == 72.0
+
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (3, 64), (2, 32)])
+def test_w4a16_zp_with_the_middle_zero_point_is_the_symmetric_consumer(bits, group):
+    """z = 2^(b-1) in every group reduces the zero-point consumer to the
+    offset-binary one, operation for operation."""
+    X, W = synth.layer_inputs(synth.small_layer(5, 256, 24, seed=71))
+    s = oracle.scales(oracle.act_stats(X).astype(np.float32), 0.5)
+    q, d = oracle.quantize(W, s, bits, group)
+    packed = oracle.pack(q, bits)
+    z = np.full(d.shape, 1 << (bits - 1), np.uint8)
+    assert np.array_equal(oracle.w4a16_zp(X, s, packed, d, z, group), oracle.w4a16(X, s, packed, d, bits, group))
+
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (3, 64), (2, 32)])
+def test_w4a16_zp_applies_the_asymmetric_quantiser(bits, group):
+    """Packed u = q + z from the MinMax quantiser, read back through the zero
+    points: the output is X S^-1 (q delta) (numpy fp64 matmul on the
+    quantiser's own codes), so a wrong nibble, group or zero-point index fails."""
+    X, W = synth.layer_inputs(synth.small_layer(7, 256, 40, seed=72))
+    W = W + 0.01                                        # groups with non-trivial zero points
+    s = oracle.scales(oracle.act_stats(X).astype(np.float32), 0.4)
+    q, d, z = oracle.quantize_asym(W, s, bits, group)
+    assert len(np.unique(z)) > 1
+    u = q.astype(np.int16) + np.repeat(z, group, axis=0).astype(np.int16)
+    Y = oracle.w4a16_zp(X, s, oracle.pack_unsigned(u), d, z, group)
+    w_hat = q * np.repeat(d, group, axis=0).astype(np.float64) / s.astype(np.float64)[:, None]
+    assert np.allclose(Y, X.double().numpy() @ w_hat, rtol=1e-12, atol=1e-12)
