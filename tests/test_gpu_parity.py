@@ -69,6 +69,23 @@ def test_act_stats(awq, N, D):
     assert np.allclose(a_mean, ref_mean, rtol=1e-5, atol=0)
 
 
+def test_act_stats_hand_worked(awq):
+    """The worked 4 x 8 example (golden file): every mean is an exact binary
+    fraction, so the fp32 statistic equals it exactly."""
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "act_stats_hand.json")))
+    X = torch.tensor(g["X_rows"], dtype=torch.float32).to(torch.bfloat16).cuda()
+    assert awq.act_stats(X, awq.STAT_MEAN).cpu().tolist() == g["mean_abs"]
+    assert awq.act_stats(X, awq.STAT_MAX).cpu().tolist() == g["max_abs"]
+
+
+def test_weight_mean_hand_worked(awq):
+    """The worked 4 x 5 example of the balanced scale's weight statistic."""
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "weight_mean_hand.json")))
+    W = torch.tensor(g["W_rows"], dtype=torch.float32).cuda()
+    got = awq.weight_mean(W).cpu().numpy()
+    assert got.tolist() == [float(np.float32(v)) for v in g["mean_abs_rows_fp32"]]
+
+
 def test_act_stats_reproducible(awq):
     X, _ = _layer(3000, 1024, 8, seed=3)
     Xd = X.cuda()

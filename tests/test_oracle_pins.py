@@ -195,6 +195,17 @@ def test_act_stats_matches_numpy():
     assert np.array_equal(oracle.act_stats(X, oracle.STAT_MAX), np.abs(xf).max(axis=0))
 
 
+def test_act_stats_hand_worked():
+    """Worked 4 x 8 example of the statistic (golden file): mean and max run
+    down each input channel's column over the N calibration rows."""
+    g = json.load(open(os.path.join(GOLDEN, "act_stats_hand.json")))
+    X = _bf16(np.array(g["X_rows"], dtype=np.float32))
+    assert X.shape == (g["N"], g["D_in"])
+    assert X.float().numpy().tolist() == g["X_rows"]          # every entry exact in bf16
+    assert oracle.act_stats(X, oracle.STAT_MEAN).tolist() == g["mean_abs"]
+    assert oracle.act_stats(X, oracle.STAT_MAX).tolist() == g["max_abs"]
+
+
 def test_scales_special_values():
     a = np.array([0.5, 2.0, 0.0, 3.0], dtype=np.float32)
     assert (oracle.scales(a, 0.0) == 1.0).all()
@@ -424,6 +435,18 @@ def test_weight_mean_closed_form():
     W = rng.standard_normal((40, 300)).astype(np.float32)
     want = np.array([math.fsum(np.abs(W[j]).astype(np.float64)) / 300 for j in range(40)], dtype=np.float32)
     assert np.allclose(oracle.weight_mean(W), want, rtol=2e-7, atol=0)
+
+
+def test_weight_mean_hand_worked():
+    """Worked 4 x 5 example of the weight statistic (golden file): the mean
+    magnitude of input channel j's row, rounded to fp32 once."""
+    g = json.load(open(os.path.join(GOLDEN, "weight_mean_hand.json")))
+    W = np.array(g["W_rows"], dtype=np.float32)
+    assert W.shape == (g["D_in"], g["D_out"])
+    got = oracle.weight_mean(W)
+    assert got.dtype == np.float32
+    assert got.tolist() == [float(np.float32(v)) for v in g["mean_abs_rows_fp32"]]
+    assert hex(int(got[3:4].view(np.uint32)[0])) == g["fp32_bits_row_3"].lower()
 
 
 def test_balanced_scale_closed_forms():
