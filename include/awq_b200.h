@@ -410,10 +410,13 @@ AWQ_API int awq_layer_output(const void* X, const float* W, int64_t N, int64_t D
  * (32 MiB) inside the library: every GPU that loads the library holds it until
  * the process exits.  Shapes whose awq_search_workspace_size exceeds it are
  * rejected with AWQ_EWORKSPACE and a message giving both sizes; they need
- * awq_search.  Arguments, outputs and results are those of awq_search.
+ * awq_search.  Arguments, outputs and results are those of awq_search, with
+ * one difference: `status` is required (AWQ_EINVAL when NULL), because a
+ * status word inside the shared array could not be read by the caller.
  *   - The first call on a device looks up the array's device address (once
- *     per device, with that device current); make that first call before any
- *     stream capture.
+ *     per device, with that device current, and once more after the device's
+ *     context has been torn down and made anew, e.g. by cudaDeviceReset);
+ *     make that first call before any stream capture.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind; each call writes every scratch byte it reads before reading it
  *     and clears the status word it uses.  Calls that may overlap on the GPU

@@ -164,16 +164,10 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_act_stats(const uint16_t* X, int64_t N, int64_t D, int stat, float* a, int num_sms,
                              cudaStream_t st) {
-  static int attr_set_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (attr_set_device != dev) {
-    for (auto fn : {act_stats_kernel<false>, act_stats_kernel<true>}) {
-      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-      if (e != cudaSuccess) return e;
-    }
-    attr_set_device = dev;
-  }
+  static SmemAttrOnce once_mean, once_max;
+  cudaError_t e = set_smem_once(act_stats_kernel<false>, kSmemBytes, once_mean);
+  if (e == cudaSuccess) e = set_smem_once(act_stats_kernel<true>, kSmemBytes, once_max);
+  if (e != cudaSuccess) return e;
   // Slab width: D / (pairs that fit) rounded up to whole lines, at most
   // kMaxSlabChunks chunks.
   const int64_t pairs = num_sms >= 2 ? num_sms / 2 : 1;

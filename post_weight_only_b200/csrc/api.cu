@@ -52,16 +52,20 @@ int device_info(int* num_sms) {
   return AWQ_OK;
 }
 
-uint64_t timeout_ns() {
-  static uint64_t t = 0;
-  if (t == 0) {
-    uint64_t ms = 2000;
-    if (const char* env = getenv("AWQ_TIMEOUT_MS")) {
-      long long v = atoll(env);
-      if (v > 0) ms = static_cast<uint64_t>(v);
-    }
-    t = ms * 1000000ull;
+uint64_t read_timeout_ns() {
+  uint64_t ms = 2000;
+  if (const char* env = getenv("AWQ_TIMEOUT_MS")) {
+    long long v = atoll(env);
+    if (v > 0) ms = static_cast<uint64_t>(v);
   }
+  return ms * 1000000ull;
+}
+
+// The bounded-wait limit of the kernels, read from AWQ_TIMEOUT_MS once (a
+// function-local static is initialised exactly once, even with several host
+// threads).
+uint64_t timeout_ns() {
+  static const uint64_t t = read_timeout_ns();
   return t;
 }
 
@@ -282,12 +286,18 @@ int check_search_args(const void* X, const float* W, const float* a, int64_t N, 
 // ---------------------------------------------------------------- scratch without allocation
 // Scratch for awq_search_noalloc: a file-scope device array.  Host code must
 // not use its name as a device address; the address comes from
-// cudaGetSymbolAddress, once per device, with that device current.
+// cudaGetSymbolAddress, once per device (and again if that device's context
+// was torn down and made anew, which reloads the module), with that device
+// current.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[AWQ_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+struct NoallocAddr {
+  unsigned long long ctx;   // current_context_id() when the address was looked up
+  void* ptr;
+};
+NoallocAddr g_noalloc[kMaxDevices] = {};
 
 int noalloc_scratch(void** out) {
   int dev = 0;
@@ -295,17 +305,49 @@ int noalloc_scratch(void** out) {
   if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(AWQ_EUNSUPPORTED, "device %d: at most %d devices", dev, kMaxDevices);
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  const unsigned long long ctx = awq::current_context_id();
+  if (ctx == 0 || g_noalloc[dev].ctx != ctx || !g_noalloc[dev].ptr) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
     if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(no-allocation scratch)");
-    g_noalloc_ptr[dev] = ptr;
+    // the lookup made the device's context current if it was not yet
+    g_noalloc[dev] = {awq::current_context_id(), ptr};
   }
-  *out = g_noalloc_ptr[dev];
+  *out = g_noalloc[dev].ptr;
   return AWQ_OK;
 }
 
 }  // namespace
+
+namespace awq {
+
+namespace {
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename F>
+F driver_fn(const char* name) {
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult qres;
+  if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+      qres == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<F>(ptr);
+  return nullptr;
+}
+}  // namespace
+
+unsigned long long current_context_id() {
+  static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+}  // namespace awq
 
 extern "C" {
 
@@ -661,14 +703,17 @@ int awq_search_noalloc(const void* X, const float* W, const float* a, int64_t N,
                 "awq_search_noalloc: this shape needs %zu bytes of scratch, the built-in scratch holds %u; "
                 "use awq_search with a workspace",
                 lay.total, static_cast<unsigned>(AWQ_NOALLOC_SCRATCH_BYTES));
-  if (status && !aligned(status, 4)) return fail(AWQ_EALIGN, "status is not 4-byte aligned");
+  // The status word is required: inside the shared scratch array a device-side
+  // timeout could not be read by the caller and the next call would clear it.
+  if (!status) return fail(AWQ_EINVAL, "status is NULL: awq_search_noalloc needs the caller's device status word");
+  AWQ_TRY(check_ptr(status, "status", 4));
   void* scratch = nullptr;
   AWQ_TRY(noalloc_scratch(&scratch));
   uint8_t* ws = static_cast<uint8_t*>(scratch);
-  int32_t* st_word = status ? status : reinterpret_cast<int32_t*>(ws + lay.status);
+  int32_t* st_word = status;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // Every scratch byte the search reads it writes first in the same call;
-  // only the status word has to start at zero.
+  // only the status word (the caller's) has to start at zero.
   cudaError_t e = cudaMemsetAsync(st_word, 0, sizeof(int32_t), st);
   if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(status)");
   awq::AlphaList al{};

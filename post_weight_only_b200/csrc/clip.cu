@@ -431,16 +431,6 @@ cudaError_t launch_recip(const float* s, int64_t D, float* r, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <typename K>
-static cudaError_t set_smem(K kernel, int bytes, int& done_dev) {
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (done_dev == dev) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done_dev = dev;
-  return e;
-}
-
 int launch_gram(const uint16_t* XT, int64_t D_in, int64_t Np, int group, uint16_t* Hb, int* status,
                 uint64_t timeout_ns, cudaStream_t st, cudaError_t* cerr, const char** what) {
   *cerr = cudaSuccess;
@@ -450,13 +440,13 @@ int launch_gram(const uint16_t* XT, int64_t D_in, int64_t Np, int group, uint16_
     return kECuda;
   }
   const unsigned grid = static_cast<unsigned>((D_in + 127) / 128);
-  static int dev64 = -1, dev128 = -1;
+  static SmemAttrOnce dev64, dev128;
   cudaError_t e;
   if (group == 64) {
-    e = set_smem(gram_kernel<64>, kGramSmem, dev64);
+    e = set_smem_once(gram_kernel<64>, kGramSmem, dev64);
     if (e == cudaSuccess) gram_kernel<64><<<grid, 192, kGramSmem, st>>>(m, D_in, Np, Hb, status, timeout_ns);
   } else {
-    e = set_smem(gram_kernel<128>, kGramSmem, dev128);
+    e = set_smem_once(gram_kernel<128>, kGramSmem, dev128);
     if (e == cudaSuccess) gram_kernel<128><<<grid, 192, kGramSmem, st>>>(m, D_in, Np, Hb, status, timeout_ns);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
@@ -495,13 +485,13 @@ int launch_clip_loss(const uint16_t* op, const uint16_t* Hb, int64_t D_in, int64
   p.status = status;
   p.timeout_ns = timeout_ns;
   const unsigned grid = static_cast<unsigned>(p.units < num_sms ? p.units : num_sms);
-  static int dev64 = -1, dev128 = -1;
+  static SmemAttrOnce dev64, dev128;
   cudaError_t e;
   if (group == 64) {
-    e = set_smem(clip_loss_kernel<64>, LossLayout<64>::kSmem, dev64);
+    e = set_smem_once(clip_loss_kernel<64>, LossLayout<64>::kSmem, dev64);
     if (e == cudaSuccess) clip_loss_kernel<64><<<grid, kLossThreads, LossLayout<64>::kSmem, st>>>(mOp, mH, p);
   } else {
-    e = set_smem(clip_loss_kernel<128>, LossLayout<128>::kSmem, dev128);
+    e = set_smem_once(clip_loss_kernel<128>, LossLayout<128>::kSmem, dev128);
     if (e == cudaSuccess) clip_loss_kernel<128><<<grid, kLossThreads, LossLayout<128>::kSmem, st>>>(mOp, mH, p);
   }
   if (e == cudaSuccess) e = cudaGetLastError();

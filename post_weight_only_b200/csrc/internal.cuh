@@ -6,9 +6,32 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace awq {
 
 constexpr int kMaxAlpha = 64;
+
+// ---- api.cu
+// An identifier of the calling thread's current CUDA context, unique for the
+// life of the process (a context made after cudaDeviceReset gets a new one);
+// 0 when there is no current context yet or the driver cannot tell.
+unsigned long long current_context_id();
+
+// Remembers the context in which a kernel's dynamic shared-memory limit was
+// last raised, so that it is raised once per context (racing threads may both
+// raise it, which is harmless); with no known context it is raised every call.
+struct SmemAttrOnce {
+  std::atomic<unsigned long long> ctx{0};
+};
+template <typename K>
+inline cudaError_t set_smem_once(K kernel, int bytes, SmemAttrOnce& once) {
+  const unsigned long long id = current_context_id();
+  if (id != 0 && once.ctx.load(std::memory_order_acquire) == id) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && id != 0) once.ctx.store(id, std::memory_order_release);
+  return e;
+}
 
 // Quantisers: delta = max / (2^(b-1) - 1), codes +-(2^(b-1) - 1); the
 // power-of-two delta = max / 2^(b-1), codes [-2^(b-1), 2^(b-1) - 1]; or the

@@ -485,30 +485,28 @@ __global__ void wait_timeout_selftest_kernel(int* status, unsigned long long tim
 }
 
 // ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 lookup_encode_fn() {
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult qres;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+      qres == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  return nullptr;
+}
+
+// Looked up once (a function-local static is initialised exactly once, even
+// with several host threads).
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult qres;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
-        qres == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = lookup_encode_fn();
   return fn;
 }
 
 template <int kForm>
 cudaError_t launch_form(int grid, const CUtensorMap& mX, const CUtensorMap& mWt, const CUtensorMap& mOp,
                         const Params& p, cudaStream_t st) {
-  static int attr_set_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (attr_set_device != dev) {
-    cudaError_t e =
-        cudaFuncSetAttribute(search_kernel<kForm>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set_device = dev;
-  }
+  static SmemAttrOnce once;
+  const cudaError_t e = set_smem_once(search_kernel<kForm>, kSmemBytes, once);
+  if (e != cudaSuccess) return e;
   search_kernel<kForm><<<grid, kThreads, kSmemBytes, st>>>(mX, mWt, mOp, p);
   return cudaGetLastError();
 }
