@@ -134,7 +134,7 @@ def act_stats(X, stat: int = STAT_MEAN) -> np.ndarray:
 def scales(a, alpha: float, w_mean=None) -> np.ndarray:
     """s_j = a_j^alpha (floored), fp32.  compassingai.com concept page, flow
     step 3.  With w_mean: the balanced scale s_j = a_j^alpha /
-    w_mean_j^(1 - alpha) (zhihu AWQ/GPTQ/SmoothQuant comparison, "the scale
+    w_mean_j^(1 - alpha) (laojiahuo2003.github.io GPTQ/AWQ/SmoothQuant notes, section 4.4, "the scale
     per channel"), both statistics floored."""
     a = _f32(a)
     s = np.empty_like(a)

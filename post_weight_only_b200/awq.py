@@ -424,9 +424,12 @@ def check_device_status(status: torch.Tensor) -> None:
 
 
 def search_batched(layers, alpha_grid: Sequence[float], bits: int = 4, group: int = 128,
-                   want_cols: bool = False, workspace: Optional[Workspace] = None, loss_form: int = LOSS_ERROR):
+                   want_cols: bool = False, workspace: Optional[Workspace] = None, loss_form: int = LOSS_ERROR,
+                   check_status: bool = True):
     """Independent searches of several layers in one call: ``awq_search_batched``.
-    ``layers`` is a sequence of (X, W, a).  Returns one SearchResult per layer."""
+    ``layers`` is a sequence of (X, W, a).  Returns one SearchResult per layer;
+    with check_status=False nothing waits for the device (check
+    ``result.status`` after synchronising)."""
     A = len(alpha_grid)
     grid = (ctypes.c_float * A)(*[float(v) for v in alpha_grid])
     descs = (AwqLayer * len(layers))()
@@ -453,7 +456,8 @@ def search_batched(layers, alpha_grid: Sequence[float], bits: int = 4, group: in
     ws = (workspace or _default_ws).get(nbytes, dev)
     _check(_batched(descs, len(layers), grid, A, bits, group, loss_form, _ptr(ws), ws.numel(), _ptr(status),
                     _stream()))
-    check_device_status(status)
+    if check_status:
+        check_device_status(status)
     for r in results:
         r.status = status
     return results
@@ -574,3 +578,115 @@ def quantize_layer_host(X_host: torch.Tensor, W_host: torch.Tensor, alpha_grid: 
     if v != 0:
         raise AwqError(v & 0xFF, f"device status {v:#x}")
     return out
+
+
+def quantize_block(xs: Sequence[torch.Tensor], layers, alpha_grid: Sequence[float], bits: int = 4,
+                   group: int = 128, stat: int = STAT_MEAN, workspace: Optional[Workspace] = None,
+                   loss_form: int = LOSS_ERROR):
+    """Every linear of a block on the device, with no host synchronisation.
+
+    ``xs`` are the block's distinct layer inputs (bf16 [N, D_in] each);
+    ``layers`` is a sequence of (input index, W fp32 [D_in, D_out]).  The
+    statistic of each input is computed once, all layers are searched in one
+    ``awq_search_batched`` call (each layer independently: compassingai.com
+    concept page, "full scale-optimisation flow", final note), and each layer
+    gets s* = a^alpha* and its quantise + pack.  Returns one LayerResult per
+    layer; check each ``result.search.status`` after synchronising."""
+    a = [act_stats(X, stat) for X in xs]
+    res = search_batched([(xs[xi], W, a[xi]) for xi, W in layers], alpha_grid, bits, group, workspace=workspace,
+                         loss_form=loss_form, check_status=False)
+    out = []
+    for (xi, W), r in zip(layers, res):
+        s_star = scales(a[xi], r.alpha_star)
+        packed, sc = quantize_pack(W, s_star, bits, group)
+        out.append(LayerResult(a[xi], r, s_star, packed, sc))
+    return out
+
+
+class BlockHostState:
+    """Device copies of a block's inputs and pinned host result buffers, kept
+    between calls of :func:`quantize_block_host` on blocks of one shape."""
+
+    def __init__(self):
+        self.xs = None
+        self.ws = None
+        self.results = None
+        self.copy_stream = None
+        self.back_stream = None
+
+
+def quantize_block_host(xs_host: Sequence[torch.Tensor], layers_host, alpha_grid: Sequence[float], bits: int = 4,
+                        group: int = 128, stat: int = STAT_MEAN, device="cuda",
+                        workspace: Optional[Workspace] = None, state: Optional[BlockHostState] = None,
+                        loss_form: int = LOSS_ERROR):
+    """A block's linears from host buffers to host results, copies overlapped
+    with compute.
+
+    ``xs_host``: the distinct layer inputs (bf16, pinned for asynchronous
+    copies); ``layers_host``: (input index, W fp32 on the host) per layer.
+    A copy stream uploads the inputs, then each layer's W in order; the current
+    stream computes each input's statistic as soon as it has landed, and each
+    layer's search (``awq_search``), s* and pack as soon as its W has landed;
+    a third stream copies each layer's L, alpha*, status, codes and scales back
+    as soon as they are done.  Synchronises, checks every status word and
+    returns a list of dicts of host tensors (reused across calls through
+    ``state``)."""
+    dev = torch.device(device)
+    st = state if state is not None else BlockHostState()
+    compute = torch.cuda.current_stream(dev)
+    if st.copy_stream is None:
+        st.copy_stream = torch.cuda.Stream(dev)
+        st.back_stream = torch.cuda.Stream(dev)
+    if st.xs is None:
+        st.xs = [torch.empty(x.shape, dtype=x.dtype, device=dev) for x in xs_host]
+        st.ws = [torch.empty(w.shape, dtype=w.dtype, device=dev) for _, w in layers_host]
+    # the previous call's device work on these buffers has finished (it synchronised)
+    st.copy_stream.wait_stream(compute)
+    x_ready, w_ready = [], []
+    with torch.cuda.stream(st.copy_stream):
+        for xd, xh in zip(st.xs, xs_host):
+            xd.copy_(xh, non_blocking=True)
+            x_ready.append(torch.cuda.Event())
+            x_ready[-1].record(st.copy_stream)
+        for wd, (_, wh) in zip(st.ws, layers_host):
+            wd.copy_(wh, non_blocking=True)
+            w_ready.append(torch.cuda.Event())
+            w_ready[-1].record(st.copy_stream)
+    a = []
+    for k, xd in enumerate(st.xs):
+        compute.wait_event(x_ready[k])
+        a.append(act_stats(xd, stat))
+    pin = all(x.is_pinned() for x in xs_host)
+    if st.results is None:
+        st.results = []
+        for (xi, _), wd in zip(layers_host, st.ws):
+            D_in, D_out = wd.shape
+            st.results.append({
+                "L": torch.empty(len(alpha_grid), dtype=torch.float64, pin_memory=pin),
+                "alpha_star": torch.empty(1, dtype=torch.float32, pin_memory=pin),
+                "status": torch.empty(1, dtype=torch.int32, pin_memory=pin),
+                "packed": torch.empty(D_in // 8, D_out, dtype=torch.int32, pin_memory=pin),
+                "scales": torch.empty(D_in // group, D_out, dtype=torch.float32, pin_memory=pin),
+            })
+    for i, ((xi, _), wd) in enumerate(zip(layers_host, st.ws)):
+        compute.wait_event(w_ready[i])
+        r = search(st.xs[xi], wd, a[xi], alpha_grid, bits, group, workspace=workspace, check_status=False,
+                   loss_form=loss_form)
+        s_star = scales(a[xi], r.alpha_star)
+        packed, sc = quantize_pack(wd, s_star, bits, group)
+        done = torch.cuda.Event()
+        done.record(compute)
+        st.back_stream.wait_event(done)
+        host = st.results[i]
+        with torch.cuda.stream(st.back_stream):
+            for name, t in (("L", r.L), ("alpha_star", r.alpha_star), ("status", r.status), ("packed", packed),
+                            ("scales", sc)):
+                t.record_stream(st.back_stream)
+                host[name].copy_(t, non_blocking=True)
+    st.back_stream.synchronize()
+    compute.synchronize()
+    for host in st.results:
+        v = int(host["status"][0])
+        if v != 0:
+            raise AwqError(v & 0xFF, f"device status {v:#x}")
+    return st.results

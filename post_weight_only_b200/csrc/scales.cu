@@ -9,7 +9,7 @@
 // 0 all scales are 1.  The power is taken in fp64 and rounded once to fp32,
 // so alpha = 0 gives exactly 1 and alpha = 1 gives exactly a_j.
 //
-// Balanced scale (zhihu AWQ/GPTQ/SmoothQuant comparison, the per-channel
+// Balanced scale (laojiahuo2003.github.io GPTQ/AWQ/SmoothQuant notes, section 4.4, the per-channel
 // scale): with a weight statistic b_j = mean_n |W_jn|, s_j = a_j^alpha /
 // b_j^(1-alpha); b is floored the same way, and the quotient of the two fp64
 // powers is rounded once.

@@ -16,6 +16,9 @@ At these sizes the oracle cannot evaluate every output column, so
     agree (identical, or the oracle's loss at the GPU's choice within 1% of
     the oracle's minimum).
 """
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -83,6 +86,34 @@ def _check_layer_path(awq, X, W, alphas, bits, group, form, cols):
     q_or, d_or = oracle.quantize(W, s_or, bits, group)
     assert np.array_equal(r.packed.cpu().numpy().view(np.uint32), oracle.pack(q_or, bits))
     assert np.array_equal(r.scales.cpu().numpy(), d_or)
+
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.mark.parametrize("name", ["llama7b_attn_proj"])
+def test_full_layer_against_full_oracle(awq, name):
+    """Every L(alpha) of the whole layer (all output columns) and alpha*
+    against the oracle's full search, stored once by
+    tests/golden/make_full_goldens.py (oracle only): relative 1e-2 per alpha,
+    alpha* identical or within 1% of the oracle's minimum."""
+    from golden.make_full_goldens import input_digest
+    g = json.load(open(os.path.join(GOLDEN, f"full_{name}.json")))
+    wl = synth.workload(name)
+    X, W = synth.layer_inputs(wl.layers[0])
+    assert input_digest(X, W) == g["input_sha1"], "the seeded inputs differ from those of the stored oracle run"
+    alphas = synth.alpha_grid(wl.n_intervals).numpy()
+    assert [float(v) for v in alphas] == g["alphas"]
+    bits, group = wl.quant[0]
+    r = awq.quantize_layer(X.cuda(), W.cuda(), alphas.tolist(), bits, group)
+    torch.cuda.synchronize()
+    awq.check_device_status(r.search.status)
+    L_or = np.array(g["L"])
+    L_gpu = r.search.L.cpu().numpy()
+    assert np.all(np.abs(L_gpu - L_or) <= L_RTOL * L_or), np.max(np.abs(L_gpu / L_or - 1))
+    idx = int(r.search.alpha_idx.item())
+    check_alpha(L_or, g["alpha_idx"], idx)
+    assert abs(float(r.a.double().sum().item()) - g["a_sum"]) <= 1e-5 * g["a_sum"]
 
 
 def test_linear_512_n256_all_columns(awq):

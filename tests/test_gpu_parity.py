@@ -11,6 +11,9 @@ Acceptance, per the contract of the search:
 Sizes span several tiles (128 output columns x 256 tokens x 64 k) and ragged
 tails in every dimension.
 """
+import json
+import os
+
 import numpy as np
 import pytest
 import torch

@@ -7,7 +7,7 @@ against the CPU oracle, through the C ABI.
     kernels, alone and with clip ratios and FP16 deltas; the search's losses
     within the arithmetic's bound and relative 1e-2, alpha* by the contract's
     rule;
-  * the balanced scale (zhihu AWQ/GPTQ/SmoothQuant comparison, the
+  * the balanced scale (laojiahuo2003.github.io GPTQ/AWQ/SmoothQuant notes, section 4.4, the
     per-channel scale s_j = mean|X_j|^alpha / mean|W_j|^(1-alpha)): the weight
     statistic within relative 1e-6 (fp64 sums in another order), the scales
     within one fp32 ulp (fp64 powers from two math libraries), the search as

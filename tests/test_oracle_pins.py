@@ -428,7 +428,7 @@ def test_pow2_quantiser_search_differs_from_symmetric():
 
 
 # ---------------------------------------------------------------- balanced scale
-# (zhihu AWQ/GPTQ/SmoothQuant comparison: s_j = mean|X_j|^alpha / mean|W_j|^(1-alpha))
+# (laojiahuo2003.github.io GPTQ/AWQ/SmoothQuant notes, section 4.4: s_j = mean|X_j|^alpha / mean|W_j|^(1-alpha))
 
 def test_weight_mean_closed_form():
     rng = np.random.default_rng(8)
