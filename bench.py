@@ -392,7 +392,7 @@ class DeviceJob:
         """statistic of every input -> search of every linear -> s* -> pack.
         No host synchronisation; returns the per-search results."""
         awq, job = self.awq, self.job
-        a = [awq.act_stats(x) for x in self.xs]
+        a = awq.act_stats_batched(self.xs) if len(self.xs) > 1 else [awq.act_stats(self.xs[0])]
         out = [None] * len(job.searches)
         for (bits, group), idx in self.groups.items():
             if len(idx) == 1:
@@ -514,7 +514,7 @@ def measure_job(job: Job, dev, steps: int, warmup: int, flush, flush_sink, form,
         "eff_tflops": job.flops() / (ms / 1e3) / 1e12,
         "pct_bf16_peak_step": job.flops() / (ms / 1e3) / 1e12 / float(peaks["bf16_tflops"]),
         "roofline": roofline_of(job, prof, steps, total),
-        "hbm_kernels": {"act_stats": hbm_in_step(prof, "act_stats", stats_bytes(job), steps),
+        "hbm_kernels": {"act_stats": hbm_in_step(prof, "act_stats", stats_bytes(job), steps),   # one launch per step
                         "quantize_pack": hbm_in_step(prof, "quantize_pack", pack_bytes(job), steps),
                         "search_operand": hbm_in_step(prof, "search_operand", operand_bytes(job), steps)},
         "kernels": {name: {"total_ms": t, "launches": n} for name, (t, n) in prof.items() if n},

@@ -93,6 +93,21 @@ enum { AWQ_LOSS_ERROR = 0, AWQ_LOSS_REFERENCE = 1 };
 AWQ_API int awq_act_stats(const void* X, int64_t N, int64_t D_in, int stat, float* a, void* stream);
 
 /*
+ * The statistic of several inputs in one launch (the distinct inputs of a
+ * transformer block: the q/k/v input, the o input, the gate/up input, the down
+ * input), each as awq_act_stats defines it (max exact; the mean's fixed fp32
+ * summation order can differ from that of a single-input call, within its
+ * rounding).  The launch's CTA pairs are shared out over the inputs in
+ * proportion to their bytes, so one wave streams them all.
+ *   Xs, Ns, D_ins, as  host arrays of n_inputs entries: device pointers X
+ *                      [N][D_in] bf16 and a [D_in] fp32 (each 16-byte aligned)
+ *   n_inputs           1 .. 16 (AWQ_EUNSUPPORTED beyond)
+ * Errors as awq_act_stats, with the failing input's index in the message.
+ */
+AWQ_API int awq_act_stats_batched(const void* const* Xs, const int64_t* Ns, const int64_t* D_ins, int n_inputs,
+                                  int stat, float* const* as, void* stream);
+
+/*
  * Scale vector for one alpha (compassingai.com concept page, flow step 3:
  * s_j = activation_scale[j]^alpha; step 6: s* = activation_scale^alpha*).
  *   s_j = (float) pow((double) max(a_j, 1e-6f * max_i a_i), (double) alpha)
@@ -165,7 +180,7 @@ AWQ_API int awq_search(const void* X, const float* W, const float* a, int64_t N,
                        int32_t* status, void* stream);
 
 /*
- * Quantiser and scale variants of the search (NEXT f2):
+ * Quantiser and scale variants of the search:
  *   quantizer  AWQ_QUANT_SYMMETRIC: delta = max|w'| / (2^(b-1)-1), codes in
  *              +-(2^(b-1)-1) (as awq_search);
  *              AWQ_QUANT_DELTA_POW2 (mudrobot.github.io notes, "analysing the
@@ -183,11 +198,17 @@ AWQ_API int awq_search(const void* X, const float* W, const float* a, int64_t N,
  *              scales are the balanced a^alpha / w_mean^(1-alpha); recover s*
  *              with awq_scales_ex.
  *   gram_form  nonzero: evaluate L(alpha) = sum_n e_n^T H e_n with H = X^T X
- *              (the Gram form of the loss, NEXT f4): H is formed once
+ *              (the Gram form of the loss): H is formed once
  *              (tensor cores, fp32, rounded to bf16), then each alpha costs
  *              2 D_in^2 D_out flops instead of 2 N D_in D_out, which is cheaper
  *              when N > D_in.  Error form only.  The workspace is
  *              awq_search_ex_workspace_size(...).
+ *   ldw        0, or the row stride of W in elements (ldw >= D_out, a multiple
+ *              of 4): row k of W starts at W + k ldw.  It lets a caller search
+ *              a slice of output columns of a wider matrix in place (W pointing
+ *              at the slice's first column), as the column-sharded multi-GPU
+ *              search does; the loss is a sum over output columns (concept
+ *              page, flow step 4c), so the slices' losses add up to the layer's.
  */
 #define AWQ_QUANT_SYMMETRIC 0
 #define AWQ_QUANT_DELTA_POW2 1
@@ -196,6 +217,7 @@ typedef struct {
   int quantizer;
   const float* w_mean;
   int gram_form;
+  int64_t ldw;
 } awq_search_options;
 
 /* Bytes of workspace awq_search_ex needs with these options (0 if invalid). */
@@ -352,7 +374,7 @@ AWQ_API int awq_quantize_pack_ex(const float* W, const float* s, const float* cl
  *   zeros   [D_in/group][D_out] uint8 output: z (device).
  * No clip ratio (the clipping search is symmetric).  An all-zero group has
  * delta = 0, z = 0 and codes 0.  Errors as awq_quantize_pack_ex.
- * awq_w4a16_gemm reads symmetric codes only.
+ * awq_w4a16_gemm_zp applies these codes to activations (fp32 deltas only).
  */
 AWQ_API int awq_quantize_pack_zp(const float* W, const float* s, int64_t D_in, int64_t D_out, int bits, int group,
                                  int flags, uint32_t* packed, void* scales, uint8_t* zeros, void* stream);
@@ -388,6 +410,27 @@ AWQ_API size_t awq_w4a16_workspace_size(int64_t N, int64_t D_in, int64_t D_out);
 AWQ_API int awq_w4a16_gemm(const void* X, const float* s, const uint32_t* packed, const float* scales, int64_t N,
                            int64_t D_in, int64_t D_out, int bits, int group, float* Y, void* workspace,
                            size_t workspace_bytes, int32_t* status, void* stream);
+
+/*
+ * awq_w4a16_gemm for asymmetric codes (the output of awq_quantize_pack_zp:
+ * compassingai.com AWQ concept page, "the AWQ mechanism", symmetric or
+ * asymmetric quantisation; "inference-time equivalent" for the product):
+ *     Y[t][n] = sum_k x_tk / s_k * (u_kn - z[k/group][n]) * scales[k/group][n]
+ * with the same two paths and roundings: the GEMV subtracts each group's zero
+ * point exactly in fp32; the tensor-core path forms bf16((u - z) * bf16(delta))
+ * (u - z is exact) from a per-(group, column) fp32 copy of 128 + z that a
+ * first small kernel writes into the workspace.
+ *   zeros     [D_in/group][D_out] uint8 zero points (device), 16-byte aligned
+ *   scales    fp32 deltas (pack without AWQ_PACK_DELTA_FP16)
+ *   workspace at least awq_w4a16_zp_workspace_size(N, D_in, D_out, group)
+ *             bytes (that of awq_w4a16_gemm plus, for N > 4, 4 bytes per
+ *             group and column)
+ * Other arguments and errors as awq_w4a16_gemm; zeros NULL is AWQ_EINVAL.
+ */
+AWQ_API size_t awq_w4a16_zp_workspace_size(int64_t N, int64_t D_in, int64_t D_out, int group);
+AWQ_API int awq_w4a16_gemm_zp(const void* X, const float* s, const uint32_t* packed, const float* scales,
+                              const uint8_t* zeros, int64_t N, int64_t D_in, int64_t D_out, int bits, int group,
+                              float* Y, void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
 
 /*
  * The layer's reference output Y = X bf16(W) computed by the search's own

@@ -329,7 +329,7 @@ void oracle_pack(const int8_t *q, int64_t D_in, int64_t D_out, int bits, uint32_
     }
 }
 
-/* Dense 3-bit packing (NEXT f2): the 32 codes of rows 32j .. 32j+31 of column
+/* Dense 3-bit packing (an option of the pack): the 32 codes of rows 32j .. 32j+31 of column
  * n as one 96-bit little-endian string, code i (u = q + 4) at bits 3i .. 3i+2,
  * stored as words (3j, n), (3j+1, n), (3j+2, n) holding bits 0-31, 32-63 and
  * 64-95.  Codes 10 and 21 straddle two words.  D_in % 32 == 0. */

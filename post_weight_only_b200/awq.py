@@ -31,7 +31,7 @@ EXPORTS = (
     "awq_search_noalloc", "awq_clip_search_workspace_size", "awq_clip_search", "awq_quantize_pack_clip",
     "awq_search_joint_workspace_size", "awq_search_joint", "awq_quantize_pack_ex", "awq_w4a16_gemm",
     "awq_w4a16_workspace_size", "awq_search_ex", "awq_weight_mean", "awq_scales_ex", "awq_search_ex_workspace_size",
-    "awq_quantize_pack_zp",
+    "awq_quantize_pack_zp", "awq_w4a16_gemm_zp", "awq_w4a16_zp_workspace_size", "awq_act_stats_batched",
 )
 STAGES = ("act_stats", "scale_table", "search_operand", "search_gemm", "loss_reduce", "quantize_pack",
           "weight_t", "clip_gram", "clip_operand", "clip_loss", "w4a16")
@@ -72,7 +72,7 @@ _search = _sig("awq_search", I, [P, P, P, I64, I64, I64, P, I, I, I, I, P, P, P,
 
 
 class AwqSearchOptions(ctypes.Structure):
-    _fields_ = [("quantizer", ctypes.c_int), ("w_mean", P), ("gram_form", ctypes.c_int)]
+    _fields_ = [("quantizer", ctypes.c_int), ("w_mean", P), ("gram_form", ctypes.c_int), ("ldw", I64)]
 
 
 QUANT_SYMMETRIC = 0
@@ -104,6 +104,9 @@ _pack_zp = _sig("awq_quantize_pack_zp", I, [P, P, I64, I64, I, I, I, P, P, P, P]
 PACK_DELTA_FP16 = 1
 _w4a16 = _sig("awq_w4a16_gemm", I, [P, P, P, P, I64, I64, I64, I, I, P, P, SZ, P, P])
 _w4a16_ws = _sig("awq_w4a16_workspace_size", SZ, [I64, I64, I64])
+_w4a16_zp = _sig("awq_w4a16_gemm_zp", I, [P, P, P, P, P, I64, I64, I64, I, I, P, P, SZ, P, P])
+_stats_batched = _sig("awq_act_stats_batched", I, [P, P, P, I, I, P, P])
+_w4a16_zp_ws = _sig("awq_w4a16_zp_workspace_size", SZ, [I64, I64, I64, I])
 _joint = _sig("awq_search_joint", I, [P, P, P, I, P, I64, I64, P, I, I, I, I, P, P, P, P, P, SZ, P, P])
 
 
@@ -145,6 +148,20 @@ def act_stats(X: torch.Tensor, stat: int = STAT_MEAN) -> torch.Tensor:
     a = torch.empty(D, dtype=torch.float32, device=X.device)
     _check(_act_stats(_ptr(X), N, D, stat, _ptr(a), _stream()))
     return a
+
+
+def act_stats_batched(Xs: Sequence[torch.Tensor], stat: int = STAT_MEAN) -> list:
+    """The statistic of several inputs in one launch: ``awq_act_stats_batched``.
+    Returns one fp32 [D_in] tensor per input."""
+    Xs = [_dev(X, torch.bfloat16, "X") for X in Xs]
+    outs = [torch.empty(X.shape[1], dtype=torch.float32, device=X.device) for X in Xs]
+    n = len(Xs)
+    xp = (ctypes.c_void_p * n)(*[X.data_ptr() for X in Xs])
+    ns = (ctypes.c_int64 * n)(*[X.shape[0] for X in Xs])
+    ds = (ctypes.c_int64 * n)(*[X.shape[1] for X in Xs])
+    ap = (ctypes.c_void_p * n)(*[a.data_ptr() for a in outs])
+    _check(_stats_batched(xp, ns, ds, n, stat, ap, _stream()))
+    return outs
 
 
 def weight_mean(W: torch.Tensor) -> torch.Tensor:
@@ -216,10 +233,17 @@ def search(X: torch.Tensor, W: torch.Tensor, a: torch.Tensor, alpha_grid: Sequen
            check_status: bool = True, loss_form: int = LOSS_ERROR, quantizer: int = QUANT_SYMMETRIC,
            w_mean: Optional[torch.Tensor] = None, gram: bool = False) -> SearchResult:
     """Grid search over alpha for one layer: ``awq_search``, or
-    ``awq_search_ex`` with a quantiser variant, the balanced scale or the
-    Gram form of the loss."""
+    ``awq_search_ex`` with a quantiser variant, the balanced scale, the Gram
+    form of the loss, or a W whose rows are further apart than D_out (a slice
+    of output columns of a wider matrix, e.g. ``W[:, c0:c1]``, searched in
+    place through the row stride ``ldw``)."""
     X = _dev(X, torch.bfloat16, "X")
-    W = _dev(W, torch.float32, "W")
+    ldw = 0
+    if (W.is_cuda and W.dtype == torch.float32 and W.dim() == 2 and W.stride(1) == 1
+            and W.stride(0) > W.shape[1] and W.stride(0) % 4 == 0 and W.data_ptr() % 16 == 0):
+        ldw = W.stride(0)           # a column slice: passed in place
+    else:
+        W = _dev(W, torch.float32, "W")
     a = _dev(a, torch.float32, "a")
     N, D_in = X.shape
     D_out = W.shape[1]
@@ -231,9 +255,9 @@ def search(X: torch.Tensor, W: torch.Tensor, a: torch.Tensor, alpha_grid: Sequen
     astar = torch.empty(1, dtype=torch.float32, device=dev)
     aidx = torch.empty(1, dtype=torch.int32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    plain = quantizer == QUANT_SYMMETRIC and w_mean is None and not gram
+    plain = quantizer == QUANT_SYMMETRIC and w_mean is None and not gram and ldw == 0
     b = None if w_mean is None else _dev(w_mean, torch.float32, "w_mean")
-    opts = AwqSearchOptions(int(quantizer), _ptr(b), 1 if gram else 0)
+    opts = AwqSearchOptions(int(quantizer), _ptr(b), 1 if gram else 0, ldw)
     nbytes = (search_workspace_size(N, D_in, D_out, A, bits, group, loss_form) if plain
               else int(_search_ex_ws(N, D_in, D_out, A, bits, group, loss_form, ctypes.byref(opts))))
     if nbytes == 0:
@@ -328,11 +352,14 @@ def quantize_pack_zp(W: torch.Tensor, s: torch.Tensor, bits: int = 4, group: int
 
 def w4a16_gemm(X: torch.Tensor, s: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, bits: int = 4,
                group: int = 128, check_status: bool = True,
-               workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Y = X diag(1/s) Dequant(packed, scales), fp32: ``awq_w4a16_gemm``.
-    ``workspace`` (uint8, at least ``w4a16_workspace_size(N, D_in, D_out)`` bytes)
-    is allocated per call when not given; ``out`` (contiguous fp32 [N, D_out]
-    on the same device) receives Y when given."""
+               workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+               zeros: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y = X diag(1/s) Dequant(packed, scales), fp32: ``awq_w4a16_gemm``, or
+    with ``zeros`` (uint8 [D_in/group, D_out], from ``quantize_pack_zp``) the
+    asymmetric codes' ``awq_w4a16_gemm_zp``.  ``workspace`` (uint8, at least
+    ``w4a16_workspace_size(N, D_in, D_out[, group, zp=True])`` bytes) is
+    allocated per call when not given; ``out`` (contiguous fp32 [N, D_out] on
+    the same device) receives Y when given."""
     X = _dev(X, torch.bfloat16, "X")
     s = _dev(s, torch.float32, "s")
     if packed.dtype not in (torch.int32, torch.uint32):
@@ -349,18 +376,27 @@ def w4a16_gemm(X: torch.Tensor, s: torch.Tensor, packed: torch.Tensor, scales: t
             raise ValueError("out must be a contiguous float32 [N, D_out] tensor on X's device")
         Y = out
     status = torch.zeros(1, dtype=torch.int32, device=X.device)
-    nbytes = _w4a16_ws(N, D_in, D_out)
+    nbytes = w4a16_workspace_size(N, D_in, D_out, group, zp=zeros is not None)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=X.device)
-    _check(_w4a16(_ptr(X), _ptr(s), _ptr(packed), _ptr(scales), N, D_in, D_out, bits, group, _ptr(Y),
-                  _ptr(workspace), workspace.numel(), _ptr(status), _stream()))
+    if zeros is None:
+        _check(_w4a16(_ptr(X), _ptr(s), _ptr(packed), _ptr(scales), N, D_in, D_out, bits, group, _ptr(Y),
+                      _ptr(workspace), workspace.numel(), _ptr(status), _stream()))
+    else:
+        zeros = _dev(zeros, torch.uint8, "zeros")
+        _check(_w4a16_zp(_ptr(X), _ptr(s), _ptr(packed), _ptr(scales), _ptr(zeros), N, D_in, D_out, bits, group,
+                         _ptr(Y), _ptr(workspace), workspace.numel(), _ptr(status), _stream()))
     if check_status:
         check_device_status(status)
     return Y
 
 
-def w4a16_workspace_size(N: int, D_in: int, D_out: int) -> int:
-    return int(_w4a16_ws(N, D_in, D_out))
+def w4a16_workspace_size(N: int, D_in: int, D_out: int, group: int = 128, zp: bool = False) -> int:
+    """Workspace bytes of ``w4a16_gemm``; zp: for asymmetric codes (zeros given)."""
+    n = int(_w4a16_zp_ws(N, D_in, D_out, group) if zp else _w4a16_ws(N, D_in, D_out))
+    if n == 0:
+        raise AwqError(AWQ_EINVAL, "w4a16 workspace size: invalid arguments")
+    return n
 
 
 def quantize_pack_clip(W: torch.Tensor, s: torch.Tensor, clip: torch.Tensor, bits: int = 4, group: int = 128):
@@ -590,9 +626,10 @@ def quantize_block(xs: Sequence[torch.Tensor], layers, alpha_grid: Sequence[floa
     statistic of each input is computed once, all layers are searched in one
     ``awq_search_batched`` call (each layer independently: compassingai.com
     concept page, "full scale-optimisation flow", final note), and each layer
-    gets s* = a^alpha* and its quantise + pack.  Returns one LayerResult per
+    gets s* = a^alpha* and its quantise + pack (the statistics of all inputs in
+    one ``awq_act_stats_batched`` launch).  Returns one LayerResult per
     layer; check each ``result.search.status`` after synchronising."""
-    a = [act_stats(X, stat) for X in xs]
+    a = act_stats_batched(xs, stat)
     res = search_batched([(xs[xi], W, a[xi]) for xi, W in layers], alpha_grid, bits, group, workspace=workspace,
                          loss_form=loss_form, check_status=False)
     out = []

@@ -56,10 +56,28 @@ __device__ __forceinline__ void fold8(float (&acc)[8], const uint4& v) {
   for (int e = 0; e < 8; ++e) acc[e] = kMax ? fmaxf(acc[e], x[e]) : acc[e] + x[e];
 }
 
-// Cluster blockIdx.x / kCluster owns channels [slab * W, min(D, (slab + 1) * W)).
+// The inputs of one launch: input i is X [N][D] bf16 with output a [D], cut
+// into slabs of slab_ch channels that are clusters first_slab[i] ..
+// first_slab[i + 1] - 1 of the grid.
+struct StatsInputs {
+  const uint16_t* X[kMaxStatsInputs];
+  float* a[kMaxStatsInputs];
+  int64_t N[kMaxStatsInputs], D[kMaxStatsInputs], slab_ch[kMaxStatsInputs];
+  int first_slab[kMaxStatsInputs + 1];
+  int n;
+};
+
+// Cluster blockIdx.x / kCluster owns channels [slab * W, min(D, (slab + 1) * W))
+// of the input whose slab range holds it.
 template <bool kMax>
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
-    act_stats_kernel(const uint16_t* __restrict__ X, int64_t N, int64_t D, int64_t slab_ch, float* __restrict__ a) {
+    act_stats_kernel(const StatsInputs in) {
+  const int slab_id = static_cast<int>(blockIdx.x / kCluster);
+  int which = 0;
+  while (which + 1 < in.n && slab_id >= in.first_slab[which + 1]) ++which;
+  const uint16_t* __restrict__ X = in.X[which];
+  float* __restrict__ a = in.a[which];
+  const int64_t N = in.N[which], D = in.D[which], slab_ch = in.slab_ch[which];
   extern __shared__ __align__(16) uint8_t smem[];
   uint4* ring = reinterpret_cast<uint4*>(smem);
   float* fold = reinterpret_cast<float*>(smem);                 // reuses the ring after the stream
@@ -67,7 +85,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
   const int t = threadIdx.x;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x / kCluster) * slab_ch;     // first channel of the slab
+  const int64_t c0 = static_cast<int64_t>(slab_id - in.first_slab[which]) * slab_ch;   // first channel of the slab
   const int64_t c1 = c0 + slab_ch < D ? c0 + slab_ch : D;
   const int nck = static_cast<int>((c1 - c0) / 8);              // chunks, >= 1
   const int RL = nck < kThreads ? kThreads / nck : 1;           // row lanes
@@ -87,27 +105,35 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
       const int64_t first = r0 + rl;
       const int nr = first < r1 ? static_cast<int>((r1 - first + RL - 1) / RL) : 0;   // rows of this lane
       const int nst = (nr + kRowsPerStage - 1) / kRowsPerStage;
-      const uint4* src = reinterpret_cast<const uint4*>(X) + c0 / 8 + ck + first * stride;
+      // The next row to copy, advanced by a pointer step (no per-row products);
+      // row i lands in ring slot i % kDepth, so stage g's slots are
+      // (g % kStages) * kRowsPerStage + q with q a compile-time offset.
+      const uint4* next = reinterpret_cast<const uint4*>(X) + c0 / 8 + ck + first * stride;
       const int64_t step = static_cast<int64_t>(RL) * stride;
-      auto issue = [&](int g) {
+      uint4* const mine = ring + t;
+      // One pass covers the prologue, the steady state and the drain: pass g
+      // issues stage g (if any) and folds stage g - (kStages - 1) (if any).
+      for (int g = 0; g < nst + kStages - 1; ++g) {
         if (g < nst) {
+          uint4* slots = mine + (g % kStages) * kRowsPerStage * kThreads;
+          const int left = nr - g * kRowsPerStage;
 #pragma unroll
           for (int q = 0; q < kRowsPerStage; ++q) {
-            const int i = g * kRowsPerStage + q;
-            if (i < nr) cp_async16(ring + (i & (kDepth - 1)) * kThreads + t, src + i * step, 16u);
+            if (q < left) {
+              cp_async16(slots + q * kThreads, next, 16u);
+              next += step;
+            }
           }
         }
         cp_async_commit();
-      };
+        const int f = g - (kStages - 1);
+        if (f >= 0) {
+          cp_async_wait<kStages - 1>();    // this thread's rows of stage f have landed
+          const uint4* slots = mine + (f % kStages) * kRowsPerStage * kThreads;
+          const int left = nr - f * kRowsPerStage;
 #pragma unroll
-      for (int g = 0; g < kStages - 1; ++g) issue(g);
-      for (int g = 0; g < nst; ++g) {
-        issue(g + kStages - 1);
-        cp_async_wait<kStages - 1>();      // this thread's rows of stage g have landed
-#pragma unroll
-        for (int q = 0; q < kRowsPerStage; ++q) {
-          const int i = g * kRowsPerStage + q;
-          if (i < nr) fold8<kMax>(acc, ring[(i & (kDepth - 1)) * kThreads + t]);
+          for (int q = 0; q < kRowsPerStage; ++q)
+            if (q < left) fold8<kMax>(acc, slots[q * kThreads]);
         }
       }
       cp_async_wait<0>();
@@ -134,8 +160,10 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
       const int nch = nck * 8;
       const int P = nch < kThreads ? kThreads / nch : 1;
       float* parts = fold + kThreads * 8;                     // after the row-lane sums
-      if (t < P * nch) {
-        const int c = t % nch, pp = t / nch;
+      // (a slab can hold more channels than the CTA has threads: then P = 1
+      // and each thread takes channels t, t + kThreads, ...)
+      for (int idx = t; idx < P * nch; idx += kThreads) {
+        const int c = idx % nch, pp = idx / nch;
         float sum = fold[pp * nch + c];
         for (int l = pp + P; l < RL; l += P) sum = kMax ? fmaxf(sum, fold[l * nch + c]) : sum + fold[l * nch + c];
         parts[pp * nch + c] = sum;
@@ -162,25 +190,49 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_act_stats(const uint16_t* X, int64_t N, int64_t D, int stat, float* a, int num_sms,
-                             cudaStream_t st) {
+cudaError_t launch_act_stats_batched(const uint16_t* const* X, const int64_t* N, const int64_t* D, int n, int stat,
+                                     float* const* a, int num_sms, cudaStream_t st) {
+  if (n < 1 || n > kMaxStatsInputs) return cudaErrorInvalidValue;
   static SmemAttrOnce once_mean, once_max;
   cudaError_t e = set_smem_once(act_stats_kernel<false>, kSmemBytes, once_mean);
   if (e == cudaSuccess) e = set_smem_once(act_stats_kernel<true>, kSmemBytes, once_max);
   if (e != cudaSuccess) return e;
-  // Slab width: D / (pairs that fit) rounded up to whole lines, at most
-  // kMaxSlabChunks chunks.
+  // The pairs that fit in one wave are shared out in proportion to the
+  // inputs' bytes (at least one each); an input's slab width is its D over
+  // its pairs, rounded up to whole lines, at most kMaxSlabChunks chunks.
   const int64_t pairs = num_sms >= 2 ? num_sms / 2 : 1;
-  int64_t slab = (D + pairs - 1) / pairs;
-  slab = (slab + kSlabAlign - 1) / kSlabAlign * kSlabAlign;
-  if (slab > static_cast<int64_t>(kMaxSlabChunks) * 8) slab = static_cast<int64_t>(kMaxSlabChunks) * 8;
-  const int64_t slabs = (D + slab - 1) / slab;
-  const dim3 grid(static_cast<unsigned>(slabs * kCluster));
+  double total = 0.0;
+  for (int i = 0; i < n; ++i) total += static_cast<double>(N[i]) * static_cast<double>(D[i]);
+  StatsInputs in{};
+  in.n = n;
+  int slabs_all = 0;
+  for (int i = 0; i < n; ++i) {
+    int64_t p = static_cast<int64_t>(static_cast<double>(pairs) * static_cast<double>(N[i]) *
+                                     static_cast<double>(D[i]) / total);
+    if (p < 1) p = 1;
+    int64_t slab = (D[i] + p - 1) / p;
+    slab = (slab + kSlabAlign - 1) / kSlabAlign * kSlabAlign;
+    if (slab > static_cast<int64_t>(kMaxSlabChunks) * 8) slab = static_cast<int64_t>(kMaxSlabChunks) * 8;
+    in.X[i] = X[i];
+    in.a[i] = a[i];
+    in.N[i] = N[i];
+    in.D[i] = D[i];
+    in.slab_ch[i] = slab;
+    in.first_slab[i] = slabs_all;
+    slabs_all += static_cast<int>((D[i] + slab - 1) / slab);
+  }
+  in.first_slab[n] = slabs_all;
+  const dim3 grid(static_cast<unsigned>(slabs_all * kCluster));
   if (stat == 1)
-    act_stats_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(X, N, D, slab, a);
+    act_stats_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(in);
   else
-    act_stats_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(X, N, D, slab, a);
+    act_stats_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(in);
   return cudaGetLastError();
+}
+
+cudaError_t launch_act_stats(const uint16_t* X, int64_t N, int64_t D, int stat, float* a, int num_sms,
+                             cudaStream_t st) {
+  return launch_act_stats_batched(&X, &N, &D, 1, stat, &a, num_sms, st);
 }
 
 }  // namespace awq

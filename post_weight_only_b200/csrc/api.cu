@@ -186,6 +186,7 @@ struct SearchOpts {
   int qmode = awq::kQuantSymmetric;
   const float* w_mean = nullptr;    // balanced scale a^alpha / w_mean^(1 - alpha) when set
   bool gram = false;                // L = sum_n e_n^T (X^T X) e_n (error form only)
+  int64_t ldw = 0;                  // row stride of W in elements (0: D_out)
 };
 
 // Workspace of the Gram form: X^T (tokens padded to 8), H = X^T X in fp32 and
@@ -221,6 +222,7 @@ int search_one(const void* X, const float* W, const float* a, int64_t N, int64_t
                float* alpha_star, int32_t* alpha_idx, uint8_t* ws, int32_t* status, cudaStream_t st,
                int num_sms, const SearchOpts& opts = SearchOpts()) {
   const SearchLayout lay = search_layout(N, D_in, D_out, A, group, form, num_sms);
+  const int64_t ldw = opts.ldw > 0 ? opts.ldw : D_out;
   float* s_tab = reinterpret_cast<float*>(ws + lay.s_tab);
   float* r_tab = reinterpret_cast<float*>(ws + lay.r_tab);
   uint16_t* op = reinterpret_cast<uint16_t*>(ws + lay.op);
@@ -238,12 +240,12 @@ int search_one(const void* X, const float* W, const float* a, int64_t N, int64_t
   {
     StageTimer t(AWQ_STAGE_SEARCH_OPERAND, st);
     const int op_form = form == awq::kFormGram ? awq::kFormError : form;   // the Gram form reads E = S^-1 Q(SW) - W
-    e = awq::launch_search_operand(W, s_tab, r_tab, D_in, D_out, A, bits, group, op_form, opts.qmode, op, st);
+    e = awq::launch_search_operand(W, ldw, s_tab, r_tab, D_in, D_out, A, bits, group, op_form, opts.qmode, op, st);
   }
   if (e != cudaSuccess) return fail_cuda(e, "search operand kernel");
   if (wt) {
     StageTimer t(AWQ_STAGE_WEIGHT_T, st);
-    e = awq::launch_weight_t(W, D_in, D_out, wt, st);
+    e = awq::launch_weight_t(W, ldw, D_in, D_out, wt, st);
   }
   if (e != cudaSuccess) return fail_cuda(e, "weight transpose kernel");
   awq::SearchShape sh{static_cast<int>(N), static_cast<int>(D_in), static_cast<int>(D_out), A, bits, group, form};
@@ -367,6 +369,31 @@ int awq_act_stats(const void* X, int64_t N, int64_t D_in, int stat, float* a, vo
   {
     StageTimer t(AWQ_STAGE_ACT_STATS, static_cast<cudaStream_t>(stream));
     e = awq::launch_act_stats(static_cast<const uint16_t*>(X), N, D_in, stat, a, sms, static_cast<cudaStream_t>(stream));
+  }
+  return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "act_stats kernel");
+}
+
+int awq_act_stats_batched(const void* const* Xs, const int64_t* Ns, const int64_t* D_ins, int n_inputs, int stat,
+                          float* const* as, void* stream) {
+  if (!Xs || !Ns || !D_ins || !as) return fail(AWQ_EINVAL, "Xs, Ns, D_ins and as must not be NULL");
+  if (n_inputs < 1 || n_inputs > awq::kMaxStatsInputs)
+    return fail(AWQ_EUNSUPPORTED, "n_inputs = %d: need 1..%d", n_inputs, awq::kMaxStatsInputs);
+  if (stat != AWQ_STAT_MEAN && stat != AWQ_STAT_MAX) return fail(AWQ_EINVAL, "stat = %d: use AWQ_STAT_MEAN or AWQ_STAT_MAX", stat);
+  for (int i = 0; i < n_inputs; ++i) {
+    if (Ns[i] < 1 || Ns[i] > kMaxDim) return fail(AWQ_EINVAL, "input %d: N = %lld: need 1 <= N <= 2^24", i, (long long)Ns[i]);
+    if (D_ins[i] < 8 || D_ins[i] > kMaxDin || D_ins[i] % 8)
+      return fail(AWQ_EINVAL, "input %d: D_in = %lld: need a multiple of 8 in [8, 2^20]", i, (long long)D_ins[i]);
+    int rc = check_ptr(Xs[i], "X", 16);
+    if (rc == AWQ_OK) rc = check_ptr(as[i], "a", 16);
+    if (rc != AWQ_OK) return fail(rc, "input %d: %s", i, g_last_error.c_str());
+  }
+  int sms = 0;
+  AWQ_TRY(device_info(&sms));
+  cudaError_t e;
+  {
+    StageTimer t(AWQ_STAGE_ACT_STATS, static_cast<cudaStream_t>(stream));
+    e = awq::launch_act_stats_batched(reinterpret_cast<const uint16_t* const*>(Xs), Ns, D_ins, n_inputs, stat, as,
+                                      sms, static_cast<cudaStream_t>(stream));
   }
   return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "act_stats kernel");
 }
@@ -515,6 +542,10 @@ int awq_search_ex(const void* X, const float* W, const float* a, int64_t N, int6
     if (options->w_mean) AWQ_TRY(check_ptr(options->w_mean, "w_mean", 4));
     o.w_mean = options->w_mean;
     o.gram = options->gram_form != 0;
+    if (options->ldw != 0 && (options->ldw < D_out || options->ldw % 4 || options->ldw > kMaxDim))
+      return fail(AWQ_EINVAL, "ldw = %lld: need 0, or a multiple of 4 with D_out = %lld <= ldw <= 2^24",
+                  (long long)options->ldw, (long long)D_out);
+    o.ldw = options->ldw;
   }
   return search_impl(X, W, a, N, D_in, D_out, alpha_grid, n_alpha, bits, group, loss_form, L, L_col, alpha_star,
                      alpha_idx, workspace, workspace_bytes, status, stream, o);
@@ -650,7 +681,7 @@ int awq_layer_output(const void* X, const float* W, int64_t N, int64_t D_in, int
   uint16_t* wt = reinterpret_cast<uint16_t*>(ws + lay.wt);
   {
     StageTimer t(AWQ_STAGE_WEIGHT_T, st);
-    e = awq::launch_weight_t(W, D_in, D_out, wt, st);
+    e = awq::launch_weight_t(W, D_out, D_in, D_out, wt, st);
   }
   if (e != cudaSuccess) return fail_cuda(e, "weight transpose kernel");
   awq::SearchShape sh{static_cast<int>(N), static_cast<int>(D_in), static_cast<int>(D_out), 0, 4, 128,
@@ -930,12 +961,17 @@ int awq_search_joint(const void* X, const float* const* Ws, const int64_t* D_out
 
 size_t awq_w4a16_workspace_size(int64_t N, int64_t D_in, int64_t D_out) {
   if (N < 1 || D_in < 1 || D_out < 1) return 0;
-  return awq::w4a16_scratch_bytes(N, D_in, D_out) + 256;
+  return awq::w4a16_scratch_bytes(N, D_in, D_out, 0) + 256;
 }
 
-int awq_w4a16_gemm(const void* X, const float* s, const uint32_t* packed, const float* scales, int64_t N,
-                   int64_t D_in, int64_t D_out, int bits, int group, float* Y, void* workspace,
-                   size_t workspace_bytes, int32_t* status, void* stream) {
+size_t awq_w4a16_zp_workspace_size(int64_t N, int64_t D_in, int64_t D_out, int group) {
+  if (N < 1 || D_in < 1 || D_out < 1 || check_quant_args(4, group) != AWQ_OK || D_in % group) return 0;
+  return awq::w4a16_scratch_bytes(N, D_in, D_out, D_in / group) + 256;
+}
+
+static int w4a16_impl(const void* X, const float* s, const uint32_t* packed, const float* scales,
+                      const uint8_t* zeros, int64_t N, int64_t D_in, int64_t D_out, int bits, int group, float* Y,
+                      void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
   if (N < 1 || N > kMaxDim) return fail(AWQ_EINVAL, "N = %lld: need 1 <= N <= 2^24", (long long)N);
   AWQ_TRY(check_quant_args(bits, group));
   if (D_in < group || D_in > kMaxDin || D_in % group)
@@ -948,8 +984,10 @@ int awq_w4a16_gemm(const void* X, const float* s, const uint32_t* packed, const 
   AWQ_TRY(check_ptr(packed, "packed", 16));
   AWQ_TRY(check_ptr(scales, "scales", 16));
   AWQ_TRY(check_ptr(Y, "Y", 4));
+  if (zeros) AWQ_TRY(check_ptr(zeros, "zeros", 16));
   if (!workspace) return fail(AWQ_EWORKSPACE, "workspace is NULL");
-  const size_t need = awq_w4a16_workspace_size(N, D_in, D_out);
+  const size_t need = zeros ? awq_w4a16_zp_workspace_size(N, D_in, D_out, group)
+                            : awq_w4a16_workspace_size(N, D_in, D_out);
   if (workspace_bytes < need) return fail(AWQ_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
   void* xs = reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(workspace) + 255) & ~uintptr_t(255));
   if (!status) return fail(AWQ_EINVAL, "status is NULL");
@@ -963,11 +1001,26 @@ int awq_w4a16_gemm(const void* X, const float* s, const uint32_t* packed, const 
   int rc;
   {
     StageTimer t(AWQ_STAGE_W4A16, st);
-    rc = awq::launch_w4a16(X, s, packed, scales, N, D_in, D_out, bits, group, Y, xs, sms, status, timeout_ns(), st,
-                           &e, &what);
+    rc = awq::launch_w4a16(X, s, packed, scales, zeros, N, D_in, D_out, bits, group, Y, xs, sms, status,
+                           timeout_ns(), st, &e, &what);
   }
   if (rc != AWQ_OK) return e != cudaSuccess ? fail_cuda(e, what) : fail(rc, "%s failed", what);
   return AWQ_OK;
+}
+
+int awq_w4a16_gemm(const void* X, const float* s, const uint32_t* packed, const float* scales, int64_t N,
+                   int64_t D_in, int64_t D_out, int bits, int group, float* Y, void* workspace,
+                   size_t workspace_bytes, int32_t* status, void* stream) {
+  return w4a16_impl(X, s, packed, scales, nullptr, N, D_in, D_out, bits, group, Y, workspace, workspace_bytes,
+                    status, stream);
+}
+
+int awq_w4a16_gemm_zp(const void* X, const float* s, const uint32_t* packed, const float* scales,
+                      const uint8_t* zeros, int64_t N, int64_t D_in, int64_t D_out, int bits, int group, float* Y,
+                      void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  if (!zeros) return fail(AWQ_EINVAL, "zeros is NULL");
+  return w4a16_impl(X, s, packed, scales, zeros, N, D_in, D_out, bits, group, Y, workspace, workspace_bytes, status,
+                    stream);
 }
 
 }  // extern "C"

@@ -54,6 +54,10 @@ struct AlphaList {
 // No scratch: the row split folds through distributed shared memory.
 cudaError_t launch_act_stats(const uint16_t* X, int64_t N, int64_t D, int stat, float* a, int num_sms,
                              cudaStream_t st);
+// Several inputs (host arrays of n <= kMaxStatsInputs entries) in one launch.
+constexpr int kMaxStatsInputs = 16;
+cudaError_t launch_act_stats_batched(const uint16_t* const* X, const int64_t* N, const int64_t* D, int n, int stat,
+                                     float* const* a, int num_sms, cudaStream_t st);
 
 // ---- scales.cu
 // s_tab [A][D] (may be null), r_tab [A][D] = fl32(1 / s) (may be null).
@@ -67,7 +71,8 @@ cudaError_t launch_weight_mean(const float* W, int64_t D_in, int64_t D_out, floa
 // ---- quant.cu
 // The search's A operand for every alpha, bf16 [A][D_out][D_in]: error form
 // (S^-1 Q(S W) - W)^T, reference form (S^-1 Q(S W))^T.  See quant.cu.
-cudaError_t launch_search_operand(const float* W, const float* s_tab, const float* r_tab, int64_t D_in,
+// W rows are ldw elements apart (ldw >= D_out).
+cudaError_t launch_search_operand(const float* W, int64_t ldw, const float* s_tab, const float* r_tab, int64_t D_in,
                                   int64_t D_out, int A, int bits, int group, int form, int qmode, uint16_t* op,
                                   cudaStream_t st);
 // The clipping search's operand for every clip ratio c of `clips`, bf16
@@ -77,7 +82,7 @@ cudaError_t launch_clip_operand(const float* W, const float* s, const float* r, 
                                 const AlphaList& clips, int n_clip, int bits, int group, uint16_t* op,
                                 cudaStream_t st);
 // bf16 W^T [D_out][D_in] for the reference output X W.
-cudaError_t launch_weight_t(const float* W, int64_t D_in, int64_t D_out, uint16_t* wt, cudaStream_t st);
+cudaError_t launch_weight_t(const float* W, int64_t ldw, int64_t D_in, int64_t D_out, uint16_t* wt, cudaStream_t st);
 // Final quantise + pack for one given scale vector s (natural nibble order);
 // clip [D_in/group][D_out] (may be null) scales each group maximum; delta16:
 // delta rounded to FP16 before the codes, scales stored as FP16 (else fp32).
@@ -116,6 +121,8 @@ struct SearchBuffers {
 };
 int search_grid_size(const SearchShape& sh, int num_sms);
 int search_token_tiles(int N);
+// Token tiles per block of the search's unit order (X tiles of a block fit an L2 budget).
+int search_token_block(const SearchShape& sh, int Tt);
 // Rows of loss partials per alpha: one per 128-token half of a token tile.
 int search_partial_rows(int N);
 // Returns 0 on success, otherwise an awq error code; *cerr gets the CUDA error.
@@ -153,13 +160,16 @@ int launch_clip_loss(const uint16_t* op, const uint16_t* Hb, int64_t D_in, int64
 // ---- w4a16.cu (the quantised layer applied to activations)
 // Y [N][D_out] fp32 = X diag(1/s) Dequant(packed, scales), tcgen05 with the
 // weights dequantised into shared memory; stream-K over the k blocks when
-// the token tile is small.  ws: scratch of w4a16_scratch_bytes(N, D_in, D_out)
-// bytes, 256-byte aligned (scaled activations, stream-K partial tiles).
-// D_out must be a multiple of 4.
-size_t w4a16_scratch_bytes(int64_t N, int64_t D_in, int64_t D_out);
-int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const float* scales, int64_t N, int64_t D_in,
-                 int64_t D_out, int bits, int group, float* Y, void* ws, int num_sms, int* status,
-                 uint64_t timeout_ns, cudaStream_t st, cudaError_t* cerr, const char** what);
+// the token tile is small.  ws: scratch of w4a16_scratch_bytes(N, D_in, D_out,
+// zrows) bytes, 256-byte aligned (scaled activations, stream-K partial tiles,
+// and with zero points the fp32 rows of 128 + z).  zeros: NULL (offset-binary
+// codes u = q + 2^(b-1)) or [D_in/group][D_out] uint8 zero points of
+// asymmetric codes u = q + z (zrows = D_in / group).  D_out must be a
+// multiple of 4.
+size_t w4a16_scratch_bytes(int64_t N, int64_t D_in, int64_t D_out, int64_t zrows);
+int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const float* scales, const uint8_t* zeros,
+                 int64_t N, int64_t D_in, int64_t D_out, int bits, int group, float* Y, void* ws, int num_sms,
+                 int* status, uint64_t timeout_ns, cudaStream_t st, cudaError_t* cerr, const char** what);
 
 // Self-test of the bounded wait: one CTA waits on an mbarrier that nothing
 // arrives at, gives up after timeout_ns and records the timeout in *status.

@@ -278,6 +278,19 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
 }
 
+// Three-input fp32 maximum and minimum (one instruction on sm_100a; finite
+// inputs here, so the NaN rules of max.f32 / min.f32 never apply).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Programmatic dependent launch: the primary lets its dependent grid start
 // early; the dependent waits for the primary's completion (and its memory)
 // before touching the primary's output.

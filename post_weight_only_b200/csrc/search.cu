@@ -50,8 +50,8 @@
 // Units are dealt round robin in whole waves, all pairs advancing through
 // alpha in step (so the operand of one alpha is read from HBM once and shared
 // through L2); the alpha passes of the last partial wave are split evenly
-// over all pairs.  The unit numbering is token-minor or weight-minor,
-// whichever keeps the data that concurrent pairs share smaller.
+// over all pairs.  Units are numbered in token blocks sized to L2 (see
+// unit_tiles and search_token_block).
 //
 // Every mbarrier wait is bounded: on a timeout the kernel records
 // AWQ_ETIMEOUT in the status word, every role leaves its loop, in-flight
@@ -79,6 +79,10 @@ constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*align*/;
 constexpr uint16_t kPairMask = 0x3;
+// L2 budget for the X tiles of one token block of the unit order, and the
+// fewest tiles worth keeping as a block.
+constexpr long long kXBlockBudgetBytes = 64ll << 20;
+constexpr int kMinBlockTiles = 8;
 static_assert(kHalfN == kBM, "operand and X half-tiles share one box shape");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
@@ -87,7 +91,8 @@ enum Site { kSiteTmaEmpty = 1, kSiteMmaAccEmpty, kSiteMmaFull, kSiteEpiAccFull, 
 
 struct Params {
   int N, D_in, D_out, A;
-  int Tt, Wt, U, KB, H, gemm_only, weight_minor;
+  int Tt, Wt, U, KB, H, gemm_only;
+  int tb;                     // token tiles per token block of the unit order (see unit_tiles)
   const uint16_t* op;         // Gram form: the operand E [A][D_out][D_in], read by the epilogue
   float* yref;
   float* partial;
@@ -140,14 +145,21 @@ struct Schedule {
   }
 };
 
+// Unit order: the token tiles are cut into blocks of tb tiles (the last block
+// may be shorter); the units of one block come before the next block's,
+// weight tile by weight tile, token tile fastest.  A wave of pairs then covers
+// a few weight tiles across the block's token tiles: the block's X tiles stay
+// in L2 through all alpha passes of the wave and the next waves of the block,
+// and each alpha's operand tile is read by the wave's pairs at about the same
+// time.
 __device__ __forceinline__ void unit_tiles(const Params& p, int u, int& wt, int& tt) {
-  if (p.weight_minor) {
-    tt = u / p.Wt;
-    wt = u % p.Wt;
-  } else {
-    wt = u / p.Tt;
-    tt = u % p.Tt;
-  }
+  const int per_block = p.tb * p.Wt;
+  const int b = u / per_block;
+  const int t0 = b * p.tb;
+  const int tc = min(p.tb, p.Tt - t0);          // token tiles in this block
+  const int r = u - b * per_block;
+  wt = r / tc;
+  tt = t0 + r % tc;
 }
 
 // Passes of a segment: the reference form starts with the reference pass,
@@ -563,6 +575,27 @@ bool make_word_map(CUtensorMap* m, const void* base, bool is_float, uint64_t inn
 
 int search_token_tiles(int N) { return (N + kBN - 1) / kBN; }
 
+// Token tiles per block of the unit order: as many as keep the block's X tiles
+// (256 tokens x D_in bf16 each) within an L2 budget, balanced over the blocks.
+// Per wave, the operand of every alpha is read once for the wave's few weight
+// tiles, and the block's X tiles once for all its waves.  When fewer than
+// kMinBlockTiles X tiles fit (a very long reduction dimension), a block is a
+// single token tile: every pair of a wave then shares that tile and reads its
+// own weight tiles.  Measured on B200 (21 alphas, N = 4096): the 28672 x 8192
+// down projection ran 28.0 ms with blocks of one token tile against 29.9 ms
+// with four and 35.3 ms with all sixteen; the 11008-input layer was fastest
+// with blocks of 8, the 8192-input layers with all 16, and the 16384-token
+// layer with 32 -- the choices this budget makes.
+int search_token_block(const SearchShape& sh, int Tt) {
+  const double tile_bytes = 2.0 * kBN * static_cast<double>(sh.D_in);
+  const double budget = static_cast<double>(kXBlockBudgetBytes);
+  int tmax = static_cast<int>(budget / tile_bytes);
+  if (tmax < kMinBlockTiles) return 1;
+  if (tmax >= Tt) return Tt;
+  const int nblk = (Tt + tmax - 1) / tmax;
+  return (Tt + nblk - 1) / nblk;
+}
+
 int search_partial_rows(int N) { return 2 * search_token_tiles(N); }
 
 // Number of CTAs (two per pair): one pair per unit of work, at most one CTA
@@ -612,15 +645,7 @@ int launch_search(const SearchShape& sh, const SearchBuffers& b, int grid, uint6
   p.KB = (sh.D_in + kBK - 1) / kBK;
   p.H = search_partial_rows(sh.N);
   p.gemm_only = gemm_only ? 1 : 0;
-  {
-    // Concurrent pairs (one wave) either share token tiles (weight-minor
-    // numbering: all of X stays hot, plus the operand of a few weight tiles)
-    // or weight tiles (token-minor: the operand of one alpha stays hot, plus
-    // a few token tiles of X).  Keep the smaller working set.
-    const double x_bytes = 2.0 * sh.N * sh.D_in;
-    const double op_per_alpha = 2.0 * sh.D_in * static_cast<double>(sh.D_out);
-    p.weight_minor = (!gemm_only && x_bytes > op_per_alpha) ? 1 : 0;
-  }
+  p.tb = search_token_block(sh, p.Tt);
   p.op = b.op;
   p.yref = b.yref;
   p.partial = b.partial;

@@ -159,14 +159,37 @@ __global__ void __launch_bounds__(256) scale_x_kernel(const uint4* __restrict__ 
   }
 }
 
+// zb[g][n] = 128 + zeros[g][n] as fp32: the per-(group, column) bias of the
+// asymmetric dequantiser, read by TMA beside the deltas.
+__global__ void __launch_bounds__(256) zero_bias_kernel(const uint8_t* __restrict__ zeros, int64_t n,
+                                                        float* __restrict__ zb) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    zb[i] = 128.0f + static_cast<float>(zeros[i]);
+}
+
+// A kernel argument copied into a register the compiler cannot see through.
+// Used for the dequantisers' magic constants: read straight from the
+// parameter bank, a constant is a second non-register operand of the
+// mask-and-OR, which then takes two logic ops instead of one.
+__device__ __forceinline__ uint32_t in_register(uint32_t v) {
+  uint32_t r;
+  asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
+  return r;
+}
+
 // ------------------------------------------------------------ the GEMM
 __device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t u) { return *reinterpret_cast<__nv_bfloat162*>(&u); }
 __device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
-template <int G>
+// kZp: asymmetric codes; each stage also holds the rows of 128 + z (fp32,
+// made by zero_bias_kernel) beside the deltas, and the dequantiser subtracts
+// that per-(group, column) value instead of 128 + off.
+template <int G, bool kZp>
 __global__ void __launch_bounds__(kW4Threads, 1)
     w4a16_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
-                 const __grid_constant__ CUtensorMap tmS, const W4Params p) {
+                 const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
+                 const W4Params p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   // 1024-byte aligned base (128-byte swizzle atoms), derived by pointer
   // arithmetic on the shared array so that accesses stay in the shared space.
@@ -223,7 +246,7 @@ __global__ void __launch_bounds__(kW4Threads, 1)
   if (warp < kW4TmaWarps) {
     // ---------------------------------------------------------- TMA: warp w fills the stages of step index = w mod issuers
     if (lane == 0 && warp < p.issuers) {
-      const uint32_t tx = static_cast<uint32_t>(xs_bytes + pk_bytes + p.scale_rows * 128 * 4);
+      const uint32_t tx = static_cast<uint32_t>(xs_bytes + pk_bytes + (kZp ? 2 : 1) * p.scale_rows * 128 * 4);
       const int step = p.issuers;
       int s = warp;                 // this warp's next stage slot (S is a multiple of `step`)
       uint32_t ph = 0;
@@ -245,6 +268,7 @@ __global__ void __launch_bounds__(kW4Threads, 1)
           tma_load_3d(sp, &tmX, &w_full[s], 0, t0, kb);
           tma_load_2d(sp + xs_bytes, &tmP, &w_full[s], n0, kb * 8);
           tma_load_2d(sp + xs_bytes + pk_bytes, &tmS, &w_full[s], n0, (kb * 64) / G);
+          if (kZp) tma_load_2d(sp + xs_bytes + pk_bytes + p.scale_rows * 512, &tmZ, &w_full[s], n0, (kb * 64) / G);
           ++fills;
           s += step;
           if (s >= S) {
@@ -325,7 +349,7 @@ __global__ void __launch_bounds__(kW4Threads, 1)
     const int n = (warp & 3) * 32 + lane;
     const int h = (warp - kW4DqWarp0) >> 2;       // half of each k block: chunks 4h..4h+3
     const uint32_t bias_bits = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(128.0f + p.off)));
-    const uint32_t magic = p.magic;
+    const uint32_t magic = in_register(p.magic);
     const __nv_bfloat162 bias = as_bf162(bias_bits | (bias_bits << 16));     // 128 + off, exact
     const int swz = n & 7;
     int s = 0, sa = 0;
@@ -357,13 +381,15 @@ __global__ void __launch_bounds__(kW4Threads, 1)
           const int srow = ((kb0 + j) * 64 + 32 * h) / G - row0;
           const float* sc = reinterpret_cast<const float*>(sp + xs_bytes + pk_bytes) + srow * 128 + n;
           const __nv_bfloat162 d2 = __float2bfloat162_rn(sc[0]);
+          __nv_bfloat162 zbias = bias;
+          if (kZp) zbias = __float2bfloat162_rn(sc[p.scale_rows * 128]);   // 128 + z, exact in bf16
           uint32_t o[16];                           // chunks 4h..4h+3 of row n: 16 bf16 pairs
 #pragma unroll
           for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const uint32_t pair = ((w[i] >> (4 * q)) & 0x000F000Fu) | magic;   // {128 + u_q, 128 + u_{q+4}}
-              o[4 * i + q] = as_u32(__hmul2(__hsub2(as_bf162(pair), bias), d2));
+              o[4 * i + q] = as_u32(__hmul2(__hsub2(as_bf162(pair), zbias), d2));
             }
           uint4* arow = reinterpret_cast<uint4*>(a_sm + sa * kW4ABytes + (n >> 3) * 1024 + (n & 7) * 128);
 #pragma unroll
@@ -518,20 +544,26 @@ constexpr int kGvUnroll = 4;                     // k8 rows in flight per warp (
 constexpr int kGvMaxSplit = 32;
 constexpr int kGvMaxTokens = 4;
 
-// magic = 0x4B000000 (2^23), a kernel argument so that it sits in a register
-// and (w & mask) | magic is one three-input logic op.
+// magic = 0x4B000000 (2^23), held in a register (see in_register) so that
+// (w & mask) | magic is one three-input logic op with the mask as its one
+// immediate operand.
 __device__ __forceinline__ float nib(uint32_t w, uint32_t mask, uint32_t magic) {
   return __uint_as_float((w & mask) | magic);
 }
 
-template <int NT>
+// kZp: asymmetric codes u = q + z with a zero point per (group, column)
+// (zeros [D_in/G][D_out] uint8); the subtracted bias is 2^23 + 16^i z of the
+// current group instead of 2^23 + 16^i off, so every term is still exact.
+template <int NT, bool kZp>
 __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 3 : 2) w4a16_gemv_kernel(const uint4* __restrict__ X,
                                                                 const float4* __restrict__ s,
                                                                 const uint4* __restrict__ packed,
-                                                                const float4* __restrict__ scales, int64_t D_in,
+                                                                const float4* __restrict__ scales,
+                                                                const uint8_t* __restrict__ zeros, int64_t D_in,
                                                                 int64_t D_out, int gshift, int off,
                                                                 uint32_t magic, int R8, float* __restrict__ out) {
   constexpr int U = NT <= 2 ? kGvUnroll : kGvUnroll / 2;     // fits two CTAs per SM at 3-4 tokens
+  magic = in_register(magic);
   __shared__ __align__(16) float xt[NT * kGvChunk8 * 8];       // x~ [NT][chunk rows * 8]
   __shared__ __align__(16) float red[8 * NT * kGvCols];         // per-warp sums
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -584,6 +616,12 @@ __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 3 : 2) w4a16_gemv_kernel
         for (int c = 0; c < 4; ++c) acc[t][c] = make_float2(0.0f, 0.0f);
       int64_t g_cur = -1;                          // the group acc belongs to
       float4 dcur = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      float2 zb01[4], zb23[4];                     // kZp: the biases of the group's zero points, per column
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        zb01[c] = bias01;
+        zb23[c] = bias23;
+      }
       auto flush = [&]() {
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
@@ -609,6 +647,15 @@ __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 3 : 2) w4a16_gemv_kernel
           if (g != g_cur) {                          // uniform over the warp
             if (g_cur >= 0) flush();
             dcur = __ldg(scales + g * D4 + n4);      // used at the group's flush
+            if (kZp) {                               // the four columns' zero points, one 32-bit load
+              const uint32_t z4 = __ldg(reinterpret_cast<const uint32_t*>(zeros + g * D_out) + n4);
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const float z = static_cast<float>((z4 >> (8 * c)) & 0xFFu);
+                zb01[c] = make_float2(-(8388608.0f + z), -(8388608.0f + 16.0f * z));
+                zb23[c] = make_float2(-(8388608.0f + 256.0f * z), -(8388608.0f + 4096.0f * z));
+              }
+            }
             g_cur = g;
           }
           float4 xa[NT], xb[NT];
@@ -622,10 +669,11 @@ __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 3 : 2) w4a16_gemv_kernel
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const uint32_t w = wv[c], wh = w >> 16;
-            const float2 v01 = __fadd2_rn(make_float2(nib(w, 0xFu, magic), nib(w, 0xF0u, magic)), bias01);
-            const float2 v23 = __fadd2_rn(make_float2(nib(w, 0xF00u, magic), nib(w, 0xF000u, magic)), bias23);
-            const float2 v45 = __fadd2_rn(make_float2(nib(wh, 0xFu, magic), nib(wh, 0xF0u, magic)), bias01);
-            const float2 v67 = __fadd2_rn(make_float2(nib(wh, 0xF00u, magic), nib(wh, 0xF000u, magic)), bias23);
+            const float2 b01 = kZp ? zb01[c] : bias01, b23 = kZp ? zb23[c] : bias23;
+            const float2 v01 = __fadd2_rn(make_float2(nib(w, 0xFu, magic), nib(w, 0xF0u, magic)), b01);
+            const float2 v23 = __fadd2_rn(make_float2(nib(w, 0xF00u, magic), nib(w, 0xF000u, magic)), b23);
+            const float2 v45 = __fadd2_rn(make_float2(nib(wh, 0xFu, magic), nib(wh, 0xF0u, magic)), b01);
+            const float2 v67 = __fadd2_rn(make_float2(nib(wh, 0xF00u, magic), nib(wh, 0xF000u, magic)), b23);
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
               float2 a2 = __ffma2_rn(v01, make_float2(xa[t].x, xa[t].y), acc[t][c]);
@@ -694,17 +742,18 @@ __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float4* __restri
 namespace {
 
 struct W4Layout {
-  size_t xs, count, partial, total;
+  size_t xs, count, partial, zb, total;
 };
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 int w4_token_tile(int64_t N) { return N >= 256 ? 256 : static_cast<int>((N + 15) / 16 * 16); }
 
-W4Layout w4_layout(int64_t N, int64_t D_in, int64_t D_out) {
+// zrows: rows of zero points (D_in / group) of the asymmetric consumer, else 0.
+W4Layout w4_layout(int64_t N, int64_t D_in, int64_t D_out, int64_t zrows = 0) {
   W4Layout l;
   if (N <= kGvMaxTokens) {                        // the GEMV: partial rows of up to kGvMaxSplit splits
-    l.xs = l.count = l.partial = 0;
+    l.xs = l.count = l.partial = l.zb = 0;
     l.total = round256(static_cast<size_t>(kGvMaxSplit) * N * D_out * 4);
     return l;
   }
@@ -715,22 +764,29 @@ W4Layout w4_layout(int64_t N, int64_t D_in, int64_t D_out) {
   l.count = round256(static_cast<size_t>(N) * static_cast<size_t>(Dp) * 2);
   l.partial = l.count + round256(static_cast<size_t>(units) * 4);
   const size_t part = Nt <= kW4MaxStreamTokens ? static_cast<size_t>(kW4MaxGrid) * 2 * N * 128 * 4 : 0;
-  l.total = l.partial + part;
+  l.zb = l.partial + round256(part);
+  l.total = l.zb + round256(static_cast<size_t>(zrows) * D_out * 4);
   return l;
 }
 
 template <int NT>
 cudaError_t launch_gemv_nt(dim3 grid, cudaStream_t st, const void* X, const float* s, const uint32_t* packed,
-                           const float* scales, int64_t D_in, int64_t D_out, int gshift, int off, int R8, float* out) {
-  w4a16_gemv_kernel<NT><<<grid, kGvThreads, 0, st>>>(
-      static_cast<const uint4*>(X), reinterpret_cast<const float4*>(s), reinterpret_cast<const uint4*>(packed),
-      reinterpret_cast<const float4*>(scales), D_in, D_out, gshift, off, 0x4B000000u, R8, out);
+                           const float* scales, const uint8_t* zeros, int64_t D_in, int64_t D_out, int gshift, int off,
+                           int R8, float* out) {
+  if (zeros)
+    w4a16_gemv_kernel<NT, true><<<grid, kGvThreads, 0, st>>>(
+        static_cast<const uint4*>(X), reinterpret_cast<const float4*>(s), reinterpret_cast<const uint4*>(packed),
+        reinterpret_cast<const float4*>(scales), zeros, D_in, D_out, gshift, off, 0x4B000000u, R8, out);
+  else
+    w4a16_gemv_kernel<NT, false><<<grid, kGvThreads, 0, st>>>(
+        static_cast<const uint4*>(X), reinterpret_cast<const float4*>(s), reinterpret_cast<const uint4*>(packed),
+        reinterpret_cast<const float4*>(scales), nullptr, D_in, D_out, gshift, off, 0x4B000000u, R8, out);
   return cudaGetLastError();
 }
 
-int launch_w4a16_gemv(const void* X, const float* s, const uint32_t* packed, const float* scales, int64_t N,
-                      int64_t D_in, int64_t D_out, int bits, int group, float* Y, void* ws, int num_sms,
-                      cudaStream_t st, cudaError_t* cerr, const char** what) {
+int launch_w4a16_gemv(const void* X, const float* s, const uint32_t* packed, const float* scales,
+                      const uint8_t* zeros, int64_t N, int64_t D_in, int64_t D_out, int bits, int group, float* Y,
+                      void* ws, int num_sms, cudaStream_t st, cudaError_t* cerr, const char** what) {
   const int64_t rows8 = D_in / 8;
   const int64_t tiles = (D_out + kGvCols - 1) / kGvCols;
   // About eight CTAs per SM over column tiles x splits; at least 8 k8 rows
@@ -751,10 +807,10 @@ int launch_w4a16_gemv(const void* X, const float* s, const uint32_t* packed, con
   const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(splits));
   cudaError_t e;
   switch (N) {
-    case 1: e = launch_gemv_nt<1>(grid, st, X, s, packed, scales, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
-    case 2: e = launch_gemv_nt<2>(grid, st, X, s, packed, scales, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
-    case 3: e = launch_gemv_nt<3>(grid, st, X, s, packed, scales, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
-    case 4: e = launch_gemv_nt<4>(grid, st, X, s, packed, scales, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
+    case 1: e = launch_gemv_nt<1>(grid, st, X, s, packed, scales, zeros, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
+    case 2: e = launch_gemv_nt<2>(grid, st, X, s, packed, scales, zeros, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
+    case 3: e = launch_gemv_nt<3>(grid, st, X, s, packed, scales, zeros, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
+    case 4: e = launch_gemv_nt<4>(grid, st, X, s, packed, scales, zeros, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
     default: *what = "gemv token count"; return kEUnsupported;
   }
   if (e != cudaSuccess) {
@@ -780,15 +836,19 @@ int launch_w4a16_gemv(const void* X, const float* s, const uint32_t* packed, con
 
 }  // namespace
 
-size_t w4a16_scratch_bytes(int64_t N, int64_t D_in, int64_t D_out) { return w4_layout(N, D_in, D_out).total; }
+size_t w4a16_scratch_bytes(int64_t N, int64_t D_in, int64_t D_out, int64_t zrows) {
+  return w4_layout(N, D_in, D_out, zrows).total;
+}
 
-int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const float* scales, int64_t N, int64_t D_in,
-                 int64_t D_out, int bits, int group, float* Y, void* ws, int num_sms, int* status,
-                 uint64_t timeout_ns, cudaStream_t st, cudaError_t* cerr, const char** what) {
+int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const float* scales, const uint8_t* zeros,
+                 int64_t N, int64_t D_in, int64_t D_out, int bits, int group, float* Y, void* ws, int num_sms,
+                 int* status, uint64_t timeout_ns, cudaStream_t st, cudaError_t* cerr, const char** what) {
   *cerr = cudaSuccess;
   if (N <= kGvMaxTokens)
-    return launch_w4a16_gemv(X, s, packed, scales, N, D_in, D_out, bits, group, Y, ws, num_sms, st, cerr, what);
-  const W4Layout lay = w4_layout(N, D_in, D_out);
+    return launch_w4a16_gemv(X, s, packed, scales, zeros, N, D_in, D_out, bits, group, Y, ws, num_sms, st, cerr,
+                             what);
+  const bool zp = zeros != nullptr;
+  const W4Layout lay = w4_layout(N, D_in, D_out, zp ? D_in / group : 0);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   void* xs = wsb + lay.xs;
   int* count = reinterpret_cast<int*>(wsb + lay.count);
@@ -825,7 +885,7 @@ int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const fl
   const int issuers = kps > 1 ? 2 : 1;
   const int KBS = (KB + kps - 1) / kps;
   const int scale_rows = kps * 64 >= group ? kps * 64 / group : 1;
-  const int stage_bytes = (kps * Nt * 128 + kps * kW4PkBytes + scale_rows * 512 + 1023) / 1024 * 1024;
+  const int stage_bytes = (kps * Nt * 128 + kps * kW4PkBytes + (zp ? 2 : 1) * scale_rows * 512 + 1023) / 1024 * 1024;
   // One CTA per SM; its shared memory goes to deep rings.
   const int budget = 220 * 1024;
   const int a_stages = Nt <= 32 ? 4 : 3;
@@ -836,15 +896,28 @@ int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const fl
   if (stages < 2) stages = 2;
   const int smem = fixed + stages * stage_bytes;
 
-  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, W4Params) = nullptr;
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, W4Params) = nullptr;
   switch (group) {
-    case 32: kern = w4a16_kernel<32>; break;
-    case 64: kern = w4a16_kernel<64>; break;
-    case 128: kern = w4a16_kernel<128>; break;
-    case 256: kern = w4a16_kernel<256>; break;
+    case 32: kern = zp ? w4a16_kernel<32, true> : w4a16_kernel<32, false>; break;
+    case 64: kern = zp ? w4a16_kernel<64, true> : w4a16_kernel<64, false>; break;
+    case 128: kern = zp ? w4a16_kernel<128, true> : w4a16_kernel<128, false>; break;
+    case 256: kern = zp ? w4a16_kernel<256, true> : w4a16_kernel<256, false>; break;
     default:
       *what = "group";
       return kEUnsupported;
+  }
+  float* zb = reinterpret_cast<float*>(wsb + lay.zb);
+  if (zp) {
+    const int64_t nz = (D_in / group) * D_out;
+    int64_t blocks = (nz + 255) / 256;
+    if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
+    zero_bias_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(zeros, nz, zb);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      *cerr = e;
+      *what = "zero_bias_kernel launch";
+      return kECuda;
+    }
   }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) {
@@ -857,7 +930,7 @@ int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const fl
 
   // X' as [KB][N][64]: dimension 1 (tokens) has stride Dp, dimension 2
   // (k blocks) stride 64 elements; one box = the X' planes of a stage.
-  CUtensorMap mX, mP, mS;
+  CUtensorMap mX, mP, mS, mZ;
   const uint64_t xdims[3] = {64, static_cast<uint64_t>(N), static_cast<uint64_t>(KB)};
   const uint64_t xstr[2] = {static_cast<uint64_t>(Dp) * 2, 128};
   const uint32_t xbox[3] = {64, static_cast<uint32_t>(Nt), static_cast<uint32_t>(kps)};
@@ -865,6 +938,9 @@ int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const fl
       !make_word_map(&mP, packed, false, static_cast<uint64_t>(D_out), static_cast<uint64_t>(D_in / 8), 128,
                      static_cast<uint32_t>(8 * kps)) ||
       !make_word_map(&mS, scales, true, static_cast<uint64_t>(D_out), static_cast<uint64_t>(D_in / group), 128,
+                     static_cast<uint32_t>(scale_rows)) ||
+      !make_word_map(&mZ, zp ? static_cast<const void*>(zb) : static_cast<const void*>(scales), true,
+                     static_cast<uint64_t>(D_out), static_cast<uint64_t>(D_in / group), 128,
                      static_cast<uint32_t>(scale_rows))) {
     *what = "tensor maps for the W4A16 GEMM";
     return kECuda;
@@ -903,7 +979,7 @@ int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const fl
     p.chunk = KBS;
     grid = units < slots ? units : slots;
   }
-  kern<<<static_cast<unsigned>(grid), kW4Threads, smem, st>>>(mX, mP, mS, p);
+  kern<<<static_cast<unsigned>(grid), kW4Threads, smem, st>>>(mX, mP, mS, mZ, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     *cerr = e;

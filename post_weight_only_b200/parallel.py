@@ -95,12 +95,15 @@ def layer_sharded_search(n_layers: int, layer_search: Callable[[int], Tuple[torc
 def cuda_shard_loss(X: torch.Tensor, W: torch.Tensor, a: torch.Tensor, alpha_grid: Sequence[float],
                     bits: int = 4, group: int = 128, loss_form: int = 0) -> Callable[[int, int], torch.Tensor]:
     """The per-shard loss of :func:`column_sharded_search` on this rank's GPU:
-    the search over columns [c0, c1) of W (X replicated), through the C ABI."""
+    the search over columns [c0, c1) of W (X replicated), through the C ABI.
+    The slice is searched in place: W + c0 with W's row stride, no copy (c0 is
+    a multiple of the 256-column tile, so the slice stays 16-byte aligned)."""
     from . import awq
 
     def fn(c0: int, c1: int) -> torch.Tensor:
         if c1 <= c0:
             return torch.zeros(len(alpha_grid), dtype=torch.float64, device=X.device)
-        res = awq.search(X, W[:, c0:c1].contiguous(), a, alpha_grid, bits, group, loss_form=loss_form)
+        Wc = W[:, c0:c1] if c1 - c0 < W.shape[1] else W
+        res = awq.search(X, Wc, a, alpha_grid, bits, group, loss_form=loss_form)
         return res.L
     return fn

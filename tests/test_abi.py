@@ -146,7 +146,8 @@ def test_argument_checks_without_gpu(lib):
     assert gcall(st=None) == 1                             # the status word is required
 
     class Opts(ctypes.Structure):
-        _fields_ = [("quantizer", ctypes.c_int), ("w_mean", ctypes.c_void_p), ("gram_form", ctypes.c_int)]
+        _fields_ = [("quantizer", ctypes.c_int), ("w_mean", ctypes.c_void_p), ("gram_form", ctypes.c_int),
+                    ("ldw", ctypes.c_int64)]
 
     x = lib.awq_search_ex
     x.argtypes = [P, P, P, I64, I64, I64, P, I, I, I, I, ctypes.POINTER(Opts), P, P, P, P, P, ctypes.c_size_t, P, P]
@@ -160,6 +161,8 @@ def test_argument_checks_without_gpu(lib):
     assert xcall(ctypes.byref(Opts(3, None, 0))) == 1        # unknown quantiser
     assert xcall(ctypes.byref(Opts(1, fake + 2, 0))) == 2    # misaligned weight means
     assert xcall(ctypes.byref(Opts(1, None, 0)), bits=5) == 3   # the common checks still apply
+    assert xcall(ctypes.byref(Opts(0, None, 0, 32))) == 1    # row stride below D_out
+    assert xcall(ctypes.byref(Opts(0, None, 0, 66))) == 1    # row stride not a multiple of 4
     xws = lib.awq_search_ex_workspace_size
     xws.argtypes = [I64, I64, I64, I, I, I, I, ctypes.POINTER(Opts)]
     xws.restype = ctypes.c_size_t

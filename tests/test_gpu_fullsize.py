@@ -91,7 +91,7 @@ def _check_layer_path(awq, X, W, alphas, bits, group, form, cols):
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
-@pytest.mark.parametrize("name", ["llama7b_attn_proj"])
+@pytest.mark.parametrize("name", ["llama7b_attn_proj", "llama7b_mlp_down"])
 def test_full_layer_against_full_oracle(awq, name):
     """Every L(alpha) of the whole layer (all output columns) and alpha*
     against the oracle's full search, stored once by

@@ -1,4 +1,4 @@
-"""GPU parity of the Gram form of the alpha search (NEXT f4, second half):
+"""GPU parity of the Gram form of the alpha search:
 L(alpha) = sum_n e_n^T H e_n with H = X^T X, the same quantity as
 ||X S^-1 Q(S W) - X W||^2 (compassingai.com concept page, flow step 4c),
 against the CPU oracle's direct evaluation.

@@ -59,6 +59,7 @@ _check_alpha = check_alpha
     (1, 8), (7, 264), (300, 520), (4096, 4096), (1000, 11008),
     (1, 4096),                                    # one row: the second CTA of each pair has none
     (3, 262144), (2, 524288), (1, 1048576),       # one row lane per chunk; one, two, four rounds
+    (64, 65536), (40, 151552),                    # slabs wider than the CTA's threads, with several row lanes
 ])
 def test_act_stats(awq, N, D):
     X, _ = _layer(N, D, 8, seed=N)
@@ -87,6 +88,22 @@ def test_weight_mean_hand_worked(awq):
     W = torch.tensor(g["W_rows"], dtype=torch.float32).cuda()
     got = awq.weight_mean(W).cpu().numpy()
     assert got.tolist() == [float(np.float32(v)) for v in g["mean_abs_rows_fp32"]]
+
+
+def test_act_stats_batched(awq):
+    """Several inputs of different shapes in one launch: each statistic as the
+    oracle's (max exact, mean within relative 1e-5)."""
+    shapes = [(4096, 8192), (300, 264), (1, 4096), (2048, 28672), (17, 8)]
+    Xs = [_layer(N, D, 8, seed=N + D)[0] for N, D in shapes]
+    for stat in (awq.STAT_MEAN, awq.STAT_MAX):
+        got = awq.act_stats_batched([X.cuda() for X in Xs], stat)
+        for X, a in zip(Xs, got):
+            ref = oracle.act_stats(X, oracle.STAT_MEAN if stat == awq.STAT_MEAN else oracle.STAT_MAX)
+            a = a.cpu().numpy().astype(np.float64)
+            if stat == awq.STAT_MAX:
+                assert np.array_equal(a, ref)
+            else:
+                assert np.allclose(a, ref, rtol=1e-5, atol=0)
 
 
 def test_act_stats_reproducible(awq):

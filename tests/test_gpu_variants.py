@@ -1,4 +1,4 @@
-"""GPU parity of the quantiser and scale variants of the search (NEXT f2)
+"""GPU parity of the quantiser and scale variants of the search
 against the CPU oracle, through the C ABI.
 
   * the power-of-two delta (mudrobot.github.io AWQ notes, "analysing the

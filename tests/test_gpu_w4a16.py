@@ -151,3 +151,52 @@ def test_w4a16_rejects_unaligned_columns(awq):
     scales = torch.ones(1, 6, device="cuda")
     with pytest.raises(awq.AwqError):
         awq.w4a16_gemm(X, s, packed, scales, 4, 128)
+
+
+# ------------------------------------------------------------ asymmetric (zero-point) codes
+def _zp_case(awq, N, D_in, D_out, bits, group, seed):
+    """Codes, deltas and zero points from the oracle's MinMax quantiser
+    (oracle.quantize_asym, packed by oracle.pack_unsigned), applied by the CUDA
+    consumer and by oracle.w4a16_zp."""
+    X, W = synth.layer_inputs(synth.small_layer(max(N, 8), D_in, D_out, seed=seed))
+    X = X[:N].contiguous()
+    s = oracle.scales(oracle.act_stats(X).astype(np.float32), 0.5)
+    q, d, z = oracle.quantize_asym(W, s, bits, group)
+    u = q.astype(np.int16) + np.repeat(z, group, axis=0).astype(np.int16)
+    packed = oracle.pack_unsigned(u)
+    Y = awq.w4a16_gemm(X.cuda(), torch.from_numpy(s).cuda(), torch.from_numpy(packed.view(np.int32)).cuda(),
+                       torch.from_numpy(d).cuda(), bits, group,
+                       zeros=torch.from_numpy(z).cuda()).cpu().numpy().astype(np.float64)
+    Y_or = oracle.w4a16_zp(X, s, packed, d, z, group)
+    w_hat = q * np.repeat(d, group, axis=0).astype(np.float64) / s.astype(np.float64)[:, None]
+    return Y, Y_or, _bound(X.double().numpy(), w_hat, group)
+
+
+@pytest.mark.parametrize("N,D_in,D_out,bits,group", [
+    (1, 4096, 512, 4, 128),       # GEMV, split K
+    (3, 1024, 132, 3, 64),        # GEMV, ragged column tile
+    (4, 256, 1000, 2, 32),        # GEMV, 2-bit, group 32
+    (2, 2048, 256, 4, 256),       # GEMV, group 256
+    (5, 512, 200, 4, 128),        # tensor cores, stream-K, ragged columns
+    (37, 384, 132, 3, 64),
+    (17, 8192, 2048, 4, 128),     # stream-K shares inside one unit
+    (300, 1024, 260, 4, 128),     # two token tiles, no split
+    (64, 1056, 96, 2, 32),        # group 32: two delta and zero rows per k block; half k block
+    (300, 768, 256, 4, 256),      # group 256, large token tile
+])
+def test_w4a16_zero_point_against_oracle(awq, N, D_in, D_out, bits, group):
+    Y, Y_or, bound = _zp_case(awq, N, D_in, D_out, bits, group, seed=N + 7 * D_in)
+    assert np.all(np.abs(Y - Y_or) <= bound), np.max(np.abs(Y - Y_or) / bound)
+
+
+def test_w4a16_zero_point_matches_symmetric_at_the_midpoint(awq):
+    """With every zero point equal to 2^(b-1) the asymmetric consumer reads the
+    offset-binary codes of the symmetric pack: both paths give the same Y bit
+    for bit (GEMV and tensor cores)."""
+    for N in (2, 40):
+        X, W = synth.layer_inputs(synth.small_layer(max(N, 8), 1024, 256, seed=N))
+        X = X[:N].contiguous().cuda()
+        s = torch.from_numpy(oracle.scales(oracle.act_stats(X.cpu()).astype(np.float32), 0.5)).cuda()
+        packed, sc = awq.quantize_pack(W.cuda(), s, 4, 128)
+        z = torch.full((1024 // 128, 256), 8, dtype=torch.uint8, device="cuda")
+        assert torch.equal(awq.w4a16_gemm(X, s, packed, sc, 4, 128, zeros=z), awq.w4a16_gemm(X, s, packed, sc, 4, 128))
