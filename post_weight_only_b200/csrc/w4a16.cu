@@ -516,55 +516,60 @@ __global__ void __launch_bounds__(kW4Threads, 1)
 }
 
 // ------------------------------------------------------------ decode: the GEMV
-// Y[t][n] = sum_k x~_tk * 16^(k%4) (u_kn - off) * delta_{k/G, n} on CUDA cores
-// for N <= 4 tokens, fp32 throughout (x / s rounded once, IEEE division; no
-// bf16 roundings of the weights; delta applied once per group).
+// Y[t][n] = sum_g delta_{g,n} (sum_{k in g} x'_tk u_kn - z_{g,n} sum_{k in g} x'_tk)
+// on CUDA cores for N <= 4 tokens, fp32 throughout: x' = x / s rounded once
+// (IEEE division), the integer weights exact, delta applied once per group;
+// z is 2^(b-1) for the offset-binary codes, the group's zero point for
+// asymmetric ones.
 //
-// Dequantisation without integer-to-float conversions: for nibble i < 4 of a
-// word (bits 4i..4i+3), (w & (0xF << 4i)) | 0x4B000000 is the float
-// 2^23 + 16^i u exactly (the nibble lies in the mantissa), and subtracting
-// 2^23 + 16^i off leaves 16^i (u - off) exactly; nibbles 4..7 are the same
-// after w >> 16.  The factor 16^i is folded into the activation side,
-// x~_k = (x_k / s_k) 16^-(k % 4) (an exact power-of-two scaling), so every
-// product x~ * 16^i (u - off) equals x' (u - off).  Per word: one shift,
-// eight mask-ORs, four paired subtractions and four paired FMAs per token.
+// Dequantisation with one logic op per weight and no conversion: a float
+// whose bit pattern p is below 2^24 (exponent field 0 or 1) has the value
+// p 2^-149 -- the subnormals and the smallest normal binade form one linear
+// scale.  So for nibble i <= 5 of a 32-bit word (bits 4i .. 4i+3 <= 23),
+// (w & (0xF << 4i)) read as a float is exactly 16^i u 2^-149; nibbles 6 and 7
+// are the same after w >> 8 (bits 16..23: 16^4 u, 16^5 u).  The power of two
+// of each nibble position is folded into the activation side: x~_k =
+// x'_k 16^-e(k) 2^64 with e = 0, 1, 2, 3, 4, 5, 4, 5 for k mod 8 = 0..7 (an
+// exact scaling), so every product x~ (w & mask) is x' u 2^-85 exactly before
+// the one rounding of its FMA.  The offset comes out once per group: the sum
+// of x' over the group's rows is staged with x~, and the group's flush adds
+// delta (2^85 acc - z sum x').  Per word: one shift, eight logic ops and four
+// paired FMAs per token.
 //
 // Work: CTA (column tile, split) owns 128 columns (lane l: columns 4l..4l+3,
-// one 16-byte load per k8 row) and a contiguous range of k8 rows, cut into
-// eight contiguous runs, one per warp.  x~ of the range is
-// staged in shared memory in chunks of kGvChunk8 rows; each row's 8 values
-// are a warp-wide broadcast.  The warps' sums are added in warp order, and
-// with several splits the partial rows [split][N][D_out] are summed in split
-// order by gemv_reduce_kernel: the result does not depend on timing.  No
-// waits between CTAs.
+// one 16-byte load per k8 row) and a contiguous range of k8 rows (a multiple
+// of 32), cut into eight contiguous runs of whole 4-row batches, one per
+// warp.  x~ and the per-row sums of x' of the range are staged in shared
+// memory in chunks of kGvChunk8 rows; each row's 8 values are a warp-wide
+// broadcast.  A warp keeps the next batch of packed words in flight while it
+// works on the current one (the first batch is issued before the staging).
+// The warps' sums are added in warp order, and with several splits the
+// partial rows [split][N][D_out] are summed in split order by
+// gemv_reduce_kernel: the result does not depend on timing.  No waits between
+// CTAs.
 constexpr int kGvThreads = 256;
 constexpr int kGvCols = 128;
-constexpr int kGvChunk8 = 128;                   // k8 rows of x~ staged at a time
-constexpr int kGvUnroll = 4;                     // k8 rows in flight per warp (2 for 3-4 tokens)
+constexpr int kGvChunk8 = 256;                   // k8 rows of x~ staged at a time, 1-2 tokens (a multiple of 32)
+constexpr int kGvBatch = 4;                      // k8 rows per batch of loads
 constexpr int kGvMaxSplit = 32;
 constexpr int kGvMaxTokens = 4;
 
-// magic = 0x4B000000 (2^23), held in a register (see in_register) so that
-// (w & mask) | magic is one three-input logic op with the mask as its one
-// immediate operand.
-__device__ __forceinline__ float nib(uint32_t w, uint32_t mask, uint32_t magic) {
-  return __uint_as_float((w & mask) | magic);
-}
+__device__ __forceinline__ float nibf(uint32_t w, uint32_t mask) { return __uint_as_float(w & mask); }
 
 // kZp: asymmetric codes u = q + z with a zero point per (group, column)
-// (zeros [D_in/G][D_out] uint8); the subtracted bias is 2^23 + 16^i z of the
-// current group instead of 2^23 + 16^i off, so every term is still exact.
+// (zeros [D_in/G][D_out] uint8) in place of 2^(b-1).
 template <int NT, bool kZp>
 __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 3 : 2) w4a16_gemv_kernel(const uint4* __restrict__ X,
                                                                 const float4* __restrict__ s,
                                                                 const uint4* __restrict__ packed,
                                                                 const float4* __restrict__ scales,
                                                                 const uint8_t* __restrict__ zeros, int64_t D_in,
-                                                                int64_t D_out, int gshift, int off,
-                                                                uint32_t magic, int R8, float* __restrict__ out) {
-  constexpr int U = NT <= 2 ? kGvUnroll : kGvUnroll / 2;     // fits two CTAs per SM at 3-4 tokens
-  magic = in_register(magic);
-  __shared__ __align__(16) float xt[NT * kGvChunk8 * 8];       // x~ [NT][chunk rows * 8]
+                                                                int64_t D_out, int gshift, int off, int R8,
+                                                                float* __restrict__ out) {
+  constexpr int U = kGvBatch;
+  constexpr int CH = NT <= 2 ? kGvChunk8 : kGvChunk8 / 2;       // chunk rows (static shared memory <= 48 KiB)
+  __shared__ __align__(16) float xt[NT * CH * 8];               // x~ [NT][chunk rows * 8]
+  __shared__ float xr[NT * CH];                                 // sum of x' over each row's 8 values
   __shared__ __align__(16) float red[8 * NT * kGvCols];         // per-warp sums
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t rows8 = D_in / 8;
@@ -574,134 +579,140 @@ __global__ void __launch_bounds__(kGvThreads, NT == 1 ? 3 : 2) w4a16_gemv_kernel
   const int64_t n4 = static_cast<int64_t>(blockIdx.x) * (kGvCols / 4) + lane;   // column quad
   const bool valid = n4 < D4;
   const float fo = static_cast<float>(off);
-  const float2 bias01 = make_float2(-(8388608.0f + fo), -(8388608.0f + 16.0f * fo));
-  const float2 bias23 = make_float2(-(8388608.0f + 256.0f * fo), -(8388608.0f + 4096.0f * fo));
-  float2 tot[NT][4];
+  float tot[NT][4];
 #pragma unroll
   for (int t = 0; t < NT; ++t)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) tot[t][c] = make_float2(0.0f, 0.0f);
+    for (int c = 0; c < 4; ++c) tot[t][c] = 0.0f;
 
-  for (int64_t cb = rb; cb < re; cb += kGvChunk8) {
-    const int nr = static_cast<int>(re - cb < kGvChunk8 ? re - cb : kGvChunk8);
+  for (int64_t cb = rb; cb < re; cb += CH) {
+    const int nr = static_cast<int>(re - cb < CH ? re - cb : CH);   // a multiple of 4
+    // this warp's rows of the chunk: whole batches
+    const int q = (((nr + 7) >> 3) + U - 1) / U * U;
+    const int r0 = warp * q, r1 = r0 + q < nr ? r0 + q : nr;
+    // the first batch of packed words, before the staging
+    uint4 pw[U];
+    const uint4* pp = packed + (cb + r0) * D4 + n4;
+    if (valid && r0 < r1) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) pw[u] = __ldcs(pp + u * D4);
+    }
     if (cb != rb) __syncthreads();                 // the previous chunk's x~ is no longer read
     for (int i = threadIdx.x; i < NT * nr; i += kGvThreads) {
       const int t = i / nr, r = i - t * nr;
       const uint4 xv = X[t * rows8 + cb + r];
       const float4 s0 = __ldg(s + 2 * (cb + r)), s1 = __ldg(s + 2 * (cb + r) + 1);
-      float4 lo, hi;
-      lo.x = __fdiv_rn(bf16_bits_to_float(xv.x & 0xFFFFu), s0.x);
-      lo.y = __fmul_rn(__fdiv_rn(bf16_bits_to_float(xv.x >> 16), s0.y), 0.0625f);
-      lo.z = __fmul_rn(__fdiv_rn(bf16_bits_to_float(xv.y & 0xFFFFu), s0.z), 0.00390625f);
-      lo.w = __fmul_rn(__fdiv_rn(bf16_bits_to_float(xv.y >> 16), s0.w), 0.000244140625f);
-      hi.x = __fdiv_rn(bf16_bits_to_float(xv.z & 0xFFFFu), s1.x);
-      hi.y = __fmul_rn(__fdiv_rn(bf16_bits_to_float(xv.z >> 16), s1.y), 0.0625f);
-      hi.z = __fmul_rn(__fdiv_rn(bf16_bits_to_float(xv.w & 0xFFFFu), s1.z), 0.00390625f);
-      hi.w = __fmul_rn(__fdiv_rn(bf16_bits_to_float(xv.w >> 16), s1.w), 0.000244140625f);
-      float4* dst = reinterpret_cast<float4*>(xt + (t * kGvChunk8 + r) * 8);
-      dst[0] = lo;
-      dst[1] = hi;
+      const float v0 = __fdiv_rn(bf16_bits_to_float(xv.x & 0xFFFFu), s0.x);
+      const float v1 = __fdiv_rn(bf16_bits_to_float(xv.x >> 16), s0.y);
+      const float v2 = __fdiv_rn(bf16_bits_to_float(xv.y & 0xFFFFu), s0.z);
+      const float v3 = __fdiv_rn(bf16_bits_to_float(xv.y >> 16), s0.w);
+      const float v4 = __fdiv_rn(bf16_bits_to_float(xv.z & 0xFFFFu), s1.x);
+      const float v5 = __fdiv_rn(bf16_bits_to_float(xv.z >> 16), s1.y);
+      const float v6 = __fdiv_rn(bf16_bits_to_float(xv.w & 0xFFFFu), s1.z);
+      const float v7 = __fdiv_rn(bf16_bits_to_float(xv.w >> 16), s1.w);
+      // x' 16^-e 2^64: e = 0, 1, 2, 3, 4, 5, 4, 5 (exact powers of two)
+      float4* dst = reinterpret_cast<float4*>(xt + (t * CH + r) * 8);
+      dst[0] = make_float4(__fmul_rn(v0, 0x1p64f), __fmul_rn(v1, 0x1p60f), __fmul_rn(v2, 0x1p56f),
+                           __fmul_rn(v3, 0x1p52f));
+      dst[1] = make_float4(__fmul_rn(v4, 0x1p48f), __fmul_rn(v5, 0x1p44f), __fmul_rn(v6, 0x1p48f),
+                           __fmul_rn(v7, 0x1p44f));
+      xr[t * CH + r] = ((v0 + v1) + (v2 + v3)) + ((v4 + v5) + (v6 + v7));
     }
     __syncthreads();
-    if (valid) {
-      // warp w: the contiguous rows [w q, min((w + 1) q, nr)) of the chunk,
-      // q = ceil(nr / 8); products are summed per quantisation group and
-      // delta is applied once per group (and at the end of the range).
-      const int q = (nr + 7) >> 3;
-      const int r0 = warp * q, r1 = r0 + q < nr ? r0 + q : nr;
-      float2 acc[NT][4];
+    if (!valid || r0 >= r1) continue;
+    // rows [r0, r1) in batches of U; a group boundary falls only between
+    // batches (g8 and every batch start are multiples of U)
+    float2 acc[NT][4];
+    float xs[NT];
 #pragma unroll
-      for (int t = 0; t < NT; ++t)
+    for (int t = 0; t < NT; ++t) {
+      xs[t] = 0.0f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[t][c] = make_float2(0.0f, 0.0f);
-      int64_t g_cur = -1;                          // the group acc belongs to
-      float4 dcur = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      float2 zb01[4], zb23[4];                     // kZp: the biases of the group's zero points, per column
+      for (int c = 0; c < 4; ++c) acc[t][c] = make_float2(0.0f, 0.0f);
+    }
+    int64_t g_cur = ((cb + r0) * 8) >> gshift;
+    auto flush = [&](int64_t g) {
+      const float4 d = __ldg(scales + g * D4 + n4);
+      float z[4] = {fo, fo, fo, fo};
+      if (kZp) {                                     // the four columns' zero points, one 32-bit load
+        const uint32_t z4 = __ldg(reinterpret_cast<const uint32_t*>(zeros + g * D_out) + n4);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        zb01[c] = bias01;
-        zb23[c] = bias23;
+        for (int c = 0; c < 4; ++c) z[c] = static_cast<float>((z4 >> (8 * c)) & 0xFFu);
       }
-      auto flush = [&]() {
+      const float dv[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float a = __fmul_rn(acc[t][c].x + acc[t][c].y, 0x1p85f);   // sum of x' u over the group
+          tot[t][c] = __fmaf_rn(dv[c], __fmaf_rn(-z[c], xs[t], a), tot[t][c]);
+          acc[t][c] = make_float2(0.0f, 0.0f);
+        }
+        xs[t] = 0.0f;
+      }
+    };
+    for (int r = r0; r < r1; r += U) {
+      const int64_t g = ((cb + r) * 8) >> gshift;
+      if (g != g_cur) {                              // uniform over the warp
+        flush(g_cur);
+        g_cur = g;
+      }
+      uint4 pn[U];                                   // the next batch, in flight during this one
+      const bool more = r + U < r1;
+      if (more) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) pn[u] = __ldcs(pp + (U + u) * D4);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int rr = r + u;
+        float4 xa[NT], xb[NT];
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-          tot[t][0] = __ffma2_rn(acc[t][0], make_float2(dcur.x, dcur.x), tot[t][0]);
-          tot[t][1] = __ffma2_rn(acc[t][1], make_float2(dcur.y, dcur.y), tot[t][1]);
-          tot[t][2] = __ffma2_rn(acc[t][2], make_float2(dcur.z, dcur.z), tot[t][2]);
-          tot[t][3] = __ffma2_rn(acc[t][3], make_float2(dcur.w, dcur.w), tot[t][3]);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) acc[t][c] = make_float2(0.0f, 0.0f);
+          const float4* src = reinterpret_cast<const float4*>(xt + (t * CH + rr) * 8);
+          xa[t] = src[0];
+          xb[t] = src[1];
+          xs[t] += xr[t * CH + rr];
         }
-      };
-      for (int r = r0; r < r1; r += U) {
-        const uint4* pp = packed + (cb + r) * D4 + n4;
-        uint4 pw[U];
+        const uint32_t wv[4] = {pw[u].x, pw[u].y, pw[u].z, pw[u].w};
 #pragma unroll
-        for (int u = 0; u < U; ++u)
-          if (r + u < r1) pw[u] = __ldcs(pp + u * D4);
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int rr = r + u;
-          if (rr >= r1) break;                       // uniform over the warp
-          const int64_t g = ((cb + rr) * 8) >> gshift;
-          if (g != g_cur) {                          // uniform over the warp
-            if (g_cur >= 0) flush();
-            dcur = __ldg(scales + g * D4 + n4);      // used at the group's flush
-            if (kZp) {                               // the four columns' zero points, one 32-bit load
-              const uint32_t z4 = __ldg(reinterpret_cast<const uint32_t*>(zeros + g * D_out) + n4);
-#pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const float z = static_cast<float>((z4 >> (8 * c)) & 0xFFu);
-                zb01[c] = make_float2(-(8388608.0f + z), -(8388608.0f + 16.0f * z));
-                zb23[c] = make_float2(-(8388608.0f + 256.0f * z), -(8388608.0f + 4096.0f * z));
-              }
-            }
-            g_cur = g;
-          }
-          float4 xa[NT], xb[NT];
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t w = wv[c], w8 = w >> 8;
+          const float2 v01 = make_float2(nibf(w, 0xFu), nibf(w, 0xF0u));
+          const float2 v23 = make_float2(nibf(w, 0xF00u), nibf(w, 0xF000u));
+          const float2 v45 = make_float2(nibf(w, 0xF0000u), nibf(w, 0xF00000u));
+          const float2 v67 = make_float2(nibf(w8, 0xF0000u), nibf(w8, 0xF00000u));
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
-            const float4* src = reinterpret_cast<const float4*>(xt + (t * kGvChunk8 + rr) * 8);
-            xa[t] = src[0];
-            xb[t] = src[1];
-          }
-          const uint32_t wv[4] = {pw[u].x, pw[u].y, pw[u].z, pw[u].w};
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint32_t w = wv[c], wh = w >> 16;
-            const float2 b01 = kZp ? zb01[c] : bias01, b23 = kZp ? zb23[c] : bias23;
-            const float2 v01 = __fadd2_rn(make_float2(nib(w, 0xFu, magic), nib(w, 0xF0u, magic)), b01);
-            const float2 v23 = __fadd2_rn(make_float2(nib(w, 0xF00u, magic), nib(w, 0xF000u, magic)), b23);
-            const float2 v45 = __fadd2_rn(make_float2(nib(wh, 0xFu, magic), nib(wh, 0xF0u, magic)), b01);
-            const float2 v67 = __fadd2_rn(make_float2(nib(wh, 0xF00u, magic), nib(wh, 0xF000u, magic)), b23);
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-              float2 a2 = __ffma2_rn(v01, make_float2(xa[t].x, xa[t].y), acc[t][c]);
-              a2 = __ffma2_rn(v23, make_float2(xa[t].z, xa[t].w), a2);
-              a2 = __ffma2_rn(v45, make_float2(xb[t].x, xb[t].y), a2);
-              acc[t][c] = __ffma2_rn(v67, make_float2(xb[t].z, xb[t].w), a2);
-            }
+            float2 a2 = __ffma2_rn(v01, make_float2(xa[t].x, xa[t].y), acc[t][c]);
+            a2 = __ffma2_rn(v23, make_float2(xa[t].z, xa[t].w), a2);
+            a2 = __ffma2_rn(v45, make_float2(xb[t].x, xb[t].y), a2);
+            acc[t][c] = __ffma2_rn(v67, make_float2(xb[t].z, xb[t].w), a2);
           }
         }
       }
-      if (g_cur >= 0) flush();
+      if (more) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) pw[u] = pn[u];
+      }
+      pp += U * D4;
     }
+    flush(g_cur);
   }
 #pragma unroll
   for (int t = 0; t < NT; ++t)
     reinterpret_cast<float4*>(red)[(warp * NT + t) * (kGvCols / 4) + lane] =
-        make_float4(tot[t][0].x + tot[t][0].y, tot[t][1].x + tot[t][1].y, tot[t][2].x + tot[t][2].y,
-                    tot[t][3].x + tot[t][3].y);
+        make_float4(tot[t][0], tot[t][1], tot[t][2], tot[t][3]);
   __syncthreads();
   if (threadIdx.x < NT * 32) {
-    const int t = threadIdx.x >> 5, q = threadIdx.x & 31;
-    const int64_t m4 = static_cast<int64_t>(blockIdx.x) * (kGvCols / 4) + q;
+    const int t = threadIdx.x >> 5, qd = threadIdx.x & 31;
+    const int64_t m4 = static_cast<int64_t>(blockIdx.x) * (kGvCols / 4) + qd;
     if (m4 < D4) {
       const float4* rv = reinterpret_cast<const float4*>(red);
-      float4 a = rv[t * (kGvCols / 4) + q];
+      float4 a = rv[t * (kGvCols / 4) + qd];
 #pragma unroll
       for (int w = 1; w < 8; ++w) {
-        const float4 b = rv[(w * NT + t) * (kGvCols / 4) + q];
+        const float4 b = rv[(w * NT + t) * (kGvCols / 4) + qd];
         a.x += b.x;
         a.y += b.y;
         a.z += b.z;
@@ -776,11 +787,11 @@ cudaError_t launch_gemv_nt(dim3 grid, cudaStream_t st, const void* X, const floa
   if (zeros)
     w4a16_gemv_kernel<NT, true><<<grid, kGvThreads, 0, st>>>(
         static_cast<const uint4*>(X), reinterpret_cast<const float4*>(s), reinterpret_cast<const uint4*>(packed),
-        reinterpret_cast<const float4*>(scales), zeros, D_in, D_out, gshift, off, 0x4B000000u, R8, out);
+        reinterpret_cast<const float4*>(scales), zeros, D_in, D_out, gshift, off, R8, out);
   else
     w4a16_gemv_kernel<NT, false><<<grid, kGvThreads, 0, st>>>(
         static_cast<const uint4*>(X), reinterpret_cast<const float4*>(s), reinterpret_cast<const uint4*>(packed),
-        reinterpret_cast<const float4*>(scales), nullptr, D_in, D_out, gshift, off, 0x4B000000u, R8, out);
+        reinterpret_cast<const float4*>(scales), nullptr, D_in, D_out, gshift, off, R8, out);
   return cudaGetLastError();
 }
 
@@ -796,7 +807,7 @@ int launch_w4a16_gemv(const void* X, const float* s, const uint32_t* packed, con
   if (splits > kGvMaxSplit) splits = kGvMaxSplit;
   if (splits < 1) splits = 1;
   int64_t R8 = (rows8 + splits - 1) / splits;
-  R8 = (R8 + 7) / 8 * 8;
+  R8 = (R8 + 31) / 32 * 32;                      // whole 4-row batches for each of the 8 warps
   splits = (rows8 + R8 - 1) / R8;
   const int gshift = group == 32 ? 5 : group == 64 ? 6 : group == 128 ? 7 : 8;
   const int off = 1 << (bits - 1);
