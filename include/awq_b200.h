@@ -387,8 +387,10 @@ AWQ_API int awq_quantize_pack_zp(const float* W, const float* s, int64_t D_in, i
  *     Y[t][n] = sum_k x_tk / s_k * (u_kn - 2^(bits-1)) * scales[k/group][n]
  * with u the offset-binary codes of `packed` (the layout of
  * awq_quantize_pack).  N <= 4 (decode): a CUDA-core GEMV in fp32 (x / s
- * rounded once, exact integer weights, delta applied once per group), split over
- * k with the split partials summed in a fixed order by a second launch.
+ * rounded once, exact integer weights, delta applied once per group): the
+ * (column tile, k rows) work is shared out evenly over a grid that fills
+ * every SM (stream-K), and a second small launch adds the CTAs' sums of
+ * each tile in a fixed order from the workspace.
  * N > 4: two launches on `stream`, X' = bf16(X / s) into the workspace, then
  * a tensor-core GEMM that dequantises the weights into shared memory as
  * bf16((u - 2^(bits-1)) * bf16(delta)) (one rounding of the product) and
@@ -401,7 +403,7 @@ AWQ_API int awq_quantize_pack_zp(const float* W, const float* s, int64_t D_in, i
  *   D_out     a multiple of 4 (the rows of packed words are read by TMA)
  *   Y         [N][D_out] fp32 output, 4-byte aligned
  *   workspace at least awq_w4a16_workspace_size(N, D_in, D_out) bytes: for
- *             N <= 4 the split partials (up to 32 x N x D_out fp32); else
+ *             N <= 4 the CTAs' sums (1024 x 2 x N x 128 fp32); else
  *             the scaled activations (N x D_in bf16) and, for N <= 64, room
  *             for the partial tiles.  No device is needed to compute the size.
  *   status    [1] int32 device status word (required), as for awq_search

@@ -375,7 +375,7 @@ def w4a16_gemm(X: torch.Tensor, s: torch.Tensor, packed: torch.Tensor, scales: t
                 or not out.is_contiguous():
             raise ValueError("out must be a contiguous float32 [N, D_out] tensor on X's device")
         Y = out
-    status = torch.zeros(1, dtype=torch.int32, device=X.device)
+    status = torch.empty(1, dtype=torch.int32, device=X.device)        # the call clears it
     nbytes = w4a16_workspace_size(N, D_in, D_out, group, zp=zeros is not None)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=X.device)

@@ -995,8 +995,11 @@ static int w4a16_impl(const void* X, const float* s, const uint32_t* packed, con
   int sms = 0;
   AWQ_TRY(device_info(&sms));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), st);
-  if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(status)");
+  cudaError_t e = cudaSuccess;
+  if (!awq::w4a16_clears_status(N)) {
+    e = cudaMemsetAsync(status, 0, sizeof(int32_t), st);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(status)");
+  }
   const char* what = "w4a16 kernel";
   int rc;
   {

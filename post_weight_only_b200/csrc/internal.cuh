@@ -165,8 +165,11 @@ int launch_clip_loss(const uint16_t* op, const uint16_t* Hb, int64_t D_in, int64
 // and with zero points the fp32 rows of 128 + z).  zeros: NULL (offset-binary
 // codes u = q + 2^(b-1)) or [D_in/group][D_out] uint8 zero points of
 // asymmetric codes u = q + z (zrows = D_in / group).  D_out must be a
-// multiple of 4.
+// multiple of 4.  For N <= 4 a CUDA-core GEMV takes the place of the
+// tensor-core kernel; it has nothing to wait on and clears *status itself
+// (w4a16_clears_status), so the caller need not.
 size_t w4a16_scratch_bytes(int64_t N, int64_t D_in, int64_t D_out, int64_t zrows);
+bool w4a16_clears_status(int64_t N);
 int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const float* scales, const uint8_t* zeros,
                  int64_t N, int64_t D_in, int64_t D_out, int bits, int group, float* Y, void* ws, int num_sms,
                  int* status, uint64_t timeout_ns, cudaStream_t st, cudaError_t* cerr, const char** what);

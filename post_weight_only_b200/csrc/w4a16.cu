@@ -536,214 +536,385 @@ __global__ void __launch_bounds__(kW4Threads, 1)
 // delta (2^85 acc - z sum x').  Per word: one shift, eight logic ops and four
 // paired FMAs per token.
 //
-// Work: CTA (column tile, split) owns 128 columns (lane l: columns 4l..4l+3,
-// one 16-byte load per k8 row) and a contiguous range of k8 rows (a multiple
-// of 32), cut into eight contiguous runs of whole 4-row batches, one per
-// warp.  x~ and the per-row sums of x' of the range are staged in shared
-// memory in chunks of kGvChunk8 rows; each row's 8 values are a warp-wide
-// broadcast.  A warp keeps the next batch of packed words in flight while it
-// works on the current one (the first batch is issued before the staging).
-// The warps' sums are added in warp order, and with several splits the
-// partial rows [split][N][D_out] are summed in split order by
-// gemv_reduce_kernel: the result does not depend on timing.  No waits between
-// CTAs.
+// Work: the (column tile, 4-row batch) pairs, tile-major, are cut into
+// equal contiguous shares, one per CTA of a grid that fills every SM
+// (stream-K), and each CTA's share into eight, one per warp; a share may
+// end in one tile and go on in the next.  Lane l of a warp owns columns
+// 4l..4l+3 of the tile.  Each thread streams its own 16 bytes of each packed
+// row through a ring of gv_slots batches in shared memory (cp.async, waited
+// on with cp.async.wait_group: nothing to spin on), so the bytes in flight
+// do not cost registers.  A warp stages x~ of its rows 32 at a time, in
+// chunks aligned to the tile's 8-batch boundaries (one row per lane), and
+// with it the sum of x' over each group's rows of the chunk (a fixed
+// butterfly over the lanes); the group size is a template argument, so
+// group boundaries cost a mask test.
+// The warps' sums of a tile are added in warp order, each CTA writes its
+// sums of the (at most two) tiles it worked on to the workspace, and
+// gemv_reduce_kernel adds, per tile, the sums of the CTAs that share it in
+// CTA order: the result does not depend on timing.  A grid of whole tiles
+// (as many CTAs as tiles) stores Y itself.  The kernel also clears the
+// status word (it has nothing to wait on).
 constexpr int kGvThreads = 256;
 constexpr int kGvCols = 128;
-constexpr int kGvChunk8 = 256;                   // k8 rows of x~ staged at a time, 1-2 tokens (a multiple of 32)
-constexpr int kGvBatch = 4;                      // k8 rows per batch of loads
-constexpr int kGvMaxSplit = 32;
+constexpr int kGvBatch = 4;                      // k8 rows per ring slot
+constexpr int kGvXRows = 32;                     // k8 rows of x~ a warp stages at a time (8 batches)
 constexpr int kGvMaxTokens = 4;
+constexpr int kGvMaxCtas = 1024;                 // bounds the workspace of CTA sums
+constexpr int kGvSlotBytes = kGvBatch * kGvCols * 4;
+
+// Ring slots per warp (two CTAs of 8 warps fit an SM).
+template <int NT>
+constexpr int gv_slots() { return NT == 1 ? 6 : NT == 2 ? 5 : NT == 3 ? 4 : 3; }
+
+template <int NT>
+constexpr size_t gv_smem_bytes() {
+  return static_cast<size_t>(8) * gv_slots<NT>() * kGvSlotBytes   // ring (later the warps' sums of the next tile)
+         + static_cast<size_t>(8) * NT * kGvXRows * 8 * 4        // x~
+         + static_cast<size_t>(8) * NT * 8 * 4                   // sums of x' per group of the chunk
+         + static_cast<size_t>(8) * NT * 32 * 16;                // the warps' sums of the CTA's first tile
+}
 
 __device__ __forceinline__ float nibf(uint32_t w, uint32_t mask) { return __uint_as_float(w & mask); }
 
 // kZp: asymmetric codes u = q + z with a zero point per (group, column)
-// (zeros [D_in/G][D_out] uint8) in place of 2^(b-1).
-template <int NT, bool kZp>
-__global__ void __launch_bounds__(kGvThreads, NT == 1 ? 3 : 2) w4a16_gemv_kernel(const uint4* __restrict__ X,
-                                                                const float4* __restrict__ s,
-                                                                const uint4* __restrict__ packed,
-                                                                const float4* __restrict__ scales,
-                                                                const uint8_t* __restrict__ zeros, int64_t D_in,
-                                                                int64_t D_out, int gshift, int off, int R8,
-                                                                float* __restrict__ out) {
-  constexpr int U = kGvBatch;
-  constexpr int CH = NT <= 2 ? kGvChunk8 : kGvChunk8 / 2;       // chunk rows (static shared memory <= 48 KiB)
-  __shared__ __align__(16) float xt[NT * CH * 8];               // x~ [NT][chunk rows * 8]
-  __shared__ float xr[NT * CH];                                 // sum of x' over each row's 8 values
-  __shared__ __align__(16) float red[8 * NT * kGvCols];         // per-warp sums
+// (zeros [D_in/G][D_out] uint8) in place of 2^(b-1).  part: [gridDim.x][2]
+// [NT][128] fp32 CTA sums (slot 0: the CTA's first tile, 1: the next), or
+// Y itself when `direct` (one CTA per tile).
+template <int NT, int G, bool kZp>
+__global__ void __launch_bounds__(kGvThreads, 2) w4a16_gemv_kernel(
+    const uint4* __restrict__ X, const float4* __restrict__ s, const uint32_t* __restrict__ packed,
+    const float4* __restrict__ scales, const uint8_t* __restrict__ zeros, int64_t D_in, int64_t D_out, int off,
+    float* __restrict__ part, float* __restrict__ Y, int y16, int direct, int S, int* __restrict__ status) {
+  constexpr int U = kGvBatch, P = gv_slots<NT>(), XR = kGvXRows, CB = XR / U;
+  constexpr int GB = G / (8 * U);                  // batches per group: 1, 2, 4 or 8
+  constexpr int GR = G / 8;                        // k8 rows per group: 4 .. 32
+  static_assert(GB >= 1 && CB % GB == 0, "whole groups per chunk");
+  extern __shared__ __align__(16) uint8_t gv_sm[];
+  uint8_t* ring = gv_sm;
+  float* xt_all = reinterpret_cast<float*>(gv_sm + 8 * P * kGvSlotBytes);
+  float* xg_all = xt_all + 8 * NT * XR * 8;
+  float4* first = reinterpret_cast<float4*>(xg_all + 8 * NT * 8);   // [8 warps][NT][32 quads]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (status && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
   const int64_t rows8 = D_in / 8;
   const int64_t D4 = D_out / 4;
-  const int64_t rb = static_cast<int64_t>(blockIdx.y) * R8;      // first k8 row of this split
-  const int64_t re = rb + R8 < rows8 ? rb + R8 : rows8;
-  const int64_t n4 = static_cast<int64_t>(blockIdx.x) * (kGvCols / 4) + lane;   // column quad
-  const bool valid = n4 < D4;
+  const int NB = static_cast<int>(rows8 / U);      // batches per tile (rows8 is a multiple of 4)
+  const int64_t tiles = (D_out + kGvCols - 1) / kGvCols;
+  const int64_t W = tiles * NB;
+  const int64_t C = gridDim.x, i = blockIdx.x;
+  int64_t cs, ce;                                  // this CTA's share
+  if (S > 0) {                                     // split S of a tile: cluster rank y of tile i / S
+    const int64_t tau = i / S, y = i % S;
+    cs = tau * NB + NB * y / S;
+    ce = tau * NB + NB * (y + 1) / S;
+  } else {
+    cs = W * i / C;
+    ce = W * (i + 1) / C;
+  }
+  const int64_t t0 = cs / NB;                      // its first tile
+  const int64_t ws = cs + (ce - cs) * warp / 8, we = cs + (ce - cs) * (warp + 1) / 8;   // this warp's
+  const int nw = static_cast<int>(we - ws);
+  uint8_t* wring = ring + warp * P * kGvSlotBytes + lane * 16;
+  float* xt = xt_all + warp * NT * XR * 8;
+  float* xg = xg_all + warp * NT * 8;
   const float fo = static_cast<float>(off);
-  float tot[NT][4];
+  const int64_t rstep = U * D_out;                 // words from one batch to the next
+
+  // the ring: this thread's 16 bytes of each row of batch n of the warp's
+  // share go to slot n % P
+  int n_iss = 0, islot = 0;
+  int iss_b = static_cast<int>(ws % NB);           // tile batch of the next copy
+  int64_t iss_q4 = (ws / NB) * (kGvCols / 4) + lane;
+  bool iss_ok = iss_q4 < D4;
+  const uint32_t* isrc = packed + iss_b * rstep + (iss_ok ? 4 * iss_q4 : 0);
+  auto issue = [&]() {
+    if (n_iss < nw) {
+      uint8_t* dst = wring + islot * kGvSlotBytes;
+      const uint32_t bytes = iss_ok ? 16u : 0u;    // columns past D_out: zero fill from a valid address
+#pragma unroll
+      for (int u = 0; u < U; ++u) cp_async16(dst + u * (kGvCols * 4), isrc + u * D_out, bytes);
+      ++n_iss;
+      if (++islot == P) islot = 0;
+      isrc += rstep;
+      if (++iss_b == NB) {                         // on to the next tile
+        iss_b = 0;
+        iss_q4 += kGvCols / 4;
+        iss_ok = iss_q4 < D4;
+        isrc = packed + (iss_ok ? 4 * iss_q4 : 0);
+      }
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int q = 0; q < P - 1; ++q) issue();
+  int rslot = 0;                                   // slot of the next batch to use
+
+#pragma unroll
+  for (int t = 0; t < NT; ++t) first[(warp * NT + t) * 32 + lane] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  float tt[NT][4];                                 // the current segment's sums (a warp meets a tile once)
+  float2 acc[NT][4];
 #pragma unroll
   for (int t = 0; t < NT; ++t)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) tot[t][c] = 0.0f;
+    for (int c = 0; c < 4; ++c) {
+      tt[t][c] = 0.0f;
+      acc[t][c] = make_float2(0.0f, 0.0f);
+    }
+  bool next_tile = false;                          // tt holds sums of the CTA's second tile
+  float dv[4] = {0.0f, 0.0f, 0.0f, 0.0f};          // the current group's deltas and zero points
+  float zv[4] = {fo, fo, fo, fo};
 
-  for (int64_t cb = rb; cb < re; cb += CH) {
-    const int nr = static_cast<int>(re - cb < CH ? re - cb : CH);   // a multiple of 4
-    // this warp's rows of the chunk: whole batches
-    const int q = (((nr + 7) >> 3) + U - 1) / U * U;
-    const int r0 = warp * q, r1 = r0 + q < nr ? r0 + q : nr;
-    // the first batch of packed words, before the staging
-    uint4 pw[U];
-    const uint4* pp = packed + (cb + r0) * D4 + n4;
-    if (valid && r0 < r1) {
-#pragma unroll
-      for (int u = 0; u < U; ++u) pw[u] = __ldcs(pp + u * D4);
-    }
-    if (cb != rb) __syncthreads();                 // the previous chunk's x~ is no longer read
-    for (int i = threadIdx.x; i < NT * nr; i += kGvThreads) {
-      const int t = i / nr, r = i - t * nr;
-      const uint4 xv = X[t * rows8 + cb + r];
-      const float4 s0 = __ldg(s + 2 * (cb + r)), s1 = __ldg(s + 2 * (cb + r) + 1);
-      const float v0 = __fdiv_rn(bf16_bits_to_float(xv.x & 0xFFFFu), s0.x);
-      const float v1 = __fdiv_rn(bf16_bits_to_float(xv.x >> 16), s0.y);
-      const float v2 = __fdiv_rn(bf16_bits_to_float(xv.y & 0xFFFFu), s0.z);
-      const float v3 = __fdiv_rn(bf16_bits_to_float(xv.y >> 16), s0.w);
-      const float v4 = __fdiv_rn(bf16_bits_to_float(xv.z & 0xFFFFu), s1.x);
-      const float v5 = __fdiv_rn(bf16_bits_to_float(xv.z >> 16), s1.y);
-      const float v6 = __fdiv_rn(bf16_bits_to_float(xv.w & 0xFFFFu), s1.z);
-      const float v7 = __fdiv_rn(bf16_bits_to_float(xv.w >> 16), s1.w);
-      // x' 16^-e 2^64: e = 0, 1, 2, 3, 4, 5, 4, 5 (exact powers of two)
-      float4* dst = reinterpret_cast<float4*>(xt + (t * CH + r) * 8);
-      dst[0] = make_float4(__fmul_rn(v0, 0x1p64f), __fmul_rn(v1, 0x1p60f), __fmul_rn(v2, 0x1p56f),
-                           __fmul_rn(v3, 0x1p52f));
-      dst[1] = make_float4(__fmul_rn(v4, 0x1p48f), __fmul_rn(v5, 0x1p44f), __fmul_rn(v6, 0x1p48f),
-                           __fmul_rn(v7, 0x1p44f));
-      xr[t * CH + r] = ((v0 + v1) + (v2 + v3)) + ((v4 + v5) + (v6 + v7));
-    }
-    __syncthreads();
-    if (!valid || r0 >= r1) continue;
-    // rows [r0, r1) in batches of U; a group boundary falls only between
-    // batches (g8 and every batch start are multiples of U)
-    float2 acc[NT][4];
-    float xs[NT];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      xs[t] = 0.0f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[t][c] = make_float2(0.0f, 0.0f);
-    }
-    int64_t g_cur = ((cb + r0) * 8) >> gshift;
-    auto flush = [&](int64_t g) {
-      const float4 d = __ldg(scales + g * D4 + n4);
-      float z[4] = {fo, fo, fo, fo};
-      if (kZp) {                                     // the four columns' zero points, one 32-bit load
-        const uint32_t z4 = __ldg(reinterpret_cast<const uint32_t*>(zeros + g * D_out) + n4);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) z[c] = static_cast<float>((z4 >> (8 * c)) & 0xFFu);
-      }
-      const float dv[4] = {d.x, d.y, d.z, d.w};
-#pragma unroll
-      for (int t = 0; t < NT; ++t) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const float a = __fmul_rn(acc[t][c].x + acc[t][c].y, 0x1p85f);   // sum of x' u over the group
-          tot[t][c] = __fmaf_rn(dv[c], __fmaf_rn(-z[c], xs[t], a), tot[t][c]);
-          acc[t][c] = make_float2(0.0f, 0.0f);
+  int64_t pos = ws;
+  while (pos < we) {                               // one segment: batches [b0, b1) of tile tau
+    const int64_t tau = pos / NB;
+    const int b0 = static_cast<int>(pos - tau * NB);
+    const int b1 = static_cast<int>(we - tau * NB < NB ? we - tau * NB : NB);
+    const int64_t q4 = tau * (kGvCols / 4) + lane;
+    const bool valid = q4 < D4;
+    for (int ch = b0 / CB; ch * CB < b1; ++ch) {   // chunks of 8 batches aligned to the tile
+      // stage x~ of the chunk's rows that lie in the segment: lane = row
+      __syncwarp();                                // the previous chunk is no longer read
+      {
+        const int r = ch * XR + lane;              // k8 row
+        const bool in = r >= b0 * U && r < b1 * U;
+        float4 s0 = make_float4(1.0f, 1.0f, 1.0f, 1.0f), s1 = s0;
+        if (in) {
+          s0 = __ldg(s + 2 * r);
+          s1 = __ldg(s + 2 * r + 1);
         }
-        xs[t] = 0.0f;
-      }
-    };
-    for (int r = r0; r < r1; r += U) {
-      const int64_t g = ((cb + r) * 8) >> gshift;
-      if (g != g_cur) {                              // uniform over the warp
-        flush(g_cur);
-        g_cur = g;
-      }
-      uint4 pn[U];                                   // the next batch, in flight during this one
-      const bool more = r + U < r1;
-      if (more) {
-#pragma unroll
-        for (int u = 0; u < U; ++u) pn[u] = __ldcs(pp + (U + u) * D4);
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int rr = r + u;
-        float4 xa[NT], xb[NT];
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-          const float4* src = reinterpret_cast<const float4*>(xt + (t * CH + rr) * 8);
-          xa[t] = src[0];
-          xb[t] = src[1];
-          xs[t] += xr[t * CH + rr];
-        }
-        const uint32_t wv[4] = {pw[u].x, pw[u].y, pw[u].z, pw[u].w};
+          float xsum = 0.0f;
+          if (in) {
+            const uint4 xv = X[t * rows8 + r];
+            const float v0 = __fdiv_rn(bf16_bits_to_float(xv.x & 0xFFFFu), s0.x);
+            const float v1 = __fdiv_rn(bf16_bits_to_float(xv.x >> 16), s0.y);
+            const float v2 = __fdiv_rn(bf16_bits_to_float(xv.y & 0xFFFFu), s0.z);
+            const float v3 = __fdiv_rn(bf16_bits_to_float(xv.y >> 16), s0.w);
+            const float v4 = __fdiv_rn(bf16_bits_to_float(xv.z & 0xFFFFu), s1.x);
+            const float v5 = __fdiv_rn(bf16_bits_to_float(xv.z >> 16), s1.y);
+            const float v6 = __fdiv_rn(bf16_bits_to_float(xv.w & 0xFFFFu), s1.z);
+            const float v7 = __fdiv_rn(bf16_bits_to_float(xv.w >> 16), s1.w);
+            // x' 16^-e 2^64: e = 0, 1, 2, 3, 4, 5, 4, 5 (exact powers of two)
+            float4* dst = reinterpret_cast<float4*>(xt + (t * XR + lane) * 8);
+            dst[0] = make_float4(__fmul_rn(v0, 0x1p64f), __fmul_rn(v1, 0x1p60f), __fmul_rn(v2, 0x1p56f),
+                                 __fmul_rn(v3, 0x1p52f));
+            dst[1] = make_float4(__fmul_rn(v4, 0x1p48f), __fmul_rn(v5, 0x1p44f), __fmul_rn(v6, 0x1p48f),
+                                 __fmul_rn(v7, 0x1p44f));
+            xsum = ((v0 + v1) + (v2 + v3)) + ((v4 + v5) + (v6 + v7));
+          }
+          // the sum of x' over each group's rows of the chunk (rows outside the
+          // segment count 0), by a butterfly over the group's GR lanes
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t w = wv[c], w8 = w >> 8;
-          const float2 v01 = make_float2(nibf(w, 0xFu), nibf(w, 0xF0u));
-          const float2 v23 = make_float2(nibf(w, 0xF00u), nibf(w, 0xF000u));
-          const float2 v45 = make_float2(nibf(w, 0xF0000u), nibf(w, 0xF00000u));
-          const float2 v67 = make_float2(nibf(w8, 0xF0000u), nibf(w8, 0xF00000u));
+          for (int o = 1; o < GR; o <<= 1) xsum += __shfl_xor_sync(0xffffffffu, xsum, o);
+          if (lane % GR == 0) xg[t * 8 + lane / GR] = xsum;
+        }
+      }
+      __syncwarp();
+      const int k0 = b0 > ch * CB ? b0 - ch * CB : 0;
+      const int k1 = b1 - ch * CB < CB ? b1 - ch * CB : CB;
+#pragma unroll 1
+      for (int k = k0; k < k1; ++k) {              // not unrolled: the loop body stays in the instruction cache
+        const int b = ch * CB + k;
+        if ((k & (GB - 1)) == 0 || b == b0) {      // a group's first batch here: its deltas (and zero points)
+          if (valid) {
+            const int64_t g = b / GB;
+            const float4 d = __ldg(scales + g * D4 + q4);
+            dv[0] = d.x;
+            dv[1] = d.y;
+            dv[2] = d.z;
+            dv[3] = d.w;
+            if (kZp) {                             // the four columns' zero points, one 32-bit load
+              const uint32_t z4 = __ldg(reinterpret_cast<const uint32_t*>(zeros + g * D_out) + q4);
+#pragma unroll
+              for (int c = 0; c < 4; ++c) zv[c] = static_cast<float>((z4 >> (8 * c)) & 0xFFu);
+            }
+          }
+        }
+        issue();                                   // the batch P - 1 ahead, into the slot used last
+        cp_async_wait<P - 1>();                    // this thread's copies of this batch have landed
+        const uint8_t* slot = wring + rslot * kGvSlotBytes;
+        if (++rslot == P) rslot = 0;
+        uint4 pw[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) pw[u] = *reinterpret_cast<const uint4*>(slot + u * (kGvCols * 4));
+        const float* xk = xt + k * U * 8;          // x~ of the batch's first row
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          float4 xa[NT], xb[NT];
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
-            float2 a2 = __ffma2_rn(v01, make_float2(xa[t].x, xa[t].y), acc[t][c]);
-            a2 = __ffma2_rn(v23, make_float2(xa[t].z, xa[t].w), a2);
-            a2 = __ffma2_rn(v45, make_float2(xb[t].x, xb[t].y), a2);
-            acc[t][c] = __ffma2_rn(v67, make_float2(xb[t].z, xb[t].w), a2);
+            const float4* src = reinterpret_cast<const float4*>(xk + (t * XR + u) * 8);
+            xa[t] = src[0];
+            xb[t] = src[1];
+          }
+          const uint32_t wv[4] = {pw[u].x, pw[u].y, pw[u].z, pw[u].w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t w = wv[c], w8 = w >> 8;
+            const float2 v01 = make_float2(nibf(w, 0xFu), nibf(w, 0xF0u));
+            const float2 v23 = make_float2(nibf(w, 0xF00u), nibf(w, 0xF000u));
+            const float2 v45 = make_float2(nibf(w, 0xF0000u), nibf(w, 0xF00000u));
+            const float2 v67 = make_float2(nibf(w8, 0xF0000u), nibf(w8, 0xF00000u));
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+              float2 a2 = __ffma2_rn(v01, make_float2(xa[t].x, xa[t].y), acc[t][c]);
+              a2 = __ffma2_rn(v23, make_float2(xa[t].z, xa[t].w), a2);
+              a2 = __ffma2_rn(v45, make_float2(xb[t].x, xb[t].y), a2);
+              acc[t][c] = __ffma2_rn(v67, make_float2(xb[t].z, xb[t].w), a2);
+            }
+          }
+        }
+        if (((k + 1) & (GB - 1)) == 0 || b == b1 - 1) {   // a group's last batch here: delta (sum x' u - z sum x')
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            const float xs = xg[t * 8 + k / GB];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float a = __fmul_rn(acc[t][c].x + acc[t][c].y, 0x1p85f);   // sum of x' u over the group
+              tt[t][c] = __fmaf_rn(dv[c], __fmaf_rn(-zv[c], xs, a), tt[t][c]);
+              acc[t][c] = make_float2(0.0f, 0.0f);
+            }
           }
         }
       }
-      if (more) {
-#pragma unroll
-        for (int u = 0; u < U; ++u) pw[u] = pn[u];
-      }
-      pp += U * D4;
     }
-    flush(g_cur);
+    pos += b1 - b0;
+    if (tau == t0) {                               // the CTA's first tile: to shared memory
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        first[(warp * NT + t) * 32 + lane] = make_float4(tt[t][0], tt[t][1], tt[t][2], tt[t][3]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tt[t][c] = 0.0f;
+      }
+    } else {
+      next_tile = true;                            // the second tile: the warp's last segment
+    }
   }
+  cp_async_wait<0>();
+  __syncthreads();                                 // the ring is free: the warps' sums of the next tile there
+  float4* second = reinterpret_cast<float4*>(ring);   // [8 warps][NT][32 quads]
 #pragma unroll
   for (int t = 0; t < NT; ++t)
-    reinterpret_cast<float4*>(red)[(warp * NT + t) * (kGvCols / 4) + lane] =
-        make_float4(tot[t][0], tot[t][1], tot[t][2], tot[t][3]);
+    second[(warp * NT + t) * 32 + lane] = next_tile ? make_float4(tt[t][0], tt[t][1], tt[t][2], tt[t][3])
+                                                    : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   __syncthreads();
-  if (threadIdx.x < NT * 32) {
+  if (S > 0) {                                     // a cluster of S splits of one tile
+    float4* fin = second + 8 * NT * 32;            // this CTA's sums, read by rank 0 (DSMEM)
     const int t = threadIdx.x >> 5, qd = threadIdx.x & 31;
-    const int64_t m4 = static_cast<int64_t>(blockIdx.x) * (kGvCols / 4) + qd;
-    if (m4 < D4) {
-      const float4* rv = reinterpret_cast<const float4*>(red);
-      float4 a = rv[t * (kGvCols / 4) + qd];
+    float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (threadIdx.x < NT * 32) {
+      a = first[t * 32 + qd];
 #pragma unroll
       for (int w = 1; w < 8; ++w) {
-        const float4 b = rv[(w * NT + t) * (kGvCols / 4) + qd];
+        const float4 b = first[(w * NT + t) * 32 + qd];
         a.x += b.x;
         a.y += b.y;
         a.z += b.z;
         a.w += b.w;
       }
-      reinterpret_cast<float4*>(out)[(static_cast<int64_t>(blockIdx.y) * NT + t) * D4 + m4] = a;
+      fin[threadIdx.x] = a;
     }
+    cluster_sync_all();                            // every rank's sums are in its shared memory
+    const bool rank0 = cluster_ctarank() == 0;
+    if (rank0 && threadIdx.x < NT * 32) {
+      const uint32_t local = smem_u32(&fin[threadIdx.x]);
+      for (int r = 1; r < S; ++r) {
+        const float4 b = ld_shared_cluster_f4(mapa_shared(local, static_cast<uint32_t>(r)));
+        a.x += b.x;
+        a.y += b.y;
+        a.z += b.z;
+        a.w += b.w;
+      }
+      const int64_t m4 = t0 * (kGvCols / 4) + qd;
+      if (m4 < D4) {
+        if (y16) {
+          reinterpret_cast<float4*>(Y)[t * D4 + m4] = a;
+        } else {
+          float* yo = Y + t * D_out + 4 * m4;
+          yo[0] = a.x;
+          yo[1] = a.y;
+          yo[2] = a.z;
+          yo[3] = a.w;
+        }
+      }
+    }
+    cluster_sync_all();                            // no rank leaves while rank 0 may read its sums
+    return;
   }
-}
-
-// Y = sum over splits of the partial rows, in split order.  y16: Y is 16-byte
-// aligned (else four scalar stores; the API asks only 4-byte alignment of Y).
-__global__ void __launch_bounds__(256) gemv_reduce_kernel(const float4* __restrict__ part, int splits, int64_t n4,
-                                                          float* __restrict__ Y, int y16) {
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    float4 a = part[i];
-    for (int k = 1; k < splits; ++k) {
-      const float4 b = part[k * n4 + i];
+  if (threadIdx.x < 2 * NT * 32) {                 // (tile k, token t, quad) in warp order
+    const int k = threadIdx.x / (NT * 32), t = (threadIdx.x / 32) % NT, qd = threadIdx.x & 31;
+    const float4* red = k == 0 ? first : second;
+    float4 a = red[t * 32 + qd];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) {
+      const float4 b = red[(w * NT + t) * 32 + qd];
       a.x += b.x;
       a.y += b.y;
       a.z += b.z;
       a.w += b.w;
     }
-    if (y16) {
-      reinterpret_cast<float4*>(Y)[i] = a;
+    if (direct) {                                  // one CTA per tile: this CTA's sums are Y
+      const int64_t m4 = t0 * (kGvCols / 4) + qd;
+      if (k == 0 && m4 < D4) {
+        if (y16) {
+          reinterpret_cast<float4*>(Y)[t * D4 + m4] = a;
+        } else {
+          float* yo = Y + t * D_out + 4 * m4;
+          yo[0] = a.x;
+          yo[1] = a.y;
+          yo[2] = a.z;
+          yo[3] = a.w;
+        }
+      }
     } else {
-      Y[4 * i] = a.x;
-      Y[4 * i + 1] = a.y;
-      Y[4 * i + 2] = a.z;
-      Y[4 * i + 3] = a.w;
+      reinterpret_cast<float4*>(part)[((i * 2 + k) * NT + t) * 32 + qd] = a;
+    }
+  }
+  pdl_launch_dependents();
+}
+
+// Y[t][n] = the sums of tile n / 128 of the CTAs whose shares touch it, in
+// CTA order (the shares of the GEMV's partition, recomputed).  Launched as a
+// programmatic dependent of the GEMV: it waits for the GEMV's writes.
+template <int NT>
+__global__ void __launch_bounds__(256) gemv_reduce_kernel(const float4* __restrict__ part, int64_t D_out,
+                                                          int64_t NB, int64_t C, float* __restrict__ Y, int y16) {
+  pdl_wait_primary();
+  const int64_t D4 = D_out / 4;
+  const int64_t tiles = (D_out + kGvCols - 1) / kGvCols;
+  const int64_t W = tiles * NB;
+  for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < NT * D4;
+       o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = o / D4, m4 = o - t * D4;
+    const int64_t tau = m4 / (kGvCols / 4), qd = m4 % (kGvCols / 4);
+    // the first CTA whose share ends past the tile's first batch
+    int64_t c = tau * NB * C / W;
+    while (c > 0 && W * c / C > tau * NB) --c;
+    while (W * (c + 1) / C <= tau * NB) ++c;
+    float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    bool first = true;
+    for (; c < C && W * c / C < (tau + 1) * NB; ++c) {
+      const int64_t k = tau - (W * c / C) / NB;    // 0: the CTA's first tile, 1: the next
+      const float4 b = part[((c * 2 + k) * NT + t) * 32 + qd];
+      if (first) {
+        a = b;
+        first = false;
+      } else {
+        a.x += b.x;
+        a.y += b.y;
+        a.z += b.z;
+        a.w += b.w;
+      }
+    }
+    if (y16) {
+      reinterpret_cast<float4*>(Y)[t * D4 + m4] = a;
+    } else {
+      float* yo = Y + t * D_out + 4 * m4;
+      yo[0] = a.x;
+      yo[1] = a.y;
+      yo[2] = a.z;
+      yo[3] = a.w;
     }
   }
 }
@@ -763,9 +934,9 @@ int w4_token_tile(int64_t N) { return N >= 256 ? 256 : static_cast<int>((N + 15)
 // zrows: rows of zero points (D_in / group) of the asymmetric consumer, else 0.
 W4Layout w4_layout(int64_t N, int64_t D_in, int64_t D_out, int64_t zrows = 0) {
   W4Layout l;
-  if (N <= kGvMaxTokens) {                        // the GEMV: partial rows of up to kGvMaxSplit splits
+  if (N <= kGvMaxTokens) {                        // the GEMV: two tiles of sums per CTA
     l.xs = l.count = l.partial = l.zb = 0;
-    l.total = round256(static_cast<size_t>(kGvMaxSplit) * N * D_out * 4);
+    l.total = round256(static_cast<size_t>(kGvMaxCtas) * 2 * N * kGvCols * 4);
     return l;
   }
   const int Nt = w4_token_tile(N);
@@ -780,69 +951,187 @@ W4Layout w4_layout(int64_t N, int64_t D_in, int64_t D_out, int64_t zrows = 0) {
   return l;
 }
 
-template <int NT>
-cudaError_t launch_gemv_nt(dim3 grid, cudaStream_t st, const void* X, const float* s, const uint32_t* packed,
-                           const float* scales, const uint8_t* zeros, int64_t D_in, int64_t D_out, int gshift, int off,
-                           int R8, float* out) {
-  if (zeros)
-    w4a16_gemv_kernel<NT, true><<<grid, kGvThreads, 0, st>>>(
-        static_cast<const uint4*>(X), reinterpret_cast<const float4*>(s), reinterpret_cast<const uint4*>(packed),
-        reinterpret_cast<const float4*>(scales), zeros, D_in, D_out, gshift, off, R8, out);
-  else
-    w4a16_gemv_kernel<NT, false><<<grid, kGvThreads, 0, st>>>(
-        static_cast<const uint4*>(X), reinterpret_cast<const float4*>(s), reinterpret_cast<const uint4*>(packed),
-        reinterpret_cast<const float4*>(scales), nullptr, D_in, D_out, gshift, off, R8, out);
-  return cudaGetLastError();
+// CTAs of the (NT, G, kZp) GEMV resident on one SM, and clusters of c
+// CTAs resident on the GPU, per device (0: not yet asked).
+constexpr int kGvMaxDevices = 64;
+constexpr int kGvMaxCluster = 8;                 // portable cluster size
+std::atomic<int> g_gv_occ[kGvMaxDevices][kGvMaxTokens][2][4];
+std::atomic<int> g_gv_clusters[kGvMaxDevices][kGvMaxTokens][2][4][kGvMaxCluster + 1];
+
+template <typename K>
+cudaError_t gemv_resident_clusters(K kern, int dev, int NT, bool zp, int G, int c, int smem, int* n) {
+  std::atomic<int>& slot =
+      g_gv_clusters[dev][NT - 1][zp ? 1 : 0][G == 32 ? 0 : G == 64 ? 1 : G == 128 ? 2 : 3][c];
+  *n = slot.load(std::memory_order_relaxed);
+  if (*n > 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(c), 1, 1);
+  cfg.blockDim = dim3(kGvThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = static_cast<unsigned>(c);
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaOccupancyMaxActiveClusters(n, kern, &cfg);
+  if (e != cudaSuccess) return e;
+  if (*n < 1) *n = 1;
+  slot.store(*n, std::memory_order_relaxed);
+  return cudaSuccess;
 }
 
-int launch_w4a16_gemv(const void* X, const float* s, const uint32_t* packed, const float* scales,
-                      const uint8_t* zeros, int64_t N, int64_t D_in, int64_t D_out, int bits, int group, float* Y,
-                      void* ws, int num_sms, cudaStream_t st, cudaError_t* cerr, const char** what) {
-  const int64_t rows8 = D_in / 8;
-  const int64_t tiles = (D_out + kGvCols - 1) / kGvCols;
-  // About eight CTAs per SM over column tiles x splits; at least 8 k8 rows
-  // (one per warp) per split.
-  int64_t splits = (static_cast<int64_t>(num_sms > 0 ? num_sms : 1) * 8 + tiles / 2) / tiles;
-  if (splits > rows8 / 8) splits = rows8 / 8;
-  if (splits > kGvMaxSplit) splits = kGvMaxSplit;
-  if (splits < 1) splits = 1;
-  int64_t R8 = (rows8 + splits - 1) / splits;
-  R8 = (R8 + 31) / 32 * 32;                      // whole 4-row batches for each of the 8 warps
-  splits = (rows8 + R8 - 1) / R8;
-  const int gshift = group == 32 ? 5 : group == 64 ? 6 : group == 128 ? 7 : 8;
-  const int off = 1 << (bits - 1);
-  // The GEMV stores 16-byte rows: straight into Y when there is one split and
-  // Y is 16-byte aligned, else into the workspace for gemv_reduce_kernel.
-  const bool y16 = (reinterpret_cast<uintptr_t>(Y) & 15u) == 0;
-  float* out = splits == 1 && y16 ? Y : static_cast<float*>(ws);
-  const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(splits));
-  cudaError_t e;
-  switch (N) {
-    case 1: e = launch_gemv_nt<1>(grid, st, X, s, packed, scales, zeros, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
-    case 2: e = launch_gemv_nt<2>(grid, st, X, s, packed, scales, zeros, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
-    case 3: e = launch_gemv_nt<3>(grid, st, X, s, packed, scales, zeros, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
-    case 4: e = launch_gemv_nt<4>(grid, st, X, s, packed, scales, zeros, D_in, D_out, gshift, off, static_cast<int>(R8), out); break;
-    default: *what = "gemv token count"; return kEUnsupported;
+template <int NT, int G, bool kZp>
+int launch_gemv_k(const void* X, const float* s, const uint32_t* packed, const float* scales, const uint8_t* zeros,
+                  int64_t D_in, int64_t D_out, int bits, float* Y, void* ws, int num_sms, int* status,
+                  cudaStream_t st, cudaError_t* cerr, const char** what) {
+  auto kern = w4a16_gemv_kernel<NT, G, kZp>;
+  const int smem = static_cast<int>(gv_smem_bytes<NT>());
+  static SmemAttrOnce once;
+  cudaError_t e = set_smem_once(kern, smem, once);
+  if (e != cudaSuccess) {
+    *cerr = e;
+    *what = "cudaFuncSetAttribute(w4a16_gemv_kernel)";
+    return kECuda;
   }
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kGvMaxDevices) {
+    *cerr = e != cudaSuccess ? e : cudaErrorInvalidDevice;
+    *what = "cudaGetDevice";
+    return kECuda;
+  }
+  std::atomic<int>& occ_slot = g_gv_occ[dev][NT - 1][kZp ? 1 : 0][G == 32 ? 0 : G == 64 ? 1 : G == 128 ? 2 : 3];
+  int occ = occ_slot.load(std::memory_order_relaxed);
+  if (occ <= 0) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGvThreads, smem);
+    if (e != cudaSuccess) {
+      *cerr = e;
+      *what = "cudaOccupancyMaxActiveBlocksPerMultiprocessor";
+      return kECuda;
+    }
+    if (occ < 1) occ = 1;
+    occ_slot.store(occ, std::memory_order_relaxed);
+  }
+  const int64_t NB = D_in / 8 / kGvBatch;
+  const int64_t tiles = (D_out + kGvCols - 1) / kGvCols;
+  const int off = 1 << (bits - 1);
+  const int y16 = (reinterpret_cast<uintptr_t>(Y) & 15u) == 0 ? 1 : 0;
+  // One launch of S splits per tile, a cluster each, when all clusters are
+  // resident at once (the most splits, at least 8 batches per split): no
+  // second launch, which costs more than the uneven load of the SMs that
+  // clusters of S bring.  Else stream-K and a reduction launch.
+  {
+    int S = 0;
+    for (int c = kGvMaxCluster; c >= 2 && S == 0; --c) {
+      if (NB < 8 * c) continue;
+      int n = 0;
+      e = gemv_resident_clusters(kern, dev, NT, kZp, G, c, smem, &n);
+      if (e != cudaSuccess) {
+        *cerr = e;
+        *what = "cudaOccupancyMaxActiveClusters";
+        return kECuda;
+      }
+      if (n >= tiles) S = c;
+    }
+    if (S > 0) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(tiles * S), 1, 1);
+      cfg.blockDim = dim3(kGvThreads, 1, 1);
+      cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+      cfg.stream = st;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = static_cast<unsigned>(S);
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      e = cudaLaunchKernelEx(&cfg, kern, static_cast<const uint4*>(X), reinterpret_cast<const float4*>(s), packed,
+                             reinterpret_cast<const float4*>(scales), zeros, D_in, D_out, off,
+                             static_cast<float*>(nullptr), Y, y16, 0, S, status);
+      if (e != cudaSuccess) {
+        *cerr = e;
+        *what = "w4a16_gemv_kernel launch (clusters)";
+        return kECuda;
+      }
+      return kOk;
+    }
+  }
+  // Every SM full; as many CTAs as tiles (each a whole tile, Y stored
+  // directly) when the tiles alone fill the GPU.
+  int64_t C = static_cast<int64_t>(occ) * (num_sms > 0 ? num_sms : 1);
+  if (C > kGvMaxCtas) C = kGvMaxCtas;
+  if (C > tiles * NB) C = tiles * NB;              // at least one batch per CTA
+  const bool direct = tiles >= C;
+  if (direct) C = tiles;
+  float* part = static_cast<float*>(ws);
+  kern<<<static_cast<unsigned>(C), kGvThreads, smem, st>>>(
+      static_cast<const uint4*>(X), reinterpret_cast<const float4*>(s), packed,
+      reinterpret_cast<const float4*>(scales), zeros, D_in, D_out, off, part, Y, y16, direct ? 1 : 0, 0, status);
+  e = cudaGetLastError();
   if (e != cudaSuccess) {
     *cerr = e;
     *what = "w4a16_gemv_kernel launch";
     return kECuda;
   }
-  if (out != Y) {
-    const int64_t n4 = N * D_out / 4;
-    int64_t blocks = (n4 + 255) / 256;
-    if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
-    gemv_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(static_cast<const float4*>(ws),
-                                                                     static_cast<int>(splits), n4, Y, y16 ? 1 : 0);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) {
-      *cerr = e;
-      *what = "gemv_reduce_kernel launch";
-      return kECuda;
-    }
+  if (direct) return kOk;
+  const int64_t outs = NT * (D_out / 4);
+  int64_t blocks = (outs + 255) / 256;
+  if (blocks > static_cast<int64_t>(num_sms) * 4) blocks = static_cast<int64_t>(num_sms) * 4;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemv_reduce_kernel<NT>, static_cast<const float4*>(ws), D_out, NB, C, Y, y16);
+  if (e != cudaSuccess) {
+    *cerr = e;
+    *what = "gemv_reduce_kernel launch";
+    return kECuda;
   }
   return kOk;
+}
+
+template <int NT, int G>
+int launch_gemv_g(const void* X, const float* s, const uint32_t* packed, const float* scales, const uint8_t* zeros,
+                  int64_t D_in, int64_t D_out, int bits, float* Y, void* ws, int num_sms, int* status,
+                  cudaStream_t st, cudaError_t* cerr, const char** what) {
+  if (zeros)
+    return launch_gemv_k<NT, G, true>(X, s, packed, scales, zeros, D_in, D_out, bits, Y, ws, num_sms, status, st,
+                                      cerr, what);
+  return launch_gemv_k<NT, G, false>(X, s, packed, scales, nullptr, D_in, D_out, bits, Y, ws, num_sms, status, st,
+                                     cerr, what);
+}
+
+template <int NT>
+int launch_gemv_nt(const void* X, const float* s, const uint32_t* packed, const float* scales, const uint8_t* zeros,
+                   int64_t D_in, int64_t D_out, int bits, int group, float* Y, void* ws, int num_sms, int* status,
+                   cudaStream_t st, cudaError_t* cerr, const char** what) {
+  switch (group) {
+    case 32: return launch_gemv_g<NT, 32>(X, s, packed, scales, zeros, D_in, D_out, bits, Y, ws, num_sms, status, st, cerr, what);
+    case 64: return launch_gemv_g<NT, 64>(X, s, packed, scales, zeros, D_in, D_out, bits, Y, ws, num_sms, status, st, cerr, what);
+    case 128: return launch_gemv_g<NT, 128>(X, s, packed, scales, zeros, D_in, D_out, bits, Y, ws, num_sms, status, st, cerr, what);
+    case 256: return launch_gemv_g<NT, 256>(X, s, packed, scales, zeros, D_in, D_out, bits, Y, ws, num_sms, status, st, cerr, what);
+    default: *what = "gemv group"; return kEUnsupported;
+  }
+}
+
+int launch_w4a16_gemv(const void* X, const float* s, const uint32_t* packed, const float* scales,
+                      const uint8_t* zeros, int64_t N, int64_t D_in, int64_t D_out, int bits, int group, float* Y,
+                      void* ws, int num_sms, int* status, cudaStream_t st, cudaError_t* cerr, const char** what) {
+  switch (N) {
+    case 1: return launch_gemv_nt<1>(X, s, packed, scales, zeros, D_in, D_out, bits, group, Y, ws, num_sms, status, st, cerr, what);
+    case 2: return launch_gemv_nt<2>(X, s, packed, scales, zeros, D_in, D_out, bits, group, Y, ws, num_sms, status, st, cerr, what);
+    case 3: return launch_gemv_nt<3>(X, s, packed, scales, zeros, D_in, D_out, bits, group, Y, ws, num_sms, status, st, cerr, what);
+    case 4: return launch_gemv_nt<4>(X, s, packed, scales, zeros, D_in, D_out, bits, group, Y, ws, num_sms, status, st, cerr, what);
+    default: *what = "gemv token count"; return kEUnsupported;
+  }
 }
 
 }  // namespace
@@ -851,13 +1140,15 @@ size_t w4a16_scratch_bytes(int64_t N, int64_t D_in, int64_t D_out, int64_t zrows
   return w4_layout(N, D_in, D_out, zrows).total;
 }
 
+bool w4a16_clears_status(int64_t N) { return N <= kGvMaxTokens; }
+
 int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const float* scales, const uint8_t* zeros,
                  int64_t N, int64_t D_in, int64_t D_out, int bits, int group, float* Y, void* ws, int num_sms,
                  int* status, uint64_t timeout_ns, cudaStream_t st, cudaError_t* cerr, const char** what) {
   *cerr = cudaSuccess;
   if (N <= kGvMaxTokens)
-    return launch_w4a16_gemv(X, s, packed, scales, zeros, N, D_in, D_out, bits, group, Y, ws, num_sms, st, cerr,
-                             what);
+    return launch_w4a16_gemv(X, s, packed, scales, zeros, N, D_in, D_out, bits, group, Y, ws, num_sms, status, st,
+                             cerr, what);
   const bool zp = zeros != nullptr;
   const W4Layout lay = w4_layout(N, D_in, D_out, zp ? D_in / group : 0);
   uint8_t* wsb = static_cast<uint8_t*>(ws);

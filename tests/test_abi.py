@@ -125,8 +125,8 @@ def test_argument_checks_without_gpu(lib):
     gws.argtypes = [I64, I64, I64]
     gws.restype = SZ
     assert gws(16, 4096, 4096) >= 16 * 4096 * 2            # the scaled activations, bf16
-    for n in (1, 2, 4):                                    # decode GEMV: up to 32 split partials of N x D_out fp32
-        assert gws(n, 4096, 4096) >= 32 * n * 4096 * 4
+    for n in (1, 2, 4):                                    # decode GEMV: two tiles of CTA sums per CTA
+        assert gws(n, 4096, 4096) >= 1024 * 2 * n * 128 * 4
     assert gws(5, 4096, 4096) >= 5 * 4096 * 2              # five tokens: the tensor-core layout
     gargs = dict(X=fake, s=fake, P=fake, sc=fake, N=16, D_in=256, D_out=64, bits=4, group=128, Y=fake, ws=fake,
                  wsb=gws(16, 256, 64), st=fake, stream=None)
