@@ -556,19 +556,27 @@ __global__ void __launch_bounds__(kW4Threads, 1)
 // status word (it has nothing to wait on).
 constexpr int kGvThreads = 256;
 constexpr int kGvCols = 128;
-constexpr int kGvBatch = 4;                      // k8 rows per ring slot
 constexpr int kGvXRows = 32;                     // k8 rows of x~ a warp stages at a time (8 batches)
 constexpr int kGvMaxTokens = 4;
 constexpr int kGvMaxCtas = 1024;                 // bounds the workspace of CTA sums
-constexpr int kGvSlotBytes = kGvBatch * kGvCols * 4;
+
+// k8 rows per batch (one ring slot): 8 when a group holds 8 or more and the
+// registers allow, so that the per-batch bookkeeping is spread over more
+// words; else 4.
+template <int NT, int G>
+constexpr int gv_batch() { return G >= 64 && NT <= 2 ? 8 : 4; }
+template <int NT, int G>
+constexpr int gv_slot_bytes() { return gv_batch<NT, G>() * kGvCols * 4; }
 
 // Ring slots per warp (two CTAs of 8 warps fit an SM).
-template <int NT>
-constexpr int gv_slots() { return NT == 1 ? 6 : NT == 2 ? 5 : NT == 3 ? 4 : 3; }
+template <int NT, int G>
+constexpr int gv_slots() {
+  return gv_batch<NT, G>() == 8 ? (NT == 1 ? 3 : 2) : (NT == 1 ? 6 : NT == 2 ? 5 : NT == 3 ? 4 : 3);
+}
 
-template <int NT>
+template <int NT, int G>
 constexpr size_t gv_smem_bytes() {
-  return static_cast<size_t>(8) * gv_slots<NT>() * kGvSlotBytes   // ring (later the warps' sums of the next tile)
+  return static_cast<size_t>(8) * gv_slots<NT, G>() * gv_slot_bytes<NT, G>()   // ring (later the warps' sums of the next tile)
          + static_cast<size_t>(8) * NT * kGvXRows * 8 * 4        // x~
          + static_cast<size_t>(8) * NT * 8 * 4                   // sums of x' per group of the chunk
          + static_cast<size_t>(8) * NT * 32 * 16;                // the warps' sums of the CTA's first tile
@@ -585,20 +593,21 @@ __global__ void __launch_bounds__(kGvThreads, 2) w4a16_gemv_kernel(
     const uint4* __restrict__ X, const float4* __restrict__ s, const uint32_t* __restrict__ packed,
     const float4* __restrict__ scales, const uint8_t* __restrict__ zeros, int64_t D_in, int64_t D_out, int off,
     float* __restrict__ part, float* __restrict__ Y, int y16, int direct, int S, int* __restrict__ status) {
-  constexpr int U = kGvBatch, P = gv_slots<NT>(), XR = kGvXRows, CB = XR / U;
+  constexpr int U = gv_batch<NT, G>(), P = gv_slots<NT, G>(), XR = kGvXRows, CB = XR / U;
+  constexpr int kSlotBytes = gv_slot_bytes<NT, G>();
   constexpr int GB = G / (8 * U);                  // batches per group: 1, 2, 4 or 8
   constexpr int GR = G / 8;                        // k8 rows per group: 4 .. 32
   static_assert(GB >= 1 && CB % GB == 0, "whole groups per chunk");
   extern __shared__ __align__(16) uint8_t gv_sm[];
   uint8_t* ring = gv_sm;
-  float* xt_all = reinterpret_cast<float*>(gv_sm + 8 * P * kGvSlotBytes);
+  float* xt_all = reinterpret_cast<float*>(gv_sm + 8 * P * kSlotBytes);
   float* xg_all = xt_all + 8 * NT * XR * 8;
   float4* first = reinterpret_cast<float4*>(xg_all + 8 * NT * 8);   // [8 warps][NT][32 quads]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (status && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
   const int64_t rows8 = D_in / 8;
   const int64_t D4 = D_out / 4;
-  const int NB = static_cast<int>(rows8 / U);      // batches per tile (rows8 is a multiple of 4)
+  const int NB = static_cast<int>(rows8 / U);      // batches per tile (rows8 is a multiple of G / 8 >= U)
   const int64_t tiles = (D_out + kGvCols - 1) / kGvCols;
   const int64_t W = tiles * NB;
   const int64_t C = gridDim.x, i = blockIdx.x;
@@ -614,7 +623,7 @@ __global__ void __launch_bounds__(kGvThreads, 2) w4a16_gemv_kernel(
   const int64_t t0 = cs / NB;                      // its first tile
   const int64_t ws = cs + (ce - cs) * warp / 8, we = cs + (ce - cs) * (warp + 1) / 8;   // this warp's
   const int nw = static_cast<int>(we - ws);
-  uint8_t* wring = ring + warp * P * kGvSlotBytes + lane * 16;
+  uint8_t* wring = ring + warp * P * kSlotBytes + lane * 16;
   float* xt = xt_all + warp * NT * XR * 8;
   float* xg = xg_all + warp * NT * 8;
   const float fo = static_cast<float>(off);
@@ -629,7 +638,7 @@ __global__ void __launch_bounds__(kGvThreads, 2) w4a16_gemv_kernel(
   const uint32_t* isrc = packed + iss_b * rstep + (iss_ok ? 4 * iss_q4 : 0);
   auto issue = [&]() {
     if (n_iss < nw) {
-      uint8_t* dst = wring + islot * kGvSlotBytes;
+      uint8_t* dst = wring + islot * kSlotBytes;
       const uint32_t bytes = iss_ok ? 16u : 0u;    // columns past D_out: zero fill from a valid address
 #pragma unroll
       for (int u = 0; u < U; ++u) cp_async16(dst + u * (kGvCols * 4), isrc + u * D_out, bytes);
@@ -733,7 +742,7 @@ __global__ void __launch_bounds__(kGvThreads, 2) w4a16_gemv_kernel(
         }
         issue();                                   // the batch P - 1 ahead, into the slot used last
         cp_async_wait<P - 1>();                    // this thread's copies of this batch have landed
-        const uint8_t* slot = wring + rslot * kGvSlotBytes;
+        const uint8_t* slot = wring + rslot * kSlotBytes;
         if (++rslot == P) rslot = 0;
         uint4 pw[U];
 #pragma unroll
@@ -987,7 +996,7 @@ int launch_gemv_k(const void* X, const float* s, const uint32_t* packed, const f
                   int64_t D_in, int64_t D_out, int bits, float* Y, void* ws, int num_sms, int* status,
                   cudaStream_t st, cudaError_t* cerr, const char** what) {
   auto kern = w4a16_gemv_kernel<NT, G, kZp>;
-  const int smem = static_cast<int>(gv_smem_bytes<NT>());
+  const int smem = static_cast<int>(gv_smem_bytes<NT, G>());
   static SmemAttrOnce once;
   cudaError_t e = set_smem_once(kern, smem, once);
   if (e != cudaSuccess) {
@@ -1014,7 +1023,7 @@ int launch_gemv_k(const void* X, const float* s, const uint32_t* packed, const f
     if (occ < 1) occ = 1;
     occ_slot.store(occ, std::memory_order_relaxed);
   }
-  const int64_t NB = D_in / 8 / kGvBatch;
+  const int64_t NB = D_in / 8 / gv_batch<NT, G>();
   const int64_t tiles = (D_out + kGvCols - 1) / kGvCols;
   const int off = 1 << (bits - 1);
   const int y16 = (reinterpret_cast<uintptr_t>(Y) & 15u) == 0 ? 1 : 0;
