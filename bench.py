@@ -455,18 +455,22 @@ def timed_steps(dj: DeviceJob, steps: int, warmup: int, flush, flush_sink, barri
     return out, step_ms, prof, clk
 
 
+SUSTAINED_MS = 500.0
+
+
 def roofline_of(job: Job, prof, steps: int, timed_ms: float):
     """The search GEMM's roofline over the timed region: the alpha-GEMM flops
     of all its launches over their summed CUDA-event durations.  A region of
-    at least a second is the sustained regime (the power-capped cuBLAS loop),
-    a shorter one the burst regime."""
+    at least half a second of back-to-back GEMMs is the sustained regime (the
+    power-capped cuBLAS loop: under the 1 kW cap the clocks settle within tens
+    of milliseconds), a shorter one the burst regime."""
     peaks, src = load_peaks()
     gemm_ms, gemm_n = prof["search_gemm"]
     flops = job.flops() * steps
     achieved = flops / (gemm_ms / 1e3) / 1e12
     burst = float(peaks["bf16_tflops"])
     sustained = float(peaks.get("bf16_tflops_sustained", burst))
-    regime = "sustained" if timed_ms >= 1000.0 else "burst"
+    regime = "sustained" if timed_ms >= SUSTAINED_MS else "burst"
     peak = sustained if regime == "sustained" else burst
     tr = committed_traffic(job.name)
     launches_per_step = gemm_n / max(steps, 1)
@@ -474,6 +478,7 @@ def roofline_of(job: Job, prof, steps: int, timed_ms: float):
             "peak_source": f"{src} bf16 dense, {regime} (cuBLAS), from MEASURED_PEAKS.json" if src == "measured"
             else "fallback 1.59 PFLOP/s burst / 1.4 sustained",
             "frac_of_burst": achieved / burst, "frac_of_sustained": achieved / sustained,
+            "regime": regime, "timed_region_ms": timed_ms,
             "kernel": "search_kernel (fused per-alpha loss GEMM)",
             "launches_per_step": launches_per_step,
             "avg_launch_ms": gemm_ms / max(gemm_n, 1),
@@ -825,21 +830,26 @@ def w4a16_section(dev, rank):
         with torch.cuda.graph(gr):
             for i in range(reps):
                 fn(i)
-        gr.replay()
+        for _ in range(2):                 # untimed replays: clocks up from an idle GPU
+            gr.replay()
         torch.cuda.synchronize()
-        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ea.record()
-        gr.replay()
-        eb.record()
-        eb.synchronize()
+        best = float("inf")
+        for _ in range(5):                 # the best of five timed replays
+            ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ea.record()
+            gr.replay()
+            eb.record()
+            eb.synchronize()
+            best = min(best, ea.elapsed_time(eb))
         del gr
-        return ea.elapsed_time(eb) / reps
+        return best / reps
 
     bits, group = 4, 128
     g4 = torch.Generator(device=dev).manual_seed(4321 + rank)
-    info = {"timing": "CUDA graph of 20 calls (status clear, then N <= 4: GEMV + split reduce, else "
-                      "pre-pass + GEMM), weights rotated over copies > 256 MiB; synthetic packed words "
-                      "and deltas",
+    info = {"timing": "best of 5 replays of a CUDA graph of 20 calls (N <= 4: one GEMV launch whose column-tile splits are "
+                      "reduced in a cluster, or a stream-K GEMV and a dependent reduce launch; else a status "
+                      "clear, the pre-pass and the GEMM), weights rotated over copies > 256 MiB; synthetic "
+                      "packed words and deltas",
             "algorithmic_bytes": "packed words + fp32 deltas + X (bf16) + s + Y (fp32), each once"}
     peaks, _ = load_peaks()
     hbm_peak, bf16_peak = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
