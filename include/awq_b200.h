@@ -484,6 +484,22 @@ AWQ_API int awq_search_noalloc(const void* X, const float* W, const float* a, in
 AWQ_API int awq_selftest_wait_timeout(int32_t* status, int64_t timeout_ns, void* stream);
 
 /*
+ * Self test of the quantisers' arithmetic that is not a plain IEEE operation:
+ * delta = fl(m / d) for the constant divisors d (2^(b-1) - 1 and 2^b - 1) is
+ * formed by Markstein's FMA correction of m * fl(1/d), and the quotients
+ * w'/delta go through a reciprocal within one ulp (hardware approximation
+ * plus one Newton step).  This runs both over every non-negative finite float
+ * (about two billion values) on the device:
+ *   divisor     1 .. 255 (AWQ_EINVAL otherwise)
+ *   mismatches  [2] uint64 device output, 8-byte aligned: [0] values whose
+ *               quotient differs from the IEEE quotient, [1] normal values up
+ *               to 2^125 whose reciprocal is more than one ulp from the
+ *               correctly rounded one.  Both are 0 for a correct build.
+ * Read the result after the stream has been synchronised.
+ */
+AWQ_API int awq_selftest_divide(int32_t divisor, uint64_t* mismatches, void* stream);
+
+/*
  * Stage timing.  While enabled, every entry point records a pair of CUDA
  * events on its stream around each kernel it launches; awq_profile_read waits
  * for the recorded events and returns, per stage, the summed device time in

@@ -26,7 +26,7 @@ MAX_ALPHA = 64
 EXPORTS = (
     "awq_act_stats", "awq_scales", "awq_scales_dev", "awq_search_workspace_size", "awq_search",
     "awq_search_batched_workspace_size", "awq_search_batched", "awq_quantize_pack",
-    "awq_layer_output_workspace_size", "awq_layer_output", "awq_selftest_wait_timeout",
+    "awq_layer_output_workspace_size", "awq_layer_output", "awq_selftest_wait_timeout", "awq_selftest_divide",
     "awq_get_last_error", "awq_version", "awq_profile_enable", "awq_profile_reset", "awq_profile_read",
     "awq_search_noalloc", "awq_clip_search_workspace_size", "awq_clip_search", "awq_quantize_pack_clip",
     "awq_search_joint_workspace_size", "awq_search_joint", "awq_quantize_pack_ex", "awq_w4a16_gemm",
@@ -90,6 +90,7 @@ _pack = _sig("awq_quantize_pack", I, [P, P, I64, I64, I, I, P, P, P])
 _out_ws = _sig("awq_layer_output_workspace_size", SZ, [I64, I64, I64])
 _out = _sig("awq_layer_output", I, [P, P, I64, I64, I64, P, P, SZ, P, P])
 _selftest = _sig("awq_selftest_wait_timeout", I, [P, I64, P])
+_selftest_div = _sig("awq_selftest_divide", I, [I, P, P])
 _last_error = _sig("awq_get_last_error", ctypes.c_char_p, [])
 _prof_enable = _sig("awq_profile_enable", I, [I])
 _prof_reset = _sig("awq_profile_reset", I, [])
@@ -527,6 +528,15 @@ def layer_output(X: torch.Tensor, W: torch.Tensor, workspace: Optional[Workspace
     _check(_out(_ptr(X), _ptr(W), N, D_in, D_out, _ptr(Y), _ptr(ws), ws.numel(), _ptr(status), _stream()))
     check_device_status(status)
     return Y
+
+
+def selftest_divide(divisor: int):
+    """``awq_selftest_divide``: (quotients that differ from the IEEE ones,
+    reciprocals more than one ulp off) over every non-negative finite float."""
+    out = torch.zeros(2, dtype=torch.int64, device="cuda")
+    _check(_selftest_div(int(divisor), _ptr(out), _stream()))
+    a, b = out.cpu().tolist()
+    return a, b
 
 
 def selftest_wait_timeout(timeout_ns: int = 1_000_000) -> int:

@@ -767,6 +767,19 @@ int awq_selftest_wait_timeout(int32_t* status, int64_t timeout_ns_arg, void* str
 }
 
 
+int awq_selftest_divide(int32_t divisor, uint64_t* mismatches, void* stream) {
+  AWQ_TRY(check_ptr(mismatches, "mismatches", 8));
+  if (divisor < 1 || divisor > 255) return fail(AWQ_EINVAL, "divisor = %d: need 1 .. 255", divisor);
+  int sms = 0;
+  AWQ_TRY(device_info(&sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(mismatches, 0, 2 * sizeof(uint64_t), st);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(mismatches)");
+  e = awq::launch_divide_selftest(static_cast<float>(divisor), reinterpret_cast<unsigned long long*>(mismatches), sms,
+                                  st);
+  return e == cudaSuccess ? AWQ_OK : fail_cuda(e, "divide self-test kernel");
+}
+
 size_t awq_clip_search_workspace_size(int64_t N, int64_t D_in, int64_t D_out, int n_clip, int bits, int group) {
   if (check_clip_args(N, D_in, D_out, n_clip, bits, group) != AWQ_OK) return 0;
   return clip_layout(N, D_in, D_out, n_clip, group).total;

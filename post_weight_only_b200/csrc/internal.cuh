@@ -178,4 +178,10 @@ int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const fl
 // arrives at, gives up after timeout_ns and records the timeout in *status.
 cudaError_t launch_wait_timeout_selftest(int* status, uint64_t timeout_ns, cudaStream_t st);
 
+// Self test of the quantisers' constant divisor and reciprocal on every
+// non-negative finite float (quant.cu): bad[0] += mismatches of the division
+// by b against the IEEE quotient, bad[1] += reciprocals more than one ulp
+// from the correctly rounded one.  bad must be zeroed by the caller.
+cudaError_t launch_divide_selftest(float b, unsigned long long* bad, int num_sms, cudaStream_t st);
+
 }  // namespace awq

@@ -195,6 +195,12 @@ def test_argument_checks_without_gpu(lib):
     t.argtypes = [P, I64, P]
     t.restype = I
     assert t(fake, 10, None) == 1                          # timeout below 1 us
+    dv = lib.awq_selftest_divide
+    dv.argtypes = [I, P, P]
+    dv.restype = I
+    assert dv(0, fake, None) == 1                          # divisor below 1
+    assert dv(256, fake, None) == 1                        # divisor above 255
+    assert dv(7, fake + 4, None) == 2                      # misaligned output
 
 
 def test_no_device_is_reported_not_crashed(lib):

@@ -325,6 +325,17 @@ def test_batched_matches_single(awq, form):
         assert int(rb.alpha_idx) == int(rs.alpha_idx)
 
 
+# ------------------------------------------------------------------ quantiser arithmetic
+@pytest.mark.parametrize("divisor", [1, 3, 7, 15, 31, 127, 255])
+def test_constant_divisor_matches_ieee_on_every_float(awq, divisor):
+    """delta = fl(m / d) by Markstein's FMA correction equals __fdiv_rn for
+    every non-negative finite float, and the fast reciprocal of the quotient
+    shortcut stays within one ulp of the correctly rounded one."""
+    bad_div, bad_rcp = awq.selftest_divide(divisor)
+    assert bad_div == 0
+    assert bad_rcp == 0
+
+
 # ------------------------------------------------------------------ failure detection
 def test_bounded_wait_gives_up_with_status(awq):
     """A wait on a barrier nothing arrives at returns AWQ_ETIMEOUT in the device
