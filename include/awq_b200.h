@@ -34,6 +34,16 @@
  *     memory-safe) results.
  *   - Supported bit widths are 2, 3 and 4 (codes are stored as 4-bit
  *     offset-binary values); group sizes are 32, 64, 128 and 256.
+ *   - Debug knobs, read once per process from the environment:
+ *       AWQ_LOG=1        one stderr line per call that works on the device
+ *                        ("[awq] name(sizes)") and one per non-OK status;
+ *       AWQ_FAULT=badarg | workspace | alloc | launch
+ *                        host-side fault injection at the entry of every such
+ *                        call, before any check or launch: AWQ_EINVAL,
+ *                        AWQ_EWORKSPACE (on the calls that take a workspace;
+ *                        "alloc" is the same, since the library allocates
+ *                        nothing), or AWQ_ECUDA as from a failed launch;
+ *       AWQ_TIMEOUT_MS   the bounded waits' limit (default 2000).
  */
 #ifndef AWQ_B200_H
 #define AWQ_B200_H

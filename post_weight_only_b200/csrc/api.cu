@@ -16,6 +16,39 @@ namespace {
 
 thread_local std::string g_last_error;
 
+// Debug knobs, read once from the environment:
+//   AWQ_LOG=1      one stderr line per entry-point call (its name and sizes),
+//                  and one per non-OK status with the message;
+//   AWQ_FAULT=...  host-side fault injection at the entry of every call that
+//                  works on the device, before any argument check or launch:
+//                  "badarg" -> AWQ_EINVAL, "workspace" (or "alloc": the
+//                  library allocates nothing, so a caller's failed allocation
+//                  reaches it as a short workspace) -> AWQ_EWORKSPACE on the
+//                  calls that take one, "launch" -> AWQ_ECUDA as from a
+//                  failed kernel launch.  Nothing reaches the GPU.
+enum FaultMode { kFaultNone, kFaultBadArg, kFaultWorkspace, kFaultLaunch };
+
+bool log_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("AWQ_LOG");
+    return e != nullptr && e[0] != '\0' && e[0] != '0';
+  }();
+  return on;
+}
+
+FaultMode fault_mode() {
+  static const FaultMode m = [] {
+    const char* e = getenv("AWQ_FAULT");
+    if (e == nullptr) return kFaultNone;
+    const std::string v(e);
+    if (v == "badarg") return kFaultBadArg;
+    if (v == "workspace" || v == "alloc") return kFaultWorkspace;
+    if (v == "launch") return kFaultLaunch;
+    return kFaultNone;
+  }();
+  return m;
+}
+
 int fail(int code, const char* fmt, ...) {
   char buf[512];
   va_list ap;
@@ -23,8 +56,38 @@ int fail(int code, const char* fmt, ...) {
   vsnprintf(buf, sizeof buf, fmt, ap);
   va_end(ap);
   g_last_error = buf;
+  if (log_enabled()) fprintf(stderr, "[awq]   -> status %d: %s\n", code, buf);
   return code;
 }
+
+enum Workspace { kNoWorkspace = 0, kTakesWorkspace = 1 };
+
+// Entry of a device-side call: the trace line and the injected fault, if any.
+int api_entry(const char* name, Workspace ws, const char* fmt, ...) {
+  if (log_enabled()) {
+    char buf[384];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    fprintf(stderr, "[awq] %s(%s)\n", name, buf);
+  }
+  switch (fault_mode()) {
+    case kFaultBadArg: return fail(AWQ_EINVAL, "%s: AWQ_FAULT=badarg (injected)", name);
+    case kFaultWorkspace:
+      if (ws == kTakesWorkspace) return fail(AWQ_EWORKSPACE, "%s: AWQ_FAULT=workspace (injected)", name);
+      return AWQ_OK;
+    case kFaultLaunch:
+      return fail(AWQ_ECUDA, "%s: AWQ_FAULT=launch (injected): %s", name, cudaGetErrorName(cudaErrorLaunchFailure));
+    default: return AWQ_OK;
+  }
+}
+
+#define AWQ_ENTRY(name, ws, ...)                                  \
+  do {                                                            \
+    const int awq_entry_rc_ = api_entry((name), (ws), __VA_ARGS__); \
+    if (awq_entry_rc_ != AWQ_OK) return awq_entry_rc_;            \
+  } while (0)
 
 int fail_cuda(cudaError_t e, const char* what) {
   return fail(AWQ_ECUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
@@ -358,6 +421,8 @@ const char* awq_get_last_error(void) { return g_last_error.c_str(); }
 int awq_version(void) { return 100; }
 
 int awq_act_stats(const void* X, int64_t N, int64_t D_in, int stat, float* a, void* stream) {
+  AWQ_ENTRY("awq_act_stats", kNoWorkspace, "N=%lld D_in=%lld stat=%d", (long long)N, (long long)D_in, stat);
+
   if (N < 1 || N > kMaxDim) return fail(AWQ_EINVAL, "N = %lld: need 1 <= N <= 2^24", (long long)N);
   if (D_in < 8 || D_in > kMaxDin || D_in % 8) return fail(AWQ_EINVAL, "D_in = %lld: need a multiple of 8 in [8, 2^20]", (long long)D_in);
   if (stat != AWQ_STAT_MEAN && stat != AWQ_STAT_MAX) return fail(AWQ_EINVAL, "stat = %d: use AWQ_STAT_MEAN or AWQ_STAT_MAX", stat);
@@ -375,6 +440,7 @@ int awq_act_stats(const void* X, int64_t N, int64_t D_in, int stat, float* a, vo
 
 int awq_act_stats_batched(const void* const* Xs, const int64_t* Ns, const int64_t* D_ins, int n_inputs, int stat,
                           float* const* as, void* stream) {
+  AWQ_ENTRY("awq_act_stats_batched", kNoWorkspace, "n_inputs=%d stat=%d", n_inputs, stat);
   if (!Xs || !Ns || !D_ins || !as) return fail(AWQ_EINVAL, "Xs, Ns, D_ins and as must not be NULL");
   if (n_inputs < 1 || n_inputs > awq::kMaxStatsInputs)
     return fail(AWQ_EUNSUPPORTED, "n_inputs = %d: need 1..%d", n_inputs, awq::kMaxStatsInputs);
@@ -417,22 +483,29 @@ static int scales_common(const float* a, const float* w_mean, int64_t D_in, floa
 }
 
 int awq_scales(const float* a, int64_t D_in, float alpha, float* s, void* stream) {
+  AWQ_ENTRY("awq_scales", kNoWorkspace, "D_in=%lld alpha=%g", (long long)D_in, alpha);
+
   return scales_common(a, nullptr, D_in, alpha, nullptr, s, stream);
 }
 
 int awq_scales_dev(const float* a, int64_t D_in, const float* alpha_dev, float* s, void* stream) {
+  AWQ_ENTRY("awq_scales_dev", kNoWorkspace, "D_in=%lld", (long long)D_in);
+
   AWQ_TRY(check_ptr(alpha_dev, "alpha_dev", 4));
   return scales_common(a, nullptr, D_in, 0.0f, alpha_dev, s, stream);
 }
 
 int awq_scales_ex(const float* a, const float* w_mean, int64_t D_in, float alpha, const float* alpha_dev, float* s,
                   void* stream) {
+  AWQ_ENTRY("awq_scales_ex", kNoWorkspace, "D_in=%lld alpha=%g weight_statistic=%d", (long long)D_in, alpha, w_mean ? 1 : 0);
   if (alpha_dev) AWQ_TRY(check_ptr(alpha_dev, "alpha_dev", 4));
   if (!alpha_dev && !(alpha >= 0.0f && alpha <= 1.0f)) return fail(AWQ_EINVAL, "alpha = %g: need 0 <= alpha <= 1", alpha);
   return scales_common(a, w_mean, D_in, alpha, alpha_dev, s, stream);
 }
 
 int awq_weight_mean(const float* W, int64_t D_in, int64_t D_out, float* w_mean, void* stream) {
+  AWQ_ENTRY("awq_weight_mean", kNoWorkspace, "D_in=%lld D_out=%lld", (long long)D_in, (long long)D_out);
+
   if (D_in < 1 || D_in > kMaxDim || D_out < 1 || D_out > kMaxDim)
     return fail(AWQ_EINVAL, "D_in = %lld, D_out = %lld out of range", (long long)D_in, (long long)D_out);
   AWQ_TRY(check_ptr(W, "W", 16));
@@ -521,6 +594,7 @@ int awq_search(const void* X, const float* W, const float* a, int64_t N, int64_t
                const float* alpha_grid, int n_alpha, int bits, int group, int loss_form, double* L, double* L_col,
                float* alpha_star, int32_t* alpha_idx, void* workspace, size_t workspace_bytes, int32_t* status,
                void* stream) {
+  AWQ_ENTRY("awq_search", kTakesWorkspace, "N=%lld D_in=%lld D_out=%lld n_alpha=%d bits=%d group=%d form=%d", (long long)N, (long long)D_in, (long long)D_out, n_alpha, bits, group, loss_form);
   return search_impl(X, W, a, N, D_in, D_out, alpha_grid, n_alpha, bits, group, loss_form, L, L_col, alpha_star,
                      alpha_idx, workspace, workspace_bytes, status, stream, SearchOpts());
 }
@@ -529,6 +603,7 @@ int awq_search_ex(const void* X, const float* W, const float* a, int64_t N, int6
                   const float* alpha_grid, int n_alpha, int bits, int group, int loss_form,
                   const awq_search_options* options, double* L, double* L_col, float* alpha_star,
                   int32_t* alpha_idx, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  AWQ_ENTRY("awq_search_ex", kTakesWorkspace, "N=%lld D_in=%lld D_out=%lld n_alpha=%d bits=%d group=%d form=%d", (long long)N, (long long)D_in, (long long)D_out, n_alpha, bits, group, loss_form);
   SearchOpts o;
   if (options) {
     switch (options->quantizer) {
@@ -577,6 +652,7 @@ size_t awq_search_batched_workspace_size(const awq_layer* layers, int n_layers, 
 int awq_search_batched(const awq_layer* layers, int n_layers, const float* alpha_grid, int n_alpha, int bits,
                        int group, int loss_form, void* workspace, size_t workspace_bytes, int32_t* status,
                        void* stream) {
+  AWQ_ENTRY("awq_search_batched", kTakesWorkspace, "n_layers=%d n_alpha=%d bits=%d group=%d form=%d", n_layers, n_alpha, bits, group, loss_form);
   if (!layers || n_layers < 1) return fail(AWQ_EINVAL, "layers is NULL or n_layers < 1");
   for (int i = 0; i < n_layers; ++i) {
     const awq_layer& l = layers[i];
@@ -615,6 +691,7 @@ int awq_search_batched(const awq_layer* layers, int n_layers, const float* alpha
 
 int awq_quantize_pack(const float* W, const float* s, int64_t D_in, int64_t D_out, int bits, int group,
                       uint32_t* packed, float* scales, void* stream) {
+  AWQ_ENTRY("awq_quantize_pack", kNoWorkspace, "D_in=%lld D_out=%lld bits=%d group=%d", (long long)D_in, (long long)D_out, bits, group);
   return awq_quantize_pack_ex(W, s, nullptr, D_in, D_out, bits, group, 0, packed, scales, stream);
 }
 
@@ -661,6 +738,7 @@ size_t awq_layer_output_workspace_size(int64_t N, int64_t D_in, int64_t D_out) {
 
 int awq_layer_output(const void* X, const float* W, int64_t N, int64_t D_in, int64_t D_out, float* Y,
                      void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  AWQ_ENTRY("awq_layer_output", kTakesWorkspace, "N=%lld D_in=%lld D_out=%lld", (long long)N, (long long)D_in, (long long)D_out);
   AWQ_TRY(check_layer_shape(N, D_in, D_out));
   AWQ_TRY(check_ptr(X, "X", 16));
   AWQ_TRY(check_ptr(W, "W", 16));
@@ -724,6 +802,7 @@ int awq_profile_read(int stage, double* total_ms, int32_t* launches) {
 int awq_search_noalloc(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
                        const float* alpha_grid, int n_alpha, int bits, int group, int loss_form, double* L,
                        double* L_col, float* alpha_star, int32_t* alpha_idx, int32_t* status, void* stream) {
+  AWQ_ENTRY("awq_search_noalloc", kTakesWorkspace, "N=%lld D_in=%lld D_out=%lld n_alpha=%d bits=%d group=%d form=%d", (long long)N, (long long)D_in, (long long)D_out, n_alpha, bits, group, loss_form);
   AWQ_TRY(check_search_args(X, W, a, N, D_in, D_out, alpha_grid, n_alpha, bits, group, loss_form, L, L_col,
                             alpha_star, alpha_idx));
   int sms = 0;
@@ -754,6 +833,8 @@ int awq_search_noalloc(const void* X, const float* W, const float* a, int64_t N,
 }
 
 int awq_selftest_wait_timeout(int32_t* status, int64_t timeout_ns_arg, void* stream) {
+  AWQ_ENTRY("awq_selftest_wait_timeout", kNoWorkspace, "timeout_ns=%lld", (long long)timeout_ns_arg);
+
   AWQ_TRY(check_ptr(status, "status", 4));
   if (timeout_ns_arg < 1000 || timeout_ns_arg > 10000000000LL)
     return fail(AWQ_EINVAL, "timeout_ns = %lld: need 1 us .. 10 s", (long long)timeout_ns_arg);
@@ -768,6 +849,8 @@ int awq_selftest_wait_timeout(int32_t* status, int64_t timeout_ns_arg, void* str
 
 
 int awq_selftest_divide(int32_t divisor, uint64_t* mismatches, void* stream) {
+  AWQ_ENTRY("awq_selftest_divide", kNoWorkspace, "divisor=%d", divisor);
+
   AWQ_TRY(check_ptr(mismatches, "mismatches", 8));
   if (divisor < 1 || divisor > 255) return fail(AWQ_EINVAL, "divisor = %d: need 1 .. 255", divisor);
   int sms = 0;
@@ -788,6 +871,7 @@ size_t awq_clip_search_workspace_size(int64_t N, int64_t D_in, int64_t D_out, in
 int awq_clip_search(const void* X, const float* W, const float* s, int64_t N, int64_t D_in, int64_t D_out,
                     const float* clip_grid, int n_clip, int bits, int group, float* clip, int32_t* clip_idx,
                     float* loss, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  AWQ_ENTRY("awq_clip_search", kTakesWorkspace, "N=%lld D_in=%lld D_out=%lld n_clip=%d bits=%d group=%d", (long long)N, (long long)D_in, (long long)D_out, n_clip, bits, group);
   AWQ_TRY(check_clip_args(N, D_in, D_out, n_clip, bits, group));
   if (!clip_grid) return fail(AWQ_EINVAL, "clip_grid is NULL");
   for (int i = 0; i < n_clip; ++i)
@@ -844,6 +928,7 @@ int awq_clip_search(const void* X, const float* W, const float* s, int64_t N, in
 
 int awq_quantize_pack_clip(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out, int bits,
                            int group, uint32_t* packed, float* scales, void* stream) {
+  AWQ_ENTRY("awq_quantize_pack_clip", kNoWorkspace, "D_in=%lld D_out=%lld bits=%d group=%d", (long long)D_in, (long long)D_out, bits, group);
   if (!clip) return fail(AWQ_EINVAL, "clip is NULL");
   return awq_quantize_pack_ex(W, s, clip, D_in, D_out, bits, group, 0, packed, scales, stream);
 }
@@ -880,6 +965,7 @@ static int quantize_pack_impl(const float* W, const float* s, const float* clip,
 
 int awq_quantize_pack_ex(const float* W, const float* s, const float* clip, int64_t D_in, int64_t D_out, int bits,
                          int group, int flags, uint32_t* packed, void* scales, void* stream) {
+  AWQ_ENTRY("awq_quantize_pack_ex", kNoWorkspace, "D_in=%lld D_out=%lld bits=%d group=%d flags=%d", (long long)D_in, (long long)D_out, bits, group, flags);
   return quantize_pack_impl(W, s, clip, D_in, D_out, bits, group, flags,
                             (flags & AWQ_PACK_DELTA_POW2) ? awq::kQuantPow2 : awq::kQuantSymmetric, packed, scales,
                             nullptr, stream);
@@ -887,6 +973,7 @@ int awq_quantize_pack_ex(const float* W, const float* s, const float* clip, int6
 
 int awq_quantize_pack_zp(const float* W, const float* s, int64_t D_in, int64_t D_out, int bits, int group, int flags,
                          uint32_t* packed, void* scales, uint8_t* zeros, void* stream) {
+  AWQ_ENTRY("awq_quantize_pack_zp", kNoWorkspace, "D_in=%lld D_out=%lld bits=%d group=%d flags=%d", (long long)D_in, (long long)D_out, bits, group, flags);
   if (flags & AWQ_PACK_DELTA_POW2) return fail(AWQ_EINVAL, "AWQ_PACK_DELTA_POW2 does not apply to the asymmetric quantiser");
   return quantize_pack_impl(W, s, nullptr, D_in, D_out, bits, group, flags, awq::kQuantAsymmetric, packed, scales,
                             zeros, stream);
@@ -921,6 +1008,7 @@ int awq_search_joint(const void* X, const float* const* Ws, const int64_t* D_out
                      int64_t N, int64_t D_in, const float* alpha_grid, int n_alpha, int bits, int group,
                      int loss_form, double* L, double* L_layers, float* alpha_star, int32_t* alpha_idx,
                      void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  AWQ_ENTRY("awq_search_joint", kTakesWorkspace, "N=%lld D_in=%lld n_layers=%d n_alpha=%d bits=%d group=%d form=%d", (long long)N, (long long)D_in, n_layers, n_alpha, bits, group, loss_form);
   int64_t Dsum = 0;
   AWQ_TRY(check_joint(D_outs, n_layers, &Dsum));
   if (!Ws) return fail(AWQ_EINVAL, "Ws is NULL");
@@ -1027,6 +1115,7 @@ static int w4a16_impl(const void* X, const float* s, const uint32_t* packed, con
 int awq_w4a16_gemm(const void* X, const float* s, const uint32_t* packed, const float* scales, int64_t N,
                    int64_t D_in, int64_t D_out, int bits, int group, float* Y, void* workspace,
                    size_t workspace_bytes, int32_t* status, void* stream) {
+  AWQ_ENTRY("awq_w4a16_gemm", kTakesWorkspace, "N=%lld D_in=%lld D_out=%lld bits=%d group=%d", (long long)N, (long long)D_in, (long long)D_out, bits, group);
   return w4a16_impl(X, s, packed, scales, nullptr, N, D_in, D_out, bits, group, Y, workspace, workspace_bytes,
                     status, stream);
 }
@@ -1034,6 +1123,7 @@ int awq_w4a16_gemm(const void* X, const float* s, const uint32_t* packed, const 
 int awq_w4a16_gemm_zp(const void* X, const float* s, const uint32_t* packed, const float* scales,
                       const uint8_t* zeros, int64_t N, int64_t D_in, int64_t D_out, int bits, int group, float* Y,
                       void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  AWQ_ENTRY("awq_w4a16_gemm_zp", kTakesWorkspace, "N=%lld D_in=%lld D_out=%lld bits=%d group=%d", (long long)N, (long long)D_in, (long long)D_out, bits, group);
   if (!zeros) return fail(AWQ_EINVAL, "zeros is NULL");
   return w4a16_impl(X, s, packed, scales, zeros, N, D_in, D_out, bits, group, Y, workspace, workspace_bytes, status,
                     stream);
