@@ -671,13 +671,16 @@ def quantize_block_host(xs_host: Sequence[torch.Tensor], layers_host, alpha_grid
 
     ``xs_host``: the distinct layer inputs (bf16, pinned for asynchronous
     copies); ``layers_host``: (input index, W fp32 on the host) per layer.
-    A copy stream uploads the inputs, then each layer's W in order; the current
-    stream computes each input's statistic as soon as it has landed, and each
-    layer's search (``awq_search``), s* and pack as soon as its W has landed;
-    a third stream copies each layer's L, alpha*, status, codes and scales back
-    as soon as they are done.  Synchronises, checks every status word and
-    returns a list of dicts of host tensors (reused across calls through
-    ``state``)."""
+    The layers run in an order that starts the device early and ends it
+    soon after the last search: the layer with the smallest W first, the
+    second smallest last, the others as given.  A copy stream uploads, in that
+    order, each input before the first layer that reads it and each layer's W;
+    the current stream computes an input's statistic before its first layer,
+    then each layer's search (``awq_search``), s* and pack as soon as its W has
+    landed; a third stream copies each layer's L, alpha*, status, codes and
+    scales back as soon as they are done.  Synchronises, checks every status
+    word and returns a list of dicts of host tensors in the layers' given
+    order (reused across calls through ``state``)."""
     dev = torch.device(device)
     st = state if state is not None else BlockHostState()
     compute = torch.cuda.current_stream(dev)
@@ -687,22 +690,25 @@ def quantize_block_host(xs_host: Sequence[torch.Tensor], layers_host, alpha_grid
     if st.xs is None:
         st.xs = [torch.empty(x.shape, dtype=x.dtype, device=dev) for x in xs_host]
         st.ws = [torch.empty(w.shape, dtype=w.dtype, device=dev) for _, w in layers_host]
+    by_size = sorted(range(len(layers_host)), key=lambda i: (layers_host[i][1].numel(), i))
+    if len(by_size) > 2:
+        first, last = by_size[0], by_size[1]
+        order = [first] + [i for i in range(len(layers_host)) if i not in (first, last)] + [last]
+    else:
+        order = by_size
     # the previous call's device work on these buffers has finished (it synchronised)
     st.copy_stream.wait_stream(compute)
-    x_ready, w_ready = [], []
+    x_ready, w_ready = {}, {}
     with torch.cuda.stream(st.copy_stream):
-        for xd, xh in zip(st.xs, xs_host):
-            xd.copy_(xh, non_blocking=True)
-            x_ready.append(torch.cuda.Event())
-            x_ready[-1].record(st.copy_stream)
-        for wd, (_, wh) in zip(st.ws, layers_host):
-            wd.copy_(wh, non_blocking=True)
-            w_ready.append(torch.cuda.Event())
-            w_ready[-1].record(st.copy_stream)
-    a = []
-    for k, xd in enumerate(st.xs):
-        compute.wait_event(x_ready[k])
-        a.append(act_stats(xd, stat))
+        for i in order:
+            xi, wh = layers_host[i]
+            if xi not in x_ready:
+                st.xs[xi].copy_(xs_host[xi], non_blocking=True)
+                x_ready[xi] = torch.cuda.Event()
+                x_ready[xi].record(st.copy_stream)
+            st.ws[i].copy_(wh, non_blocking=True)
+            w_ready[i] = torch.cuda.Event()
+            w_ready[i].record(st.copy_stream)
     pin = all(x.is_pinned() for x in xs_host)
     if st.results is None:
         st.results = []
@@ -715,7 +721,13 @@ def quantize_block_host(xs_host: Sequence[torch.Tensor], layers_host, alpha_grid
                 "packed": torch.empty(D_in // 8, D_out, dtype=torch.int32, pin_memory=pin),
                 "scales": torch.empty(D_in // group, D_out, dtype=torch.float32, pin_memory=pin),
             })
-    for i, ((xi, _), wd) in enumerate(zip(layers_host, st.ws)):
+    a = {}
+    for i in order:
+        xi, _ = layers_host[i]
+        wd = st.ws[i]
+        if xi not in a:                            # the input's statistic, before its first layer
+            compute.wait_event(x_ready[xi])
+            a[xi] = act_stats(st.xs[xi], stat)
         compute.wait_event(w_ready[i])
         r = search(st.xs[xi], wd, a[xi], alpha_grid, bits, group, workspace=workspace, check_status=False,
                    loss_form=loss_form)
