@@ -107,12 +107,21 @@ struct Segment {
 
 // The sequence of segments a CTA pair processes.  Every role of both CTAs
 // walks the same sequence, so ring positions and barrier phases agree.
+// The (unit, alpha) passes of the last partial wave are shared out evenly
+// over all pairs: when alpha_major, numbered alpha-major and dealt round
+// robin, one pass per segment, so that at any time the pairs work on one or
+// two alphas and each alpha's operand tiles are fetched about once; else as
+// contiguous runs of the unit-major numbering (segments of consecutive alphas
+// of one unit: the reference form, whose segments each start with a
+// reference pass).
 struct Schedule {
   int U, A, G, c;
   int full_waves, head;
   long long j, te;
   int i;
-  __device__ Schedule(int U_, int A_, int G_, int c_) : U(U_), A(A_), G(G_), c(c_), i(0) {
+  bool alpha_major;
+  __device__ Schedule(int U_, int A_, int G_, int c_, bool am)
+      : U(U_), A(A_), G(G_), c(c_), i(0), alpha_major(am) {
     if (A == 0) {                       // reference output only: whole units round robin
       full_waves = (U - c + G - 1) / G;
       head = U;
@@ -121,8 +130,13 @@ struct Schedule {
       full_waves = U / G;
       head = full_waves * G;
       const long long items = static_cast<long long>(U - head) * A;
-      j = items * c / G;
-      te = items * (c + 1) / G;
+      if (alpha_major) {                // every G-th pass: all pairs on the same alpha or two
+        j = c;
+        te = items;
+      } else {
+        j = items * c / G;
+        te = items * (c + 1) / G;
+      }
     }
   }
   __device__ bool next(Segment& s) {
@@ -131,6 +145,14 @@ struct Schedule {
       s.a0 = 0;
       s.a1 = A;
       ++i;
+      return true;
+    }
+    if (j < te && alpha_major) {
+      const int rem = U - head;
+      s.u = head + static_cast<int>(j % rem);
+      s.a0 = static_cast<int>(j / rem);
+      s.a1 = s.a0 + 1;
+      j += G;
       return true;
     }
     if (j < te) {
@@ -228,7 +250,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      Schedule sch(p.U, p.A, npairs, pair);
+      Schedule sch(p.U, p.A, npairs, pair, kForm != kFormReference);
       Segment sg;
       uint32_t it = 0;
       int last_round[kStages];
@@ -279,7 +301,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (lane == 0 && leader) {
-      Schedule sch(p.U, p.A, npairs, pair);
+      Schedule sch(p.U, p.A, npairs, pair, kForm != kFormReference);
       Segment sg;
       uint32_t it = 0, acc_it = 0;
       const uint32_t idesc = idesc_bf16_f32(kPairM, kBN);
@@ -327,7 +349,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int h = (warp - 2) >> 2;                 // token half of the accumulator
     const int nl = q * 32 + lane;
-    Schedule sch(p.U, p.A, npairs, pair);
+    Schedule sch(p.U, p.A, npairs, pair, kForm != kFormReference);
     Segment sg;
     uint32_t acc_it = 0;
     bool ok = true;
