@@ -652,67 +652,113 @@ def quantize_block(xs: Sequence[torch.Tensor], layers, alpha_grid: Sequence[floa
 
 class BlockHostState:
     """Device copies of a block's inputs and pinned host result buffers, kept
-    between calls of :func:`quantize_block_host` on blocks of one shape."""
+    between calls of :func:`quantize_block_host` on blocks of one shape: two
+    sets of device buffers (one being computed on, one receiving the next
+    block's upload when a call is given ``prefetch``), the copy and result
+    streams, and the upload issued ahead, if any."""
 
     def __init__(self):
-        self.xs = None
-        self.ws = None
+        self.bufs = [None, None]       # per set: (device inputs, device weights)
+        self.cur = 0
+        self.pending = None            # (host key, set, input events, weight events) of an upload ahead
         self.results = None
         self.copy_stream = None
         self.back_stream = None
 
 
+def _block_order(layers_host):
+    """The order the block's layers run in: the smallest W first (the device
+    starts early), the second smallest last (the last results to copy back are
+    small), the others as given."""
+    by_size = sorted(range(len(layers_host)), key=lambda i: (layers_host[i][1].numel(), i))
+    if len(by_size) > 2:
+        first, last = by_size[0], by_size[1]
+        return [first] + [i for i in range(len(layers_host)) if i not in (first, last)] + [last]
+    return by_size
+
+
+def _host_key(xs_host, layers_host):
+    return (tuple((x.data_ptr(), tuple(x.shape)) for x in xs_host),
+            tuple((xi, w.data_ptr(), tuple(w.shape)) for xi, w in layers_host))
+
+
+def _block_buffers(st, b, xs_host, layers_host, dev):
+    """Device buffers of set b for a block of this shape (reallocated if the shape changed)."""
+    shapes = ([tuple(x.shape) for x in xs_host], [tuple(w.shape) for _, w in layers_host])
+    cur = st.bufs[b]
+    if cur is None or ([tuple(x.shape) for x in cur[0]], [tuple(w.shape) for w in cur[1]]) != shapes:
+        st.bufs[b] = ([torch.empty(x.shape, dtype=x.dtype, device=dev) for x in xs_host],
+                      [torch.empty(w.shape, dtype=w.dtype, device=dev) for _, w in layers_host])
+    return st.bufs[b]
+
+
+def _block_upload(st, b, order, xs_host, layers_host):
+    """On the copy stream, in the layers' run order: each input before the first
+    layer that reads it, and each layer's W; returns the ready events."""
+    xs_d, ws_d = st.bufs[b]
+    x_ready, w_ready = {}, {}
+    with torch.cuda.stream(st.copy_stream):
+        for i in order:
+            xi, wh = layers_host[i]
+            if xi not in x_ready:
+                xs_d[xi].copy_(xs_host[xi], non_blocking=True)
+                x_ready[xi] = torch.cuda.Event()
+                x_ready[xi].record(st.copy_stream)
+            ws_d[i].copy_(wh, non_blocking=True)
+            w_ready[i] = torch.cuda.Event()
+            w_ready[i].record(st.copy_stream)
+    return x_ready, w_ready
+
+
 def quantize_block_host(xs_host: Sequence[torch.Tensor], layers_host, alpha_grid: Sequence[float], bits: int = 4,
                         group: int = 128, stat: int = STAT_MEAN, device="cuda",
                         workspace: Optional[Workspace] = None, state: Optional[BlockHostState] = None,
-                        loss_form: int = LOSS_ERROR):
+                        loss_form: int = LOSS_ERROR, prefetch=None):
     """A block's linears from host buffers to host results, copies overlapped
     with compute.
 
     ``xs_host``: the distinct layer inputs (bf16, pinned for asynchronous
     copies); ``layers_host``: (input index, W fp32 on the host) per layer.
-    The layers run in an order that starts the device early and ends it
-    soon after the last search: the layer with the smallest W first, the
-    second smallest last, the others as given.  A copy stream uploads, in that
-    order, each input before the first layer that reads it and each layer's W;
-    the current stream computes an input's statistic before its first layer,
-    then each layer's search (``awq_search``), s* and pack as soon as its W has
-    landed; a third stream copies each layer's L, alpha*, status, codes and
-    scales back as soon as they are done.  Synchronises, checks every status
-    word and returns a list of dicts of host tensors in the layers' given
-    order (reused across calls through ``state``)."""
+    The layers run smallest W first, second smallest last, the others as
+    given.  A copy stream uploads, in that order, each input before the first
+    layer that reads it and each layer's W; the current stream computes an
+    input's statistic before its first layer, then each layer's search
+    (``awq_search``), s* and pack as soon as its W has landed; a third stream
+    copies each layer's L, alpha*, status, codes and scales back as soon as
+    they are done.
+
+    ``prefetch``: the next block's ``(xs_host, layers_host)``.  Their upload is
+    queued on the copy stream behind this block's, into the state's other set
+    of device buffers, so that it runs while this block computes; the next
+    call with the same host buffers (and ``state``) finds them uploaded and
+    starts at once.  Those host buffers must keep their contents until that
+    call.  Synchronises the compute and result streams (not an upload ahead),
+    checks every status word and returns a list of dicts of host tensors in
+    the layers' given order (reused across calls through ``state``: read them
+    before the next call)."""
     dev = torch.device(device)
     st = state if state is not None else BlockHostState()
     compute = torch.cuda.current_stream(dev)
     if st.copy_stream is None:
         st.copy_stream = torch.cuda.Stream(dev)
         st.back_stream = torch.cuda.Stream(dev)
-    if st.xs is None:
-        st.xs = [torch.empty(x.shape, dtype=x.dtype, device=dev) for x in xs_host]
-        st.ws = [torch.empty(w.shape, dtype=w.dtype, device=dev) for _, w in layers_host]
-    by_size = sorted(range(len(layers_host)), key=lambda i: (layers_host[i][1].numel(), i))
-    if len(by_size) > 2:
-        first, last = by_size[0], by_size[1]
-        order = [first] + [i for i in range(len(layers_host)) if i not in (first, last)] + [last]
+    order = _block_order(layers_host)
+    key = _host_key(xs_host, layers_host)
+    if st.pending is not None and st.pending[0] == key:
+        _, b, x_ready, w_ready = st.pending    # uploaded ahead by the previous call
     else:
-        order = by_size
-    # the previous call's device work on these buffers has finished (it synchronised)
-    st.copy_stream.wait_stream(compute)
-    x_ready, w_ready = {}, {}
-    with torch.cuda.stream(st.copy_stream):
-        for i in order:
-            xi, wh = layers_host[i]
-            if xi not in x_ready:
-                st.xs[xi].copy_(xs_host[xi], non_blocking=True)
-                x_ready[xi] = torch.cuda.Event()
-                x_ready[xi].record(st.copy_stream)
-            st.ws[i].copy_(wh, non_blocking=True)
-            w_ready[i] = torch.cuda.Event()
-            w_ready[i].record(st.copy_stream)
+        b = st.cur
+        _block_buffers(st, b, xs_host, layers_host, dev)
+        # the previous call's device work on these buffers has finished (it synchronised)
+        st.copy_stream.wait_stream(compute)
+        x_ready, w_ready = _block_upload(st, b, order, xs_host, layers_host)
+    st.pending = None
+    st.cur = b
+    xs_d, ws_d = st.bufs[b]
     pin = all(x.is_pinned() for x in xs_host)
-    if st.results is None:
+    if st.results is None or len(st.results) != len(layers_host):
         st.results = []
-        for (xi, _), wd in zip(layers_host, st.ws):
+        for (xi, _), wd in zip(layers_host, ws_d):
             D_in, D_out = wd.shape
             st.results.append({
                 "L": torch.empty(len(alpha_grid), dtype=torch.float64, pin_memory=pin),
@@ -724,12 +770,12 @@ def quantize_block_host(xs_host: Sequence[torch.Tensor], layers_host, alpha_grid
     a = {}
     for i in order:
         xi, _ = layers_host[i]
-        wd = st.ws[i]
+        wd = ws_d[i]
         if xi not in a:                            # the input's statistic, before its first layer
             compute.wait_event(x_ready[xi])
-            a[xi] = act_stats(st.xs[xi], stat)
+            a[xi] = act_stats(xs_d[xi], stat)
         compute.wait_event(w_ready[i])
-        r = search(st.xs[xi], wd, a[xi], alpha_grid, bits, group, workspace=workspace, check_status=False,
+        r = search(xs_d[xi], wd, a[xi], alpha_grid, bits, group, workspace=workspace, check_status=False,
                    loss_form=loss_form)
         s_star = scales(a[xi], r.alpha_star)
         packed, sc = quantize_pack(wd, s_star, bits, group)
@@ -742,6 +788,13 @@ def quantize_block_host(xs_host: Sequence[torch.Tensor], layers_host, alpha_grid
                             ("scales", sc)):
                 t.record_stream(st.back_stream)
                 host[name].copy_(t, non_blocking=True)
+    if prefetch is not None:
+        nxs, nlayers = prefetch
+        nb = 1 - b
+        # set nb was last read by an earlier call, whose device work has finished
+        _block_buffers(st, nb, nxs, nlayers, dev)
+        nx_ready, nw_ready = _block_upload(st, nb, _block_order(nlayers), nxs, nlayers)
+        st.pending = (_host_key(nxs, nlayers), nb, nx_ready, nw_ready)
     st.back_stream.synchronize()
     compute.synchronize()
     for host in st.results:

@@ -93,3 +93,26 @@ def test_quantize_block_host_layer_against_oracle(awq):
     assert np.allclose(L, L_or, rtol=1e-2, atol=0)
     check_alpha(L_or, best_or, int(np.argmin(L)))
     assert float(res[2]["alpha_star"][0]) == np.float32(GRID[int(np.argmin(L))])
+
+
+def test_quantize_block_host_prefetch_chain(awq):
+    """Blocks in a row, each call queueing the next block's upload
+    (``prefetch``): every block's results equal the single-layer calls; a
+    call whose inputs are not the prefetched ones uploads its own."""
+    blocks = [_block(20 + 3 * i) for i in range(3)] + [_block(40)]
+    pinned = [([x.pin_memory() for x in xs], [(xi, w.pin_memory()) for xi, w in layers]) for xs, layers in blocks]
+    state, ws = awq.BlockHostState(), awq.Workspace()
+    # 0 -> 1 -> 2 with prefetch, then 3, whose upload was not queued (2 queued block 0 again)
+    plan = [(0, 1), (1, 2), (2, 0), (3, None)]
+    for cur, nxt in plan:
+        xs_h, layers_h = pinned[cur]
+        res = awq.quantize_block_host(xs_h, layers_h, GRID, 4, 128, workspace=ws, state=state,
+                                      prefetch=None if nxt is None else pinned[nxt])
+        got = [{k: v.clone() for k, v in r.items()} for r in res]
+        ref = _single(awq, *blocks[cur])
+        for host, (L, a_star, packed, sc) in zip(got, ref):
+            assert int(host["status"][0]) == 0
+            assert torch.equal(host["L"], L)
+            assert torch.equal(host["alpha_star"], a_star)
+            assert torch.equal(host["packed"], packed)
+            assert torch.equal(host["scales"], sc)
