@@ -48,10 +48,11 @@
 // Work: a unit is (256 output columns) x (256 tokens) for a pair; per unit the
 // passes are the alphas (after the reference pass in the reference form).
 // Units are dealt round robin in whole waves, all pairs advancing through
-// alpha in step (so the operand of one alpha is read from HBM once and shared
-// through L2); the alpha passes of the last partial wave are split evenly
-// over all pairs.  Units are numbered in token blocks sized to L2 (see
-// unit_tiles and search_token_block).
+// alpha in step (so the operand of one alpha is read from HBM about once and
+// shared through L2); the alpha passes of the last partial wave are dealt
+// round robin over all pairs, alpha-major (see Schedule).  Units are numbered
+// in token blocks sized to L2 (see unit_tiles and search_token_block).  The
+// TMA loads mark X tiles evict-last and operand tiles evict-first in L2.
 //
 // Every mbarrier wait is bounded: on a timeout the kernel records
 // AWQ_ETIMEOUT in the status word, every role leaves its loop, in-flight
