@@ -76,6 +76,8 @@ def _case(awq, N, D_in, D_out, bits, group, seed):
     (1, 256, 38912, 4, 128),      # GEMV: more column tiles (304) than resident CTAs, one CTA per whole tile
     (2, 1024, 38916, 4, 64),      # the same with a ragged last tile of one column quad, 8-row batches
     (1, 128, 2048, 4, 64),        # GEMV: too few batches for clusters, stream-K shares and the reduce launch
+    (4, 1024, 32768, 4, 128),     # GEMV, four tokens: more tiles than resident clusters, stream-K
+    (3, 1024, 32768, 2, 32),      # GEMV, three tokens, 2-bit, group 32: stream-K
     (5, 512, 200, 4, 128),        # ragged columns, a few tokens
     (16, 96, 36, 4, 32),          # D_in not a multiple of 64: a half k block
     (37, 384, 132, 3, 64),
@@ -180,6 +182,8 @@ def _zp_case(awq, N, D_in, D_out, bits, group, seed):
     (3, 1024, 132, 3, 64),        # GEMV, ragged column tile
     (4, 256, 1000, 2, 32),        # GEMV, 2-bit, group 32
     (2, 2048, 256, 4, 256),       # GEMV, group 256
+    (1, 1024, 32768, 4, 128),     # GEMV: stream-K shares and the reduce launch
+    (3, 256, 38912, 4, 64),       # GEMV: one CTA per whole tile
     (5, 512, 200, 4, 128),        # tensor cores, stream-K, ragged columns
     (37, 384, 132, 3, 64),
     (17, 8192, 2048, 4, 128),     # stream-K shares inside one unit
