@@ -325,6 +325,30 @@ def test_batched_matches_single(awq, form):
         assert int(rb.alpha_idx) == int(rs.alpha_idx)
 
 
+def _batched_layers(awq, shapes, seed):
+    layers = []
+    for i, (N, D_in, D_out) in enumerate(shapes):
+        X, W = _layer(N, D_in, D_out, seed=seed + i)
+        layers.append((X.cuda(), W.cuda(), awq.act_stats(X.cuda())))
+    return layers
+
+
+def test_batched_overlap_varied_inputs(awq):
+    """Layers whose D_in and D_out shrink and grow (so every workspace region
+    changes its layout from one layer to the next, ragged token and column
+    tails included) give bit for bit the single-layer L, per-column L and
+    alpha* when searched in one batched call."""
+    shapes = [(300, 512, 128), (300, 256, 64), (257, 1024, 256), (300, 256, 132), (64, 512, 68)]
+    layers = _batched_layers(awq, shapes, 40)
+    grid = synth.alpha_grid(20).tolist()
+    batched = awq.search_batched(layers, grid, 4, 128, want_cols=True)
+    for (X, W, a), rb in zip(layers, batched):
+        rs = awq.search(X, W, a, grid, 4, 128, want_cols=True)
+        assert torch.equal(rb.L, rs.L)
+        assert torch.equal(rb.L_col, rs.L_col)
+        assert int(rb.alpha_idx) == int(rs.alpha_idx)
+
+
 # ------------------------------------------------------------------ quantiser arithmetic
 @pytest.mark.parametrize("divisor", [1, 3, 7, 15, 31, 127, 255])
 def test_constant_divisor_matches_ieee_on_every_float(awq, divisor):
