@@ -25,7 +25,9 @@
  *     only enqueue work; they are asynchronous with respect to the host and
  *     do not synchronise.  Scratch space comes from a caller-provided
  *     workspace whose size is queried (or, for awq_search_noalloc, a fixed
- *     array inside the library).  The library calls no allocator.
+ *     array inside the library).  The library calls no allocator.  A
+ *     workspace serves one call at a time: two calls in flight on different
+ *     streams need two workspaces.
  *   - The return value is an awq_status.  A non-OK status from argument
  *     checking is returned before any work is enqueued; awq_get_last_error()
  *     then describes it.  Errors found on the device (a wait that timed out)
@@ -183,6 +185,10 @@ AWQ_API size_t awq_search_workspace_size(int64_t N, int64_t D_in, int64_t D_out,
  *               call, then AWQ_ETIMEOUT | (site << 8) if a pipeline wait gave
  *               up; the outputs are then invalid.  Read it after the stream
  *               has been synchronised.
+ * The kernel's CTAs keep their alpha passes in step through a counter in the
+ * workspace (zeroed by the call on `stream`).  A CTA that has waited 2 ms for
+ * the others (another kernel holding the SMs some of them need) stops waiting
+ * for the rest of the launch; the results never depend on it.
  */
 AWQ_API int awq_search(const void* X, const float* W, const float* a, int64_t N, int64_t D_in, int64_t D_out,
                        const float* alpha_grid, int n_alpha, int bits, int group, int loss_form, double* L,

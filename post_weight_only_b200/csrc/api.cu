@@ -133,7 +133,7 @@ uint64_t timeout_ns() {
 }
 
 struct SearchLayout {
-  size_t s_tab, r_tab, op, wt, yref, partial, blk, status, total;
+  size_t s_tab, r_tab, op, wt, yref, partial, blk, status, sync, total;
   int grid, H, nblk;
 };
 
@@ -159,6 +159,7 @@ SearchLayout search_layout(int64_t N, int64_t D_in, int64_t D_out, int A, int gr
   L.partial = take(a * L.H * D_out * 4);
   L.blk = take(a * L.nblk * 8);
   L.status = take(4);
+  L.sync = take(4);
   L.total = off;
   return L;
 }
@@ -312,7 +313,7 @@ int search_one(const void* X, const float* W, const float* a, int64_t N, int64_t
   }
   if (e != cudaSuccess) return fail_cuda(e, "weight transpose kernel");
   awq::SearchShape sh{static_cast<int>(N), static_cast<int>(D_in), static_cast<int>(D_out), A, bits, group, form};
-  awq::SearchBuffers b{X, wt, op, yref, partial, nullptr, status};
+  awq::SearchBuffers b{X, wt, op, yref, partial, nullptr, status, reinterpret_cast<unsigned*>(ws + lay.sync)};
   const char* what = "search kernel";
   int rc;
   {

@@ -118,6 +118,7 @@ struct SearchBuffers {
   float* partial;             // [A][search_partial_rows(N)][D_out]
   float* y_out;               // gemm-only mode: [N][D_out]
   int* status;
+  unsigned* sync = nullptr;   // 4 bytes of device memory for the producers' pass counter, or null (no sync)
 };
 int search_grid_size(const SearchShape& sh, int num_sms);
 int search_token_tiles(int N);

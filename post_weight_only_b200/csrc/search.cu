@@ -48,11 +48,14 @@
 // Work: a unit is (256 output columns) x (256 tokens) for a pair; per unit the
 // passes are the alphas (after the reference pass in the reference form).
 // Units are dealt round robin in whole waves, all pairs advancing through
-// alpha in step (so the operand of one alpha is read from HBM about once and
-// shared through L2); the alpha passes of the last partial wave are dealt
-// round robin over all pairs, alpha-major (see Schedule).  Units are numbered
-// in token blocks sized to L2 (see unit_tiles and search_token_block).  The
-// TMA loads mark X tiles evict-last and operand tiles evict-first in L2.
+// alpha in step: the producers meet at every pass boundary of the full waves
+// (a soft barrier on a global counter, see pass_sync_wait), so that the pairs
+// sharing an operand tile read it at about the same time and it is fetched
+// from HBM about once and shared through L2.  The alpha passes of the last
+// partial wave are dealt round robin over all pairs, alpha-major (see
+// Schedule).  Units are numbered in token blocks sized to L2 (see unit_tiles
+// and search_token_block).  The TMA loads mark X tiles evict-last and
+// operand tiles evict-first in L2.
 //
 // Every mbarrier wait is bounded: on a timeout the kernel records
 // AWQ_ETIMEOUT in the status word, every role leaves its loop, in-flight
@@ -80,10 +83,8 @@ constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*align*/;
 constexpr uint16_t kPairMask = 0x3;
-// L2 budget for the X tiles of one token block of the unit order, and the
-// fewest tiles worth keeping as a block.
+// L2 budget for the X tiles of one token block of the unit order.
 constexpr long long kXBlockBudgetBytes = 64ll << 20;
-constexpr int kMinBlockTiles = 8;
 static_assert(kHalfN == kBM, "operand and X half-tiles share one box shape");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
@@ -94,6 +95,7 @@ struct Params {
   int N, D_in, D_out, A;
   int Tt, Wt, U, KB, H, gemm_only;
   int tb;                     // token tiles per token block of the unit order (see unit_tiles)
+  unsigned* sync;             // pass counter of the full waves (see pass_sync_wait), or null
   const uint16_t* op;         // Gram form: the operand E [A][D_out][D_in], read by the epilogue
   float* yref;
   float* partial;
@@ -167,6 +169,35 @@ struct Schedule {
     return false;
   }
 };
+
+// The producers of all CTAs keep their passes of the full waves in step: at
+// the start of pass q (q >= 1) each one adds 1 to *sync (it has issued every
+// load of pass q - 1) and waits until all gridDim.x producers have done so.
+// The pairs that share an operand tile (one weight tile, a block's token
+// tiles) then read each of its k-slices within a short interval, so the
+// slice is fetched from DRAM about once and served from L2 to the others;
+// left to drift apart by up to a few passes, they fetched it ~10x.  The wait
+// is a hint, not a dependency of the result: a producer that has waited
+// kSyncPatienceNs (another kernel holding SMs that a CTA of this grid needs,
+// say) stops waiting for the rest of the launch and only keeps counting.
+constexpr uint64_t kSyncPatienceNs = 2000000;
+
+__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned* ptr) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+
+// true: all producers reached `target`; false: gave up (or the CTA aborted).
+__device__ bool pass_sync_wait(const unsigned* ctr, unsigned target, volatile int* abort_flag) {
+  if (static_cast<int>(ld_relaxed_gpu(ctr) - target) >= 0) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    __nanosleep(64);
+    if (static_cast<int>(ld_relaxed_gpu(ctr) - target) >= 0) return true;
+    if (*abort_flag || globaltimer_ns() - t0 > kSyncPatienceNs) return false;
+  }
+}
 
 // Unit order: the token tiles are cut into blocks of tb tiles (the last block
 // may be shorter); the units of one block come before the next block's,
@@ -259,6 +290,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int s = 0; s < kStages; ++s) last_round[s] = -1;
       bool ok = true;
       const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
+      unsigned q = 0;                   // passes of the full waves begun
+      bool in_step = p.sync != nullptr;
       while (ok && sch.next(sg)) {
         int wt, tt;
         unit_tiles(p, sg.u, wt, tt);
@@ -266,6 +299,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int tok0 = tt * kBN + static_cast<int>(rank) * kHalfN;     // this CTA's tokens
         for (int pass = first_pass<kForm>(sg); ok && pass < sg.a1; ++pass) {
           const bool ref = is_ref_pass<kForm>(sg, pass);
+          if (p.sync && sg.u < sch.head) {
+            if (q > 0) {
+              atomicAdd(p.sync, 1u);
+              if (in_step) in_step = pass_sync_wait(p.sync, q * gridDim.x, abort_flag);
+            }
+            ++q;
+          }
           for (int kb = 0; kb < p.KB; ++kb, ++it) {
             const int s = it % kStages;
             const uint32_t r = it / kStages;
@@ -601,21 +641,18 @@ bool make_word_map(CUtensorMap* m, const void* base, bool is_float, uint64_t inn
 int search_token_tiles(int N) { return (N + kBN - 1) / kBN; }
 
 // Token tiles per block of the unit order: as many as keep the block's X tiles
-// (256 tokens x D_in bf16 each) within an L2 budget, balanced over the blocks.
-// Per wave, the operand of every alpha is read once for the wave's few weight
-// tiles, and the block's X tiles once for all its waves.  When fewer than
-// kMinBlockTiles X tiles fit (a very long reduction dimension), a block is a
-// single token tile: every pair of a wave then shares that tile and reads its
-// own weight tiles.  Measured on B200 (21 alphas, N = 4096): the 28672 x 8192
-// down projection ran 28.0 ms with blocks of one token tile against 29.9 ms
-// with four and 35.3 ms with all sixteen; the 11008-input layer was fastest
-// with blocks of 8, the 8192-input layers with all 16, and the 16384-token
-// layer with 32 -- the choices this budget makes.
+// (256 tokens x D_in bf16 each) within an L2 budget, balanced over the blocks
+// (one tile when not even one fits).  Per wave, the operand of every alpha is
+// read once for the wave's few weight tiles, and the block's X tiles once for
+// all its waves.  Measured on B200 with the pass barrier (21 alphas, N = 4096,
+// the 70B block): the 28672 x 8192 down projection took 32.8-34.0 ms with
+// blocks of four token tiles against 34.4 with one and 31.6-34.7 with two,
+// the whole step 122.7-123.3 ms against 124.6-125.0 and 125.6-126.0.
 int search_token_block(const SearchShape& sh, int Tt) {
   const double tile_bytes = 2.0 * kBN * static_cast<double>(sh.D_in);
   const double budget = static_cast<double>(kXBlockBudgetBytes);
   int tmax = static_cast<int>(budget / tile_bytes);
-  if (tmax < kMinBlockTiles) return 1;
+  if (tmax < 1) return 1;
   if (tmax >= Tt) return Tt;
   const int nblk = (Tt + tmax - 1) / tmax;
   return (Tt + nblk - 1) / nblk;
@@ -677,6 +714,17 @@ int launch_search(const SearchShape& sh, const SearchBuffers& b, int grid, uint6
   p.y_out = b.y_out;
   p.status = b.status;
   p.timeout_ns = timeout_ns;
+  // the pass counter, for a grid with at least one full wave of units
+  const bool sync = b.sync && !gemm_only && p.U >= grid / 2 && grid >= 4;
+  p.sync = sync ? b.sync : nullptr;
+  if (sync) {
+    const cudaError_t e0 = cudaMemsetAsync(b.sync, 0, sizeof(unsigned), st);
+    if (e0 != cudaSuccess) {
+      *cerr = e0;
+      *what = "cudaMemsetAsync(pass counter)";
+      return kECuda;
+    }
+  }
 
   cudaError_t e = form == kFormError  ? launch_form<kFormError>(grid, mX, mWt, mOp, p, st)
                   : form == kFormGram ? launch_form<kFormGram>(grid, mX, mWt, mOp, p, st)

@@ -349,6 +349,36 @@ def test_batched_overlap_varied_inputs(awq):
         assert int(rb.alpha_idx) == int(rs.alpha_idx)
 
 
+def test_concurrent_searches_on_two_streams(awq):
+    """Two searches in flight at once on two streams, each with its own
+    workspace.  Each grid has a full wave of units (16 token tiles x 5 weight
+    tiles on 74 CTA pairs), so its producers meet at every pass boundary; a
+    grid whose CTAs wait for SMs that the other grid holds must stop waiting
+    rather than stall.  The results equal those of the same searches run one
+    after the other."""
+    grid = synth.alpha_grid(20).tolist()
+    layers = []
+    for i in range(2):
+        X, W = _layer(4096, 512, 1280, seed=80 + i)
+        X, W = X.cuda(), W.cuda()
+        layers.append((X, W, awq.act_stats(X)))
+    ref = [awq.search(X, W, a, grid, 4, 128, want_cols=True) for X, W, a in layers]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    out = []
+    for (X, W, a), st in zip(layers, streams):
+        st.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(st):
+            out.append(awq.search(X, W, a, grid, 4, 128, want_cols=True, workspace=awq.Workspace(),
+                                  check_status=False))
+    torch.cuda.synchronize()
+    for r, rr in zip(out, ref):
+        awq.check_device_status(r.status)
+        assert torch.equal(r.L, rr.L)
+        assert torch.equal(r.L_col, rr.L_col)
+        assert int(r.alpha_idx) == int(rr.alpha_idx)
+
+
 # ------------------------------------------------------------------ quantiser arithmetic
 @pytest.mark.parametrize("divisor", [1, 3, 7, 15, 31, 127, 255])
 def test_constant_divisor_matches_ieee_on_every_float(awq, divisor):
