@@ -32,6 +32,7 @@ Prints one JSON line (rank 0).
 from __future__ import annotations
 
 import argparse
+import gc
 import hashlib
 import json
 import os
@@ -741,17 +742,27 @@ def clip_section(dev, flush, flush_sink):
     torch.cuda.synchronize()
     reps = 10
     times = []
-    for _ in range(reps):
-        flush.zero_()
-        flush_sink.add_(flush.amax())
-        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ea.record()
-        cr = awq.clip_search(X, W, r.s_star, cgrid, bits, group, workspace=cws, check_status=False)
-        eb.record()
-        times.append((ea, eb))
-    torch.cuda.synchronize()
+    # The call is a few short launches: a host-side pause inside the region
+    # (a collection of the earlier sections' garbage) would leave the device
+    # idle between them, so collection is held off while it is timed and the
+    # median call is reported beside the mean.
+    gc.collect()
+    gc.disable()
+    try:
+        for _ in range(reps):
+            flush.zero_()
+            flush_sink.add_(flush.amax())
+            ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ea.record()
+            cr = awq.clip_search(X, W, r.s_star, cgrid, bits, group, workspace=cws, check_status=False)
+            eb.record()
+            times.append((ea, eb))
+        torch.cuda.synchronize()
+    finally:
+        gc.enable()
     awq.check_device_status(cr.status)
-    call_ms = sum(a_.elapsed_time(b_) for a_, b_ in times) / reps
+    per_call = sorted(a_.elapsed_time(b_) for a_, b_ in times)
+    call_ms = per_call[reps // 2]
     awq.profile_enable(True)
     awq.profile_reset()
     for _ in range(3):
@@ -764,7 +775,8 @@ def clip_section(dev, flush, flush_sink):
     hbm = float(load_peaks()[0]["hbm_gbs"])
     return {
         "layer": f"{spec.name} (N={spec.N}, D_in={spec.D_in}, D_out={spec.D_out}), {C} ratios, 4-bit g128",
-        "ms_per_call": call_ms, "n_clip": C,
+        "ms_per_call": call_ms, "ms_per_call_mean": sum(per_call) / reps, "ms_per_call_max": per_call[-1],
+        "n_clip": C,
         "stages_ms": {k: cprof[k][0] / max(cprof[k][1], 1) for k in ("clip_gram", "clip_operand", "clip_loss")},
         "loss_kernel": {"algorithmic_bytes": op_bytes, "achieved_gbs": op_bytes / (loss_ms / 1e3) / 1e9,
                         "frac_hbm": op_bytes / (loss_ms / 1e3) / 1e9 / hbm,
@@ -857,14 +869,15 @@ def w4a16_section(dev, rank):
     bits, group = 4, 128
     g4 = torch.Generator(device=dev).manual_seed(4321 + rank)
     info = {"timing": "best of 5 replays of a CUDA graph of 20 calls (N <= 4: one GEMV launch whose column-tile splits are "
-                      "reduced in a cluster, or a stream-K GEMV and a dependent reduce launch; else a status "
+                      "reduced in a cluster (N = 1-2 on the CUDA cores, 3-4 on mma.sync tiles), or a stream-K GEMV "
+                      "and a dependent reduce launch; else a status "
                       "clear, the pre-pass and the GEMM), weights rotated over copies > 256 MiB; synthetic "
                       "packed words and deltas",
             "algorithmic_bytes": "packed words + fp32 deltas + X (bf16) + s + Y (fp32), each once"}
     peaks, _ = load_peaks()
     hbm_peak, bf16_peak = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
-    for name, (Dk, Dn, Ns) in (("down_proj_28672x8192", (28672, 8192, (1, 4, 16))),
-                                ("attn_proj_4096x4096", (4096, 4096, (1, 16, 4096))),
+    for name, (Dk, Dn, Ns) in (("down_proj_28672x8192", (28672, 8192, (1, 2, 4, 16))),
+                                ("attn_proj_4096x4096", (4096, 4096, (1, 4, 16, 4096))),
                                 ("square_8192x8192", (8192, 8192, (4096,)))):
         packed_q = torch.randint(-2 ** 31, 2 ** 31 - 1, (Dk // 8, Dn), generator=g4, device=dev,
                                  dtype=torch.int64).to(torch.int32)
@@ -881,7 +894,7 @@ def w4a16_section(dev, rank):
             gbs = nbytes / (ms / 1e3) / 1e9
             tf = 2.0 * Nq * Dk * Dn / (ms / 1e3) / 1e12
             info[f"{name}_N{Nq}"] = {
-                "path": "cuda-core GEMV" if Nq <= 4 else "tcgen05 GEMM", "ms": ms, "algorithmic_bytes": nbytes,
+                "path": ("cuda-core GEMV" if Nq <= 2 else "mma.sync GEMV") if Nq <= 4 else "tcgen05 GEMM", "ms": ms, "algorithmic_bytes": nbytes,
                 "achieved_gbs": gbs, "frac_hbm": gbs / hbm_peak, "tflops": tf, "frac_bf16": tf / bf16_peak}
         del weights, packed_q
     torch.cuda.empty_cache()

@@ -402,11 +402,18 @@ AWQ_API int awq_quantize_pack_zp(const float* W, const float* s, int64_t D_in, i
  * AWQ paper, TinyChat section, "on-the-fly weight dequantization"):
  *     Y[t][n] = sum_k x_tk / s_k * (u_kn - 2^(bits-1)) * scales[k/group][n]
  * with u the offset-binary codes of `packed` (the layout of
- * awq_quantize_pack).  N <= 4 (decode): a CUDA-core GEMV in fp32 (x / s
+ * awq_quantize_pack).  N <= 2 (decode): a CUDA-core GEMV in fp32 (x / s
  * rounded once, exact integer weights, delta applied once per group): the
- * (column tile, k rows) work is shared out evenly over a grid that fills
- * every SM (stream-K), and a second small launch adds the CTAs' sums of
- * each tile in a fixed order from the workspace.
+ * splits of each column tile form a thread-block cluster whose first CTA
+ * adds the others' sums in a fixed order, or, when the clusters do not fit
+ * in one wave, the (column tile, k rows) work is shared out evenly over a
+ * grid that fills every SM (stream-K) and a second small launch adds the
+ * CTAs' sums of each tile in a fixed order from the workspace.
+ * N = 3 or 4 with D_in <= 65536: one launch of warp-level tensor-core tiles
+ * (x / s rounded once to bf16, exact integer codes, fp32 accumulation, the
+ * fp32 delta applied once per group), the splits of each column tile summed
+ * in a fixed order inside a cluster; no workspace is used.  Longer rows take
+ * the CUDA-core GEMV.
  * N > 4: two launches on `stream`, X' = bf16(X / s) into the workspace, then
  * a tensor-core GEMM that dequantises the weights into shared memory as
  * bf16((u - 2^(bits-1)) * bf16(delta)) (one rounding of the product) and
@@ -434,8 +441,9 @@ AWQ_API int awq_w4a16_gemm(const void* X, const float* s, const uint32_t* packed
  * compassingai.com AWQ concept page, "the AWQ mechanism", symmetric or
  * asymmetric quantisation; "inference-time equivalent" for the product):
  *     Y[t][n] = sum_k x_tk / s_k * (u_kn - z[k/group][n]) * scales[k/group][n]
- * with the same two paths and roundings: the GEMV subtracts each group's zero
- * point exactly in fp32; the tensor-core path forms bf16((u - z) * bf16(delta))
+ * with the same paths and roundings: the CUDA-core GEMV subtracts each
+ * group's zero point exactly in fp32, the tensor-core GEMV adds
+ * (2^(bits-1) - z) times the group's sum of bf16 x / s; the tensor-core path forms bf16((u - z) * bf16(delta))
  * (u - z is exact) from a per-(group, column) fp32 copy of 128 + z that a
  * first small kernel writes into the workspace.
  *   zeros     [D_in/group][D_out] uint8 zero points (device), 16-byte aligned

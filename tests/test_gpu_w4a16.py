@@ -2,10 +2,12 @@
 applied to activations) against the oracle, on codes packed by the library
 itself.
 
-Two CUDA paths: N <= 4 tokens run the CUDA-core GEMV (fp32 throughout: x / s
-rounded once to fp32, exact integer weights, delta applied per k8 row); more
-tokens run the tensor-core GEMM.  The bound below, derived for the GEMM,
-covers the GEMV's smaller errors too.
+Three CUDA paths: one or two tokens run the CUDA-core GEMV (fp32 throughout:
+x / s rounded once to fp32, exact integer weights, delta applied per group);
+three or four tokens run the mma.sync GEMV (x / s rounded once to bf16, exact
+integer codes, fp32 accumulation, the fp32 delta applied per group); more
+tokens run the tcgen05 GEMM.  The bound below, derived for the GEMM, covers the GEMVs'
+smaller errors too.
 
 Tolerance, from the arithmetic of the tensor-core path: x_tk / s_k is rounded to
 bf16 once, each weight q * bf16(delta) is rounded to bf16 once (relative
@@ -92,6 +94,10 @@ def _case(awq, N, D_in, D_out, bits, group, seed):
     (32, 2048, 640, 4, 64),       # the largest 4-k-block-stage token tile (Nt = 32), group 64
     (33, 2048, 640, 4, 128),      # the smallest 2-k-block-stage token tile (Nt = 48)
     (3, 1056, 96, 2, 32),         # group 32 (two groups per k block), 2-bit, D_in not a multiple of 256
+    (3, 65536, 128, 4, 128),      # 3-4 tokens: eight CTAs of 8192 rows, the largest X' in shared memory
+    (3, 65792, 64, 4, 256),       # past that range: the CUDA-core GEMV at three tokens
+    (4, 4096, 1280, 3, 64),       # 3-4 tokens: ten tiles split eight ways
+    (4, 96, 4, 4, 32),            # 3-4 tokens: three groups over eight warps, one column quad
 ])
 def test_w4a16_against_oracle(awq, N, D_in, D_out, bits, group):
     Y, Y_or, bound = _case(awq, N, D_in, D_out, bits, group, seed=N + D_in)
