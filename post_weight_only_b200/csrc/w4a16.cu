@@ -958,8 +958,11 @@ __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float4* __restri
 // split one tile's groups form a cluster, and rank 0 adds their sums in rank
 // order from their shared memory (DSMEM), so the result does not depend on
 // timing.  Each lane keeps 7 steps of 16 bytes in flight (a ring of cp.async
-// copies in shared memory).  The host takes cw = 4: 256-column tiles and a
-// ring of 16 steps were both measured slower on a 28672 x 8192 layer.  A group's
+// copies in shared memory); the loop runs over the warp's groups with the
+// group's steps unrolled (the group size is a template argument), which cut
+// the loop's bookkeeping by a sixth of the time.  The host takes cw = 4:
+// 256-column tiles and a ring of 16 steps were both measured slower on a
+// 28672 x 8192 layer.  A group's
 // delta is applied once, after its last step; the zero-point form adds
 // (off - z) times the group's sum of X' at the same point.  No waits on other
 // CTAs beyond the cluster barrier, no workspace.
@@ -1013,10 +1016,10 @@ __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
 // Y [NT][D_out] fp32 (any 4-byte alignment).  Grid: tiles x S CTAs, clusters
 // of S along x; a tile is 32 cw columns.  k8max / gmax: k8 rows / groups of
 // the largest CTA range.
-template <int NT, bool kZp>
+template <int NT, int G, bool kZp>
 __global__ void __launch_bounds__(kMmThreads, 2) w4a16_gemv_mma_kernel(
     const uint4* __restrict__ X, const float4* __restrict__ s, const uint32_t* __restrict__ packed,
-    const float4* __restrict__ scales, const uint8_t* __restrict__ zeros, int64_t D_in, int64_t D_out, int G,
+    const float4* __restrict__ scales, const uint8_t* __restrict__ zeros, int64_t D_in, int64_t D_out,
     int off, int S, int cw, int k8max, int gmax, float* __restrict__ Y, int* __restrict__ status) {
   static_assert(NT >= 2 && NT <= 4, "2-4 token slots");
   extern __shared__ __align__(16) uint8_t mm_sm[];
@@ -1031,7 +1034,7 @@ __global__ void __launch_bounds__(kMmThreads, 2) w4a16_gemv_mma_kernel(
   const int rank = static_cast<int>(cluster_ctarank());
   const int64_t tile = blockIdx.x / S;
   const int64_t ng = D_in / G, rows8 = D_in / 8;
-  const int gr8 = G / 8, spg = G / 32;            // k8 rows and steps (4 k8 rows each) per group
+  constexpr int gr8 = G / 8, spg = G / 32;        // k8 rows and steps (4 k8 rows each) per group
   const int64_t ga = ng * rank / S, gb = ng * (rank + 1) / S;   // this CTA's groups
   const int kw = 8 / cw, cols = 32 * cw;          // warps per slice, columns per tile
   const int part = warp / cw, slice = warp % cw;
@@ -1118,53 +1121,54 @@ __global__ void __launch_bounds__(kMmThreads, 2) w4a16_gemv_mma_kernel(
     dcur = __ldg(scales + wa * D4 + c0 / 4);
     if (kZp) zcur = __ldg(reinterpret_cast<const uint32_t*>(zeros + wa * D_out + c0));
   }
-  int sg = 0;
 #pragma unroll 1
-  for (int st = 0; st < nsteps; ++st) {
-    issue();                                      // the step kMmRing - 1 ahead, into the entry used last
-    cp_async_wait<kMmRing - 1>();                 // this lane's copy of step st has landed
-    const uint4 w = my_ring[(st & (kMmRing - 1)) * kMmThreads];
-    uint4 xb = make_uint4(0u, 0u, 0u, 0u);
-    if (xin) xb = *reinterpret_cast<const uint4*>(xrow + st * 64);
-    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+  for (int gl = 0; gl < nsteps / spg; ++gl) {     // one group of this warp: spg steps, then its delta
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {                 // columns c0 + 2h (A row g) and c0 + 2h + 1 (A row g + 8)
-      const uint32_t lo = wv[2 * h], hi = wv[2 * h + 1];
-      mma_bf16_16816(acc[h], code_pair(lo, 0, bias), code_pair(hi, 0, bias), code_pair(lo, 1, bias),
-                     code_pair(hi, 1, bias), xb.x, xb.y);
-      mma_bf16_16816(acc[h], code_pair(lo, 2, bias), code_pair(hi, 2, bias), code_pair(lo, 3, bias),
-                     code_pair(hi, 3, bias), xb.z, xb.w);
+    for (int q = 0; q < spg; ++q) {
+      const int st = gl * spg + q;
+      issue();                                    // the step kMmRing - 1 ahead, into the entry used last
+      cp_async_wait<kMmRing - 1>();               // this lane's copy of step st has landed
+      const uint4 w = my_ring[(st & (kMmRing - 1)) * kMmThreads];
+      uint4 xb = make_uint4(0u, 0u, 0u, 0u);
+      if (xin) xb = *reinterpret_cast<const uint4*>(xrow + st * 64);
+      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {               // columns c0 + 2h (A row g) and c0 + 2h + 1 (A row g + 8)
+        const uint32_t lo = wv[2 * h], hi = wv[2 * h + 1];
+        mma_bf16_16816(acc[h], code_pair(lo, 0, bias), code_pair(hi, 0, bias), code_pair(lo, 1, bias),
+                       code_pair(hi, 1, bias), xb.x, xb.y);
+        mma_bf16_16816(acc[h], code_pair(lo, 2, bias), code_pair(hi, 2, bias), code_pair(lo, 3, bias),
+                       code_pair(hi, 3, bias), xb.z, xb.w);
+      }
     }
-    if (++sg == spg) {                            // the group's last step: delta (sum q x' + (off - z) sum x')
-      sg = 0;
-      const float dv[4] = {dcur.x, dcur.y, dcur.z, dcur.w};
-      float corr[4][2];
+    // the group's delta (and, with zero points, (off - z) sum x')
+    const float dv[4] = {dcur.x, dcur.y, dcur.z, dcur.w};
+    float corr[4][2];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) corr[c][0] = corr[c][1] = 0.0f;
-      if (kZp) {
-        const int gl = static_cast<int>(gi - ga);
+    for (int c = 0; c < 4; ++c) corr[c][0] = corr[c][1] = 0.0f;
+    if (kZp) {
+      const int gc = static_cast<int>(gi - ga);
 #pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          const int t = 2 * j + tt;
-          const float xsum = t < NT ? xg[t * gmax + gl] : 0.0f;
+      for (int tt = 0; tt < 2; ++tt) {
+        const int t = 2 * j + tt;
+        const float xsum = t < NT ? xg[t * gmax + gc] : 0.0f;
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            corr[c][tt] = __fmul_rn(static_cast<float>(off - static_cast<int>((zcur >> (8 * c)) & 0xFFu)), xsum);
-        }
+        for (int c = 0; c < 4; ++c)
+          corr[c][tt] = __fmul_rn(static_cast<float>(off - static_cast<int>((zcur >> (8 * c)) & 0xFFu)), xsum);
       }
-      ++gi;
-      if (valid && gi < wb) {                     // the next group's delta, a group's steps ahead of its use
-        dcur = __ldg(scales + gi * D4 + c0 / 4);
-        if (kZp) zcur = __ldg(reinterpret_cast<const uint32_t*>(zeros + gi * D_out + c0));
-      }
+    }
+    ++gi;
+    if (valid && gi < wb) {                       // the next group's delta, a group's steps ahead of its use
+      dcur = __ldg(scales + gi * D4 + c0 / 4);
+      if (kZp) zcur = __ldg(reinterpret_cast<const uint32_t*>(zeros + gi * D_out + c0));
+    }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 4; ++c) {
 #pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          float& a = acc[c >> 1][2 * (c & 1) + tt];
-          tot[c][tt] = __fmaf_rn(dv[c], a + corr[c][tt], tot[c][tt]);
-          a = 0.0f;
-        }
+      for (int tt = 0; tt < 2; ++tt) {
+        float& a = acc[c >> 1][2 * (c & 1) + tt];
+        tot[c][tt] = __fmaf_rn(dv[c], kZp ? a + corr[c][tt] : a, tot[c][tt]);
+        a = 0.0f;
       }
     }
   }
@@ -1407,7 +1411,7 @@ int launch_gemv_nt(const void* X, const float* s, const uint32_t* packed, const 
 // columns; S CTAs per tile, as many as keep two CTAs on every SM (at most 8,
 // at least enough that no CTA's range of groups exceeds kMmMaxRows rows), in
 // clusters of S.
-template <int NT, bool kZp>
+template <int NT, int G, bool kZp>
 int launch_gemv_mma_k(const void* X, const float* s, const uint32_t* packed, const float* scales,
                       const uint8_t* zeros, int64_t D_in, int64_t D_out, int bits, int group, float* Y, int num_sms,
                       int* status, cudaStream_t st, cudaError_t* cerr, const char** what) {
@@ -1426,7 +1430,7 @@ int launch_gemv_mma_k(const void* X, const float* s, const uint32_t* packed, con
   const MmLayout Lm = mm_layout(NT, k8max, gmax);
   // the attribute covers the largest layout any call can ask for
   const MmLayout Lmax = mm_layout(NT, (kMmMaxRows + 256) / 8, (kMmMaxRows + 256) / 32);
-  auto kern = w4a16_gemv_mma_kernel<NT, kZp>;
+  auto kern = w4a16_gemv_mma_kernel<NT, G, kZp>;
   static SmemAttrOnce once;
   cudaError_t e = set_smem_once(kern, Lmax.total, once);
   if (e != cudaSuccess) {
@@ -1447,7 +1451,7 @@ int launch_gemv_mma_k(const void* X, const float* s, const uint32_t* packed, con
   cfg.attrs = at;
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<const uint4*>(X), reinterpret_cast<const float4*>(s), packed,
-                         reinterpret_cast<const float4*>(scales), zeros, D_in, D_out, group, 1 << (bits - 1),
+                         reinterpret_cast<const float4*>(scales), zeros, D_in, D_out, 1 << (bits - 1),
                          static_cast<int>(S), cw, k8max, gmax, Y, status);
   if (e != cudaSuccess) {
     *cerr = e;
@@ -1457,15 +1461,28 @@ int launch_gemv_mma_k(const void* X, const float* s, const uint32_t* packed, con
   return kOk;
 }
 
+template <int NT, int G>
+int launch_gemv_mma_g(const void* X, const float* s, const uint32_t* packed, const float* scales,
+                      const uint8_t* zeros, int64_t D_in, int64_t D_out, int bits, float* Y, int num_sms, int* status,
+                      cudaStream_t st, cudaError_t* cerr, const char** what) {
+  if (zeros)
+    return launch_gemv_mma_k<NT, G, true>(X, s, packed, scales, zeros, D_in, D_out, bits, G, Y, num_sms, status, st,
+                                          cerr, what);
+  return launch_gemv_mma_k<NT, G, false>(X, s, packed, scales, nullptr, D_in, D_out, bits, G, Y, num_sms, status,
+                                         st, cerr, what);
+}
+
 template <int NT>
 int launch_gemv_mma(const void* X, const float* s, const uint32_t* packed, const float* scales, const uint8_t* zeros,
                     int64_t D_in, int64_t D_out, int bits, int group, float* Y, int num_sms, int* status,
                     cudaStream_t st, cudaError_t* cerr, const char** what) {
-  if (zeros)
-    return launch_gemv_mma_k<NT, true>(X, s, packed, scales, zeros, D_in, D_out, bits, group, Y, num_sms, status, st,
-                                       cerr, what);
-  return launch_gemv_mma_k<NT, false>(X, s, packed, scales, nullptr, D_in, D_out, bits, group, Y, num_sms, status,
-                                      st, cerr, what);
+  switch (group) {
+    case 32: return launch_gemv_mma_g<NT, 32>(X, s, packed, scales, zeros, D_in, D_out, bits, Y, num_sms, status, st, cerr, what);
+    case 64: return launch_gemv_mma_g<NT, 64>(X, s, packed, scales, zeros, D_in, D_out, bits, Y, num_sms, status, st, cerr, what);
+    case 128: return launch_gemv_mma_g<NT, 128>(X, s, packed, scales, zeros, D_in, D_out, bits, Y, num_sms, status, st, cerr, what);
+    case 256: return launch_gemv_mma_g<NT, 256>(X, s, packed, scales, zeros, D_in, D_out, bits, Y, num_sms, status, st, cerr, what);
+    default: *what = "gemv group"; return kEUnsupported;
+  }
 }
 
 int launch_w4a16_gemv(const void* X, const float* s, const uint32_t* packed, const float* scales,
@@ -1473,8 +1490,8 @@ int launch_w4a16_gemv(const void* X, const float* s, const uint32_t* packed, con
                       void* ws, int num_sms, int* status, cudaStream_t st, cudaError_t* cerr, const char** what) {
   // 3-4 tokens on the tensor cores while a CTA's share of the rows fits its
   // shared memory.  Two tokens stay on the CUDA cores: measured faster there
-  // (41.8 against 53.4 us on a 28672 x 8192 layer; at four tokens 73.2
-  // against 54.3 us).
+  // (41.8 against ~44.5 us on a 28672 x 8192 layer; at four tokens 73.2
+  // against 45.3 us).
   if (N >= 3 && D_in <= static_cast<int64_t>(kMmMaxSplit) * kMmMaxRows) {
     switch (N) {
       case 3: return launch_gemv_mma<3>(X, s, packed, scales, zeros, D_in, D_out, bits, group, Y, num_sms, status, st, cerr, what);
