@@ -138,11 +138,11 @@ def test_w4a16_decode_full_size(awq, N, D_in, D_out):
     assert np.all(np.abs(Y[:, cols] - Y_or) <= bound), np.max(np.abs(Y[:, cols] - Y_or) / bound)
 
 
-@pytest.mark.parametrize("N,D_in,D_out", [(1, 4096, 512), (2, 64, 128), (8, 1024, 256)])
+@pytest.mark.parametrize("N,D_in,D_out", [(1, 4096, 512), (2, 64, 128), (3, 1024, 256), (8, 1024, 256)])
 def test_w4a16_output_only_4_byte_aligned(awq, N, D_in, D_out):
-    """Y may be 4-byte aligned only (the ABI's requirement): the GEMV then
-    stores scalars; the values are those of an aligned Y, bit for bit (the
-    same sums in the same order)."""
+    """Y may be 4-byte aligned only (the ABI's requirement): the GEMVs then
+    store scalars (the mma.sync GEMV always does); the values are those of an
+    aligned Y, bit for bit (the same sums in the same order)."""
     X, W = synth.layer_inputs(synth.small_layer(max(N, 8), D_in, D_out, seed=3))
     X = X[:N].contiguous().cuda()
     s = torch.from_numpy(oracle.scales(oracle.act_stats(X.cpu()).astype(np.float32), 0.5)).cuda()
