@@ -868,15 +868,15 @@ def w4a16_section(dev, rank):
 
     bits, group = 4, 128
     g4 = torch.Generator(device=dev).manual_seed(4321 + rank)
-    info = {"timing": "best of 5 replays of a CUDA graph of 20 calls (N <= 4: one GEMV launch whose column-tile splits are "
-                      "reduced in a cluster (N = 1-2 on the CUDA cores, 3-4 on mma.sync tiles), or a stream-K GEMV "
+    info = {"timing": "best of 5 replays of a CUDA graph of 20 calls (N <= 8: one GEMV launch whose column-tile splits are "
+                      "reduced in a cluster (N = 1-2 on the CUDA cores, 3-8 on mma.sync tiles), or a stream-K GEMV "
                       "and a dependent reduce launch; else a status "
                       "clear, the pre-pass and the GEMM), weights rotated over copies > 256 MiB; synthetic "
                       "packed words and deltas",
             "algorithmic_bytes": "packed words + fp32 deltas + X (bf16) + s + Y (fp32), each once"}
     peaks, _ = load_peaks()
     hbm_peak, bf16_peak = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
-    for name, (Dk, Dn, Ns) in (("down_proj_28672x8192", (28672, 8192, (1, 2, 4, 16))),
+    for name, (Dk, Dn, Ns) in (("down_proj_28672x8192", (28672, 8192, (1, 2, 4, 8, 16))),
                                 ("attn_proj_4096x4096", (4096, 4096, (1, 4, 16, 4096))),
                                 ("square_8192x8192", (8192, 8192, (4096,)))):
         packed_q = torch.randint(-2 ** 31, 2 ** 31 - 1, (Dk // 8, Dn), generator=g4, device=dev,
@@ -894,7 +894,7 @@ def w4a16_section(dev, rank):
             gbs = nbytes / (ms / 1e3) / 1e9
             tf = 2.0 * Nq * Dk * Dn / (ms / 1e3) / 1e12
             info[f"{name}_N{Nq}"] = {
-                "path": ("cuda-core GEMV" if Nq <= 2 else "mma.sync GEMV") if Nq <= 4 else "tcgen05 GEMM", "ms": ms, "algorithmic_bytes": nbytes,
+                "path": ("cuda-core GEMV" if Nq <= 2 else "mma.sync GEMV") if Nq <= 8 else "tcgen05 GEMM", "ms": ms, "algorithmic_bytes": nbytes,
                 "achieved_gbs": gbs, "frac_hbm": gbs / hbm_peak, "tflops": tf, "frac_bf16": tf / bf16_peak}
         del weights, packed_q
     torch.cuda.empty_cache()

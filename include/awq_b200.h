@@ -409,12 +409,14 @@ AWQ_API int awq_quantize_pack_zp(const float* W, const float* s, int64_t D_in, i
  * in one wave, the (column tile, k rows) work is shared out evenly over a
  * grid that fills every SM (stream-K) and a second small launch adds the
  * CTAs' sums of each tile in a fixed order from the workspace.
- * N = 3 or 4 with D_in <= 65536: one launch of warp-level tensor-core tiles
- * (x / s rounded once to bf16, exact integer codes, fp32 accumulation, the
- * fp32 delta applied once per group), the splits of each column tile summed
- * in a fixed order inside a cluster; no workspace is used.  Longer rows take
- * the CUDA-core GEMV.
- * N > 4: two launches on `stream`, X' = bf16(X / s) into the workspace, then
+ * N = 3 to 8 with D_in <= 65536 (N <= 4) or 32768 (N >= 5): one launch of
+ * warp-level tensor-core tiles (x / s rounded once to bf16, exact integer
+ * codes, fp32 accumulation, the fp32 delta applied once per group), the
+ * splits of each column tile summed in a fixed order inside a cluster; no
+ * workspace is used.  Longer rows take the CUDA-core GEMV (N <= 4) or the
+ * GEMM below.
+ * N > 8 (and the longer rows at N 5..8): two launches on `stream`,
+ * X' = bf16(X / s) into the workspace, then
  * a tensor-core GEMM that dequantises the weights into shared memory as
  * bf16((u - 2^(bits-1)) * bf16(delta)) (one rounding of the product) and
  * accumulates in fp32.  For N <= 64 the k blocks of all output tiles are

@@ -44,9 +44,10 @@
 // Decode (N <= 4 tokens) takes a GEMV instead: there the work is a stream of
 // packed words with a few multiply-adds per weight, bound by HBM, and a
 // tcgen05 tile of 16+ tokens would sit mostly idle.  One or two tokens run on
-// the CUDA cores (w4a16_gemv_kernel); 3-4 tokens hand the products to
+// the CUDA cores (w4a16_gemv_kernel); 3-8 tokens hand the products to
 // warp-level mma.sync tiles of 8 token slots (w4a16_gemv_mma_kernel), since
-// four paired FMAs per word and token make the FMA pipe the bound.
+// from three tokens on the paired FMAs per word and token make the FMA pipe
+// the bound.
 //
 // Work: a unit is a 128-column x Nt-token output tile of KBS = ceil(KB /
 // KPS) stage steps.  Large N: units are dealt out to a persistent grid,
@@ -931,13 +932,13 @@ __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float4* __restri
 }
 
 
-// ------------------------------------------------------------ decode, 2-4 tokens, on the tensor cores
+// ------------------------------------------------------------ decode, 3-8 tokens, on the tensor cores
 //
-// With 3-4 tokens the GEMV above spends four paired FMAs per packed word and
-// token and the FMA pipe sets its time.  This form keeps the dequantisation on
+// With three or more tokens the GEMV above spends four paired FMAs per packed
+// word and token and the FMA pipe sets its time.  This form keeps the dequantisation on
 // the CUDA cores and hands the products to the tensor cores through warp-level
 // mma.sync m16n8k16 (bf16 operands, fp32 accumulation; N = 8 token slots, of
-// which 2-4 carry tokens).
+// which 3-8 carry tokens).
 //
 // Operands.  A packed word holds rows r0..r0+7 of one column.  The mask-and-OR
 // of (word >> 4i) with 0x000F000F | 0x43004300 is the exact bf16 pair
@@ -968,8 +969,13 @@ __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float4* __restri
 // CTAs beyond the cluster barrier, no workspace.
 constexpr int kMmThreads = 256;
 constexpr int kMmRing = 8;                       // 16-byte steps per lane in the ring (7 in flight)
-constexpr int kMmMaxRows = 8192;                 // rows of one CTA's range (X' in shared memory)
 constexpr int kMmMaxSplit = 8;                   // CTAs per tile: a portable cluster
+constexpr int kMmMaxTokens = 8;                  // the MMA's token slots
+// Rows of one CTA's range (X' of all tokens in shared memory) and warp slices
+// of 32 columns per CTA: 5-8 tokens take half the rows and twice the columns,
+// so that two CTAs still fit an SM and the tiles x splits still fill one wave.
+__host__ __device__ constexpr int mm_max_rows(int nt) { return nt <= 4 ? 8192 : 4096; }
+__host__ __device__ constexpr int mm_slices(int nt) { return nt <= 4 ? 4 : 8; }
 
 // Shared memory: X', the zero-point form's group sums of X', the ring; after
 // the main loop the ring holds the warps' sums (red) and the CTA's (fin).
@@ -988,7 +994,8 @@ __host__ __device__ inline MmLayout mm_layout(int nt, int k8max, int gmax) {
   L.total = L.ring + kMmRing * kMmThreads * 16;
   return L;
 }
-static_assert(2 * 4 * 256 * 4 + 4 * 256 * 4 <= kMmRing * kMmThreads * 16, "the sums fit in the ring");
+static_assert(2 * kMmMaxTokens * 256 * 4 + kMmMaxTokens * 256 * 4 <= kMmRing * kMmThreads * 16,
+              "the sums fit in the ring");
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
@@ -1021,7 +1028,7 @@ __global__ void __launch_bounds__(kMmThreads, 2) w4a16_gemv_mma_kernel(
     const uint4* __restrict__ X, const float4* __restrict__ s, const uint32_t* __restrict__ packed,
     const float4* __restrict__ scales, const uint8_t* __restrict__ zeros, int64_t D_in, int64_t D_out,
     int off, int S, int cw, int k8max, int gmax, float* __restrict__ Y, int* __restrict__ status) {
-  static_assert(NT >= 2 && NT <= 4, "2-4 token slots");
+  static_assert(NT >= 2 && NT <= kMmMaxTokens, "2-8 token slots");
   extern __shared__ __align__(16) uint8_t mm_sm[];
   const MmLayout Lm = mm_layout(NT, k8max, gmax);
   uint8_t* xs = mm_sm + Lm.xs;
@@ -1407,18 +1414,18 @@ int launch_gemv_nt(const void* X, const float* s, const uint32_t* packed, const 
   }
 }
 
-// The tensor-core GEMV for 3-4 tokens (w4a16_gemv_mma_kernel): tiles of 128
-// columns; S CTAs per tile, as many as keep two CTAs on every SM (at most 8,
-// at least enough that no CTA's range of groups exceeds kMmMaxRows rows), in
-// clusters of S.
+// The tensor-core GEMV for 3-8 tokens (w4a16_gemv_mma_kernel): tiles of
+// 32 mm_slices(NT) columns; S CTAs per tile, as many as keep two CTAs on every
+// SM (at most 8, at least enough that no CTA's range of groups exceeds
+// mm_max_rows(NT) rows), in clusters of S.
 template <int NT, int G, bool kZp>
 int launch_gemv_mma_k(const void* X, const float* s, const uint32_t* packed, const float* scales,
                       const uint8_t* zeros, int64_t D_in, int64_t D_out, int bits, int group, float* Y, int num_sms,
                       int* status, cudaStream_t st, cudaError_t* cerr, const char** what) {
   const int64_t ng = D_in / group;
   const int64_t sms = num_sms > 0 ? num_sms : 1;
-  const int64_t smin = (D_in + kMmMaxRows - 1) / kMmMaxRows;
-  const int cw = 4;
+  const int64_t smin = (D_in + mm_max_rows(NT) - 1) / mm_max_rows(NT);
+  const int cw = mm_slices(NT);
   const int64_t tiles = (D_out + 32 * cw - 1) / (32 * cw);
   int64_t S = 2 * sms / tiles;
   if (S > kMmMaxSplit) S = kMmMaxSplit;
@@ -1429,7 +1436,7 @@ int launch_gemv_mma_k(const void* X, const float* s, const uint32_t* packed, con
   const int k8max = gmax * (group / 8);
   const MmLayout Lm = mm_layout(NT, k8max, gmax);
   // the attribute covers the largest layout any call can ask for
-  const MmLayout Lmax = mm_layout(NT, (kMmMaxRows + 256) / 8, (kMmMaxRows + 256) / 32);
+  const MmLayout Lmax = mm_layout(NT, (mm_max_rows(NT) + 256) / 8, (mm_max_rows(NT) + 256) / 32);
   auto kern = w4a16_gemv_mma_kernel<NT, G, kZp>;
   static SmemAttrOnce once;
   cudaError_t e = set_smem_once(kern, Lmax.total, once);
@@ -1492,7 +1499,7 @@ int launch_w4a16_gemv(const void* X, const float* s, const uint32_t* packed, con
   // shared memory.  Two tokens stay on the CUDA cores: measured faster there
   // (41.8 against ~44.5 us on a 28672 x 8192 layer; at four tokens 73.2
   // against 45.3 us).
-  if (N >= 3 && D_in <= static_cast<int64_t>(kMmMaxSplit) * kMmMaxRows) {
+  if (N >= 3 && D_in <= static_cast<int64_t>(kMmMaxSplit) * mm_max_rows(static_cast<int>(N))) {
     switch (N) {
       case 3: return launch_gemv_mma<3>(X, s, packed, scales, zeros, D_in, D_out, bits, group, Y, num_sms, status, st, cerr, what);
       case 4: return launch_gemv_mma<4>(X, s, packed, scales, zeros, D_in, D_out, bits, group, Y, num_sms, status, st, cerr, what);
@@ -1523,6 +1530,17 @@ int launch_w4a16(const void* X, const float* s, const uint32_t* packed, const fl
   if (N <= kGvMaxTokens)
     return launch_w4a16_gemv(X, s, packed, scales, zeros, N, D_in, D_out, bits, group, Y, ws, num_sms, status, st,
                              cerr, what);
+  // 5-8 tokens fill the token slots of the GEMV's MMA tiles: one launch and
+  // no workspace, where a tcgen05 tile of 16 tokens would sit half idle.
+  if (N <= kMmMaxTokens && D_in <= static_cast<int64_t>(kMmMaxSplit) * mm_max_rows(static_cast<int>(N))) {
+    switch (N) {
+      case 5: return launch_gemv_mma<5>(X, s, packed, scales, zeros, D_in, D_out, bits, group, Y, num_sms, status, st, cerr, what);
+      case 6: return launch_gemv_mma<6>(X, s, packed, scales, zeros, D_in, D_out, bits, group, Y, num_sms, status, st, cerr, what);
+      case 7: return launch_gemv_mma<7>(X, s, packed, scales, zeros, D_in, D_out, bits, group, Y, num_sms, status, st, cerr, what);
+      case 8: return launch_gemv_mma<8>(X, s, packed, scales, zeros, D_in, D_out, bits, group, Y, num_sms, status, st, cerr, what);
+      default: break;
+    }
+  }
   const bool zp = zeros != nullptr;
   const W4Layout lay = w4_layout(N, D_in, D_out, zp ? D_in / group : 0);
   uint8_t* wsb = static_cast<uint8_t*>(ws);

@@ -4,9 +4,10 @@ itself.
 
 Three CUDA paths: one or two tokens run the CUDA-core GEMV (fp32 throughout:
 x / s rounded once to fp32, exact integer weights, delta applied per group);
-three or four tokens run the mma.sync GEMV (x / s rounded once to bf16, exact
-integer codes, fp32 accumulation, the fp32 delta applied per group); more
-tokens run the tcgen05 GEMM.  The bound below, derived for the GEMM, covers the GEMVs'
+three to eight tokens run the mma.sync GEMV (x / s rounded once to bf16,
+exact integer codes, fp32 accumulation, the fp32 delta applied per group;
+longer rows than it stages take the neighbouring path); more tokens run the
+tcgen05 GEMM.  The bound below, derived for the GEMM, covers the GEMVs'
 smaller errors too.
 
 Tolerance, from the arithmetic of the tensor-core path: x_tk / s_k is rounded to
@@ -98,6 +99,9 @@ def _case(awq, N, D_in, D_out, bits, group, seed):
     (3, 65792, 64, 4, 256),       # past that range: the CUDA-core GEMV at three tokens
     (4, 4096, 1280, 3, 64),       # 3-4 tokens: ten tiles split eight ways
     (4, 96, 4, 4, 32),            # 3-4 tokens: three groups over eight warps, one column quad
+    (6, 4096, 1028, 2, 32),       # 5-8 tokens: 256-column tiles, ragged last tile, 2-bit
+    (8, 32768, 512, 4, 128),      # eight tokens: eight CTAs of 4096 rows, the largest X' in shared memory
+    (5, 33024, 64, 4, 256),       # past that range: the tcgen05 GEMM at five tokens
 ])
 def test_w4a16_against_oracle(awq, N, D_in, D_out, bits, group):
     Y, Y_or, bound = _case(awq, N, D_in, D_out, bits, group, seed=N + D_in)
@@ -190,7 +194,9 @@ def _zp_case(awq, N, D_in, D_out, bits, group, seed):
     (2, 2048, 256, 4, 256),       # GEMV, group 256
     (1, 1024, 32768, 4, 128),     # GEMV: stream-K shares and the reduce launch
     (3, 256, 38912, 4, 64),       # GEMV: one CTA per whole tile
-    (5, 512, 200, 4, 128),        # tensor cores, stream-K, ragged columns
+    (5, 512, 200, 4, 128),        # mma.sync GEMV, ragged columns
+    (7, 1024, 520, 3, 64),        # mma.sync GEMV, seven tokens
+    (9, 512, 200, 4, 128),        # tensor cores, stream-K, ragged columns
     (37, 384, 132, 3, 64),
     (17, 8192, 2048, 4, 128),     # stream-K shares inside one unit
     (300, 1024, 260, 4, 128),     # two token tiles, no split
