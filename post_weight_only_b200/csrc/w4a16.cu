@@ -935,10 +935,11 @@ __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float4* __restri
 // ------------------------------------------------------------ decode, 3-8 tokens, on the tensor cores
 //
 // With three or more tokens the GEMV above spends four paired FMAs per packed
-// word and token and the FMA pipe sets its time.  This form keeps the dequantisation on
-// the CUDA cores and hands the products to the tensor cores through warp-level
-// mma.sync m16n8k16 (bf16 operands, fp32 accumulation; N = 8 token slots, of
-// which 3-8 carry tokens).
+// word and token and the FMA pipe sets its time; up to 16 tokens the tcgen05
+// GEMM below pads them to one 16-token tile.  This form keeps the
+// dequantisation on the CUDA cores and hands the products to the tensor cores
+// through warp-level mma.sync m16n8k16 (bf16 operands, fp32 accumulation;
+// N = 8 token slots, of which 3-8 carry tokens).
 //
 // Operands.  A packed word holds rows r0..r0+7 of one column.  The mask-and-OR
 // of (word >> 4i) with 0x000F000F | 0x43004300 is the exact bf16 pair
@@ -954,19 +955,19 @@ __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float4* __restri
 // c0+1 are A rows g and g+8 of one accumulator, c0+2 and c0+3 of another, so
 // each lane ends with the sums of its own four columns for tokens 2j and 2j+1.
 //
-// Work: a CTA takes 32 cw columns (cw = 8 or 4 warp slices of 32) and a range
-// of whole groups, split between the 8 / cw warps of a slice; the S CTAs that
-// split one tile's groups form a cluster, and rank 0 adds their sums in rank
-// order from their shared memory (DSMEM), so the result does not depend on
-// timing.  Each lane keeps 7 steps of 16 bytes in flight (a ring of cp.async
-// copies in shared memory); the loop runs over the warp's groups with the
-// group's steps unrolled (the group size is a template argument), which cut
-// the loop's bookkeeping by a sixth of the time.  The host takes cw = 4:
-// 256-column tiles and a ring of 16 steps were both measured slower on a
-// 28672 x 8192 layer.  A group's
-// delta is applied once, after its last step; the zero-point form adds
-// (off - z) times the group's sum of X' at the same point.  No waits on other
-// CTAs beyond the cluster barrier, no workspace.
+// Work: a CTA takes 32 cw columns (cw = mm_slices(NT) warp slices of 32: 4
+// for 3-4 tokens, 8 for 5-8) and a range of whole groups, split between the
+// 8 / cw warps of a slice; the S CTAs that split one tile's groups form a
+// cluster, and rank 0 adds their sums in rank order from their shared memory
+// (DSMEM), so the result does not depend on timing.  Each lane keeps 7 steps
+// of 16 bytes in flight (a ring of cp.async copies in shared memory); the loop
+// runs over the warp's groups with the group's steps unrolled (the group size
+// is a template argument), which cut the time by a sixth at four tokens.  At
+// four tokens on a 28672 x 8192 layer, 256-column tiles and a ring of 16 steps
+// were both measured slower.  A group's delta is applied once, after its last
+// step; the zero-point form adds (off - z) times the group's sum of X' at the
+// same point.  No waits on other CTAs beyond the cluster barrier, no
+// workspace.
 constexpr int kMmThreads = 256;
 constexpr int kMmRing = 8;                       // 16-byte steps per lane in the ring (7 in flight)
 constexpr int kMmMaxSplit = 8;                   // CTAs per tile: a portable cluster
