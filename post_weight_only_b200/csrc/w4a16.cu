@@ -41,7 +41,7 @@
 //               contiguous over n) and writes chunks 4h..4h+3 of row n of
 //               the A tile.
 //   warps 11-14 epilogue: TMEM lanes 32 (w % 4) .. + 31 -> Y.
-// Decode (N <= 4 tokens) takes a GEMV instead: there the work is a stream of
+// Decode (N <= 8 tokens) takes a GEMV instead: there the work is a stream of
 // packed words with a few multiply-adds per weight, bound by HBM, and a
 // tcgen05 tile of 16+ tokens would sit mostly idle.  One or two tokens run on
 // the CUDA cores (w4a16_gemv_kernel); 3-8 tokens hand the products to
@@ -520,7 +520,8 @@ __global__ void __launch_bounds__(kW4Threads, 1)
 
 // ------------------------------------------------------------ decode: the GEMV
 // Y[t][n] = sum_g delta_{g,n} (sum_{k in g} x'_tk u_kn - z_{g,n} sum_{k in g} x'_tk)
-// on CUDA cores for N <= 4 tokens, fp32 throughout: x' = x / s rounded once
+// on CUDA cores for one or two tokens (and for three or four on rows longer
+// than the mma.sync GEMV below stages), fp32 throughout: x' = x / s rounded once
 // (IEEE division), the integer weights exact, delta applied once per group;
 // z is 2^(b-1) for the offset-binary codes, the group's zero point for
 // asymmetric ones.

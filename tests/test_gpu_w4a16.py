@@ -72,15 +72,15 @@ def _case(awq, N, D_in, D_out, bits, group, seed):
 @pytest.mark.parametrize("N,D_in,D_out,bits,group", [
     (1, 4096, 4096, 4, 128),      # one decode token: the GEMV, split K
     (2, 512, 200, 4, 128),        # GEMV: ragged second column tile
-    (4, 1024, 132, 3, 64),        # GEMV at its largest token count
+    (4, 1024, 132, 3, 64),        # mma.sync GEMV, 3-bit, ragged column tile
     (1, 32, 4, 4, 32),            # GEMV: one group, four k8 rows (fewer than the warps), one column quad
     (2, 2048, 256, 4, 256),       # GEMV, group 256
-    (3, 256, 1000, 2, 32),        # GEMV, 2-bit, group 32
+    (3, 256, 1000, 2, 32),        # mma.sync GEMV, 2-bit, group 32
     (1, 256, 38912, 4, 128),      # GEMV: more column tiles (304) than resident CTAs, one CTA per whole tile
     (2, 1024, 38916, 4, 64),      # the same with a ragged last tile of one column quad, 8-row batches
     (1, 128, 2048, 4, 64),        # GEMV: too few batches for clusters, stream-K shares and the reduce launch
-    (4, 1024, 32768, 4, 128),     # GEMV, four tokens: more tiles than resident clusters, stream-K
-    (3, 1024, 32768, 2, 32),      # GEMV, three tokens, 2-bit, group 32: stream-K
+    (4, 1024, 32768, 4, 128),     # mma.sync GEMV, four tokens: 256 tiles, unsplit
+    (3, 1024, 32768, 2, 32),      # mma.sync GEMV, three tokens, 2-bit, group 32: 256 tiles, unsplit
     (5, 512, 200, 4, 128),        # ragged columns, a few tokens
     (16, 96, 36, 4, 32),          # D_in not a multiple of 64: a half k block
     (37, 384, 132, 3, 64),
